@@ -1,0 +1,418 @@
+"""CPU oracle of the Wan2.1-style I2V DiT denoising step and its CFG Euler sampler.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+module.  The CUDA library never calls it and shares no code with it.
+
+Plain, slow and obviously correct: float64 numpy, materialised softmax per
+query row, library matmul/erf as the only primitives, no blocking or fusion.
+Every function cites the passage of the source pages it follows:
+
+* [I2V]  "图解 Wan2.1 I2V：从一张图到一段视频，模型到底发生了什么" (liyongzhi.xyz)
+* [WAN]  "Wan（通义万相）：大规模视频生成基础模型 — 技术深度解析 & Wan2.1 vs Wan2.2对比"
+         (devpress.csdn.net)
+* [MLQM] "从热词到架构：Wan2.1到底在解决什么问题" (mlqm.cn)
+
+Where the pages are silent the oracle takes the plainest reading; each one is
+marked "Reading:" below.  Storage rounding: with ``rnd=True`` the oracle rounds
+to bfloat16 (round-to-nearest-even) at exactly the points where the GPU path
+stores a bf16 tensor (GEMM operands, q/k/v, attention outputs, FFN hidden, the
+cross-attention K/V cache), so a bf16 run is compared with the same function.
+Parity pins: see tests/test_oracle_*.py.  Functions whose full output no page
+pins ("parity unpinned"): dit_forward / block_forward values beyond the
+invariants (AdaLN-Zero identity, attention and RoPE special cases) checked in
+the tests; the pages print no tensor values.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+from scipy.special import erf as _erf
+
+F64 = np.float64
+
+
+# ---------------------------------------------------------------- storage rounding
+def bf16(a) -> np.ndarray:
+    """Round to the nearest bfloat16 value, ties to even (8 significant bits).
+
+    Reading: the pages fix no precision; bf16 storage with round-to-nearest-even
+    is the GPU path's storage type.  frexp gives a = m * 2**e with |m| in
+    [0.5, 1); keeping 8 significant bits means rounding m * 2**8 to an integer
+    (numpy's rint rounds halves to even).
+    """
+    a = np.asarray(a, dtype=F64)
+    m, e = np.frexp(a)
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
+
+
+def _st(a, rnd: bool):
+    return bf16(a) if rnd else np.asarray(a, dtype=F64)
+
+
+# ---------------------------------------------------------------- shapes
+def token_count(F: int, H: int, W: int) -> int:
+    """Tokens of an F-frame H x W video: latent (1+(F-1)/4) x H/8 x W/8, then the
+    (1,2,2) patch halves each spatial side ([I2V] 2, 5.1; [WAN] 2.2, 2.5)."""
+    T = 1 + (F - 1) // 4
+    return T * (H // 16) * (W // 16)
+
+
+def grid_positions(T: int, Hp: int, Wp: int):
+    """Token order l = (f*Hp + y)*Wp + x, the flattening of the Conv3d output grid
+    [T, Hp, Wp] ([I2V] 5.1).  Returns the (frame, row, column) of every token."""
+    f, y, x = np.meshgrid(np.arange(T), np.arange(Hp), np.arange(Wp), indexing="ij")
+    return f.reshape(-1), y.reshape(-1), x.reshape(-1)
+
+
+# ---------------------------------------------------------------- conditioning y
+def mask_frames(T: int, known_pixel_frames=(0,)) -> np.ndarray:
+    """Temporal mask m [4, T] of [I2V] 4.1 step 3 (and Q3, Q6).
+
+    A pixel-frame mask of length F = 4(T-1)+1 holds 1 at known frames.  Frame 0
+    is repeated 4 times in front of frames 1..F-1, giving 4T entries s, which
+    are grouped into consecutive runs of 4: m[c, f] = s[4f + c].
+    Reading: the grouping is by consecutive runs (one latent frame = 4 pixel
+    frames), which puts all ones of the default mask on latent frame 0.
+    """
+    F = 4 * (T - 1) + 1
+    known = set(int(p) for p in known_pixel_frames)
+    pix = np.array([1.0 if p in known else 0.0 for p in range(F)])
+    s = np.concatenate([np.repeat(pix[:1], 4), pix[1:]])
+    assert s.shape[0] == 4 * T
+    m = np.empty((4, T))
+    for f in range(T):
+        for c in range(4):
+            m[c, f] = s[4 * f + c]
+    return m
+
+
+def build_cond_y(img_lat: np.ndarray, known_pixel_frames=(0,)) -> np.ndarray:
+    """y = concat(mask [4,T,H,W], image latent [16,T,H,W]) -> [20,T,H,W]
+    ([I2V] 4.1 step 4)."""
+    C, T, H, W = img_lat.shape
+    m = mask_frames(T, known_pixel_frames)
+    mask = np.broadcast_to(m[:, :, None, None], (4, T, H, W))
+    return np.concatenate([mask, np.asarray(img_lat, F64)], axis=0)
+
+
+# ---------------------------------------------------------------- elementwise pieces
+def silu(x):
+    x = np.asarray(x, F64)
+    return x / (1.0 + np.exp(-x))
+
+
+def gelu(x):
+    """Exact GELU x * Phi(x) ([I2V] 5.5: Linear -> GELU -> Linear).
+    Reading: the erf form (no tanh approximation)."""
+    x = np.asarray(x, F64)
+    return 0.5 * x * (1.0 + _erf(x / math.sqrt(2.0)))
+
+
+def linear(x, w, b=None):
+    """y = x W^T + b with W stored [out, in]."""
+    y = np.asarray(x, F64) @ np.asarray(w, F64).T
+    if b is not None:
+        y = y + np.asarray(b, F64)
+    return y
+
+
+def layer_norm(x, eps: float, gamma=None, beta=None):
+    x = np.asarray(x, F64)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    y = (x - mu) / np.sqrt(var + eps)
+    if gamma is not None:
+        y = y * np.asarray(gamma, F64)
+    if beta is not None:
+        y = y + np.asarray(beta, F64)
+    return y
+
+
+def rms_norm(x, eps: float, gamma=None):
+    x = np.asarray(x, F64)
+    y = x / np.sqrt((x * x).mean(axis=-1, keepdims=True) + eps)
+    if gamma is not None:
+        y = y * np.asarray(gamma, F64)
+    return y
+
+
+def adaln_modulate(x, shift, scale, eps: float, norm: str = "layer"):
+    """x' = norm(x) * (1 + scale) + shift ([I2V] 5.2).
+    Reading: norm is LayerNorm without affine, eps 1e-6 (the page names
+    LayerNorm); norm="rms" selects RMSNorm instead."""
+    n = layer_norm(x, eps) if norm == "layer" else rms_norm(x, eps)
+    return n * (1.0 + np.asarray(scale, F64)) + np.asarray(shift, F64)
+
+
+# ---------------------------------------------------------------- timestep embedding
+def sinusoid(tau: float, dim: int = 256) -> np.ndarray:
+    """sinusoidal_embedding_1d(256, t) of [I2V] 5.2.
+    Reading: [cos(tau w_i), sin(tau w_i)], w_i = 10000^(-i/128), i = 0..127."""
+    half = dim // 2
+    w = np.power(10000.0, -np.arange(half, dtype=F64) / half)
+    a = float(tau) * w
+    return np.concatenate([np.cos(a), np.sin(a)])
+
+
+def time_mod(wts: dict, tau: float, D: int):
+    """Shared time MLP ([I2V] 5.2; [WAN] 2.5 "shared MLP + per-block bias").
+
+    e  = Linear2(SiLU(Linear1(sinusoid(tau))))          [D]
+    e0 = time_projection(SiLU(e)) reshaped to [6, D] in the order
+         (shift1, scale1, gate1, shift2, scale2, gate2).
+    Reading: SiLU activations as in the DiT reference design the page cites.
+    """
+    es = sinusoid(tau, 256)
+    e = linear(silu(linear(es, wts["t1.w"], wts["t1.b"])), wts["t2.w"], wts["t2.b"])
+    e0 = linear(silu(e), wts["tp.w"], wts["tp.b"]).reshape(6, D)
+    return e, e0
+
+
+# ---------------------------------------------------------------- 3D RoPE
+def rope_split(dh: int):
+    """Per-head split of [I2V] 5.3: frame d - 4(d/6), row 2(d/6), column 2(d/6)."""
+    s = dh // 6
+    return dh - 4 * s, 2 * s, 2 * s
+
+
+def rope_3d(x, pos_f, pos_y, pos_x):
+    """Factorised 3D rotary embedding on x [N, heads, dh] ([I2V] 5.3).
+
+    Each head is cut into segments (frame, row, column) of rope_split(dh)
+    channels; each segment gets 1D RoPE with its own coordinate.
+    Reading: channel pairs (2j, 2j+1) are (real, imaginary) and pair j of a
+    segment of size d_s turns by pos * 10000^(-2j/d_s).
+    """
+    x = np.asarray(x, F64)
+    N, h, dh = x.shape
+    out = np.empty_like(x)
+    off = 0
+    for size, pos in zip(rope_split(dh), (pos_f, pos_y, pos_x)):
+        j = np.arange(size // 2, dtype=F64)
+        freq = np.power(10000.0, -2.0 * j / size)
+        theta = np.asarray(pos, F64)[:, None] * freq[None, :]          # [N, size/2]
+        c, s = np.cos(theta)[:, None, :], np.sin(theta)[:, None, :]
+        re = x[:, :, off:off + size:2]
+        im = x[:, :, off + 1:off + size:2]
+        out[:, :, off:off + size:2] = re * c - im * s
+        out[:, :, off + 1:off + size:2] = re * s + im * c
+        off += size
+    return out
+
+
+# ---------------------------------------------------------------- attention
+def attention(q, k, v):
+    """softmax(q k^T / sqrt(dh)) v per head, no mask ([I2V] 5.3, 5.4).
+
+    q [Nq, h, dh], k/v [Nk, h, dh] -> [Nq, h, dh].  The softmax is
+    materialised per query row (subtracting the row maximum).
+    Reading: scale 1/sqrt(dh); no key mask (the pages show none).
+    """
+    q, k, v = (np.asarray(a, F64) for a in (q, k, v))
+    Nq, h, dh = q.shape
+    out = np.empty((Nq, h, v.shape[2]))
+    for hh in range(h):
+        s = (q[:, hh, :] @ k[:, hh, :].T) / math.sqrt(dh)
+        s = s - s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        p = p / p.sum(axis=1, keepdims=True)
+        out[:, hh, :] = p @ v[:, hh, :]
+    return out
+
+
+# ---------------------------------------------------------------- patchify / unpatchify
+def patchify(x_in):
+    """[B, C, T, H, W] -> [B, L, C*4]: the receptive fields of Conv3d(k=(1,2,2),
+    s=(1,2,2)) ([I2V] 5.1), flattened in the weight order (c, kh, kw)."""
+    x_in = np.asarray(x_in, F64)
+    B, C, T, H, W = x_in.shape
+    Hp, Wp = H // 2, W // 2
+    p = x_in.reshape(B, C, T, Hp, 2, Wp, 2)
+    p = p.transpose(0, 2, 3, 5, 1, 4, 6)              # B, T, Hp, Wp, C, kh, kw
+    return p.reshape(B, T * Hp * Wp, C * 4)
+
+
+def unpatchify(p, T: int, Hp: int, Wp: int, C: int = 16):
+    """Inverse of patchify: v[b, c, f, 2y+kh, 2x+kw] = p[b, l, c*4 + kh*2 + kw]
+    with l = (f*Hp + y)*Wp + x ([I2V] 5.5 "Head ... and unpatchify").
+    Reading: output feature order (c, kh, kw), mirroring the Conv3d weight."""
+    p = np.asarray(p, F64)
+    B = p.shape[0]
+    v = p.reshape(B, T, Hp, Wp, C, 2, 2).transpose(0, 4, 1, 2, 5, 3, 6)
+    return v.reshape(B, C, T, 2 * Hp, 2 * Wp)
+
+
+def patch_embed(x_t, y, w_pe, b_pe, rnd: bool = False):
+    """tokens = Conv3d(36, D, (1,2,2), stride (1,2,2))(concat(x_t, y)) as a GEMM
+    ([I2V] 4.2 for the 36-channel concat, 5.1 for the patchify).
+    x_t [B,16,T,H,W]; y [20,T,H,W] shared by the batch -> [B, L, D]."""
+    x_t = np.asarray(x_t, F64)
+    B = x_t.shape[0]
+    yb = np.broadcast_to(np.asarray(y, F64)[None], (B,) + np.shape(y))
+    x_in = np.concatenate([x_t, yb], axis=1)
+    return linear(_st(patchify(x_in), rnd), w_pe, b_pe)
+
+
+# ---------------------------------------------------------------- context (once per video)
+def context_embed(w: dict, txt, clip, rnd: bool = False):
+    """Text MLP [n_txt, c_txt] -> [n_txt, D] and CLIP MLPProj [n_img, c_img] ->
+    [n_img, D] ([I2V] 7 steps 1-2).  txt is [B, n_txt, c_txt] (the
+    unconditional row carries zeroed text, [I2V] Q5); clip is [n_img, c_img].
+    Reading: each MLP is Linear -> GELU -> Linear with biases."""
+    t = _st(gelu(linear(txt, w["txt1.w"], w["txt1.b"])), rnd)
+    ctx_txt = _st(linear(t, w["txt2.w"], w["txt2.b"]), rnd)
+    i = _st(gelu(linear(clip, w["img1.w"], w["img1.b"])), rnd)
+    ctx_img = _st(linear(i, w["img2.w"], w["img2.b"]), rnd)
+    return ctx_txt, ctx_img
+
+
+def cross_kv(w: dict, blk: int, ctx_txt, ctx_img, rnd: bool = False):
+    """Per-block cross-attention keys/values of [I2V] 5.4: the text branch uses
+    Linear_k / Linear_v, the image branch its own k_img / v_img."""
+    p = f"blk{blk}."
+    return dict(
+        k_txt=_st(linear(ctx_txt, w[p + "ck.w"], w[p + "ck.b"]), rnd),
+        v_txt=_st(linear(ctx_txt, w[p + "cv.w"], w[p + "cv.b"]), rnd),
+        k_img=_st(linear(ctx_img, w[p + "cki.w"], w[p + "cki.b"]), rnd),
+        v_img=_st(linear(ctx_img, w[p + "cvi.w"], w[p + "cvi.b"]), rnd),
+    )
+
+
+# ---------------------------------------------------------------- one DiT block
+def block_forward(X, e0, w: dict, blk: int, kv: dict, dims, rnd: bool = False, rows=None):
+    """One DiT block ([I2V] 5.2-5.5), order self-attention -> cross -> FFN.
+
+    X [B, L, D] residual stream; e0 [6, D]; kv from cross_kv (k_txt/v_txt
+    [B, n_txt, D], k_img/v_img [n_img, D]).  ``rows`` (optional index array)
+    computes the output only for those token rows of every sample; keys and
+    values still cover all L tokens, so the result is exact for those rows.
+
+    mod = e0 + b_i                                    ([WAN] 2.5)
+    h   = norm(X)(1 + scale1) + shift1                ([I2V] 5.2)
+    q,k = RMSNorm(Linear_q/k h), v = Linear_v h       ([I2V] 5.3 (1))
+    q,k = RoPE3D(q), RoPE3D(k)                        ([I2V] 5.3 (2))
+    X  += gate1 * Linear_o(attn(q, k, v))             ([I2V] 5.2, 5.3)
+    X  += Linear_co(attn(qc, K_img, V_img) + attn(qc, K_txt, V_txt)),
+          qc = Linear_cq(LN_affine(X))                ([I2V] 5.4; no adaLN, no gate)
+    X  += gate2 * Linear_2(GELU(Linear_1(norm(X)(1+scale2)+shift2)))   ([I2V] 5.5)
+    Readings: QK-RMSNorm over the full width D with learned gains, before the
+    head split; the cross-attention input gets a LayerNorm with affine gains.
+    """
+    p = f"blk{blk}."
+    D, nh, dh, eps = dims.D, dims.heads, dims.dh, dims.eps
+    X = np.asarray(X, F64)
+    B, L, _ = X.shape
+    rows = np.arange(L) if rows is None else np.asarray(rows)
+    mod = np.asarray(e0, F64) + np.asarray(w[p + "mod"], F64)
+    shift1, scale1, gate1, shift2, scale2, gate2 = mod
+    pf, py, px = grid_positions(dims.T, dims.Hp, dims.Wp)
+
+    out = np.empty((B, len(rows), D))
+    for b in range(B):
+        x = X[b]
+        # ---- self-attention (keys and values need every token)
+        h = _st(adaln_modulate(x, shift1, scale1, eps, dims.norm), rnd)
+        qkv = _st(linear(h, w[p + "qkv.w"], w[p + "qkv.b"]), rnd)
+        q, k, v = qkv[:, :D], qkv[:, D:2 * D], qkv[:, 2 * D:]
+        q = rms_norm(q[rows], eps, w[p + "gq"]).reshape(len(rows), nh, dh)
+        k = rms_norm(k, eps, w[p + "gk"]).reshape(L, nh, dh)
+        q = _st(rope_3d(q, pf[rows], py[rows], px[rows]), rnd)
+        k = _st(rope_3d(k, pf, py, px), rnd)
+        v = v.reshape(L, nh, dh)
+        o = _st(attention(q, k, v).reshape(len(rows), D), rnd)
+        xr = x[rows] + gate1 * linear(o, w[p + "o.w"], w[p + "o.b"])
+        # ---- decoupled cross-attention (not modulated, not gated)
+        hc = _st(layer_norm(xr, eps, w[p + "cn.g"], w[p + "cn.b"]), rnd)
+        qc = _st(linear(hc, w[p + "cq.w"], w[p + "cq.b"]), rnd).reshape(len(rows), nh, dh)
+        kt, vt = kv["k_txt"][b], kv["v_txt"][b]
+        ki, vi = kv["k_img"], kv["v_img"]
+        o_img = attention(qc, ki.reshape(-1, nh, dh), vi.reshape(-1, nh, dh))
+        o_txt = attention(qc, kt.reshape(-1, nh, dh), vt.reshape(-1, nh, dh))
+        oc = _st((o_img + o_txt).reshape(len(rows), D), rnd)
+        xr = xr + linear(oc, w[p + "co.w"], w[p + "co.b"])
+        # ---- gated FFN
+        h2 = _st(adaln_modulate(xr, shift2, scale2, eps, dims.norm), rnd)
+        u = _st(gelu(linear(h2, w[p + "f1.w"], w[p + "f1.b"])), rnd)
+        out[b] = xr + gate2 * linear(u, w[p + "f2.w"], w[p + "f2.b"])
+    return out
+
+
+# ---------------------------------------------------------------- head
+def head_unpatchify(X, e, w: dict, dims, rnd: bool = False):
+    """Head with adaLN and unpatchify ([I2V] 5.5): z = LN(X)(1+sc)+sh with
+    (sh, sc) = e + b_head; p = Linear(D -> 16*1*2*2)(z); v = unpatchify(p).
+    Reading: shift then scale rows of b_head [2, D], added to e (not e0)."""
+    sh = np.asarray(e, F64) + np.asarray(w["head.mod"][0], F64)
+    sc = np.asarray(e, F64) + np.asarray(w["head.mod"][1], F64)
+    z = _st(adaln_modulate(X, sh, sc, dims.eps, "layer"), rnd)
+    p = linear(z, w["head.w"], w["head.b"])
+    return unpatchify(p, dims.T, dims.Hp, dims.Wp)
+
+
+# ---------------------------------------------------------------- whole DiT
+def dit_forward(x_t, y, tau: float, w: dict, kvs: list, dims, rnd: bool = False):
+    """v = DiT(concat(x_t, y), tau, context) for a batch ([I2V] 5, 7)."""
+    e, e0 = time_mod(w, tau, dims.D)
+    X = patch_embed(x_t, y, w["pe.w"], w["pe.b"], rnd)
+    for i in range(dims.blocks):
+        X = block_forward(X, e0, w, i, kvs[i], dims, rnd)
+    return head_unpatchify(X, e, w, dims, rnd)
+
+
+# ---------------------------------------------------------------- flow matching + sampler
+def fm_path(x0, x1, t: float):
+    """x_t = (1-t) x0 + t x1 with x0 noise and x1 data ([WAN] 2.7)."""
+    return (1.0 - t) * np.asarray(x0, F64) + t * np.asarray(x1, F64)
+
+
+def fm_velocity(x0, x1):
+    """v = x1 - x0 ([WAN] 2.7)."""
+    return np.asarray(x1, F64) - np.asarray(x0, F64)
+
+
+def cfg_combine(v_c, v_u, s: float):
+    """v = v_u + s (v_c - v_u) ([I2V] 7)."""
+    v_c, v_u = np.asarray(v_c, F64), np.asarray(v_u, F64)
+    return v_u + s * (v_c - v_u)
+
+
+def euler_cfg_step(x, v_c, v_u, s: float, dt: float):
+    """Explicit Euler step of dx/dt = v from t to t+dt ([WAN] 2.7 "20-50 Euler
+    steps"; [MLQM] 3.2), with CFG ([I2V] 7).  v_u None means no guidance."""
+    v = np.asarray(v_c, F64) if v_u is None else cfg_combine(v_c, v_u, s)
+    return np.asarray(x, F64) + dt * v
+
+
+def schedule(N: int):
+    """Uniform grid t_k = k/N on [0, 1] with dt = 1/N; the model sees
+    tau_k = 1000 (1 - t_k).  Reading: the [WAN] 2.7 convention (x0 noise at
+    t=0, data at t=1) integrated forward; tau is the noise level x 1000, which
+    is the [I2V] 7 schedule (1.0 at noise) on a 0..1000 scale."""
+    return [(k / N, 1.0 / N, 1000.0 * (1.0 - k / N)) for k in range(N)]
+
+
+def sample(x0, img_lat, w: dict, txt, clip, dims, steps: int, cfg_scale: float,
+           rnd: bool = False, model=None, known_pixel_frames=(0,)):
+    """The inference loop of [I2V] 7: prepare y and the context once, then
+    `steps` CFG Euler steps.  The cond row sees the text, the uncond row zeroed
+    text with CLIP and y kept ([I2V] Q5).  ``model(x, tau)`` (optional) stands
+    in for the DiT and returns (v_c, v_u).  Returns the final latent and the
+    per-step velocities."""
+    if model is None:
+        y = build_cond_y(img_lat, known_pixel_frames)
+        txt2 = np.stack([np.asarray(txt, F64), np.zeros_like(txt, dtype=F64)])
+        ctx_txt, ctx_img = context_embed(w, txt2, clip, rnd)
+        kvs = [cross_kv(w, i, ctx_txt, ctx_img, rnd) for i in range(dims.blocks)]
+
+        def model(x, tau):
+            v = dit_forward(np.stack([x, x]), y, tau, w, kvs, dims, rnd)
+            return v[0], v[1]
+    x = np.asarray(x0, F64)
+    trace = []
+    for t, dt, tau in schedule(steps):
+        v_c, v_u = model(x, tau)
+        trace.append((v_c, v_u))
+        x = euler_cfg_step(x, v_c, v_u, cfg_scale, dt)
+    return x, trace
