@@ -1,0 +1,317 @@
+// k_gemm_tc.cu — bf16 GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA)
+// with the epilogues of the DiT block fused in: bias, bias+GELU, bias then
+// gate * (.) added into the fp32 residual stream, fp32 store, unpatchify.
+//
+// C[m, n] = sum_k A[m, k] * B[n, k]: A = activations [M, K], B = a Linear
+// weight [N, K]; both K-major, loaded by TMA into 128-byte-swizzled shared
+// memory tiles of 64 K-elements.
+//
+// CTA = 6 warps, persistent over output tiles of 128 x BN:
+//   warp 0     TMA producer (one lane): STAGES-deep ring of (A, B) tiles
+//   warp 1     TMEM owner + MMA issuer (one lane): 128 x BN x 16 UMMAs,
+//              accumulating in one of two TMEM buffers
+//   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter of the
+//              accumulator, epilogue math, global stores; they release the
+//              TMEM buffer so the next tile's MMAs overlap this epilogue.
+#include "wd_internal.cuh"
+
+#include <cudaTypedefs.h>
+
+namespace wd {
+namespace tcg {
+
+constexpr int BM = 128, BK = 64;
+constexpr int THREADS = 192;
+
+template <int BN>
+struct Cfg {
+  static constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr uint32_t IDESC = idesc_bf16(BM, BN, 0, 0);
+};
+
+// Wait-site ids recorded in the device error word on a timeout.
+enum : unsigned { SITE_EMPTY = 0x101, SITE_FULL = 0x102, SITE_TFULL = 0x103, SITE_TEMPTY = 0x104, SITE_DRAIN = 0x105 };
+
+// ------------------------------------------------------------------ epilogue on 32 columns
+// One thread = one output row m; columns n .. n+31 come from the accumulator.
+template <int MODE>
+__device__ __forceinline__ void epilogue32(const Epi& ep, int64_t m, int n, const uint32_t (&r)[32]) {
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+  if (ep.bias) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      const float4 b = __ldg(reinterpret_cast<const float4*>(ep.bias + n + j));
+      v[j] += b.x; v[j + 1] += b.y; v[j + 2] += b.z; v[j + 3] += b.w;
+    }
+  }
+  if constexpr (MODE == EPI_STORE || MODE == EPI_GELU) {
+    if constexpr (MODE == EPI_GELU) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<bf16*>(ep.out) + m * ep.ldo + n);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                          pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+    }
+  } else if constexpr (MODE == EPI_F32) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(ep.out) + m * ep.ldo + n);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  } else if constexpr (MODE == EPI_RESID) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(ep.out) + m * ep.ldo + n);
+    const bool gated = ep.gate_a || ep.gate_b;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float4 g = make_float4(1.f, 1.f, 1.f, 1.f);
+      if (gated) {
+        const float4 ga = ep.gate_a ? __ldg(reinterpret_cast<const float4*>(ep.gate_a + n + 4 * j))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 gb = ep.gate_b ? __ldg(reinterpret_cast<const float4*>(ep.gate_b + n + 4 * j))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+        g = make_float4(ga.x + gb.x, ga.y + gb.y, ga.z + gb.z, ga.w + gb.w);
+      }
+      float4 x = dst[j];
+      x.x += g.x * v[4 * j]; x.y += g.y * v[4 * j + 1]; x.z += g.z * v[4 * j + 2]; x.w += g.w * v[4 * j + 3];
+      dst[j] = x;
+    }
+  } else {   // EPI_UNPATCH
+    float* out = static_cast<float*>(ep.out);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) out[unpatch_index(ep, m, n + j)] = v[j];
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+template <int BN, int MODE>
+__global__ void __launch_bounds__(THREADS, 1)
+k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Epi ep, int M,
+          int N, int K) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;   // [2]
+  uint64_t* tempty = tfull + 2;          // [2]
+  uint64_t* tdone = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tdone + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = N / BN;
+  const int m_tiles = (M + BM - 1) / BM;
+  const int tiles = m_tiles * n_tiles;
+  const int k_iters = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 4); }
+    mbar_init(tdone, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) { tmem_alloc(tmem_slot, C::TMEM_COLS); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, last_par = 0;   // per-stage bit masks
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        const int m0 = (t / n_tiles) * BM, n0 = (t % n_tiles) * BN;
+        for (int k = 0; k < k_iters; ++k) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, SITE_EMPTY)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          tma_load_2d(sA + stage * C::A_BYTES, &tmA, k * BK, m0, &full[stage]);
+          tma_load_2d(sB + stage * C::B_BYTES, &tmB, k * BK, n0, &full[stage]);
+          issued |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Let every copy this thread issued land before the CTA can exit.
+      for (int s = 0; s < C::STAGES; ++s)
+        if (issued & (1u << s)) mbar_wait(&full[s], (last_par >> s) & 1u, SITE_DRAIN);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, SITE_TEMPTY)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d = tmem + acc * BN;
+        for (int k = 0; k < k_iters; ++k) {
+          if (!mbar_wait(&full[stage], phase, SITE_FULL)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            umma_ss(d, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), C::IDESC,
+                    (k | kk) != 0);
+          }
+          umma_commit(&empty[stage]);   // frees the smem slot once these MMAs have read it
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);       // accumulator ready for the epilogue
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      // Every MMA issued above has completed once tdone flips.
+      umma_commit(tdone);
+      mbar_wait(tdone, 0, SITE_DRAIN);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------- epilogue warps
+    const int q = warp & 3;   // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+      const int m0 = (t / n_tiles) * BM, n0 = (t % n_tiles) * BN;
+      if (!mbar_wait(&tfull[acc], acc_phase, SITE_TFULL)) break;
+      tc_fence_after();
+      const int64_t m = m0 + q * 32 + lane;
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tbase + c, r);
+        tmem_wait_ld();
+        if (m < M) epilogue32<MODE>(ep, m, n0 + c, r);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace tcg
+
+// ------------------------------------------------------------------ host side
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 tensor map over a row-major [rows, cols] matrix with row stride
+// `ld` elements; box = box_cols x box_rows, 128-byte swizzle.
+static wd_status make_tmap_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                                int box_cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) { set_error("cuTensorMapEncodeTiled unavailable"); return WD_ERR_CUDA; }
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) { set_error("cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r)); return WD_ERR_CUDA; }
+  return WD_OK;
+}
+
+static int sm_count() {
+  static int cnt[16] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!cnt[dev & 15]) cudaDeviceGetAttribute(&cnt[dev & 15], cudaDevAttrMultiProcessorCount, dev);
+  return cnt[dev & 15];
+}
+
+template <int BN, int MODE>
+static wd_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const Epi& ep, int M, int N, int K,
+                           cudaStream_t st) {
+  using C = tcg::Cfg<BN>;
+  static bool attr[16] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr[dev & 15]) {
+    cudaFuncSetAttribute(tcg::k_gemm_tc<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    attr[dev & 15] = true;
+  }
+  const int tiles = ((M + tcg::BM - 1) / tcg::BM) * (N / BN);
+  const int grid = tiles < sm_count() ? tiles : sm_count();
+  tcg::k_gemm_tc<BN, MODE><<<grid, tcg::THREADS, C::SMEM, st>>>(ta, tb, ep, M, N, K);
+  return launch_status("gemm_tc");
+}
+
+template <int BN>
+static wd_status dispatch_mode(int mode, const CUtensorMap& ta, const CUtensorMap& tb, const Epi& ep, int M, int N,
+                               int K, cudaStream_t st) {
+  switch (mode) {
+    case EPI_STORE: return launch_tc<BN, EPI_STORE>(ta, tb, ep, M, N, K, st);
+    case EPI_GELU: return launch_tc<BN, EPI_GELU>(ta, tb, ep, M, N, K, st);
+    case EPI_F32: return launch_tc<BN, EPI_F32>(ta, tb, ep, M, N, K, st);
+    case EPI_RESID: return launch_tc<BN, EPI_RESID>(ta, tb, ep, M, N, K, st);
+    case EPI_UNPATCH: return launch_tc<BN, EPI_UNPATCH>(ta, tb, ep, M, N, K, st);
+  }
+  set_error("gemm_tc: bad epilogue %d", mode);
+  return WD_ERR_ARG;
+}
+
+wd_status gemm_tc(int M, int N, int K, const bf16* A, int64_t lda, const bf16* B, int64_t ldb, int mode,
+                  const Epi& ep, cudaStream_t st) {
+  if (M <= 0 || N <= 0 || K <= 0) { set_error("gemm: empty shape %d x %d x %d", M, N, K); return WD_ERR_SHAPE; }
+  // TMA rules: 16-byte aligned base and row strides.
+  if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B)) & 15u) {
+    set_error("gemm_tc: operands must be 16-byte aligned");
+    return WD_ERR_ALIGN;
+  }
+  if ((lda % 8) || (ldb % 8) || (K % 8)) {
+    set_error("gemm_tc: K=%d, lda=%lld, ldb=%lld must be multiples of 8", K, (long long)lda, (long long)ldb);
+    return WD_ERR_SHAPE;
+  }
+  if (N % 64) { set_error("gemm_tc: N=%d must be a multiple of 64", N); return WD_ERR_SHAPE; }
+  if (mode != EPI_UNPATCH && (ep.ldo % 8 || (reinterpret_cast<uintptr_t>(ep.out) & 15u))) {
+    set_error("gemm_tc: output must be 16-byte aligned with ldo %% 8 == 0");
+    return WD_ERR_ALIGN;
+  }
+  const int BN = (N % 256 == 0) ? 256 : ((N % 128 == 0) ? 128 : 64);
+  CUtensorMap ta, tb;
+  WD_TRY(make_tmap_bf16(&ta, A, M, K, lda, tcg::BK, tcg::BM));
+  WD_TRY(make_tmap_bf16(&tb, B, N, K, ldb, tcg::BK, BN));
+  switch (BN) {
+    case 256: return dispatch_mode<256>(mode, ta, tb, ep, M, N, K, st);
+    case 128: return dispatch_mode<128>(mode, ta, tb, ep, M, N, K, st);
+    default: return dispatch_mode<64>(mode, ta, tb, ep, M, N, K, st);
+  }
+}
+
+}  // namespace wd

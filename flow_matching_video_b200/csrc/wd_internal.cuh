@@ -1,0 +1,103 @@
+// wd_internal.cuh — declarations shared by the kernels of libwd (one
+// translation unit: wd_lib.cu includes every kernel file).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <string>
+
+#include "../../include/wd.h"
+#include "wd_ptx.cuh"
+
+namespace wd {
+
+using bf16 = __nv_bfloat16;
+
+// ------------------------------------------------------------------ errors
+void set_error(const char* fmt, ...);
+
+#define WD_TRY(expr)                       \
+  do {                                     \
+    wd_status _s = (expr);                 \
+    if (_s != WD_OK) return _s;            \
+  } while (0)
+
+wd_status launch_status(const char* what);   // cudaGetLastError -> WD_ERR_CUDA + message
+
+// ------------------------------------------------------------------ element conversions
+template <typename T> __device__ __forceinline__ float to_f(T v);
+template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f<bf16>(bf16 v) { return __bfloat162float(v); }
+template <typename T> __device__ __forceinline__ T from_f(float v);
+template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ bf16 from_f<bf16>(float v) { return __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
+  __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
+  return __bfloat1622float2(h);
+}
+
+// Exact GELU x * Phi(x) (erf form).
+__device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+
+// ------------------------------------------------------------------ GEMM epilogues
+// Every GEMM computes acc[m, n] = sum_k A[m, k] * B[n, k] (B is a Linear weight
+// [out, in]) and then one of these epilogues, with v = acc + bias[n]:
+enum EpiMode : int {
+  EPI_STORE = 0,      // out[m, n] = v                        (out in the activation type)
+  EPI_GELU = 1,       // out[m, n] = GELU(v)                  (out in the activation type)
+  EPI_F32 = 2,        // out[m, n] = v                        (out fp32)
+  EPI_RESID = 3,      // out[m, n] += g[n] * v, g = ga + gb   (out fp32 residual, in place)
+  EPI_UNPATCH = 4,    // unpatchify scatter of v into [B, 16, T, H, W] fp32
+};
+
+struct Epi {
+  void* out;
+  int64_t ldo;            // row stride of out, elements (unused by EPI_UNPATCH)
+  const float* bias;      // [N] or null
+  const float* gate_a;    // EPI_RESID: gate = gate_a[n] + gate_b[n]; both null -> 1
+  const float* gate_b;
+  int T, Hp, Wp, L;       // EPI_UNPATCH geometry
+};
+
+// Unpatchify address of GEMM element (row m = b*L + l, column n = c*4+kh*2+kw).
+__device__ __forceinline__ int64_t unpatch_index(const Epi& ep, int64_t m, int n) {
+  const int64_t b = m / ep.L;
+  const int l = static_cast<int>(m - b * ep.L);
+  const int x = l % ep.Wp, y = (l / ep.Wp) % ep.Hp, f = l / (ep.Wp * ep.Hp);
+  const int c = n >> 2, kh = (n >> 1) & 1, kw = n & 1;
+  const int H = 2 * ep.Hp, W = 2 * ep.Wp;
+  return (((b * 16 + c) * ep.T + f) * H + (2 * y + kh)) * static_cast<int64_t>(W) + (2 * x + kw);
+}
+
+// ------------------------------------------------------------------ internal launchers
+// C = epilogue(A[M,K] * B[N,K]^T): A, B in T (float or bf16).
+template <typename T>
+wd_status gemm_simt(int M, int N, int K, const T* A, int64_t lda, const T* B, int64_t ldb, int mode,
+                    const Epi& ep, cudaStream_t st);
+// Tensor-core (tcgen05 + TMA) bf16 GEMM.
+wd_status gemm_tc(int M, int N, int K, const bf16* A, int64_t lda, const bf16* B, int64_t ldb, int mode,
+                  const Epi& ep, cudaStream_t st);
+
+// Multi-head attention O = softmax(Q K^T / sqrt(dh)) V per (batch, head),
+// optionally summed with a second, independently normalised key/value
+// segment (the decoupled image/text cross-attention).
+template <typename T>
+struct AttnArgs {
+  const T* q; int64_t q_rs;                    // q row (b, l): q + (b*Lq + l)*q_rs + h*dh
+  const T* k1; const T* v1; int64_t kv1_rs; int64_t kv1_bs; int n1;
+  const T* k2; const T* v2; int64_t kv2_rs; int64_t kv2_bs; int n2;   // k2 == null: one segment
+  T* o; int64_t o_rs;
+  int batch, Lq, heads, dh;
+};
+template <typename T>
+wd_status attention_simt(const AttnArgs<T>& a, cudaStream_t st);
+wd_status attention_tc(const AttnArgs<bf16>& a, cudaStream_t st);
+
+}  // namespace wd

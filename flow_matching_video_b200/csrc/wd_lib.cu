@@ -1,0 +1,7 @@
+// wd_lib.cu — libwd is built as one translation unit so that every kernel
+// sees the same device error word without relocatable device code.
+#include "k_small.cu"
+#include "k_simt.cu"
+#include "k_gemm_tc.cu"
+#include "k_attn_tc.cu"
+#include "wd_api.cu"

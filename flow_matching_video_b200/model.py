@@ -1,0 +1,126 @@
+"""Device-side Wan2.1-style I2V DiT built on the libwd C ABI.
+
+Holds the weights and buffers in device memory (torch tensors) and sequences
+the entry points of libwd for one denoising forward and one CFG Euler step
+("图解 Wan2.1 I2V" section 7).  Every arithmetic step runs in libwd's kernels;
+this module only allocates, fills structs of pointers and calls.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import synth
+from . import wd
+
+MATRIX_SUFFIX = ".w"
+
+
+def _tdtype(dims: synth.Dims):
+    return torch.bfloat16 if dims.dtype == "bf16" else torch.float32
+
+
+def weights_to_device(w_host: dict, dims: synth.Dims, device) -> dict:
+    """numpy weights from synth.model_weights -> device tensors (matrices in the
+    storage type, everything else fp32).  Time-MLP matrices stay fp32."""
+    out = {}
+    for k, a in w_host.items():
+        is_mat = k.endswith(MATRIX_SUFFIX) and not k.startswith(("t1.", "t2.", "tp."))
+        dt = _tdtype(dims) if is_mat else torch.float32
+        out[k] = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device=device, dtype=dt)
+    return out
+
+
+def random_weights_on_device(wl: synth.Workload, device) -> dict:
+    """Seeded N(0, 0.02) weights drawn directly on the device (large stacks)."""
+    d, s = wl.dims, wl.seed
+    td = _tdtype(d)
+    D, F = d.D, d.ffn
+    std = synth.WEIGHT_STD
+    w = {}
+
+    def g(name, shape, dt=torch.float32, mean=0.0):
+        w[name] = synth.device_normal(shape, std, mean, s, name, device, dt)
+
+    g("t1.w", (D, synth.T_EMB)); g("t1.b", (D,)); g("t2.w", (D, D)); g("t2.b", (D,))
+    g("tp.w", (6 * D, D)); g("tp.b", (6 * D,))
+    g("pe.w", (D, synth.PATCH_K), td); g("pe.b", (D,))
+    g("txt1.w", (D, d.c_txt), td); g("txt1.b", (D,)); g("txt2.w", (D, D), td); g("txt2.b", (D,))
+    g("img1.w", (D, d.c_img), td); g("img1.b", (D,)); g("img2.w", (D, D), td); g("img2.b", (D,))
+    for i in range(d.blocks):
+        p = f"blk{i}."
+        for nm, shp in (("qkv", (3 * D, D)), ("o", (D, D)), ("cq", (D, D)), ("ck", (D, D)), ("cv", (D, D)),
+                        ("cki", (D, D)), ("cvi", (D, D)), ("co", (D, D)), ("f1", (F, D)), ("f2", (D, F))):
+            g(p + nm + ".w", shp, td)
+            g(p + nm + ".b", (shp[0],))
+        g(p + "gq", (D,), mean=1.0); g(p + "gk", (D,), mean=1.0)
+        g(p + "cn.g", (D,), mean=1.0); g(p + "cn.b", (D,))
+        g(p + "mod", (6, D))
+    g("head.mod", (2, D)); g("head.w", (synth.OUT_P, D), td); g("head.b", (synth.OUT_P,))
+    return w
+
+
+class DiT:
+    """The DiT of one workload on one device, with its buffers for `batch` rows."""
+
+    def __init__(self, dims: synth.Dims, weights: dict, batch: int, device="cuda"):
+        self.dims = dims
+        self.cd = wd.make_dims(dims)
+        self.batch = batch
+        self.device = torch.device(device)
+        self.w = weights
+        self.tdtype = _tdtype(dims)
+        p = lambda k: self.w[k].data_ptr()
+        self.time_w = wd.wd_time_weights(*(p(k) for k in ("t1.w", "t1.b", "t2.w", "t2.b", "tp.w", "tp.b")))
+        self.ctx_w = wd.wd_ctx_weights(*(p(k) for k in ("txt1.w", "txt1.b", "txt2.w", "txt2.b",
+                                                        "img1.w", "img1.b", "img2.w", "img2.b")))
+        names = {"qkv_w": "qkv.w", "qkv_b": "qkv.b", "g_q": "gq", "g_k": "gk", "o_w": "o.w", "o_b": "o.b",
+                 "cn_g": "cn.g", "cn_b": "cn.b", "cq_w": "cq.w", "cq_b": "cq.b", "ck_w": "ck.w", "ck_b": "ck.b",
+                 "cv_w": "cv.w", "cv_b": "cv.b", "cki_w": "cki.w", "cki_b": "cki.b", "cvi_w": "cvi.w",
+                 "cvi_b": "cvi.b", "co_w": "co.w", "co_b": "co.b", "f1_w": "f1.w", "f1_b": "f1.b",
+                 "f2_w": "f2.w", "f2_b": "f2.b", "mod": "mod"}
+        self.block_w = [wd.wd_block_weights(*(p(f"blk{i}." + names[f]) for f in wd.BLOCK_FIELDS))
+                        for i in range(dims.blocks)]
+        self.head_w = wd.wd_head_weights(p("head.mod"), p("head.w"), p("head.b"))
+        L, D = dims.L, dims.D
+        dev = self.device
+        self.ws = torch.empty(wd.wd_workspace_bytes(self.cd, batch), dtype=torch.uint8, device=dev)
+        self.ctx = torch.empty(wd.wd_ctx_bytes(self.cd, batch), dtype=torch.uint8, device=dev)
+        kvb = wd.wd_kv_bytes(self.cd, batch)
+        self.kv = torch.empty((dims.blocks, kvb), dtype=torch.uint8, device=dev)
+        self.X = torch.empty((batch, L, D), dtype=torch.float32, device=dev)
+        self.e = torch.empty(D, dtype=torch.float32, device=dev)
+        self.e0 = torch.empty((6, D), dtype=torch.float32, device=dev)
+        self.v = torch.empty((batch, 16, dims.T, dims.H, dims.W), dtype=torch.float32, device=dev)
+
+    # -------------------------------------------------------------- once per video
+    def build_cond_y(self, img_lat: torch.Tensor, known_frames=None) -> torch.Tensor:
+        y = torch.empty((20,) + tuple(img_lat.shape[1:]), dtype=torch.float32, device=self.device)
+        wd.wd_build_cond_y(self.cd, img_lat, y, known_frames)
+        return y
+
+    def prepare_context(self, txt: torch.Tensor, clip: torch.Tensor):
+        """txt [batch, n_txt, c_txt], clip [n_img, c_img] in the storage type."""
+        wd.wd_context_embed(self.cd, self.ctx_w, txt, clip, self.batch, self.ctx)
+        for i in range(self.dims.blocks):
+            wd.wd_cross_kv(self.cd, self.block_w[i], self.ctx, self.batch, self.kv[i])
+
+    # -------------------------------------------------------------- per step
+    def forward(self, x_t: torch.Tensor, y: torch.Tensor, tau: float, stream=None) -> torch.Tensor:
+        """v = DiT(concat(x_t, y), tau) for x_t [batch, 16, T, H, W]; returns self.v."""
+        wd.wd_time_mod(self.cd, self.time_w, tau, self.e, self.e0, stream)
+        wd.wd_patch_embed(self.cd, x_t, y, self.w["pe.w"], self.w["pe.b"], self.batch, self.X, self.ws, stream)
+        for i in range(self.dims.blocks):
+            wd.wd_block_forward(self.cd, self.block_w[i], self.e0, self.kv[i], self.batch, self.X, self.ws, stream)
+        wd.wd_unpatchify(self.cd, self.head_w, self.e, self.batch, self.X, self.v, self.ws, stream)
+        return self.v
+
+    def cfg_euler_step(self, xb: torch.Tensor, y: torch.Tensor, tau: float, dt: float, cfg_scale: float,
+                       stream=None):
+        """One CFG Euler step on xb [2, 16, T, H, W] (both rows hold x; row 0
+        sees the text, row 1 zeroed text): x += dt (v_u + s (v_c - v_u))."""
+        assert self.batch == 2
+        v = self.forward(xb, y, tau, stream)
+        wd.wd_euler_cfg_step(xb[0], v[0], v[1], cfg_scale, dt, stream=stream)
+        xb[1].copy_(xb[0])
+        return xb

@@ -1,0 +1,232 @@
+/*
+ * wd.h — C ABI of libwd, the B200 (sm_100a) denoising step of a Wan2.1-style
+ * image-to-video DiT driven by a classifier-free-guided Euler flow-matching
+ * sampler.
+ *
+ * Sources (cited by page title and section):
+ *   [I2V] "图解 Wan2.1 I2V：从一张图到一段视频，模型到底发生了什么" (liyongzhi.xyz)
+ *   [WAN] "Wan（通义万相）：大规模视频生成基础模型 — 技术深度解析 & Wan2.1 vs Wan2.2对比"
+ *         (devpress.csdn.net)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers are DEVICE pointers (cudaMalloc'd or torch tensors) unless a
+ *   comment says "host".  The caller owns every buffer; the library never
+ *   allocates device memory.  Scratch comes from a caller-provided workspace
+ *   whose size the *_bytes queries return.
+ * - Tensors are dense, row-major, in the layouts written next to each
+ *   argument.  Every device pointer must be 16-byte aligned, otherwise the
+ *   call returns WD_ERR_ALIGN before launching anything.
+ * - dtype: wd_dims.dtype selects the storage type of weight matrices and of
+ *   activations handed between kernels: WD_F32 (float, all-fp32 SIMT path)
+ *   or WD_BF16 (bfloat16 tensor-core path, fp32 accumulation).  Arguments
+ *   typed `const void*` below have that type; `float*` arguments are always
+ *   fp32 (residual stream, latents, biases, gains, modulation vectors).
+ * - Calls are asynchronous on `stream` (a cudaStream_t).  Validation failures
+ *   return before any launch; a failed launch returns WD_ERR_CUDA.  Device
+ *   kernels never trap: bounded waits that run out set a device error word,
+ *   which wd_check() reports as WD_ERR_TIMEOUT.
+ * - No exception crosses the ABI.  wd_last_error() gives the calling thread's
+ *   last message.
+ */
+#ifndef WD_H_
+#define WD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* wd_stream; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  WD_OK = 0,
+  WD_ERR_ARG = 1,         /* null pointer or bad scalar argument          */
+  WD_ERR_SHAPE = 2,       /* dimensions the kernels do not support        */
+  WD_ERR_DTYPE = 3,       /* unknown dtype                                */
+  WD_ERR_ALIGN = 4,       /* a device pointer is not 16-byte aligned      */
+  WD_ERR_WORKSPACE = 5,   /* workspace smaller than the *_bytes query     */
+  WD_ERR_CUDA = 6,        /* CUDA launch or runtime error                 */
+  WD_ERR_TIMEOUT = 7,     /* a bounded device wait ran out                */
+  WD_ERR_UNSUPPORTED = 8  /* feature not built for this configuration     */
+} wd_status;
+
+typedef enum { WD_F32 = 0, WD_BF16 = 1 } wd_dtype;
+typedef enum { WD_NORM_LAYER = 0, WD_NORM_RMS = 1 } wd_norm;
+
+/* Model and video dimensions.  D = model width, heads x (D/heads) attention
+ * heads, ffn = FFN hidden width, blocks = DiT blocks; T, H, W = latent frames,
+ * height and width (H, W even); the token grid is T x H/2 x W/2 and the token
+ * count L = T*(H/2)*(W/2) ([I2V] 5.1).  n_txt x c_txt text tokens (umT5,
+ * [I2V] 3.1), n_img x c_img CLIP tokens ([I2V] 3.2).  norm selects the adaLN
+ * norm (LayerNorm without affine by default, [I2V] 5.2); eps its epsilon. */
+typedef struct {
+  int D, heads, ffn, blocks;
+  int T, H, W;
+  int n_txt, c_txt, n_img, c_img;
+  int dtype; /* wd_dtype */
+  int norm;  /* wd_norm  */
+  float eps;
+} wd_dims;
+
+/* Shared time MLP: e = t2(SiLU(t1(sin(tau)))), e0 = tp(SiLU(e)) ([I2V] 5.2).
+ * All fp32.  t1_w [D,256], t2_w [D,D], tp_w [6D,D]; biases [D], [D], [6D]. */
+typedef struct {
+  const float *t1_w, *t1_b, *t2_w, *t2_b, *tp_w, *tp_b;
+} wd_time_weights;
+
+/* Text MLP (c_txt -> D -> D) and CLIP MLPProj (c_img -> D -> D), each
+ * Linear -> GELU -> Linear ([I2V] 7 steps 1-2).  Matrices [out,in] in dtype. */
+typedef struct {
+  const void *txt1_w; const float *txt1_b; const void *txt2_w; const float *txt2_b;
+  const void *img1_w; const float *img1_b; const void *img2_w; const float *img2_b;
+} wd_ctx_weights;
+
+/* One DiT block ([I2V] 5.2-5.5).  Matrices [out,in] in dtype, vectors fp32.
+ *   qkv_w [3D,D] rows (q; k; v), qkv_b [3D]; g_q, g_k [D] QK-RMSNorm gains;
+ *   o_w [D,D]; cn_g, cn_b [D] cross-attention pre-norm affine;
+ *   cq_w, ck_w, cv_w (text K/V), cki_w, cvi_w (image K/V), co_w: [D,D];
+ *   f1_w [ffn,D], f2_w [D,ffn]; mod [6,D] the block's modulation bias b_i
+ *   ([WAN] 2.5), rows (shift1, scale1, gate1, shift2, scale2, gate2). */
+typedef struct {
+  const void *qkv_w; const float *qkv_b;
+  const float *g_q, *g_k;
+  const void *o_w; const float *o_b;
+  const float *cn_g, *cn_b;
+  const void *cq_w; const float *cq_b;
+  const void *ck_w; const float *ck_b;
+  const void *cv_w; const float *cv_b;
+  const void *cki_w; const float *cki_b;
+  const void *cvi_w; const float *cvi_b;
+  const void *co_w; const float *co_b;
+  const void *f1_w; const float *f1_b;
+  const void *f2_w; const float *f2_b;
+  const float *mod;
+} wd_block_weights;
+
+/* Head ([I2V] 5.5): mod [2,D] (shift, scale biases added to e), w [64,D]
+ * in dtype, b [64] fp32.  Output feature c*4 + kh*2 + kw. */
+typedef struct {
+  const float *mod;
+  const void *w;
+  const float *b;
+} wd_head_weights;
+
+/* ------------------------------------------------------------------ queries */
+const char* wd_last_error(void);
+const char* wd_version(void);
+
+/* Synchronises `stream`, then reports any pending asynchronous CUDA error
+ * (WD_ERR_CUDA) or a device wait that ran out (WD_ERR_TIMEOUT; the error
+ * word is cleared by the call). */
+wd_status wd_check(wd_stream stream);
+
+/* Token count L = T*(H/2)*(W/2) ([I2V] 5.1), or 0 for invalid dims. */
+int64_t wd_token_count(const wd_dims* d);
+
+/* Workspace bytes that wd_patch_embed, wd_block_forward and wd_unpatchify
+ * need for a batch of `batch` samples (one buffer serves all three). */
+size_t wd_workspace_bytes(const wd_dims* d, int batch);
+
+/* Bytes of the context buffer written by wd_context_embed:
+ * ctx_txt [batch, n_txt, D] then ctx_img [n_img, D], dtype elements, plus
+ * the MLP hidden scratch behind them. */
+size_t wd_ctx_bytes(const wd_dims* d, int batch);
+
+/* Bytes of ONE block's cross-attention K/V cache written by wd_cross_kv:
+ * k_img [n_img,D], v_img [n_img,D], k_txt [batch,n_txt,D], v_txt [batch,n_txt,D]
+ * in that order, dtype elements, each part starting on a 256-byte boundary. */
+size_t wd_kv_bytes(const wd_dims* d, int batch);
+
+/* ------------------------------------------------------------------ the path */
+
+/* Conditioning y = concat(mask, image latent) ([I2V] 4.1, Q3, Q6).
+ * img_lat [16,T,H,W] fp32 -> y [20,T,H,W] fp32.  known_frames (HOST array of
+ * n_known pixel-frame indices in [0, 4(T-1)]; NULL or n_known = 0 means {0})
+ * marks the known frames; the mask channel c of latent frame f is 1 when
+ * entry 4f+c of (frame 0 repeated 4 times, frames 1..F-1) is known. */
+wd_status wd_build_cond_y(const wd_dims* d, const float* img_lat, const int* known_frames,
+                          int n_known, float* y, wd_stream stream);
+
+/* Text and CLIP projections, once per video ([I2V] 7 steps 1-2, 6).
+ * txt [batch, n_txt, c_txt] and clip [n_img, c_img] in dtype (the CFG
+ * unconditional row carries zeroed text, [I2V] Q5).  ctx receives
+ * wd_ctx_bytes(d, batch) bytes: ctx_txt [batch,n_txt,D], ctx_img [n_img,D]
+ * (dtype), then scratch. */
+wd_status wd_context_embed(const wd_dims* d, const wd_ctx_weights* w, const void* txt,
+                           const void* clip, int batch, void* ctx, wd_stream stream);
+
+/* One block's cross-attention keys and values from the context written by
+ * wd_context_embed ([I2V] 5.4: text uses Linear_k/Linear_v, image its own
+ * k_img/v_img).  kv receives wd_kv_bytes(d, batch) bytes. */
+wd_status wd_cross_kv(const wd_dims* d, const wd_block_weights* w, const void* ctx, int batch,
+                      void* kv, wd_stream stream);
+
+/* Time modulation ([I2V] 5.2): tau (the noise level x 1000) -> e [D] and
+ * e0 [6,D], both fp32. */
+wd_status wd_time_mod(const wd_dims* d, const wd_time_weights* w, float tau, float* e, float* e0,
+                      wd_stream stream);
+
+/* Patch embedding of concat(x_t, y) ([I2V] 4.2, 5.1): Conv3d(36, D, (1,2,2),
+ * stride (1,2,2)) as a GEMM.  x_t [batch,16,T,H,W] fp32, y [20,T,H,W] fp32
+ * shared by the batch, w [D,144] (Conv3d weight [D,36,1,2,2] flattened) in
+ * dtype, b [D] fp32 -> X [batch, L, D] fp32, token l = (f*(H/2)+y)*(W/2)+x. */
+wd_status wd_patch_embed(const wd_dims* d, const float* x_t, const float* y, const void* w,
+                         const float* b, int batch, float* X, void* ws, size_t ws_bytes,
+                         wd_stream stream);
+
+/* One DiT block, in place on the fp32 residual stream X [batch, L, D]
+ * ([I2V] 5.2-5.5): adaLN-modulated full 3D self-attention with QK-RMSNorm and
+ * 3D RoPE, gate1 residual; decoupled image/text cross-attention, plain
+ * residual; adaLN-modulated GELU FFN, gate2 residual.  e0 [6,D] fp32 from
+ * wd_time_mod; kv from wd_cross_kv for this block. */
+wd_status wd_block_forward(const wd_dims* d, const wd_block_weights* w, const float* e0,
+                           const void* kv, int batch, float* X, void* ws, size_t ws_bytes,
+                           wd_stream stream);
+
+/* Head and unpatchify ([I2V] 5.5): z = LN(X)(1 + e + mod[1]) + e + mod[0],
+ * p = z w^T + b, v[b,c,f,2y+kh,2x+kw] = p[b, l, c*4+kh*2+kw].
+ * X [batch,L,D] fp32, e [D] fp32 -> v [batch,16,T,H,W] fp32. */
+wd_status wd_unpatchify(const wd_dims* d, const wd_head_weights* w, const float* e, int batch,
+                        const float* X, float* v, void* ws, size_t ws_bytes, wd_stream stream);
+
+/* CFG-combined Euler step ([I2V] 7; [WAN] 2.7):
+ * x[i] += dt * (v_uncond[i] + cfg_scale * (v_cond[i] - v_uncond[i])), or
+ * x[i] += dt * v_cond[i] when v_uncond is NULL.  n fp32 elements.  x may
+ * not overlap the velocities. */
+wd_status wd_euler_cfg_step(float* x, const float* v_cond, const float* v_uncond, float cfg_scale,
+                            float dt, size_t n, wd_stream stream);
+
+/* ------------------------------------------------------------------ building blocks
+ * The kernels of the path, exposed one by one so that each can be checked on
+ * its own.  Same conventions as above. */
+
+/* C = epilogue(A B^T + bias) for A [M,K] and B [N,K] (a Linear weight), both
+ * in `dtype` (wd_dtype), row-major with leading dimension K; bias [N] fp32 or
+ * NULL.  epilogue 0: out [M,N] = v in dtype; 1: out = GELU(v) (erf form,
+ * [I2V] 5.5) in dtype; 2: out = v in fp32; 3: out [M,N] fp32 += g*v with
+ * g = gate_a + gate_b (either may be NULL; both NULL means 1) — the gated
+ * residual of [I2V] 5.2.  bf16 runs on the tcgen05 tensor cores (N a
+ * multiple of 64, K a multiple of 8), fp32 on the CUDA cores. */
+wd_status wd_gemm(int dtype, int M, int N, int K, const void* A, const void* B, const float* bias, int epilogue,
+                  void* out, const float* gate_a, const float* gate_b, wd_stream stream);
+
+/* Multi-head attention without mask ([I2V] 5.3, 5.4): for every batch b and
+ * head h, o = softmax(q k1^T / sqrt(dh)) v1 [+ softmax(q k2^T / sqrt(dh)) v2].
+ * q, o [batch, Lq, heads*dh]; k1, v1 [batch, n1, heads*dh] or, with
+ * kv1_shared != 0, [n1, heads*dh] shared by the batch; k2/v2 likewise, or
+ * NULL for one segment.  dh in {32, 64, 128}. */
+wd_status wd_attention(int dtype, int batch, int Lq, int heads, int dh, const void* q, const void* k1, const void* v1,
+                       int n1, int kv1_shared, const void* k2, const void* v2, int n2, int kv2_shared, void* o,
+                       wd_stream stream);
+
+/* Debugging aid: bit 0 routes bf16 GEMMs, bit 1 bf16 attention, to the
+ * CUDA-core kernels instead of the tensor-core ones.  Process-wide. */
+void wd_set_debug_flags(unsigned flags);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* WD_H_ */

@@ -1,0 +1,100 @@
+"""The C ABI library loads, exports every function include/wd.h declares, and
+its host-side logic (sizes, validation) behaves; no GPU is needed.
+
+Validation failures return before any CUDA call, so they can be exercised on
+a machine without a GPU.
+"""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from flow_matching_video_b200 import synth
+from oracle import wan_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def wd():
+    from flow_matching_video_b200 import build
+    build.build()
+    from flow_matching_video_b200 import wd as _wd
+    return _wd
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "wd.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(wd_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_path():
+    fns = header_functions()
+    for name in ("wd_build_cond_y", "wd_patch_embed", "wd_time_mod", "wd_block_forward", "wd_unpatchify",
+                 "wd_euler_cfg_step", "wd_context_embed", "wd_cross_kv"):
+        assert name in fns
+
+
+def test_every_declared_symbol_is_exported_and_bound(wd):
+    lib = wd.lib()
+    for name in header_functions():
+        assert hasattr(lib, name), name
+        assert name in wd.SIGNATURES, name
+
+
+def test_token_count_and_sizes_match_oracle(wd):
+    for wl in synth.WORKLOADS.values():
+        d = wd.make_dims(wl.dims)
+        F = wl.dims.F_pix
+        assert wd.wd_token_count(d) == O.token_count(F, 8 * wl.dims.H, 8 * wl.dims.W) == wl.dims.L
+        ws = wd.wd_workspace_bytes(d, wl.batch)
+        rows = wl.batch * wl.dims.L
+        es = 2 if wl.dims.dtype == "bf16" else 4
+        assert ws >= rows * (max(3 * wl.dims.D, wl.dims.ffn) + max(wl.dims.D, 144)) * es
+        kv = wd.wd_kv_bytes(d, wl.batch)
+        assert kv >= 2 * (wl.dims.n_img + wl.batch * wl.dims.n_txt) * wl.dims.D * es
+        assert wd.wd_ctx_bytes(d, wl.batch) >= (wl.batch * wl.dims.n_txt + wl.dims.n_img) * wl.dims.D * es
+
+
+def test_invalid_dims_rejected(wd):
+    d = wd.make_dims(synth.TINY.dims)
+    d.heads = 3            # D % heads != 0
+    assert wd.wd_workspace_bytes(d, 2) == 0
+    d = wd.make_dims(synth.TINY.dims)
+    d.H = 7                # odd latent height
+    assert wd.wd_workspace_bytes(d, 2) == 0
+    d = wd.make_dims(synth.TINY.dims)
+    d.dtype = 9
+    assert wd.wd_workspace_bytes(d, 2) == 0
+    assert wd.wd_workspace_bytes(wd.make_dims(synth.TINY.dims), 0) == 0
+
+
+def test_null_and_misaligned_pointers_rejected_before_launch(wd):
+    lib = wd.lib()
+    d = wd.make_dims(synth.TINY.dims)
+    # NULL latent -> WD_ERR_ARG
+    assert lib.wd_euler_cfg_step(None, None, None, 5.0, 0.5, 16, None) == 1
+    assert "NULL" in wd.wd_last_error()
+    # misaligned pointers -> WD_ERR_ALIGN, never dereferenced
+    assert lib.wd_euler_cfg_step(0x1004, 0x2000, None, 5.0, 0.5, 16, None) == 4
+    assert lib.wd_build_cond_y(C.byref(d), 0x1000, None, 0, 0x2008, None) == 4
+    # workspace too small -> WD_ERR_WORKSPACE
+    hw = wd.wd_head_weights(0x1000, 0x2000, 0x3000)
+    assert lib.wd_unpatchify(C.byref(d), C.byref(hw), 0x4000, 2, 0x5000, 0x6000, 0x7000, 16, None) == 5
+    # known frame out of range -> WD_ERR_ARG
+    kf = (C.c_int * 1)(99)
+    assert lib.wd_build_cond_y(C.byref(d), 0x1000, kf, 1, 0x2000, None) == 1
+    # bad dtype for the building blocks
+    assert lib.wd_gemm(7, 8, 64, 8, 0x1000, 0x2000, None, 0, 0x3000, None, None, None) == 3
+    assert lib.wd_attention(7, 1, 8, 1, 32, 0x1000, 0x2000, 0x3000, 8, 0, None, None, 0, 0, 0x4000, None) == 3
+
+
+def test_product_path_has_no_oracle_import():
+    pkg = os.path.join(ROOT, "flow_matching_video_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh")):
+                src = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert not re.search(r"(from|import)\s+oracle|wan_oracle|liboracle", src), f

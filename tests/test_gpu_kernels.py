@@ -1,0 +1,226 @@
+"""Kernel-by-kernel parity of the CUDA path against the CPU oracle.
+
+Each test calls one libwd entry point through the C ABI and compares every
+output element with the oracle on the same seeded inputs.  Tolerances
+(max |gpu - oracle| / rms(oracle)): 1e-4 for fp32 arithmetic, 2e-2 for
+bf16-stored outputs (fp32 accumulation), as stated for the path; exact for
+the 0/1 mask and copies.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import wan_oracle as O
+from flow_matching_video_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-4
+TOL_BF16 = 2e-2
+
+
+@pytest.fixture(scope="module")
+def wd():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from flow_matching_video_b200 import build
+    build.build()
+    from flow_matching_video_b200 import wd as _wd
+    return _wd
+
+
+def rel(gpu, ref):
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    assert np.all(np.isfinite(gpu))
+    return float(np.abs(gpu - ref).max() / max(np.sqrt((ref * ref).mean()), 1e-30))
+
+
+def dev(a, dtype=torch.float32):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to("cuda", dtype)
+
+
+def host(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def bf(a):
+    return O.bf16(a)
+
+
+# ------------------------------------------------------------------ Euler / CFG
+@pytest.mark.parametrize("n", [1, 7, 4096 + 3, 16 * 21 * 60 * 104])
+def test_euler_cfg(wd, n):
+    rng = np.random.default_rng(n)
+    x, vc, vu = (rng.standard_normal(n).astype(np.float32) for _ in range(3))
+    gx = dev(x)
+    wd.wd_euler_cfg_step(gx, dev(vc), dev(vu), 5.0, 1 / 12)
+    wd.wd_check()
+    assert rel(host(gx), O.euler_cfg_step(x, vc, vu, 5.0, 1 / 12)) < 1e-6
+    gx = dev(x)
+    wd.wd_euler_cfg_step(gx, dev(vc), None, 5.0, 0.5)
+    wd.wd_check()
+    assert rel(host(gx), O.euler_cfg_step(x, vc, None, 5.0, 0.5)) < 1e-6
+
+
+def test_euler_exact_velocity_lands_on_data(wd):
+    rng = np.random.default_rng(3)
+    x0, x1 = rng.standard_normal((2, 16, 3, 8, 8)).astype(np.float32)
+    v = (x1.astype(np.float64) - x0).astype(np.float32)
+    gx = dev(x0)
+    wd.wd_euler_cfg_step(gx, dev(v), dev(v), 5.0, 1.0)
+    wd.wd_check()
+    np.testing.assert_allclose(host(gx), x1, atol=1e-6)
+
+
+# ------------------------------------------------------------------ conditioning
+@pytest.mark.parametrize("known", [None, [0], [0, 80], [5, 17, 80]])
+def test_build_cond_y_exact(wd, known):
+    d = synth.Dims(D=128, heads=4, ffn=512, blocks=1, T=21, H=6, W=10, n_txt=4, c_txt=8, n_img=2, c_img=8,
+                   dtype="f32")
+    img = np.random.default_rng(1).standard_normal((16, 21, 6, 10)).astype(np.float32)
+    y = torch.empty((20, 21, 6, 10), device="cuda")
+    wd.wd_build_cond_y(wd.make_dims(d), dev(img), y, known)
+    wd.wd_check()
+    want = O.build_cond_y(img, known or (0,))
+    np.testing.assert_array_equal(host(y), want)
+
+
+# ------------------------------------------------------------------ time MLP
+@pytest.mark.parametrize("wl", [synth.TINY, synth.STACK_480P81], ids=lambda w: w.name)
+@pytest.mark.parametrize("tau", [1000.0, 437.5, 0.0])
+def test_time_mod(wd, wl, tau):
+    w = synth.model_weights(wl, blocks=[])
+    D = wl.dims.D
+    tw = {k: dev(w[k]) for k in ("t1.w", "t1.b", "t2.w", "t2.b", "tp.w", "tp.b")}
+    st = wd.wd_time_weights(*(tw[k].data_ptr() for k in ("t1.w", "t1.b", "t2.w", "t2.b", "tp.w", "tp.b")))
+    e, e0 = torch.empty(D, device="cuda"), torch.empty((6, D), device="cuda")
+    wd.wd_time_mod(wd.make_dims(wl.dims), st, tau, e, e0)
+    wd.wd_check()
+    re, re0 = O.time_mod(w, tau, D)
+    assert rel(host(e), re) < TOL_F32
+    assert rel(host(e0), re0) < TOL_F32
+
+
+# ------------------------------------------------------------------ GEMM with fused epilogues
+GEMM_SHAPES = [(300, 192, 72), (128, 256, 64), (1000, 384, 1536), (257, 64, 144), (4096, 4608, 1536),
+               (2000, 8960, 1536), (1500, 1536, 8960)]
+
+
+def _gemm_case(wd, dtype, M, N, K, epi, seed=0):
+    rng = np.random.default_rng(seed + M + N + K + epi)
+    A = rng.standard_normal((M, K)).astype(np.float32)
+    B = (rng.standard_normal((N, K)) * 0.05).astype(np.float32)
+    bias = rng.standard_normal(N).astype(np.float32) * 0.1
+    ga, gb = rng.standard_normal(N).astype(np.float32), rng.standard_normal(N).astype(np.float32) * 0.1
+    is_bf = dtype == wd.WD_BF16
+    if is_bf:
+        A, B = bf(A).astype(np.float32), bf(B).astype(np.float32)
+    tdt = torch.bfloat16 if is_bf else torch.float32
+    acc = O.linear(A, B, bias)
+    if epi == wd.EPI_RESID:
+        X0 = rng.standard_normal((M, N)).astype(np.float32)
+        out = dev(X0)
+        want = X0 + (ga.astype(np.float64) + gb) * acc
+    else:
+        out = torch.empty((M, N), device="cuda", dtype=torch.float32 if epi == wd.EPI_F32 else tdt)
+        want = O.gelu(acc) if epi == wd.EPI_GELU else acc
+        if is_bf and epi != wd.EPI_F32:
+            want = bf(want)
+    wd.wd_gemm(dtype, M, N, K, dev(A, tdt), dev(B, tdt), dev(bias), epi, out,
+               dev(ga) if epi == wd.EPI_RESID else None, dev(gb) if epi == wd.EPI_RESID else None)
+    wd.wd_check()
+    if epi == wd.EPI_RESID:     # compare the update itself, not the residual it lands on
+        return host(out) - X0, want - X0
+    return host(out), want
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+@pytest.mark.parametrize("epi", [0, 1, 2, 3])
+def test_gemm_bf16_tensor_cores(wd, M, N, K, epi):
+    got, want = _gemm_case(wd, wd.WD_BF16, M, N, K, epi)
+    # bf16-stored outputs carry one rounding; fp32 outputs only accumulation order
+    tol = TOL_BF16 if epi in (0, 1) else 1e-4
+    assert rel(got, want) < tol
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 192, 72), (97, 64, 144), (513, 128, 300)])
+@pytest.mark.parametrize("epi", [0, 1, 2, 3])
+def test_gemm_f32_cuda_cores(wd, M, N, K, epi):
+    got, want = _gemm_case(wd, wd.WD_F32, M, N, K, epi)
+    assert rel(got, want) < TOL_F32
+
+
+def test_gemm_bf16_simt_reference_kernel(wd):
+    wd.wd_set_debug_flags(1)
+    try:
+        got, want = _gemm_case(wd, wd.WD_BF16, 300, 192, 72, 0)
+    finally:
+        wd.wd_set_debug_flags(0)
+    assert rel(got, want) < TOL_BF16
+
+
+# ------------------------------------------------------------------ attention
+ATTN_CASES = [  # batch, Lq, heads, dh, n1, shared1, n2, shared2
+    (1, 200, 2, 128, 200, 0, 0, 0),
+    (2, 130, 3, 128, 257, 1, 512, 0),
+    (1, 513, 1, 128, 1, 1, 0, 0),
+    (1, 64, 2, 64, 9, 1, 16, 0),
+    (2, 32, 4, 32, 32, 0, 0, 0),
+    (1, 1000, 2, 128, 1000, 0, 0, 0),
+]
+
+
+def _attn_case(wd, dtype, b, Lq, h, dh, n1, s1, n2, s2, seed=0):
+    rng = np.random.default_rng(seed + Lq + n1 + n2 + dh)
+    D = h * dh
+    q = rng.standard_normal((b, Lq, D)).astype(np.float32)
+    k1 = rng.standard_normal(((1 if s1 else b), n1, D)).astype(np.float32)
+    v1 = rng.standard_normal(((1 if s1 else b), n1, D)).astype(np.float32)
+    k2 = v2 = None
+    if n2:
+        k2 = rng.standard_normal(((1 if s2 else b), n2, D)).astype(np.float32)
+        v2 = rng.standard_normal(((1 if s2 else b), n2, D)).astype(np.float32)
+    is_bf = dtype == wd.WD_BF16
+    if is_bf:
+        q, k1, v1 = bf(q), bf(k1), bf(v1)
+        if n2:
+            k2, v2 = bf(k2), bf(v2)
+    tdt = torch.bfloat16 if is_bf else torch.float32
+    o = torch.empty((b, Lq, D), device="cuda", dtype=tdt)
+    wd.wd_attention(dtype, b, Lq, h, dh, dev(q, tdt), dev(k1, tdt), dev(v1, tdt), n1, s1, o,
+                    dev(k2, tdt) if n2 else None, dev(v2, tdt) if n2 else None, n2, s2)
+    wd.wd_check()
+    want = np.empty((b, Lq, D))
+    for bb in range(b):
+        kk, vv = k1[0 if s1 else bb], v1[0 if s1 else bb]
+        r = O.attention(q[bb].reshape(Lq, h, dh), kk.reshape(n1, h, dh), vv.reshape(n1, h, dh))
+        if n2:
+            kk, vv = k2[0 if s2 else bb], v2[0 if s2 else bb]
+            r = r + O.attention(q[bb].reshape(Lq, h, dh), kk.reshape(n2, h, dh), vv.reshape(n2, h, dh))
+        want[bb] = r.reshape(Lq, D)
+    if is_bf:
+        want = bf(want)
+    return host(o), want
+
+
+@pytest.mark.parametrize("case", ATTN_CASES)
+def test_attention_bf16(wd, case):
+    got, want = _attn_case(wd, wd.WD_BF16, *case)
+    assert rel(got, want) < TOL_BF16
+
+
+@pytest.mark.parametrize("case", ATTN_CASES)
+def test_attention_f32(wd, case):
+    got, want = _attn_case(wd, wd.WD_F32, *case)
+    assert rel(got, want) < TOL_F32
+
+
+def test_attention_bf16_simt_reference_kernel(wd):
+    wd.wd_set_debug_flags(2)
+    try:
+        got, want = _attn_case(wd, wd.WD_BF16, 2, 130, 3, 128, 257, 1, 512, 0)
+    finally:
+        wd.wd_set_debug_flags(0)
+    assert rel(got, want) < TOL_BF16
