@@ -1,7 +1,385 @@
-// k_attn_tc.cu — attention on the sm_100a tensor cores (placeholder: routes
-// to the CUDA-core kernel until the tcgen05 version is in place).
+// k_attn_tc.cu — non-causal multi-head attention on the sm_100a tensor cores
+// (tcgen05 + TMEM + TMA), head dim 128, bf16 in / bf16 out, fp32 softmax and
+// accumulation ("图解 Wan2.1 I2V" 5.3: full spatio-temporal self-attention;
+// 5.4: decoupled image/text cross-attention, two softmaxes summed).
+//
+// A CTA owns NQ query tiles of 128 rows of one (batch, head) and streams the
+// keys/values of NSEG segments in 128-key blocks:
+//   warp 0           TMA loader: the Q tiles once, then K_j, V_j through a
+//                    3-slot ring of 32 KB tiles
+//   warp 1           TMEM owner + MMA issuer: S_t = Q_t K_j^T into TMEM,
+//                    O_t (+)= P_t V_j with P_t from shared memory
+//   warps 2..        one warpgroup (128 threads, thread = query row) per Q
+//                    tile: online softmax on S_t read from TMEM, P_t written
+//                    as bf16 into a 128-byte-swizzled shared tile, O_t
+//                    rescaled in TMEM only when the running max grows by more
+//                    than 8 (log2 units; the final 1/l keeps the result
+//                    exact), then the normalised output written out.
+// With NQ = 2 the two tiles ping-pong: while one warpgroup runs its softmax,
+// the tensor cores compute the other tile's P V and next S.
 #include "wd_internal.cuh"
 
 namespace wd {
-wd_status attention_tc(const AttnArgs<bf16>& a, cudaStream_t st) { return attention_simt<bf16>(a, st); }
+namespace tca {
+
+constexpr int BQ = 128, BKV = 128, DH = 128;
+constexpr int TILE_BYTES = 128 * 128 * 2;   // one 128 x 128 bf16 tile (two 64-column halves)
+constexpr int HALF_BYTES = TILE_BYTES / 2;
+constexpr int RING = 3;
+constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
+
+template <int NQ, int NSEG>
+struct Cfg {
+  static constexpr int THREADS = 64 + 128 * NQ;
+  static constexpr int Q_OFF = 0;
+  static constexpr int P_OFF = NQ * TILE_BYTES;
+  static constexpr int RING_OFF = 2 * NQ * TILE_BYTES;
+  static constexpr int BAR_OFF = RING_OFF + RING * TILE_BYTES;
+  static constexpr int SMEM = 1024 + BAR_OFF + 256;
+  static constexpr int TMEM_COLS = 512;
+  // TMEM columns: S_t, O_t (per tile); with two segments one tile has O and O'
+  __host__ __device__ static constexpr int s_col(int t) { return NSEG == 1 ? t * 256 : 0; }
+  __host__ __device__ static constexpr int o_col(int t, int seg) { return NSEG == 1 ? t * 256 + 128 : 128 + 128 * seg; }
+  static constexpr uint32_t IDESC_S = idesc_bf16(128, 128, 0, 0);    // Q K^T: both K-major
+  static constexpr uint32_t IDESC_O = idesc_bf16(128, 128, 0, 1);    // P V: V is MN-major (dh contiguous)
+};
+
+enum : unsigned { SITE_Q = 0x201, SITE_KVF = 0x202, SITE_KVE = 0x203, SITE_S = 0x204, SITE_P = 0x205,
+                  SITE_O = 0x206, SITE_DRAIN = 0x207 };
+
+struct Seg {
+  int n;        // keys
+  int shared;   // keys shared by the batch (tensor map batch extent 1)
+};
+
+// Every tensor map starts at its operand's first column, so head h's columns
+// are [h*128, h*128 + 128) in all of them.
+struct Params {
+  int Lq;       // query rows per batch
+  Seg seg[2];
+  bf16* o;
+  int64_t o_rs;
+  float scale_log2;
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int NQ, int NSEG>
+__global__ void __launch_bounds__(Cfg<NQ, NSEG>::THREADS, 1)
+k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK0,
+          const __grid_constant__ CUtensorMap tmV0, const __grid_constant__ CUtensorMap tmK1,
+          const __grid_constant__ CUtensorMap tmV1, const Params p) {
+  using C = Cfg<NQ, NSEG>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* q_full = bars;                 // 1
+  uint64_t* kv_full = bars + 1;            // RING
+  uint64_t* kv_empty = kv_full + RING;     // RING
+  uint64_t* s_full = kv_empty + RING;      // NQ
+  uint64_t* p_full = s_full + NQ;          // NQ
+  uint64_t* o_done = p_full + NQ;          // NQ
+  uint64_t* tdone = o_done + NQ;           // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tdone + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int l0 = qb * BQ * NQ;
+  const int nk0 = p.seg[0].n, nk1 = p.seg[1].n;
+  const int sh0 = p.seg[0].shared, sh1 = p.seg[1].shared;
+  const int nb0 = (nk0 + BKV - 1) / BKV;
+  const int nb1 = NSEG == 2 ? (nk1 + BKV - 1) / BKV : 0;
+  const int NB = nb0 + nb1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < RING; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+    for (int t = 0; t < NQ; ++t) { mbar_init(&s_full[t], 1); mbar_init(&p_full[t], 128); mbar_init(&o_done[t], 1); }
+    mbar_init(tdone, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) { tmem_alloc(tmem_slot, C::TMEM_COLS); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA loader
+    if (lane == 0) {
+      bool ok = true;
+      uint32_t issued = 0, last_par = 0;
+      mbar_arrive_expect_tx(q_full, NQ * TILE_BYTES);
+      for (int t = 0; t < NQ; ++t)
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_3d(smem + C::Q_OFF + t * TILE_BYTES + hf * HALF_BYTES, &tmQ, h * DH + hf * 64,
+                      l0 + t * BQ, b, q_full);
+      for (int n = 0; n < NB && ok; ++n) {
+        const int sg = n < nb0 ? 0 : 1;
+        const int j0 = (n - (sg ? nb0 : 0)) * BKV;
+        const CUtensorMap* tk = sg ? &tmK1 : &tmK0;
+        const CUtensorMap* tv = sg ? &tmV1 : &tmV0;
+        const int bb = (sg ? sh1 : sh0) ? 0 : b;
+        for (int kv = 0; kv < 2; ++kv) {
+          const int seq = 2 * n + kv, slot = seq % RING;
+          const uint32_t ph = (seq / RING) & 1u;
+          if (!mbar_wait(&kv_empty[slot], ph ^ 1u, SITE_KVE)) { ok = false; break; }
+          mbar_arrive_expect_tx(&kv_full[slot], TILE_BYTES);
+          const int col = h * DH;
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_3d(smem + C::RING_OFF + slot * TILE_BYTES + hf * HALF_BYTES, kv ? tv : tk, col + hf * 64, j0,
+                        bb, &kv_full[slot]);
+          issued |= 1u << slot;
+          last_par = (last_par & ~(1u << slot)) | (ph << slot);
+        }
+      }
+      mbar_wait(q_full, 0, SITE_DRAIN);
+      for (int s = 0; s < RING; ++s)
+        if (issued & (1u << s)) mbar_wait(&kv_full[s], (last_par >> s) & 1u, SITE_DRAIN);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(q_full, 0, SITE_Q);
+      tc_fence_after();
+      const uint32_t q0 = smem_u32(smem + C::Q_OFF), p0 = smem_u32(smem + C::P_OFF);
+      const uint32_t r0 = smem_u32(smem + C::RING_OFF);
+      // P_t V_j for block n-1 of tile t
+      auto issue_pv = [&](int t, int n) -> bool {
+        if (!mbar_wait(&p_full[t], n & 1u, SITE_P)) return false;
+        const int vseq = 2 * n + 1, vslot = vseq % RING;
+        if (!mbar_wait(&kv_full[vslot], (vseq / RING) & 1u, SITE_KVF)) return false;
+        tc_fence_after();
+        const int sg = n < nb0 ? 0 : 1;
+        const int first = (n == 0) || (n == nb0);
+        const uint32_t d = tmem + C::o_col(t, sg);
+        const uint32_t pa = p0 + t * TILE_BYTES, vb = r0 + vslot * TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(pa + (kk >> 2) * HALF_BYTES + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(vb + kk * 2048, HALF_BYTES, 1024);
+          umma_ss(d, ad, bd, C::IDESC_O, (!first || kk) ? 1u : 0u);
+        }
+        if (t == NQ - 1) umma_commit(&kv_empty[vslot]);
+        return true;
+      };
+      for (int n = 0; n < NB && ok; ++n) {
+        const int kseq = 2 * n, kslot = kseq % RING;
+        if (!mbar_wait(&kv_full[kslot], (kseq / RING) & 1u, SITE_KVF)) { ok = false; break; }
+        tc_fence_after();
+        for (int t = 0; t < NQ && ok; ++t) {
+          if (n > 0 && !issue_pv(t, n - 1)) { ok = false; break; }
+          const uint32_t d = tmem + C::s_col(t);
+          const uint32_t qa = q0 + t * TILE_BYTES, kb = r0 + kslot * TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < DH / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+            umma_ss(d, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), C::IDESC_S, kk ? 1u : 0u);
+          }
+          umma_commit(&s_full[t]);
+        }
+        if (ok) umma_commit(&kv_empty[kslot]);
+      }
+      for (int t = 0; t < NQ && ok; ++t) {
+        if (!issue_pv(t, NB - 1)) { ok = false; break; }
+        umma_commit(&o_done[t]);
+      }
+      umma_commit(tdone);
+      mbar_wait(tdone, 0, SITE_DRAIN);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int t = (warp - 2) >> 2;       // Q tile of this warpgroup
+    const int quarter = warp & 3;        // TMEM lanes this warp may access
+    const int r = quarter * 32 + lane;   // query row within the tile
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t s_addr = tmem + lane_base + C::s_col(t);
+    uint8_t* prow = smem + C::P_OFF + t * TILE_BYTES + r * 128;
+    float m = -INFINITY, l = 0.f, l_first = 0.f;
+    bool ok = true;
+    for (int n = 0; n < NB; ++n) {
+      const int sg = n < nb0 ? 0 : 1;
+      const bool first = (n == 0) || (n == nb0);
+      if (NSEG == 2 && n == nb0) { l_first = l; m = -INFINITY; l = 0.f; }
+      if (!mbar_wait_warp(&s_full[t], n & 1u, SITE_S)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t s[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, s[c]);
+      tmem_wait_ld();
+      const int valid = (sg ? nk1 : nk0) - (n - (sg ? nb0 : 0)) * BKV;   // keys of this block that exist
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          float v = __uint_as_float(s[c][k]) * p.scale_log2;
+          if (c * 32 + k >= valid) v = -INFINITY;
+          s[c][k] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
+      // lazy rescale: move the reference max only when it grew by more than the threshold
+      const bool grow = mx > m + RESCALE_THRESHOLD;
+      const float m_new = grow ? mx : m;
+      const float alpha = grow ? ex2(m - m_new) : 1.f;
+      m = m_new;
+      // P = exp2(s - m) as bf16 into the swizzled shared tile (the S registers die here)
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {        // 8 keys -> one 16-byte chunk
+          float e[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            e[k] = ex2(__uint_as_float(s[c][g * 8 + k]) - m);
+            rs += e[k];
+          }
+          const int chunk = c * 4 + g;               // 0..15 over the 128 keys
+          const int atom = chunk >> 3, cc = chunk & 7;
+          uint4 pk = make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
+                                pack_bf16x2(e[6], e[7]));
+          *reinterpret_cast<uint4*>(prow + atom * HALF_BYTES + ((cc ^ (r & 7)) << 4)) = pk;
+        }
+      }
+      l = l * alpha + rs;
+      // O_t *= alpha for the rows whose reference max moved (P V of the previous
+      // block has completed: its commit precedes the S commit waited on above)
+      if (__any_sync(0xffffffffu, grow) && !first) {
+        const uint32_t o_addr = tmem + lane_base + C::o_col(t, sg);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_addr + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_st32(o_addr + c * 32, o);
+        }
+        tmem_wait_st();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+    }
+    // ---------------------------------------------------------- epilogue
+    if (ok && mbar_wait_warp(&o_done[t], 0, SITE_O)) {
+      tc_fence_after();
+      const int row = l0 + t * BQ + r;
+      const float inv1 = 1.f / l;
+      const float inv0 = NSEG == 2 ? 1.f / l_first : 0.f;
+      bf16* dst = p.o + (static_cast<int64_t>(b) * p.Lq + row) * p.o_rs + h * DH;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_base + C::o_col(t, NSEG - 1) + c * 32, o);
+        tmem_wait_ld();
+        float v[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(o[k]) * inv1;
+        if (NSEG == 2) {
+          uint32_t o2[32];
+          tmem_ld32(tmem + lane_base + C::o_col(t, 0) + c * 32, o2);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) v[k] += __uint_as_float(o2[k]) * inv0;
+        }
+        if (row < p.Lq) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            d4[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                               pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace tca
+
+// ------------------------------------------------------------------ host side
+// 3D bf16 tensor map over [batches, rows, cols] (cols contiguous, row stride
+// `rs` elements, batch stride `bs` elements); box = 64 cols x 128 rows x 1.
+static wd_status make_tmap_3d(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int64_t batches,
+                              int64_t rs, int64_t bs) {
+  auto fn = encode_fn();
+  if (!fn) { set_error("cuTensorMapEncodeTiled unavailable"); return WD_ERR_CUDA; }
+  if (batches > 1 && (bs * 2) % 16) { set_error("attention: batch stride not 16-byte aligned"); return WD_ERR_ALIGN; }
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(batches)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(rs) * 2,
+                           static_cast<cuuint64_t>(batches > 1 ? bs : rs * rows) * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) { set_error("cuTensorMapEncodeTiled (3d) failed (%d)", static_cast<int>(r)); return WD_ERR_CUDA; }
+  return WD_OK;
+}
+
+template <int NQ, int NSEG>
+static wd_status launch_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk0, const CUtensorMap& tv0,
+                                const CUtensorMap& tk1, const CUtensorMap& tv1, const tca::Params& p, int batch,
+                                int heads, cudaStream_t st) {
+  using C = tca::Cfg<NQ, NSEG>;
+  static bool attr[16] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr[dev & 15]) {
+    cudaFuncSetAttribute(tca::k_attn_tc<NQ, NSEG>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    attr[dev & 15] = true;
+  }
+  dim3 grid((p.Lq + tca::BQ * NQ - 1) / (tca::BQ * NQ), heads, batch);
+  tca::k_attn_tc<NQ, NSEG><<<grid, C::THREADS, C::SMEM, st>>>(tq, tk0, tv0, tk1, tv1, p);
+  return launch_status("attention_tc");
+}
+
+// The q/k/v pointers of AttnArgs may point into the middle of a row (the
+// fused q|k|v buffer); the tensor maps start at the row's first element that
+// is 16-byte aligned (the pointer itself) and use the row stride as extent.
+wd_status attention_tc(const AttnArgs<bf16>& a, cudaStream_t st) {
+  if (a.dh != tca::DH) return attention_simt<bf16>(a, st);
+  if (a.n1 <= 0 || (a.k2 && a.n2 <= 0)) { set_error("attention: empty key segment"); return WD_ERR_SHAPE; }
+  const int D = a.heads * a.dh;
+  auto al = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; };
+  if (!al(a.q) || !al(a.k1) || !al(a.v1) || (a.k2 && (!al(a.k2) || !al(a.v2))) || !al(a.o) || (a.q_rs % 8) ||
+      (a.kv1_rs % 8) || (a.kv2_rs % 8) || (a.o_rs % 8)) {
+    set_error("attention_tc: operands must be 16-byte aligned with row strides multiple of 8");
+    return WD_ERR_ALIGN;
+  }
+  CUtensorMap tq, tk0, tv0, tk1, tv1;
+  // Each map covers D columns from its own base pointer.
+  WD_TRY(make_tmap_3d(&tq, a.q, D, a.Lq, a.batch, a.q_rs, a.q_rs * a.Lq));
+  const int64_t b1 = a.kv1_bs ? a.batch : 1;
+  WD_TRY(make_tmap_3d(&tk0, a.k1, D, a.n1, b1, a.kv1_rs, a.kv1_bs));
+  WD_TRY(make_tmap_3d(&tv0, a.v1, D, a.n1, b1, a.kv1_rs, a.kv1_bs));
+  tca::Params p{};
+  p.Lq = a.Lq;
+  p.seg[0] = tca::Seg{a.n1, a.kv1_bs == 0};
+  p.o = a.o;
+  p.o_rs = a.o_rs;
+  p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(a.dh));
+  if (a.k2) {
+    const int64_t b2 = a.kv2_bs ? a.batch : 1;
+    WD_TRY(make_tmap_3d(&tk1, a.k2, D, a.n2, b2, a.kv2_rs, a.kv2_bs));
+    WD_TRY(make_tmap_3d(&tv1, a.v2, D, a.n2, b2, a.kv2_rs, a.kv2_bs));
+    p.seg[1] = tca::Seg{a.n2, a.kv2_bs == 0};
+    return launch_attn_tc<1, 2>(tq, tk0, tv0, tk1, tv1, p, a.batch, a.heads, st);
+  }
+  return launch_attn_tc<2, 1>(tq, tk0, tv0, tk0, tv0, p, a.batch, a.heads, st);
+}
+
 }  // namespace wd

@@ -191,7 +191,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
       const int m0 = (t / n_tiles) * BM, n0 = (t % n_tiles) * BN;
-      if (!mbar_wait(&tfull[acc], acc_phase, SITE_TFULL)) break;
+      if (!mbar_wait_warp(&tfull[acc], acc_phase, SITE_TFULL)) break;
       tc_fence_after();
       const int64_t m = m0 + q * 32 + lane;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
