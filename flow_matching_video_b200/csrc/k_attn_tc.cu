@@ -6,12 +6,13 @@
 // A CTA owns NQ query tiles of 128 rows of one (batch, head) and streams the
 // keys/values of NSEG segments in 128-key blocks:
 //   warp 0           TMA loader: the Q tiles once, then K_j, V_j through a
-//                    3-slot ring of 32 KB tiles
+//                    ring of RING 32 KB tiles
 //   warp 1           TMEM owner + MMA issuer: S_t = Q_t K_j^T into TMEM,
-//                    O_t (+)= P_t V_j with P_t from shared memory
+//                    O_t (+)= P_t V_j with P_t read from TMEM (TS form), so
+//                    this product reads only V from shared memory
 //   warps 2..        one warpgroup (128 threads, thread = query row) per Q
 //                    tile: online softmax on S_t read from TMEM, P_t written
-//                    as bf16 into a 128-byte-swizzled shared tile, O_t
+//                    back as bf16 over the first half of S_t's columns, O_t
 //                    rescaled in TMEM only when the running max grows by more
 //                    than 8 (log2 units; the final 1/l keeps the result
 //                    exact), then the normalised output written out.
@@ -25,15 +26,17 @@ namespace tca {
 constexpr int BQ = 128, BKV = 128, DH = 128;
 constexpr int TILE_BYTES = 128 * 128 * 2;   // one 128 x 128 bf16 tile (two 64-column halves)
 constexpr int HALF_BYTES = TILE_BYTES / 2;
-constexpr int RING = 3;
+#ifndef WD_ATTN_RING
+#define WD_ATTN_RING 5   // K/V tiles in flight (32 KB each)
+#endif
+constexpr int RING = WD_ATTN_RING;
 constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
 
 template <int NQ, int NSEG>
 struct Cfg {
   static constexpr int THREADS = 64 + 128 * NQ;
   static constexpr int Q_OFF = 0;
-  static constexpr int P_OFF = NQ * TILE_BYTES;
-  static constexpr int RING_OFF = 2 * NQ * TILE_BYTES;
+  static constexpr int RING_OFF = NQ * TILE_BYTES;
   static constexpr int BAR_OFF = RING_OFF + RING * TILE_BYTES;
   static constexpr int SMEM = 1024 + BAR_OFF + 256;
   static constexpr int TMEM_COLS = 512;
@@ -41,11 +44,11 @@ struct Cfg {
   __host__ __device__ static constexpr int s_col(int t) { return NSEG == 1 ? t * 256 : 0; }
   __host__ __device__ static constexpr int o_col(int t, int seg) { return NSEG == 1 ? t * 256 + 128 : 128 + 128 * seg; }
   static constexpr uint32_t IDESC_S = idesc_bf16(128, 128, 0, 0);    // Q K^T: both K-major
-  static constexpr uint32_t IDESC_O = idesc_bf16(128, 128, 0, 1);    // P V: V is MN-major (dh contiguous)
+  static constexpr uint32_t IDESC_O = idesc_bf16(128, 128, 0, 1);    // P V: P from TMEM, V MN-major (dh contiguous)
 };
 
 enum : unsigned { SITE_Q = 0x201, SITE_KVF = 0x202, SITE_KVE = 0x203, SITE_S = 0x204, SITE_P = 0x205,
-                  SITE_O = 0x206, SITE_DRAIN = 0x207 };
+                  SITE_O = 0x206, SITE_DRAIN = 0x207, SITE_TOK = 0x208 };
 
 struct Seg {
   int n;        // keys
@@ -68,6 +71,27 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x on the FMA/ALU pipes, to take part of the exponentials off the MUFU
+// unit (the softmax otherwise saturates it at the same rate as the tensor
+// cores).  Range reduction x = j + f with j = round(x): adding 1.5 * 2^23
+// leaves round(x) in the low mantissa bits of the sum (round-to-nearest-even);
+// 2^f on [-1/2, 1/2] is a degree-3 polynomial whose coefficients were fitted
+// for this library (iteratively reweighted least squares on the relative
+// error, max relative error 7.5e-5 in fp32, far below a bf16 half-ulp); the
+// factor 2^j is added to the exponent field.  Arguments below -127 give 0.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -127.f);
+  const float t = x + 12582912.f;
+  const int j = __float_as_int(t) - 0x4B400000;
+  const float f = x - (t - 12582912.f);
+  const float q = fmaf(fmaf(fmaf(0.0551716648f, f, 0.2426111251f), f, 0.6932609677f), f, 0.9999280572f);
+  return __int_as_float(__float_as_int(q) + (j << 23));
+}
+
+#ifndef WD_EXP2_EMU_PER8
+#define WD_EXP2_EMU_PER8 0   // of every 8 exponentials, this many run on the FMA pipe
+#endif
+
 template <int NQ, int NSEG>
 __global__ void __launch_bounds__(Cfg<NQ, NSEG>::THREADS, 1)
 k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK0,
@@ -84,7 +108,8 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   uint64_t* p_full = s_full + NQ;          // NQ
   uint64_t* o_done = p_full + NQ;          // NQ
   uint64_t* tdone = o_done + NQ;           // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tdone + 1);
+  uint64_t* tok = tdone + 1;               // 2: exp-phase token between the two softmax warpgroups
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tok + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -98,8 +123,10 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < RING; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
-    for (int t = 0; t < NQ; ++t) { mbar_init(&s_full[t], 1); mbar_init(&p_full[t], 128); mbar_init(&o_done[t], 1); }
+    for (int t = 0; t < NQ; ++t) { mbar_init(&s_full[t], 1); mbar_init(&p_full[t], 4); mbar_init(&o_done[t], 1); }
     mbar_init(tdone, 1);
+    mbar_init(&tok[0], 4);
+    mbar_init(&tok[1], 4);
     fence_mbar_init();
   }
   if (warp == 1) { tmem_alloc(tmem_slot, C::TMEM_COLS); tmem_relinquish(); }
@@ -147,7 +174,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     if (lane == 0) {
       bool ok = mbar_wait(q_full, 0, SITE_Q);
       tc_fence_after();
-      const uint32_t q0 = smem_u32(smem + C::Q_OFF), p0 = smem_u32(smem + C::P_OFF);
+      const uint32_t q0 = smem_u32(smem + C::Q_OFF);
       const uint32_t r0 = smem_u32(smem + C::RING_OFF);
       // P_t V_j for block n-1 of tile t
       auto issue_pv = [&](int t, int n) -> bool {
@@ -158,12 +185,12 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         const int sg = n < nb0 ? 0 : 1;
         const int first = (n == 0) || (n == nb0);
         const uint32_t d = tmem + C::o_col(t, sg);
-        const uint32_t pa = p0 + t * TILE_BYTES, vb = r0 + vslot * TILE_BYTES;
+        const uint32_t pa = tmem + C::s_col(t), vb = r0 + vslot * TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(pa + (kk >> 2) * HALF_BYTES + (kk & 3) * 32, 16, 1024);
+          // A = P: 16 keys = 8 TMEM columns of packed bf16 pairs
           const uint64_t bd = sdesc_sw128(vb + kk * 2048, HALF_BYTES, 1024);
-          umma_ss(d, ad, bd, C::IDESC_O, (!first || kk) ? 1u : 0u);
+          umma_ts(d, pa + kk * 8, bd, C::IDESC_O, (!first || kk) ? 1u : 0u);
         }
         if (t == NQ - 1) umma_commit(&kv_empty[vslot]);
         return true;
@@ -200,7 +227,6 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const int r = quarter * 32 + lane;   // query row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_addr = tmem + lane_base + C::s_col(t);
-    uint8_t* prow = smem + C::P_OFF + t * TILE_BYTES + r * 128;
     float m = -INFINITY, l = 0.f, l_first = 0.f;
     bool ok = true;
     for (int n = 0; n < NB; ++n) {
@@ -209,45 +235,70 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       if (NSEG == 2 && n == nb0) { l_first = l; m = -INFINITY; l = 0.f; }
       if (!mbar_wait_warp(&s_full[t], n & 1u, SITE_S)) { ok = false; break; }
       tc_fence_after();
-      uint32_t s[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, s[c]);
-      tmem_wait_ld();
       const int valid = (sg ? nk1 : nk0) - (n - (sg ? nb0 : 0)) * BKV;   // keys of this block that exist
+      const bool ragged = valid < BKV;                                      // warp-uniform
+      // pass 1: row maximum of the raw scores, 64 columns in registers at a time
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t a[32], c[32];
+        tmem_ld32(s_addr + hf * 64, a);
+        tmem_ld32(s_addr + hf * 64 + 32, c);
+        tmem_wait_ld();
+        if (ragged) {
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          float v = __uint_as_float(s[c][k]) * p.scale_log2;
-          if (c * 32 + k >= valid) v = -INFINITY;
-          s[c][k] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
+          for (int k = 0; k < 32; ++k) {
+            if (hf * 64 + k >= valid) a[k] = __float_as_uint(-INFINITY);
+            if (hf * 64 + 32 + k >= valid) c[k] = __float_as_uint(-INFINITY);
+          }
         }
+#pragma unroll
+        for (int k = 0; k < 32; ++k) mx = fmax3(mx, __uint_as_float(a[k]), __uint_as_float(c[k]));
+      }
+      mx *= p.scale_log2;
       // lazy rescale: move the reference max only when it grew by more than the threshold
       const bool grow = mx > m + RESCALE_THRESHOLD;
       const float m_new = grow ? mx : m;
       const float alpha = grow ? ex2(m - m_new) : 1.f;
       m = m_new;
-      // P = exp2(s - m) as bf16 into the swizzled shared tile (the S registers die here)
-      float rs = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {        // 8 keys -> one 16-byte chunk
-          float e[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            e[k] = ex2(__uint_as_float(s[c][g * 8 + k]) - m);
-            rs += e[k];
-          }
-          const int chunk = c * 4 + g;               // 0..15 over the 128 keys
-          const int atom = chunk >> 3, cc = chunk & 7;
-          uint4 pk = make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
-                                pack_bf16x2(e[6], e[7]));
-          *reinterpret_cast<uint4*>(prow + atom * HALF_BYTES + ((cc ^ (r & 7)) << 4)) = pk;
-        }
+      const float neg_m = -m;
+      // The two warpgroups take turns with the exponentials (MUFU), so that one
+      // tile's softmax overlaps the other tile's MMAs instead of both sharing
+      // the unit at the same time.
+      if (NQ == 2 && !(t == 0 && n == 0)) {
+        if (!mbar_wait_warp(&tok[t], (t == 0 ? n - 1 : n) & 1u, SITE_TOK)) { ok = false; break; }
       }
+      // pass 2: P = exp2(s * scale - m) as packed bf16 pairs into TMEM, over
+      // the first 64 columns of S_t (each half is written after it was read)
+      float2 rs2 = make_float2(0.f, 0.f);
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(neg_m, neg_m);
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t a[64];
+        tmem_ld32(s_addr + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+        tmem_ld32(s_addr + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+        tmem_wait_ld();
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 64; k += 2) {
+          const float2 arg = ffma2(make_float2(__uint_as_float(a[k]), __uint_as_float(a[k + 1])), sc2, nm2);
+          float e0 = ((k & 7) >= 8 - WD_EXP2_EMU_PER8) ? exp2_fma(arg.x) : ex2(arg.x);
+          float e1 = (((k + 1) & 7) >= 8 - WD_EXP2_EMU_PER8) ? exp2_fma(arg.y) : ex2(arg.y);
+          if (ragged) {
+            if (hf * 64 + k >= valid) e0 = 0.f;
+            if (hf * 64 + k + 1 >= valid) e1 = 0.f;
+          }
+          rs2 = fadd2(rs2, make_float2(e0, e1));
+          pk[k >> 1] = pack_bf16x2(e0, e1);
+        }
+        tmem_st32(s_addr + hf * 32, pk);
+      }
+      tmem_wait_st();
+      if (NQ == 2) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tok[1 - t]);
+      }
+      const float rs = rs2.x + rs2.y;
       l = l * alpha + rs;
       // O_t *= alpha for the rows whose reference max moved (P V of the previous
       // block has completed: its commit precedes the S commit waited on above)
@@ -264,9 +315,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         }
         tmem_wait_st();
       }
-      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full[t]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[t]);
     }
     // ---------------------------------------------------------- epilogue
     if (ok && mbar_wait_warp(&o_done[t], 0, SITE_O)) {
@@ -343,6 +394,7 @@ static wd_status launch_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk0, c
     attr[dev & 15] = true;
   }
   dim3 grid((p.Lq + tca::BQ * NQ - 1) / (tca::BQ * NQ), heads, batch);
+  Trace tr(NSEG == 2 ? KC_ATTN_CROSS : KC_ATTN_SELF, st);
   tca::k_attn_tc<NQ, NSEG><<<grid, C::THREADS, C::SMEM, st>>>(tq, tk0, tv0, tk1, tv1, p);
   return launch_status("attention_tc");
 }

@@ -6,13 +6,14 @@
 // weight [N, K]; both K-major, loaded by TMA into 128-byte-swizzled shared
 // memory tiles of 64 K-elements.
 //
-// CTA = 6 warps, persistent over output tiles of 128 x BN:
+// CTA = 2 + 4 * EPI_WG warps, persistent over output tiles of 128 x BN:
 //   warp 0     TMA producer (one lane): STAGES-deep ring of (A, B) tiles
 //   warp 1     TMEM owner + MMA issuer (one lane): 128 x BN x 16 UMMAs,
 //              accumulating in one of two TMEM buffers
-//   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter of the
-//              accumulator, epilogue math, global stores; they release the
-//              TMEM buffer so the next tile's MMAs overlap this epilogue.
+//   warps 2..  epilogue, EPI_WG warpgroups: each warp reads its 32-lane
+//              quarter of the accumulator for its warpgroup's share of the
+//              columns (tcgen05.ld), applies the epilogue and stores; they
+//              release the TMEM buffer so the next tile's MMAs overlap it.
 #include "wd_internal.cuh"
 
 #include <cudaTypedefs.h>
@@ -21,7 +22,11 @@ namespace wd {
 namespace tcg {
 
 constexpr int BM = 128, BK = 64;
-constexpr int THREADS = 192;
+#ifndef WD_GEMM_EPI_WG
+#define WD_GEMM_EPI_WG 1   // epilogue warpgroups; each takes an equal share of the tile's columns
+#endif
+constexpr int EPI_WG = WD_GEMM_EPI_WG;
+constexpr int THREADS = 64 + 128 * EPI_WG;
 
 template <int BN>
 struct Cfg {
@@ -41,7 +46,8 @@ enum : unsigned { SITE_EMPTY = 0x101, SITE_FULL = 0x102, SITE_TFULL = 0x103, SIT
 // ------------------------------------------------------------------ epilogue on 32 columns
 // One thread = one output row m; columns n .. n+31 come from the accumulator.
 template <int MODE>
-__device__ __forceinline__ void epilogue32(const Epi& ep, int64_t m, int n, const uint32_t (&r)[32]) {
+__device__ __forceinline__ void epilogue32(const Epi& ep, int64_t m, int n, const uint32_t (&r)[32],
+                                           const float4 (&xres)[8]) {
   float v[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
@@ -80,7 +86,7 @@ __device__ __forceinline__ void epilogue32(const Epi& ep, int64_t m, int n, cons
                                     : make_float4(0.f, 0.f, 0.f, 0.f);
         g = make_float4(ga.x + gb.x, ga.y + gb.y, ga.z + gb.z, ga.w + gb.w);
       }
-      float4 x = dst[j];
+      float4 x = xres[j];
       x.x += g.x * v[4 * j]; x.y += g.y * v[4 * j + 1]; x.z += g.z * v[4 * j + 2]; x.w += g.w * v[4 * j + 3];
       dst[j] = x;
     }
@@ -116,7 +122,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 4); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 4 * EPI_WG); }
     mbar_init(tdone, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -187,6 +193,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   } else {
     // ---------------------------------------------------------- epilogue warps
     const int q = warp & 3;   // TMEM lane quarter this warp may access
+    constexpr int COLS = BN / EPI_WG;
+    const int c_begin = ((warp - 2) >> 2) * COLS;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
@@ -196,11 +204,19 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       const int64_t m = m0 + q * 32 + lane;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
+      for (int c = c_begin; c < c_begin + COLS; c += 32) {
+        float4 xres[8];
+        if constexpr (MODE == EPI_RESID) {   // residual loads in flight while TMEM is read
+          if (m < M) {
+            const float4* src = reinterpret_cast<const float4*>(static_cast<float*>(ep.out) + m * ep.ldo + n0 + c);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) xres[j] = src[j];
+          }
+        }
         uint32_t r[32];
         tmem_ld32(tbase + c, r);
         tmem_wait_ld();
-        if (m < M) epilogue32<MODE>(ep, m, n0 + c, r);
+        if (m < M) epilogue32<MODE>(ep, m, n0 + c, r, xres);
       }
       tc_fence_before();
       __syncwarp();
@@ -268,6 +284,7 @@ static wd_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const E
   }
   const int tiles = ((M + tcg::BM - 1) / tcg::BM) * (N / BN);
   const int grid = tiles < sm_count() ? tiles : sm_count();
+  Trace tr(KC_GEMM, st);
   tcg::k_gemm_tc<BN, MODE><<<grid, tcg::THREADS, C::SMEM, st>>>(ta, tb, ep, M, N, K);
   return launch_status("gemm_tc");
 }

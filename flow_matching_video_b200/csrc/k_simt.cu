@@ -75,6 +75,7 @@ wd_status gemm_simt(int M, int N, int K, const T* A, int64_t lda, const T* B, in
   if (M <= 0 || N <= 0 || K <= 0) { set_error("gemm: empty shape %d x %d x %d", M, N, K); return WD_ERR_SHAPE; }
   dim3 grid((N + 63) / 64, (M + 63) / 64);
   if (grid.y > 65535u) { set_error("gemm_simt: M=%d too large", M); return WD_ERR_SHAPE; }
+  Trace tr(KC_GEMM, st);
   k_gemm_simt<T><<<grid, 256, 0, st>>>(M, N, K, A, lda, B, ldb, mode, ep);
   return launch_status("gemm_simt");
 }
@@ -208,6 +209,7 @@ static wd_status launch_attn_simt(const AttnArgs<T>& a, cudaStream_t st) {
   }
   dim3 grid((a.Lq + 63) / 64, a.heads, a.batch);
   const float qscale = 1.4426950408889634f / sqrtf(static_cast<float>(DH));
+  Trace tr(a.k2 ? KC_ATTN_CROSS : KC_ATTN_SELF, st);
   k_attn_simt<T, DH><<<grid, 256, smem, st>>>(a, qscale);
   return launch_status("attention_simt");
 }

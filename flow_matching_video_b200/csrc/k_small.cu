@@ -167,6 +167,7 @@ template <typename OutT>
 wd_status norm_mod(const NormArgs& a, cudaStream_t st) {
   if (a.D % 128 != 0) { set_error("norm: D=%d must be a multiple of 128", a.D); return WD_ERR_SHAPE; }
   const unsigned grid = static_cast<unsigned>((a.rows * 32 + 255) / 256);
+  Trace tr(KC_NORM, st);
   switch (a.D / 128) {
     case 1: k_norm_mod<OutT, 1><<<grid, 256, 0, st>>>(a); break;
     case 2: k_norm_mod<OutT, 2><<<grid, 256, 0, st>>>(a); break;
@@ -278,6 +279,7 @@ wd_status qknorm_rope(T* qkv, int64_t rows, const wd_dims& d, const float* gq, c
   const int D = d.D, dh = D / d.heads;
   const int L = d.T * (d.H / 2) * (d.W / 2);
   const unsigned grid = static_cast<unsigned>((2 * rows * 32 + 255) / 256);
+  Trace tr(KC_ROPE, st);
 #define WD_QKR(NC)                                                                                       \
   k_qknorm_rope<T, NC><<<grid, 256, 0, st>>>(qkv, rows, D, dh, L, d.H / 2, d.W / 2, d.T, gq, gk, tab, d.eps); \
   break;

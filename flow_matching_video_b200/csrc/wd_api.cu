@@ -157,7 +157,7 @@ static wd_status block_forward_t(const wd_dims* d, const wd_block_weights* w, co
   // 2. q|k|v = h Wqkv^T + b
   WD_TRY(gemm<T>(M, 3 * D, D, Bf, D, w->qkv_w, D, EPI_STORE, epi(A, 3 * D, w->qkv_b), st));
   // 3. QK-RMSNorm + 3D RoPE in place
-  k_rope_table<<<64, 256, 0, st>>>(ws.rope, d->T, d->H / 2, d->W / 2, dh);
+  { Trace tr(KC_SMALL, st); k_rope_table<<<64, 256, 0, st>>>(ws.rope, d->T, d->H / 2, d->W / 2, dh); }
   WD_TRY(launch_status("rope_table"));
   WD_TRY(qknorm_rope<T>(A, rows, *d, w->g_q, w->g_k, ws.rope, st));
   // 4. full self-attention -> o
@@ -270,6 +270,7 @@ wd_status wd_build_cond_y(const wd_dims* d, const float* img_lat, const int* kno
   const int64_t HW = static_cast<int64_t>(d->H) * d->W;
   const int64_t n = 20 * d->T * HW;
   const unsigned grid = static_cast<unsigned>((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  Trace tr(KC_SMALL, static_cast<cudaStream_t>(stream));
   k_cond_y<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(img_lat, mb, d->T, HW, y);
   return launch_status("build_cond_y");
 }
@@ -285,6 +286,7 @@ wd_status wd_euler_cfg_step(float* x, const float* v_cond, const float* v_uncond
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const size_t want = (n / 4 + 255) / 256;
   const unsigned grid = static_cast<unsigned>(want < static_cast<size_t>(sms) * 8 ? (want ? want : 1) : sms * 8);
+  Trace tr(KC_EULER, static_cast<cudaStream_t>(stream));
   k_euler_cfg<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, v_cond, v_uncond, cfg_scale, dt,
                                                                    static_cast<int64_t>(n));
   return launch_status("euler_cfg_step");
@@ -299,9 +301,9 @@ wd_status wd_time_mod(const wd_dims* d, const wd_time_weights* w, float tau, flo
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int D = d->D;
   // h1 = t1(sin(tau)) is written to e0 (scratch until the last launch)
-  k_time_matvec<<<(D * 32 + 255) / 256, 256, 0, st>>>(w->t1_w, w->t1_b, nullptr, tau, 0, D, 256, e0);
-  k_time_matvec<<<(D * 32 + 255) / 256, 256, 0, st>>>(w->t2_w, w->t2_b, e0, 0.f, 1, D, D, e);
-  k_time_matvec<<<(6 * D * 32 + 255) / 256, 256, 0, st>>>(w->tp_w, w->tp_b, e, 0.f, 1, 6 * D, D, e0);
+  { Trace tr(KC_SMALL, st); k_time_matvec<<<(D * 32 + 255) / 256, 256, 0, st>>>(w->t1_w, w->t1_b, nullptr, tau, 0, D, 256, e0); }
+  { Trace tr(KC_SMALL, st); k_time_matvec<<<(D * 32 + 255) / 256, 256, 0, st>>>(w->t2_w, w->t2_b, e0, 0.f, 1, D, D, e); }
+  { Trace tr(KC_SMALL, st); k_time_matvec<<<(6 * D * 32 + 255) / 256, 256, 0, st>>>(w->tp_w, w->tp_b, e, 0.f, 1, 6 * D, D, e0); }
   return launch_status("time_mod");
 }
 
@@ -382,11 +384,11 @@ wd_status wd_patch_embed(const wd_dims* d, const float* x_t, const float* y, con
   const int64_t n = rows * 144;
   const unsigned grid = static_cast<unsigned>((n + 255) / 256 < 65536 ? (n + 255) / 256 : 65536);
   if (d->dtype == WD_BF16) {
-    k_patch_gather<bf16><<<grid, 256, 0, st>>>(x_t, y, batch, d->T, d->H, d->W, static_cast<bf16*>(L.b));
+    { Trace tr(KC_SMALL, st); k_patch_gather<bf16><<<grid, 256, 0, st>>>(x_t, y, batch, d->T, d->H, d->W, static_cast<bf16*>(L.b)); }
     WD_TRY(launch_status("patch_gather"));
     WD_TRY(gemm<bf16>(static_cast<int>(rows), d->D, 144, L.b, 144, w, 144, EPI_F32, epi(X, d->D, b), st));
   } else {
-    k_patch_gather<float><<<grid, 256, 0, st>>>(x_t, y, batch, d->T, d->H, d->W, static_cast<float*>(L.b));
+    { Trace tr(KC_SMALL, st); k_patch_gather<float><<<grid, 256, 0, st>>>(x_t, y, batch, d->T, d->H, d->W, static_cast<float*>(L.b)); }
     WD_TRY(launch_status("patch_gather"));
     WD_TRY(gemm<float>(static_cast<int>(rows), d->D, 144, L.b, 144, w, 144, EPI_F32, epi(X, d->D, b), st));
   }

@@ -26,6 +26,20 @@ void set_error(const char* fmt, ...);
 
 wd_status launch_status(const char* what);   // cudaGetLastError -> WD_ERR_CUDA + message
 
+// ------------------------------------------------------------------ tracing
+// Kernel classes for launch accounting (same order as wd_kernel_class in wd.h).
+enum KClass : int { KC_GEMM = 0, KC_ATTN_SELF = 1, KC_ATTN_CROSS = 2, KC_NORM = 3, KC_ROPE = 4, KC_EULER = 5,
+                    KC_SMALL = 6, KC_COUNT = 7 };
+// Scope guard around one launch: counts it and, with timing on, records an
+// event on `st` at construction and another at destruction.
+struct Trace {
+  Trace(int cls, cudaStream_t st);
+  ~Trace();
+  int cls_;
+  cudaStream_t st_;
+  int slot_;
+};
+
 // ------------------------------------------------------------------ element conversions
 template <typename T> __device__ __forceinline__ float to_f(T v);
 template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }

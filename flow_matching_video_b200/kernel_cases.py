@@ -1,0 +1,84 @@
+"""Run one libwd kernel at the benchmark's shapes, for timing and profiling.
+
+    python -m flow_matching_video_b200.kernel_cases CASE [--batch B] [--iters N] [--warmup W]
+
+CASE is one of attn_self, attn_cross, gemm_qkv, gemm_o, gemm_ffn1, gemm_ffn2,
+norm, qknorm_rope, euler.  Shapes are those of one block of the 30-block
+480p/81-frame model (L = 32760 tokens per sample, D = 1536, 12 heads x 128,
+FFN 8960, 257 image + 512 text keys).  Inputs are seeded random values; the
+case prints the mean device time per launch (CUDA events) and the
+algorithmic FLOPs or bytes per launch.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import build
+
+build.build()
+from . import model, synth, wd  # noqa: E402
+
+L, D, H, F, NI, NT = 32760, 1536, 12, 8960, 257, 512
+
+
+def bf(*shape):
+    return torch.randn(*shape, device="cuda").to(torch.bfloat16)
+
+
+def make_case(name: str, B: int):
+    rows = B * L
+    if name == "attn_self":
+        q, k, v, o = bf(B, L, D), bf(B, L, D), bf(B, L, D), torch.empty(B, L, D, device="cuda", dtype=torch.bfloat16)
+        return (lambda: wd.wd_attention(wd.WD_BF16, B, L, H, 128, q, k, v, L, 0, o)), 4.0 * B * L * L * D, "FLOP"
+    if name == "attn_cross":
+        q, o = bf(B, L, D), torch.empty(B, L, D, device="cuda", dtype=torch.bfloat16)
+        ki, vi, kt, vt = bf(NI, D), bf(NI, D), bf(B, NT, D), bf(B, NT, D)
+        return (lambda: wd.wd_attention(wd.WD_BF16, B, L, H, 128, q, ki, vi, NI, 1, o, kt, vt, NT, 0),
+                4.0 * B * L * (NI + NT) * D, "FLOP")
+    gemms = {"gemm_qkv": (3 * D, D, wd.EPI_STORE), "gemm_o": (D, D, wd.EPI_RESID),
+             "gemm_ffn1": (F, D, wd.EPI_GELU), "gemm_ffn2": (D, F, wd.EPI_RESID)}
+    if name in gemms:
+        N, K, epi = gemms[name]
+        A, W, bias = bf(rows, K), bf(N, K) * 0.02, torch.zeros(N, device="cuda")
+        out = torch.zeros(rows, N, device="cuda", dtype=torch.float32 if epi == wd.EPI_RESID else torch.bfloat16)
+        g = torch.zeros(N, device="cuda")
+        return (lambda: wd.wd_gemm(wd.WD_BF16, rows, N, K, A, W, bias, epi, out,
+                                   g if epi == wd.EPI_RESID else None)), 2.0 * rows * N * K, "FLOP"
+    d = synth.Dims(D=D, heads=H, ffn=F, blocks=1, T=21, H=60, W=104, n_txt=NT, c_txt=4096, n_img=NI,
+                   c_img=1280, dtype="bf16")
+    if name == "euler":
+        n = 16 * 21 * 60 * 104
+        x, vc, vu = (torch.randn(n, device="cuda") for _ in range(3))
+        return (lambda: wd.wd_euler_cfg_step(x, vc, vu, 5.0, 1 / 12)), 16.0 * n, "B"
+    raise SystemExit(f"unknown case {name}")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case")
+    ap.add_argument("--batch", type=int, default=2)
+    ap.add_argument("--iters", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=2)
+    a = ap.parse_args()
+    torch.manual_seed(0)
+    run, work, unit = make_case(a.case, a.batch)
+    for _ in range(a.warmup):
+        run()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(a.iters):
+        run()
+    e.record()
+    torch.cuda.synchronize()
+    wd.wd_check()
+    ms = s.elapsed_time(e) / a.iters
+    rate = work / (ms / 1e3) / (1e12 if unit == "FLOP" else 1e9)
+    print(f"{a.case} batch={a.batch}: {ms:.4f} ms/launch, {work:.4g} {unit}/launch, "
+          f"{rate:.1f} {'TFLOP/s' if unit == 'FLOP' else 'GB/s'}")
+
+
+if __name__ == "__main__":
+    main()

@@ -100,8 +100,14 @@ WIDE_720P81 = Workload("bf16-40blk-D5120-L75600-cfg",
                             n_txt=512, c_txt=4096, n_img=257, c_img=1280, dtype="bf16"),
                        batch=2, seed=1004, steps=1, cfg_scale=5.0)
 SAMPLE_480P81 = replace(STACK_480P81, name="bf16-30blk-L32760-12step-cfg", seed=1005, steps=12)
+# A small bf16 model with 128-wide heads (so every tensor-core kernel runs) and
+# a ragged token grid (L = 3*5*7 = 105): smoke runs and fast parity checks.
+SMALL_BF16 = Workload("small-bf16-dh128-L105",
+                      Dims(D=256, heads=2, ffn=512, blocks=2, T=3, H=10, W=14, n_txt=24, c_txt=64,
+                           n_img=9, c_img=32, dtype="bf16"),
+                      batch=2, seed=1012, steps=1, txt_valid=(5, 24))
 
-WORKLOADS = {w.name: w for w in (TINY, BLOCK_480P17, STACK_480P81, WIDE_720P81, SAMPLE_480P81)}
+WORKLOADS = {w.name: w for w in (TINY, BLOCK_480P17, STACK_480P81, WIDE_720P81, SAMPLE_480P81, SMALL_BF16)}
 
 
 def stream(seed: int, name: str) -> np.random.Generator:

@@ -70,7 +70,10 @@ SIGNATURES = {
     "wd_gemm": (_I, [_I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P]),
     "wd_attention": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P, _I, _I, _P, _P]),
     "wd_set_debug_flags": (None, [C.c_uint]),
+    "wd_trace_enable": (None, [_I]),
+    "wd_trace_read": (_I, [C.POINTER(C.c_int64), C.POINTER(C.c_double)]),
 }
+KERNEL_CLASSES = ("gemm", "attn_self", "attn_cross", "norm", "qknorm_rope", "euler", "small")
 for _name, (_res, _args) in SIGNATURES.items():
     _fn = getattr(_lib, _name)
     _fn.restype = _res
@@ -189,3 +192,15 @@ def wd_attention(dtype, batch, Lq, heads, dh, q, k1, v1, n1, kv1_shared, o, k2=N
 
 def wd_set_debug_flags(flags: int):
     _lib.wd_set_debug_flags(flags)
+
+
+def wd_trace_enable(on: bool):
+    _lib.wd_trace_enable(1 if on else 0)
+
+
+def wd_trace_read():
+    """{class: (launches, total device ms)} since the previous read."""
+    n = (C.c_int64 * len(KERNEL_CLASSES))()
+    ms = (C.c_double * len(KERNEL_CLASSES))()
+    _ok(_lib.wd_trace_read(n, ms), "wd_trace_read")
+    return {k: (int(n[i]), float(ms[i])) for i, k in enumerate(KERNEL_CLASSES)}

@@ -222,6 +222,20 @@ wd_status wd_attention(int dtype, int batch, int Lq, int heads, int dh, const vo
                        int n1, int kv1_shared, const void* k2, const void* v2, int n2, int kv2_shared, void* o,
                        wd_stream stream);
 
+/* ------------------------------------------------------------------ tracing
+ * Every kernel launch is counted by class.  With timing enabled, each launch
+ * is also bracketed by two CUDA events recorded on its own stream, so the
+ * device time of each class can be read for any region of work. */
+typedef enum {
+  WD_KC_GEMM = 0, WD_KC_ATTN_SELF = 1, WD_KC_ATTN_CROSS = 2, WD_KC_NORM = 3, WD_KC_ROPE = 4,
+  WD_KC_EULER = 5, WD_KC_SMALL = 6, WD_KC_COUNT = 7
+} wd_kernel_class;
+void wd_trace_enable(int on);
+/* Waits for the recorded events, writes per-class launch counts and summed
+ * device milliseconds since the previous read (either array may be NULL;
+ * both have WD_KC_COUNT entries), then starts a new region. */
+wd_status wd_trace_read(int64_t* launches, double* total_ms);
+
 /* Debugging aid: bit 0 routes bf16 GEMMs, bit 1 bf16 attention, to the
  * CUDA-core kernels instead of the tensor-core ones.  Process-wide. */
 void wd_set_debug_flags(unsigned flags);

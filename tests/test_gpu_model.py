@@ -98,10 +98,7 @@ def test_tiny_fp32_rms_norm_variant(mods):
 
 
 # ------------------------------------------------------------------ small bf16: whole forward, ragged tiles
-SMALL_BF16 = synth.Workload("small-bf16-dh128-L105",
-                            synth.Dims(D=256, heads=2, ffn=512, blocks=2, T=3, H=10, W=14, n_txt=24, c_txt=64,
-                                       n_img=9, c_img=32, dtype="bf16"),
-                            batch=2, seed=1012, txt_valid=(5, 24))
+SMALL_BF16 = synth.SMALL_BF16
 
 
 def test_small_bf16_forward(mods):
