@@ -10,14 +10,16 @@
 //   warp 1           TMEM owner + MMA issuer: S_t = Q_t K_j^T into TMEM,
 //                    O_t (+)= P_t V_j with P_t read from TMEM (TS form), so
 //                    this product reads only V from shared memory
-//   warps 2..        one warpgroup (128 threads, thread = query row) per Q
-//                    tile: online softmax on S_t read from TMEM, P_t written
-//                    back as bf16 over the first half of S_t's columns, O_t
-//                    rescaled in TMEM only when the running max grows by more
-//                    than 8 (log2 units; the final 1/l keeps the result
-//                    exact), then the normalised output written out.
-// With NQ = 2 the two tiles ping-pong: while one warpgroup runs its softmax,
-// the tensor cores compute the other tile's P V and next S.
+//   warps 2..        8 softmax warps per Q tile: two per TMEM lane quarter
+//                    (32 query rows), each owning 64 of the 128 key columns.
+//                    Online softmax on S_t read from TMEM (the pair swaps its
+//                    row maxima through shared memory), P_t written back as
+//                    bf16 over the warp's own S columns, O_t rescaled in TMEM
+//                    only when the running max grows by more than 8 (log2
+//                    units; the final 1/l keeps the result exact), then the
+//                    normalised output written out.
+// With NQ = 2 the two tiles ping-pong: while one tile's warps run their
+// softmax, the tensor cores compute the other tile's P V and next S.
 #include "wd_internal.cuh"
 
 namespace wd {
@@ -27,18 +29,24 @@ constexpr int BQ = 128, BKV = 128, DH = 128;
 constexpr int TILE_BYTES = 128 * 128 * 2;   // one 128 x 128 bf16 tile (two 64-column halves)
 constexpr int HALF_BYTES = TILE_BYTES / 2;
 #ifndef WD_ATTN_RING
-#define WD_ATTN_RING 5   // K/V tiles in flight (32 KB each)
+#define WD_ATTN_RING 4   // K/V tiles in flight (32 KB each)
 #endif
 constexpr int RING = WD_ATTN_RING;
 constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
 
 template <int NQ, int NSEG>
 struct Cfg {
-  static constexpr int THREADS = 64 + 128 * NQ;
+  // 2 warps (loader, MMA) + per Q tile 8 softmax warps: two per TMEM lane
+  // quarter, each owning 64 of the 128 key columns of its 32 rows.
+  static constexpr int SM_WARPS = 8;
+  static constexpr int THREADS = 64 + 32 * SM_WARPS * NQ;
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = NQ * TILE_BYTES;
-  static constexpr int BAR_OFF = RING_OFF + RING * TILE_BYTES;
-  static constexpr int SMEM = 1024 + BAR_OFF + 256;
+  static constexpr int XCH_OFF = RING_OFF + RING * TILE_BYTES;     // row-max / row-sum exchange
+  static constexpr int XCH_BYTES = NQ * (2 * 2 * 128 + 2 * 2 * 128) * 4;
+  static constexpr int BAR_OFF = XCH_OFF + XCH_BYTES;
+  static constexpr int SMEM = 1024 + BAR_OFF + 512;
+  static_assert(SMEM <= 232448, "shared memory budget of one CTA exceeded (reduce WD_ATTN_RING)");
   static constexpr int TMEM_COLS = 512;
   // TMEM columns: S_t, O_t (per tile); with two segments one tile has O and O'
   __host__ __device__ static constexpr int s_col(int t) { return NSEG == 1 ? t * 256 : 0; }
@@ -48,7 +56,7 @@ struct Cfg {
 };
 
 enum : unsigned { SITE_Q = 0x201, SITE_KVF = 0x202, SITE_KVE = 0x203, SITE_S = 0x204, SITE_P = 0x205,
-                  SITE_O = 0x206, SITE_DRAIN = 0x207, SITE_TOK = 0x208 };
+                  SITE_O = 0x206, SITE_DRAIN = 0x207 };
 
 struct Seg {
   int n;        // keys
@@ -64,6 +72,15 @@ struct Params {
   int64_t o_rs;
   float scale_log2;
 };
+
+#ifndef WD_ATTN_MMA_SPIN
+#define WD_ATTN_MMA_SPIN 0   // MMA thread polls its barriers without suspending
+#endif
+#if WD_ATTN_MMA_SPIN
+#define MMA_WAIT mbar_wait_spin
+#else
+#define MMA_WAIT mbar_wait
+#endif
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -108,8 +125,11 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   uint64_t* p_full = s_full + NQ;          // NQ
   uint64_t* o_done = p_full + NQ;          // NQ
   uint64_t* tdone = o_done + NQ;           // 1
-  uint64_t* tok = tdone + 1;               // 2: exp-phase token between the two softmax warpgroups
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tok + 2);
+  uint64_t* mx_bar = tdone + 1;            // NQ x 4: the two warps of a lane quarter swap row maxima
+  uint64_t* fin_bar = mx_bar + 4 * NQ;     // NQ x 4: ... and their row sums at the end
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin_bar + 4 * NQ);
+  float* xmax = reinterpret_cast<float*>(smem + C::XCH_OFF);   // [2 parity][NQ][2 halves][128 rows]
+  float* xsum = xmax + 2 * NQ * 2 * 128;                        // [NQ][2 halves][2 (l, l_first)][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -123,10 +143,13 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < RING; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
-    for (int t = 0; t < NQ; ++t) { mbar_init(&s_full[t], 1); mbar_init(&p_full[t], 4); mbar_init(&o_done[t], 1); }
+    for (int t = 0; t < NQ; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], C::SM_WARPS);
+      mbar_init(&o_done[t], 1);
+    }
     mbar_init(tdone, 1);
-    mbar_init(&tok[0], 4);
-    mbar_init(&tok[1], 4);
+    for (int i = 0; i < 4 * NQ; ++i) { mbar_init(&mx_bar[i], 2); mbar_init(&fin_bar[i], 2); }
     fence_mbar_init();
   }
   if (warp == 1) { tmem_alloc(tmem_slot, C::TMEM_COLS); tmem_relinquish(); }
@@ -178,7 +201,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       const uint32_t r0 = smem_u32(smem + C::RING_OFF);
       // P_t V_j for block n-1 of tile t
       auto issue_pv = [&](int t, int n) -> bool {
-        if (!mbar_wait(&p_full[t], n & 1u, SITE_P)) return false;
+        if (!MMA_WAIT(&p_full[t], n & 1u, SITE_P)) return false;
         const int vseq = 2 * n + 1, vslot = vseq % RING;
         if (!mbar_wait(&kv_full[vslot], (vseq / RING) & 1u, SITE_KVF)) return false;
         tc_fence_after();
@@ -188,19 +211,24 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         const uint32_t pa = tmem + C::s_col(t), vb = r0 + vslot * TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk) {
-          // A = P: 16 keys = 8 TMEM columns of packed bf16 pairs
+          // A = P: 16 keys = 8 TMEM columns of packed bf16 pairs; keys 0-63 sit
+          // over S columns 0-31, keys 64-127 over S columns 64-95
           const uint64_t bd = sdesc_sw128(vb + kk * 2048, HALF_BYTES, 1024);
-          umma_ts(d, pa + kk * 8, bd, C::IDESC_O, (!first || kk) ? 1u : 0u);
+          umma_ts(d, pa + (kk >> 2) * 64 + (kk & 3) * 8, bd, C::IDESC_O, (!first || kk) ? 1u : 0u);
         }
         if (t == NQ - 1) umma_commit(&kv_empty[vslot]);
         return true;
       };
       for (int n = 0; n < NB && ok; ++n) {
         const int kseq = 2 * n, kslot = kseq % RING;
-        if (!mbar_wait(&kv_full[kslot], (kseq / RING) & 1u, SITE_KVF)) { ok = false; break; }
-        tc_fence_after();
         for (int t = 0; t < NQ && ok; ++t) {
+          // P_t V of the previous block first: it needs only P_t and that V tile,
+          // not the next K tile.
           if (n > 0 && !issue_pv(t, n - 1)) { ok = false; break; }
+          if (t == 0) {
+            if (!MMA_WAIT(&kv_full[kslot], (kseq / RING) & 1u, SITE_KVF)) { ok = false; break; }
+            tc_fence_after();
+          }
           const uint32_t d = tmem + C::s_col(t);
           const uint32_t qa = q0 + t * TILE_BYTES, kb = r0 + kslot * TILE_BYTES;
 #pragma unroll
@@ -221,12 +249,15 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax warpgroups
-    const int t = (warp - 2) >> 2;       // Q tile of this warpgroup
-    const int quarter = warp & 3;        // TMEM lanes this warp may access
-    const int r = quarter * 32 + lane;   // query row within the tile
+    // ------------------------------------------------------------ softmax warps
+    const int sw = warp - 2;
+    const int t = sw >> 3;                 // Q tile
+    const int hc = (sw >> 2) & 1;          // key half of this warp: columns [64 hc, 64 hc + 64)
+    const int quarter = warp & 3;          // TMEM lanes this warp may access
+    const int r = quarter * 32 + lane;     // query row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t s_addr = tmem + lane_base + C::s_col(t);
+    const uint32_t s_addr = tmem + lane_base + C::s_col(t) + hc * 64;
+    uint64_t* my_mx = &mx_bar[t * 4 + quarter];
     float m = -INFINITY, l = 0.f, l_first = 0.f;
     bool ok = true;
     for (int n = 0; n < NB; ++n) {
@@ -235,25 +266,34 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       if (NSEG == 2 && n == nb0) { l_first = l; m = -INFINITY; l = 0.f; }
       if (!mbar_wait_warp(&s_full[t], n & 1u, SITE_S)) { ok = false; break; }
       tc_fence_after();
-      const int valid = (sg ? nk1 : nk0) - (n - (sg ? nb0 : 0)) * BKV;   // keys of this block that exist
-      const bool ragged = valid < BKV;                                      // warp-uniform
-      // pass 1: row maximum of the raw scores, 64 columns in registers at a time
+      // keys of this block that exist, counted from this warp's first column
+      const int valid = (sg ? nk1 : nk0) - (n - (sg ? nb0 : 0)) * BKV - hc * 64;
+      const bool ragged = valid < 64;                                       // warp-uniform
+      // one read of this warp's 64 score columns; they stay in registers
+      uint32_t a[2][32];
+      tmem_ld32(s_addr, a[0]);
+      tmem_ld32(s_addr + 32, a[1]);
+      tmem_wait_ld();
+      if (ragged) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            if (c * 32 + k >= valid) a[c][k] = __float_as_uint(-INFINITY);
+      }
+      // row maximum over these 64 columns, then over both halves of the row
       float mx = -INFINITY;
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t a[32], c[32];
-        tmem_ld32(s_addr + hf * 64, a);
-        tmem_ld32(s_addr + hf * 64 + 32, c);
-        tmem_wait_ld();
-        if (ragged) {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            if (hf * 64 + k >= valid) a[k] = __float_as_uint(-INFINITY);
-            if (hf * 64 + 32 + k >= valid) c[k] = __float_as_uint(-INFINITY);
-          }
-        }
-#pragma unroll
-        for (int k = 0; k < 32; ++k) mx = fmax3(mx, __uint_as_float(a[k]), __uint_as_float(c[k]));
+      for (int k = 0; k < 32; k += 2)
+        mx = fmax3(mx, fmax3(__uint_as_float(a[0][k]), __uint_as_float(a[0][k + 1]), __uint_as_float(a[1][k])),
+                   __uint_as_float(a[1][k + 1]));
+      {
+        float* slot = xmax + ((n & 1) * NQ + t) * 256;
+        slot[hc * 128 + r] = mx;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(my_mx);
+        if (!mbar_wait_warp(my_mx, n & 1u, SITE_S)) { ok = false; break; }
+        mx = fmaxf(mx, slot[(1 - hc) * 128 + r]);
       }
       mx *= p.scale_log2;
       // lazy rescale: move the reference max only when it grew by more than the threshold
@@ -262,50 +302,35 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       const float alpha = grow ? ex2(m - m_new) : 1.f;
       m = m_new;
       const float neg_m = -m;
-      // The two warpgroups take turns with the exponentials (MUFU), so that one
-      // tile's softmax overlaps the other tile's MMAs instead of both sharing
-      // the unit at the same time.
-      if (NQ == 2 && !(t == 0 && n == 0)) {
-        if (!mbar_wait_warp(&tok[t], (t == 0 ? n - 1 : n) & 1u, SITE_TOK)) { ok = false; break; }
-      }
-      // pass 2: P = exp2(s * scale - m) as packed bf16 pairs into TMEM, over
-      // the first 64 columns of S_t (each half is written after it was read)
+      // P = exp2(s * scale - m) as packed bf16 pairs into TMEM over this warp's
+      // own S columns: chunk c of 16 keys -> 8 columns at 8c (masked keys hold
+      // -inf, so their exponential is 0)
       float2 rs2 = make_float2(0.f, 0.f);
       const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(neg_m, neg_m);
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t a[64];
-        tmem_ld32(s_addr + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
-        tmem_ld32(s_addr + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
-        tmem_wait_ld();
-        uint32_t pk[32];
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[8];
 #pragma unroll
-        for (int k = 0; k < 64; k += 2) {
-          const float2 arg = ffma2(make_float2(__uint_as_float(a[k]), __uint_as_float(a[k + 1])), sc2, nm2);
-          float e0 = ((k & 7) >= 8 - WD_EXP2_EMU_PER8) ? exp2_fma(arg.x) : ex2(arg.x);
-          float e1 = (((k + 1) & 7) >= 8 - WD_EXP2_EMU_PER8) ? exp2_fma(arg.y) : ex2(arg.y);
-          if (ragged) {
-            if (hf * 64 + k >= valid) e0 = 0.f;
-            if (hf * 64 + k + 1 >= valid) e1 = 0.f;
-          }
+        for (int k = 0; k < 16; k += 2) {
+          const int kk = (c & 1) * 16 + k;
+          const float2 arg = ffma2(make_float2(__uint_as_float(a[c >> 1][kk]), __uint_as_float(a[c >> 1][kk + 1])),
+                                   sc2, nm2);
+          const float e0 = ((k & 7) >= 8 - WD_EXP2_EMU_PER8) ? exp2_fma(arg.x) : ex2(arg.x);
+          const float e1 = (((k + 1) & 7) >= 8 - WD_EXP2_EMU_PER8) ? exp2_fma(arg.y) : ex2(arg.y);
           rs2 = fadd2(rs2, make_float2(e0, e1));
           pk[k >> 1] = pack_bf16x2(e0, e1);
         }
-        tmem_st32(s_addr + hf * 32, pk);
+        tmem_st8(s_addr + c * 8, pk);
       }
       tmem_wait_st();
-      if (NQ == 2) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tok[1 - t]);
-      }
-      const float rs = rs2.x + rs2.y;
-      l = l * alpha + rs;
-      // O_t *= alpha for the rows whose reference max moved (P V of the previous
-      // block has completed: its commit precedes the S commit waited on above)
+      l = l * alpha + (rs2.x + rs2.y);     // this warp's share of the row sum
+      // O_t *= alpha on this warp's 64 output columns for rows whose reference
+      // max moved (P V of the previous block has completed: its commit precedes
+      // the S commit waited on above)
       if (__any_sync(0xffffffffu, grow) && !first) {
-        const uint32_t o_addr = tmem + lane_base + C::o_col(t, sg);
+        const uint32_t o_addr = tmem + lane_base + C::o_col(t, sg) + hc * 64;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t o[32];
           tmem_ld32(o_addr + c * 32, o);
           tmem_wait_ld();
@@ -320,23 +345,36 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       if (lane == 0) mbar_arrive(&p_full[t]);
     }
     // ---------------------------------------------------------- epilogue
+    if (ok) {
+      // combine the two halves' row sums
+      float* xs = xsum + t * 512;
+      xs[hc * 256 + r] = l;
+      xs[hc * 256 + 128 + r] = l_first;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&fin_bar[t * 4 + quarter]);
+      ok = mbar_wait_warp(&fin_bar[t * 4 + quarter], 0, SITE_O);
+      if (ok) {
+        l += xs[(1 - hc) * 256 + r];
+        l_first += xs[(1 - hc) * 256 + 128 + r];
+      }
+    }
     if (ok && mbar_wait_warp(&o_done[t], 0, SITE_O)) {
       tc_fence_after();
       const int row = l0 + t * BQ + r;
       const float inv1 = 1.f / l;
       const float inv0 = NSEG == 2 ? 1.f / l_first : 0.f;
-      bf16* dst = p.o + (static_cast<int64_t>(b) * p.Lq + row) * p.o_rs + h * DH;
+      bf16* dst = p.o + (static_cast<int64_t>(b) * p.Lq + row) * p.o_rs + h * DH + hc * 64;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_base + C::o_col(t, NSEG - 1) + c * 32, o);
+        tmem_ld32(tmem + lane_base + C::o_col(t, NSEG - 1) + hc * 64 + c * 32, o);
         tmem_wait_ld();
         float v[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(o[k]) * inv1;
         if (NSEG == 2) {
           uint32_t o2[32];
-          tmem_ld32(tmem + lane_base + C::o_col(t, 0) + c * 32, o2);
+          tmem_ld32(tmem + lane_base + C::o_col(t, 0) + hc * 64 + c * 32, o2);
           tmem_wait_ld();
 #pragma unroll
           for (int k = 0; k < 32; ++k) v[k] += __uint_as_float(o2[k]) * inv0;
