@@ -73,13 +73,15 @@ struct Params {
   float scale_log2;
 };
 
-#ifndef WD_ATTN_MMA_SPIN
-#define WD_ATTN_MMA_SPIN 0   // MMA thread polls its barriers without suspending
+#ifndef WD_ATTN_POLL_NS
+#define WD_ATTN_POLL_NS 0    // > 0: the MMA thread and the softmax warps poll their barriers with this sleep
 #endif
-#if WD_ATTN_MMA_SPIN
-#define MMA_WAIT mbar_wait_spin
+#if WD_ATTN_POLL_NS > 0
+#define MMA_WAIT(bar, par, site) mbar_wait_poll(bar, par, site, WD_ATTN_POLL_NS)
+#define SM_WAIT(bar, par, site) __all_sync(0xffffffffu, mbar_wait_poll(bar, par, site, WD_ATTN_POLL_NS))
 #else
-#define MMA_WAIT mbar_wait
+#define MMA_WAIT(bar, par, site) mbar_wait(bar, par, site)
+#define SM_WAIT(bar, par, site) mbar_wait_warp(bar, par, site)
 #endif
 
 __device__ __forceinline__ float ex2(float x) {
@@ -95,18 +97,18 @@ __device__ __forceinline__ float ex2(float x) {
 // 2^f on [-1/2, 1/2] is a degree-3 polynomial whose coefficients were fitted
 // for this library (iteratively reweighted least squares on the relative
 // error, max relative error 7.5e-5 in fp32, far below a bf16 half-ulp); the
-// factor 2^j is added to the exponent field.  Arguments below -127 give 0.
+// factor 2^j is added to the exponent field.  Arguments below -125 give 2^-125 (~0).
 __device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -127.f);
+  x = fmaxf(x, -125.f);   // keeps q * 2^round(x) a normal float (q >= 0.7)
   const float t = x + 12582912.f;
-  const int j = __float_as_int(t) - 0x4B400000;
   const float f = x - (t - 12582912.f);
   const float q = fmaf(fmaf(fmaf(0.0551716648f, f, 0.2426111251f), f, 0.6932609677f), f, 0.9999280572f);
-  return __int_as_float(__float_as_int(q) + (j << 23));
+  // round(x) sits in the low bits of t's encoding; 0x4B400000 << 23 is 0 mod 2^32
+  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
 }
 
 #ifndef WD_EXP2_EMU_PER8
-#define WD_EXP2_EMU_PER8 0   // of every 8 exponentials, this many run on the FMA pipe
+#define WD_EXP2_EMU_PER8 1   // of every 8 exponentials, this many run on the FMA pipe
 #endif
 
 template <int NQ, int NSEG>
@@ -264,7 +266,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       const int sg = n < nb0 ? 0 : 1;
       const bool first = (n == 0) || (n == nb0);
       if (NSEG == 2 && n == nb0) { l_first = l; m = -INFINITY; l = 0.f; }
-      if (!mbar_wait_warp(&s_full[t], n & 1u, SITE_S)) { ok = false; break; }
+      if (!SM_WAIT(&s_full[t], n & 1u, SITE_S)) { ok = false; break; }
       tc_fence_after();
       // keys of this block that exist, counted from this warp's first column
       const int valid = (sg ? nk1 : nk0) - (n - (sg ? nb0 : 0)) * BKV - hc * 64;
@@ -292,7 +294,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         slot[hc * 128 + r] = mx;
         __syncwarp();
         if (lane == 0) mbar_arrive(my_mx);
-        if (!mbar_wait_warp(my_mx, n & 1u, SITE_S)) { ok = false; break; }
+        if (!SM_WAIT(my_mx, n & 1u, SITE_S)) { ok = false; break; }
         mx = fmaxf(mx, slot[(1 - hc) * 128 + r]);
       }
       mx *= p.scale_log2;
