@@ -6,3 +6,4 @@
 #include "k_gemm_tc.cu"
 #include "k_attn_tc.cu"
 #include "wd_api.cu"
+#include "wd_noalloc.cu"

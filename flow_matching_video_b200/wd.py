@@ -64,6 +64,7 @@ SIGNATURES = {
     "wd_cross_kv": (_I, [_PD, C.POINTER(wd_block_weights), _P, _I, _P, _P]),
     "wd_time_mod": (_I, [_PD, C.POINTER(wd_time_weights), _F, _P, _P, _P]),
     "wd_patch_embed": (_I, [_PD, _P, _P, _P, _P, _I, _P, _P, _S, _P]),
+    "wd_patch_embed_noalloc": (_I, [_PD, _P, _P, _P, _P, _I, _P, _P]),
     "wd_block_forward": (_I, [_PD, C.POINTER(wd_block_weights), _P, _P, _I, _P, _P, _S, _P]),
     "wd_unpatchify": (_I, [_PD, C.POINTER(wd_head_weights), _P, _I, _P, _P, _P, _S, _P]),
     "wd_euler_cfg_step": (_I, [_P, _P, _P, _F, _F, _S, _P]),
@@ -161,6 +162,13 @@ def wd_time_mod(dims, w: wd_time_weights, tau: float, e, e0, stream=None):
 def wd_patch_embed(dims, x_t, y, w, b, batch, X, ws, stream=None):
     _ok(_lib.wd_patch_embed(C.byref(dims), _p(x_t), _p(y), _p(w), _p(b), batch, _p(X), _p(ws), ws.numel() * ws.element_size(),
                             _stream(stream)), "wd_patch_embed")
+
+
+def wd_patch_embed_noalloc(dims, x_t, y, w, b, batch, X, stream=None):
+    """wd_patch_embed without a workspace: the library's fixed scratch array
+    is used instead (for callers that cannot allocate device memory)."""
+    _ok(_lib.wd_patch_embed_noalloc(C.byref(dims), _p(x_t), _p(y), _p(w), _p(b), batch, _p(X), _stream(stream)),
+        "wd_patch_embed_noalloc")
 
 
 def wd_block_forward(dims, w: wd_block_weights, e0, kv, batch, X, ws, stream=None):

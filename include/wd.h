@@ -199,6 +199,32 @@ wd_status wd_unpatchify(const wd_dims* d, const wd_head_weights* w, const float*
 wd_status wd_euler_cfg_step(float* x, const float* v_cond, const float* v_uncond, float cfg_scale,
                             float dt, size_t n, wd_stream stream);
 
+/* ------------------------------------------------------------------ no-allocation variant
+ * No counterpart in the source pages: an integration aid.  Some callers
+ * cannot hand the library a workspace: code running inside a host framework
+ * that owns the whole device memory pool and gives plug-ins no scratch, or a
+ * latency-critical loop that must not call cudaMalloc (it can synchronise the
+ * device and stall the other streams).  For them, wd_patch_embed_noalloc does
+ * the work of wd_patch_embed with its patch-gather scratch in a fixed array of
+ * this library, WD_NOALLOC_PATCH_SCRATCH_BYTES large, which every GPU that
+ * loads the library reserves until the process exits.
+ * - Same arguments and results as wd_patch_embed, minus the workspace.
+ * - Sizes beyond the array (batch * L * 144 * element size bytes, i.e. more
+ *   than 174762 token rows in bf16 or 87381 in fp32) return WD_ERR_WORKSPACE
+ *   before any launch.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before capturing the stream into a graph.
+ * - It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * - Every call shares the one array, which keeps the last call's contents
+ *   (each call overwrites all of the part it uses, so nothing needs
+ *   clearing); calls that overlap on the GPU — on different streams, or
+ *   from different threads — race on it and must be serialised by the
+ *   caller. */
+#define WD_NOALLOC_PATCH_SCRATCH_BYTES (48u << 20)
+wd_status wd_patch_embed_noalloc(const wd_dims* d, const float* x_t, const float* y, const void* w,
+                                 const float* b, int batch, float* X, wd_stream stream);
+
 /* ------------------------------------------------------------------ building blocks
  * The kernels of the path, exposed one by one so that each can be checked on
  * its own.  Same conventions as above. */
