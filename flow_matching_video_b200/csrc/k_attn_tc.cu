@@ -34,11 +34,18 @@ constexpr int HALF_BYTES = TILE_BYTES / 2;
 constexpr int RING = WD_ATTN_RING;
 constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
 
+#ifndef WD_ATTN_SPLIT
+#define WD_ATTN_SPLIT 1   // softmax warps per TMEM lane quarter (1 or 2), each owning 128/SPLIT key columns
+#endif
+constexpr int SPLIT = WD_ATTN_SPLIT;
+static_assert(SPLIT == 1 || SPLIT == 2, "WD_ATTN_SPLIT must be 1 or 2");
+
 template <int NQ, int NSEG>
 struct Cfg {
-  // 2 warps (loader, MMA) + per Q tile 8 softmax warps: two per TMEM lane
-  // quarter, each owning 64 of the 128 key columns of its 32 rows.
-  static constexpr int SM_WARPS = 8;
+  // 2 warps (loader, MMA) + per Q tile 4*SPLIT softmax warps: SPLIT per TMEM
+  // lane quarter (32 query rows), each owning 128/SPLIT of the key columns.
+  static constexpr int SM_WARPS = 4 * SPLIT;
+  static constexpr int COLS = BKV / SPLIT;
   static constexpr int THREADS = 64 + 32 * SM_WARPS * NQ;
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = NQ * TILE_BYTES;
@@ -76,9 +83,15 @@ struct Params {
 #ifndef WD_ATTN_POLL_NS
 #define WD_ATTN_POLL_NS 0    // > 0: the MMA thread and the softmax warps poll their barriers with this sleep
 #endif
+#ifndef WD_ATTN_WAIT_HINT_NS
+#define WD_ATTN_WAIT_HINT_NS 0   // > 0: suspend-time hint for the MMA thread's and softmax warps' try_wait
+#endif
 #if WD_ATTN_POLL_NS > 0
 #define MMA_WAIT(bar, par, site) mbar_wait_poll(bar, par, site, WD_ATTN_POLL_NS)
 #define SM_WAIT(bar, par, site) __all_sync(0xffffffffu, mbar_wait_poll(bar, par, site, WD_ATTN_POLL_NS))
+#elif WD_ATTN_WAIT_HINT_NS > 0
+#define MMA_WAIT(bar, par, site) mbar_wait_hint(bar, par, site, WD_ATTN_WAIT_HINT_NS)
+#define SM_WAIT(bar, par, site) __all_sync(0xffffffffu, mbar_wait_hint(bar, par, site, WD_ATTN_WAIT_HINT_NS))
 #else
 #define MMA_WAIT(bar, par, site) mbar_wait(bar, par, site)
 #define SM_WAIT(bar, par, site) mbar_wait_warp(bar, par, site)
@@ -124,8 +137,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   uint64_t* kv_full = bars + 1;            // RING
   uint64_t* kv_empty = kv_full + RING;     // RING
   uint64_t* s_full = kv_empty + RING;      // NQ
-  uint64_t* p_full = s_full + NQ;          // NQ
-  uint64_t* o_done = p_full + NQ;          // NQ
+  uint64_t* p_full = s_full + NQ;          // NQ: all of P_t written
+  uint64_t* p_half = p_full + NQ;          // NQ: keys 0-63 of P_t written
+  uint64_t* o_done = p_half + NQ;          // NQ
   uint64_t* tdone = o_done + NQ;           // 1
   uint64_t* mx_bar = tdone + 1;            // NQ x 4: the two warps of a lane quarter swap row maxima
   uint64_t* fin_bar = mx_bar + 4 * NQ;     // NQ x 4: ... and their row sums at the end
@@ -148,6 +162,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     for (int t = 0; t < NQ; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], C::SM_WARPS);
+      mbar_init(&p_half[t], C::SM_WARPS);
       mbar_init(&o_done[t], 1);
     }
     mbar_init(tdone, 1);
@@ -203,20 +218,31 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       const uint32_t r0 = smem_u32(smem + C::RING_OFF);
       // P_t V_j for block n-1 of tile t
       auto issue_pv = [&](int t, int n) -> bool {
-        if (!MMA_WAIT(&p_full[t], n & 1u, SITE_P)) return false;
         const int vseq = 2 * n + 1, vslot = vseq % RING;
-        if (!mbar_wait(&kv_full[vslot], (vseq / RING) & 1u, SITE_KVF)) return false;
-        tc_fence_after();
         const int sg = n < nb0 ? 0 : 1;
         const int first = (n == 0) || (n == nb0);
         const uint32_t d = tmem + C::o_col(t, sg);
         const uint32_t pa = tmem + C::s_col(t), vb = r0 + vslot * TILE_BYTES;
+        // With one softmax warp per lane quarter, P arrives in two halves (keys
+        // 0-63, then 64-127): the first four k-steps start as soon as the first
+        // half is in TMEM.
 #pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk) {
-          // A = P: 16 keys = 8 TMEM columns of packed bf16 pairs; keys 0-63 sit
-          // over S columns 0-31, keys 64-127 over S columns 64-95
-          const uint64_t bd = sdesc_sw128(vb + kk * 2048, HALF_BYTES, 1024);
-          umma_ts(d, pa + (kk >> 2) * 64 + (kk & 3) * 8, bd, C::IDESC_O, (!first || kk) ? 1u : 0u);
+        for (int half = 0; half < 2; ++half) {
+          if (SPLIT == 1 || half == 0) {
+            uint64_t* bar = (SPLIT == 1 && half == 0) ? &p_half[t] : &p_full[t];
+            if (!MMA_WAIT(bar, n & 1u, SITE_P)) return false;
+          }
+          if (half == 0 && !MMA_WAIT(&kv_full[vslot], (vseq / RING) & 1u, SITE_KVF)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = half * 4; kk < half * 4 + 4; ++kk) {
+            // A = P: 16 keys = 8 TMEM columns of packed bf16 pairs; each softmax
+            // warp's keys sit over the first half of its own S columns:
+            // key 16 kk lives at column (16kk / COLS) * COLS + (16kk % COLS) / 2
+            const uint64_t bd = sdesc_sw128(vb + kk * 2048, HALF_BYTES, 1024);
+            umma_ts(d, pa + (16 * kk / C::COLS) * C::COLS + (16 * kk % C::COLS) / 2, bd, C::IDESC_O,
+                    (!first || kk) ? 1u : 0u);
+          }
         }
         if (t == NQ - 1) umma_commit(&kv_empty[vslot]);
         return true;
@@ -252,14 +278,15 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax warps
+    constexpr int COLS = C::COLS, CH = COLS / 32;
     const int sw = warp - 2;
-    const int t = sw >> 3;                 // Q tile
-    const int hc = (sw >> 2) & 1;          // key half of this warp: columns [64 hc, 64 hc + 64)
+    const int t = sw / C::SM_WARPS;        // Q tile
+    const int hc = SPLIT == 2 ? (sw >> 2) & 1 : 0;   // key part of this warp: columns [COLS hc, COLS hc + COLS)
     const int quarter = warp & 3;          // TMEM lanes this warp may access
     const int r = quarter * 32 + lane;     // query row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t s_addr = tmem + lane_base + C::s_col(t) + hc * 64;
-    uint64_t* my_mx = &mx_bar[t * 4 + quarter];
+    const uint32_t s_addr = tmem + lane_base + C::s_col(t) + hc * COLS;
+    [[maybe_unused]] uint64_t* my_mx = &mx_bar[t * 4 + quarter];
     float m = -INFINITY, l = 0.f, l_first = 0.f;
     bool ok = true;
     for (int n = 0; n < NB; ++n) {
@@ -269,27 +296,28 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       if (!SM_WAIT(&s_full[t], n & 1u, SITE_S)) { ok = false; break; }
       tc_fence_after();
       // keys of this block that exist, counted from this warp's first column
-      const int valid = (sg ? nk1 : nk0) - (n - (sg ? nb0 : 0)) * BKV - hc * 64;
-      const bool ragged = valid < 64;                                       // warp-uniform
-      // one read of this warp's 64 score columns; they stay in registers
-      uint32_t a[2][32];
-      tmem_ld32(s_addr, a[0]);
-      tmem_ld32(s_addr + 32, a[1]);
+      const int valid = (sg ? nk1 : nk0) - (n - (sg ? nb0 : 0)) * BKV - hc * COLS;
+      const bool ragged = valid < COLS;                                     // warp-uniform
+      // one read of this warp's score columns; they stay in registers
+      uint32_t a[CH][32];
+#pragma unroll
+      for (int c = 0; c < CH; ++c) tmem_ld32(s_addr + c * 32, a[c]);
       tmem_wait_ld();
       if (ragged) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
+        for (int c = 0; c < CH; ++c)
 #pragma unroll
           for (int k = 0; k < 32; ++k)
             if (c * 32 + k >= valid) a[c][k] = __float_as_uint(-INFINITY);
       }
-      // row maximum over these 64 columns, then over both halves of the row
       float mx = -INFINITY;
 #pragma unroll
-      for (int k = 0; k < 32; k += 2)
-        mx = fmax3(mx, fmax3(__uint_as_float(a[0][k]), __uint_as_float(a[0][k + 1]), __uint_as_float(a[1][k])),
-                   __uint_as_float(a[1][k + 1]));
-      {
+      for (int c = 0; c < CH; c += 2)
+#pragma unroll
+        for (int k = 0; k < 32; k += 2)
+          mx = fmax3(mx, fmax3(__uint_as_float(a[c][k]), __uint_as_float(a[c][k + 1]), __uint_as_float(a[c + 1][k])),
+                     __uint_as_float(a[c + 1][k + 1]));
+      if constexpr (SPLIT == 2) {   // the two warps of a lane quarter swap their row maxima
         float* slot = xmax + ((n & 1) * NQ + t) * 256;
         slot[hc * 128 + r] = mx;
         __syncwarp();
@@ -304,13 +332,29 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       const float alpha = grow ? ex2(m - m_new) : 1.f;
       m = m_new;
       const float neg_m = -m;
+      // O_t *= alpha on this warp's output columns for rows whose reference
+      // max moved, before any of this block's P V can start (P V of the previous
+      // block has completed: its commit precedes the S commit waited on above)
+      if (__any_sync(0xffffffffu, grow) && !first) {
+        const uint32_t o_addr = tmem + lane_base + C::o_col(t, sg) + hc * COLS;
+#pragma unroll 1
+        for (int c = 0; c < CH; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_addr + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_st32(o_addr + c * 32, o);
+        }
+        tmem_wait_st();
+      }
       // P = exp2(s * scale - m) as packed bf16 pairs into TMEM over this warp's
       // own S columns: chunk c of 16 keys -> 8 columns at 8c (masked keys hold
       // -inf, so their exponential is 0)
       float2 rs2 = make_float2(0.f, 0.f);
       const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(neg_m, neg_m);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2 * CH; ++c) {
         uint32_t pk[8];
 #pragma unroll
         for (int k = 0; k < 16; k += 2) {
@@ -323,32 +367,22 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           pk[k >> 1] = pack_bf16x2(e0, e1);
         }
         tmem_st8(s_addr + c * 8, pk);
+        if (SPLIT == 1 && c == CH - 1) {   // keys 0-63 of P are written: release the first half of P V
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_half[t]);
+        }
       }
       tmem_wait_st();
       l = l * alpha + (rs2.x + rs2.y);     // this warp's share of the row sum
-      // O_t *= alpha on this warp's 64 output columns for rows whose reference
-      // max moved (P V of the previous block has completed: its commit precedes
-      // the S commit waited on above)
-      if (__any_sync(0xffffffffu, grow) && !first) {
-        const uint32_t o_addr = tmem + lane_base + C::o_col(t, sg) + hc * 64;
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          uint32_t o[32];
-          tmem_ld32(o_addr + c * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st32(o_addr + c * 32, o);
-        }
-        tmem_wait_st();
-      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[t]);
     }
     // ---------------------------------------------------------- epilogue
-    if (ok) {
-      // combine the two halves' row sums
+    if (SPLIT == 2 && ok) {
+      // combine the two parts' row sums
       float* xs = xsum + t * 512;
       xs[hc * 256 + r] = l;
       xs[hc * 256 + 128 + r] = l_first;
@@ -365,18 +399,18 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       const int row = l0 + t * BQ + r;
       const float inv1 = 1.f / l;
       const float inv0 = NSEG == 2 ? 1.f / l_first : 0.f;
-      bf16* dst = p.o + (static_cast<int64_t>(b) * p.Lq + row) * p.o_rs + h * DH + hc * 64;
+      bf16* dst = p.o + (static_cast<int64_t>(b) * p.Lq + row) * p.o_rs + h * DH + hc * COLS;
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < CH; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_base + C::o_col(t, NSEG - 1) + hc * 64 + c * 32, o);
+        tmem_ld32(tmem + lane_base + C::o_col(t, NSEG - 1) + hc * COLS + c * 32, o);
         tmem_wait_ld();
         float v[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(o[k]) * inv1;
         if (NSEG == 2) {
           uint32_t o2[32];
-          tmem_ld32(tmem + lane_base + C::o_col(t, 0) + hc * 64 + c * 32, o2);
+          tmem_ld32(tmem + lane_base + C::o_col(t, 0) + hc * COLS + c * 32, o2);
           tmem_wait_ld();
 #pragma unroll
           for (int k = 0; k < 32; ++k) v[k] += __uint_as_float(o2[k]) * inv0;

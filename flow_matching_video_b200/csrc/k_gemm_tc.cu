@@ -26,6 +26,12 @@ constexpr int BM = 128, BK = 64;
 #define WD_GEMM_EPI_WG 1   // epilogue warpgroups; each takes an equal share of the tile's columns
 #endif
 constexpr int EPI_WG = WD_GEMM_EPI_WG;
+#ifndef WD_GEMM_RESID_PIPE
+#define WD_GEMM_RESID_PIPE 0   // residual epilogue loads one chunk ahead
+#endif
+#ifndef WD_GEMM_RESID_PREFETCH
+#define WD_GEMM_RESID_PREFETCH 0   // producer prefetches each tile's fp32 residual block into L2
+#endif
 constexpr int THREADS = 64 + 128 * EPI_WG;
 
 template <int BN>
@@ -100,8 +106,8 @@ __device__ __forceinline__ void epilogue32(const Epi& ep, int64_t m, int n, cons
 // ------------------------------------------------------------------ kernel
 template <int BN, int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
-k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Epi ep, int M,
-          int N, int K) {
+k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+          const __grid_constant__ CUtensorMap tmX, const Epi ep, int M, int N, int K) {
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -143,6 +149,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       bool ok = true;
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
         const int m0 = (t / n_tiles) * BM, n0 = (t % n_tiles) * BN;
+        // the epilogue of this tile reads and rewrites X[m0:m0+128, n0:n0+BN]
+        // one mainloop from now: have it in L2 by then
+        if (MODE == EPI_RESID && WD_GEMM_RESID_PREFETCH) tma_prefetch_l2_2d(&tmX, n0, m0);
         for (int k = 0; k < k_iters; ++k) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, SITE_EMPTY)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
@@ -203,20 +212,41 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       tc_fence_after();
       const int64_t m = m0 + q * 32 + lane;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
-#pragma unroll 1
-      for (int c = c_begin; c < c_begin + COLS; c += 32) {
-        float4 xres[8];
-        if constexpr (MODE == EPI_RESID) {   // residual loads in flight while TMEM is read
-          if (m < M) {
-            const float4* src = reinterpret_cast<const float4*>(static_cast<float*>(ep.out) + m * ep.ldo + n0 + c);
+      if constexpr (MODE == EPI_RESID && WD_GEMM_RESID_PIPE) {
+        // residual loads run one 32-column chunk ahead of the TMEM reads
+        const float4* row_x = reinterpret_cast<const float4*>(static_cast<float*>(ep.out) + m * ep.ldo + n0);
+        float4 xres[2][8];
+        if (m < M) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) xres[j] = src[j];
-          }
+          for (int j = 0; j < 8; ++j) xres[0][j] = row_x[c_begin / 4 + j];
         }
-        uint32_t r[32];
-        tmem_ld32(tbase + c, r);
-        tmem_wait_ld();
-        if (m < M) epilogue32<MODE>(ep, m, n0 + c, r, xres);
+#pragma unroll
+        for (int c = c_begin, i = 0; c < c_begin + COLS; c += 32, ++i) {
+          if (c + 32 < c_begin + COLS && m < M) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) xres[(i + 1) & 1][j] = row_x[(c + 32) / 4 + j];
+          }
+          uint32_t r[32];
+          tmem_ld32(tbase + c, r);
+          tmem_wait_ld();
+          if (m < M) epilogue32<MODE>(ep, m, n0 + c, r, xres[i & 1]);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = c_begin; c < c_begin + COLS; c += 32) {
+          float4 xres[8];
+          if constexpr (MODE == EPI_RESID) {   // residual loads in flight while TMEM is read
+            if (m < M) {
+              const float4* src = reinterpret_cast<const float4*>(static_cast<float*>(ep.out) + m * ep.ldo + n0 + c);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) xres[j] = src[j];
+            }
+          }
+          uint32_t r[32];
+          tmem_ld32(tbase + c, r);
+          tmem_wait_ld();
+          if (m < M) epilogue32<MODE>(ep, m, n0 + c, r, xres);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -271,6 +301,23 @@ static int sm_count() {
   return cnt[dev & 15];
 }
 
+// 2D fp32 tensor map over the residual stream [rows, cols], box BN x 128, no swizzle
+// (used only for L2 prefetches).
+static wd_status make_tmap_f32(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_cols,
+                               int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) { set_error("cuTensorMapEncodeTiled unavailable"); return WD_ERR_CUDA; }
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 4};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) { set_error("cuTensorMapEncodeTiled (f32) failed (%d)", static_cast<int>(r)); return WD_ERR_CUDA; }
+  return WD_OK;
+}
+
 template <int BN, int MODE>
 static wd_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const Epi& ep, int M, int N, int K,
                            cudaStream_t st) {
@@ -284,8 +331,10 @@ static wd_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const E
   }
   const int tiles = ((M + tcg::BM - 1) / tcg::BM) * (N / BN);
   const int grid = tiles < sm_count() ? tiles : sm_count();
+  CUtensorMap tx = ta;   // unused unless the epilogue adds into the fp32 residual
+  if (MODE == EPI_RESID) WD_TRY(make_tmap_f32(&tx, ep.out, M, N, ep.ldo, BN, tcg::BM));
   Trace tr(KC_GEMM, st);
-  tcg::k_gemm_tc<BN, MODE><<<grid, tcg::THREADS, C::SMEM, st>>>(ta, tb, ep, M, N, K);
+  tcg::k_gemm_tc<BN, MODE><<<grid, tcg::THREADS, C::SMEM, st>>>(ta, tb, tx, ep, M, N, K);
   return launch_status("gemm_tc");
 }
 
