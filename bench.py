@@ -157,6 +157,23 @@ def blas_threads():
         return os.cpu_count()
 
 
+# ---------------------------------------------------------------------- multi-rank reduction
+def reduce_over_ranks(ms_local: float, tokens_local: float, world: int, device=None):
+    """Step time = max over ranks; throughput = all ranks' tokens / that time.
+    Every rank takes the same collective calls (one all_reduce MAX, one SUM)."""
+    import torch
+    ms, tokens = ms_local, tokens_local
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms_local], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        n = torch.tensor([tokens_local], dtype=torch.float64, device=device)
+        dist.all_reduce(n, op=dist.ReduceOp.SUM)
+        tokens = float(n.item())
+    return ms, tokens / (ms / 1e3)
+
+
 # ---------------------------------------------------------------------- reference arm
 def run_reference(args, rank):
     if rank != 0:
@@ -270,11 +287,8 @@ def run_ours(args, rank, world, local_rank):
     wd.wd_trace_enable(False)
     tr = wd.wd_trace_read()
     wd.wd_check()
-    ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    tokens_step = B * d.L * d.blocks
+    ms, value = reduce_over_ranks(e0.elapsed_time(e1) / args.steps, tokens_step, world, dev)
 
     # ------------------------------------------------ end to end through the API, host buffers
     torch.cuda.synchronize()
@@ -289,19 +303,13 @@ def run_ours(args, rank, world, local_rank):
     h1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms_e2e = h0.elapsed_time(h1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e, value_e2e = reduce_over_ranks(h0.elapsed_time(h1) / args.steps, tokens_step, world, dev)
     if not np.all(np.isfinite(out_host.numpy())):
         raise RuntimeError("non-finite latent after the timed steps")
 
     if rank != 0:
         return 0
     pk = peaks()
-    tokens_step = B * d.L * d.blocks
-    value = world * tokens_step / (ms / 1e3)
     flops = step_flops(d, B)
     tflops = flops / (ms / 1e3) / 1e12
     # roofline of the dominant kernel (self-attention), timed live with events
@@ -329,7 +337,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "no flush: per-step working set (3.1 GB weights, 0.4 GB residual stream) exceeds L2"},
         "tflops": tflops, "pct_bf16_peak": tflops / pk["bf16_tflops"],
         "pct_bf16_peak_sustained": tflops / peak_s, "s_per_step": ms / 1e3,
-        "e2e": {"value": world * tokens_step / (ms_e2e / 1e3), "unit": "tokens/s",
+        "e2e": {"value": value_e2e, "unit": "tokens/s",
                 "h2d_bytes_per_step": x_host.numel() * 4, "d2h_bytes_per_step": out_host.numel() * 4},
         "gpu_launches": launches,
         "roofline": {"bound": "tensor", "kernel": "attention_tc self (k_attn_tc<2,1>)",

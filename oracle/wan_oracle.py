@@ -314,9 +314,12 @@ def block_forward(X, e0, w: dict, blk: int, kv: dict, dims, rnd: bool = False, r
         x = X[b]
         # ---- self-attention (keys and values need every token)
         h = _st(adaln_modulate(x, shift1, scale1, eps, dims.norm), rnd)
-        qkv = _st(linear(h, w[p + "qkv.w"], w[p + "qkv.b"]), rnd)
-        q, k, v = qkv[:, :D], qkv[:, D:2 * D], qkv[:, 2 * D:]
-        q = rms_norm(q[rows], eps, w[p + "gq"]).reshape(len(rows), nh, dh)
+        wqkv, bqkv = w[p + "qkv.w"], w[p + "qkv.b"]
+        # the fused projection's rows (q; k; v); q is needed only for the requested rows
+        q = _st(linear(h[rows], wqkv[:D], bqkv[:D]), rnd)
+        k = _st(linear(h, wqkv[D:2 * D], bqkv[D:2 * D]), rnd)
+        v = _st(linear(h, wqkv[2 * D:], bqkv[2 * D:]), rnd)
+        q = rms_norm(q, eps, w[p + "gq"]).reshape(len(rows), nh, dh)
         k = rms_norm(k, eps, w[p + "gk"]).reshape(L, nh, dh)
         q = _st(rope_3d(q, pf[rows], py[rows], px[rows]), rnd)
         k = _st(rope_3d(k, pf, py, px), rnd)

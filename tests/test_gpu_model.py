@@ -147,6 +147,30 @@ def test_block_bf16_480p81_batch2(mods):
     _block_parity(mods, synth.STACK_480P81, 192, 1000.0)
 
 
+def test_block_bf16_720p81_wide_batch2(mods):
+    # D=5120, 40 heads x 128, FFN 13824, L=75600 (ragged last tile: 75600 = 590*128 + 80)
+    _block_parity(mods, synth.WIDE_720P81, 96, 500.0)
+
+
+def test_sampler_12_steps_full_model_short_grid(mods):
+    """The 12-step CFG loop with the full 30-block D=1536 model on a small
+    latent grid (L = 2*4*4 = 32), every element of the final latent."""
+    model, wd = mods
+    base = synth.SAMPLE_480P81
+    d = synth.Dims(**{**base.dims.__dict__, "T": 2, "H": 8, "W": 8})
+    wl = synth.Workload("short-grid-12step", d, batch=2, seed=base.seed, steps=base.steps,
+                        cfg_scale=base.cfg_scale)
+    net, w, x, txt, y, d = setup(mods, wl)
+    xb = dev(np.stack([x["x0"], x["x0"]]))
+    for t, dt, tau in O.schedule(wl.steps):
+        net.cfg_euler_step(xb, y, tau, dt, wl.cfg_scale)
+    wd.wd_check()
+    want_x, _ = O.sample(x["x0"], x["img_lat"], w, x["txt"], x["clip"], d, wl.steps, wl.cfg_scale, rnd=True)
+    assert rel(host(xb[0]), want_x) < TOL_BF16
+    # the step changes the latent by far more than the tolerance
+    assert rel(host(xb[0]), x["x0"]) > 10 * TOL_BF16
+
+
 def test_head_unpatchify_bf16_480p81(mods):
     model, wd = mods
     wl = synth.STACK_480P81
