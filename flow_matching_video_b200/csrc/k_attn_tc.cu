@@ -1,5 +1,6 @@
 // k_attn_tc.cu — non-causal multi-head attention on the sm_100a tensor cores
-// (tcgen05 + TMEM + TMA), head dim 128, bf16 in / bf16 out, fp32 softmax and
+// (tcgen05 + TMEM + TMA), head dim 128, bf16 or IEEE half operands (q, k, v
+// and the probabilities P share one type), bf16 out, fp32 softmax and
 // accumulation ("图解 Wan2.1 I2V" 5.3: full spatio-temporal self-attention;
 // 5.4: decoupled image/text cross-attention, two softmaxes summed).
 //
@@ -9,12 +10,14 @@
 //                    ring of RING 32 KB tiles
 //   warp 1           TMEM owner + MMA issuer: S_t = Q_t K_j^T into TMEM,
 //                    O_t (+)= P_t V_j with P_t read from TMEM (TS form), so
-//                    this product reads only V from shared memory
-//   warps 2..        8 softmax warps per Q tile: two per TMEM lane quarter
-//                    (32 query rows), each owning 64 of the 128 key columns.
-//                    Online softmax on S_t read from TMEM (the pair swaps its
-//                    row maxima through shared memory), P_t written back as
-//                    bf16 over the warp's own S columns, O_t rescaled in TMEM
+//                    this product reads only V from shared memory; P V is
+//                    issued in two 64-key halves as the softmax writes P
+//   warps 2..        4 * SPLIT softmax warps per Q tile, SPLIT per TMEM lane
+//                    quarter (32 query rows), each owning 128 / SPLIT key
+//                    columns (SPLIT = 1 by default: one thread holds a whole
+//                    row of S in registers, so no row maxima are exchanged).
+//                    Online softmax on S_t read from TMEM, P_t written back
+//                    over the warp's own S columns, O_t rescaled in TMEM
 //                    only when the running max grows by more than 8 (log2
 //                    units; the final 1/l keeps the result exact), then the
 //                    normalised output written out.
@@ -26,7 +29,7 @@ namespace wd {
 namespace tca {
 
 constexpr int BQ = 128, BKV = 128, DH = 128;
-constexpr int TILE_BYTES = 128 * 128 * 2;   // one 128 x 128 bf16 tile (two 64-column halves)
+constexpr int TILE_BYTES = 128 * 128 * 2;   // one 128 x 128 tile of 2-byte elements (two 64-column halves)
 constexpr int HALF_BYTES = TILE_BYTES / 2;
 #ifndef WD_ATTN_RING
 #define WD_ATTN_RING 4   // K/V tiles in flight (32 KB each)
@@ -40,7 +43,7 @@ constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
 constexpr int SPLIT = WD_ATTN_SPLIT;
 static_assert(SPLIT == 1 || SPLIT == 2, "WD_ATTN_SPLIT must be 1 or 2");
 
-template <int NQ, int NSEG>
+template <int NQ, int NSEG, typename TI>
 struct Cfg {
   // 2 warps (loader, MMA) + per Q tile 4*SPLIT softmax warps: SPLIT per TMEM
   // lane quarter (32 query rows), each owning 128/SPLIT of the key columns.
@@ -58,8 +61,11 @@ struct Cfg {
   // TMEM columns: S_t, O_t (per tile); with two segments one tile has O and O'
   __host__ __device__ static constexpr int s_col(int t) { return NSEG == 1 ? t * 256 : 0; }
   __host__ __device__ static constexpr int o_col(int t, int seg) { return NSEG == 1 ? t * 256 + 128 : 128 + 128 * seg; }
-  static constexpr uint32_t IDESC_S = idesc_bf16(128, 128, 0, 0);    // Q K^T: both K-major
-  static constexpr uint32_t IDESC_O = idesc_bf16(128, 128, 0, 1);    // P V: P from TMEM, V MN-major (dh contiguous)
+  // Q K^T: both K-major; P V: P from TMEM, V MN-major (dh contiguous).  P is
+  // held in the operands' type (A and B of one MMA share their type).
+  static constexpr bool HALF = std::is_same<TI, f16>::value;
+  static constexpr uint32_t IDESC_S = HALF ? idesc_f16(128, 128, 0, 0) : idesc_bf16(128, 128, 0, 0);
+  static constexpr uint32_t IDESC_O = HALF ? idesc_f16(128, 128, 0, 1) : idesc_bf16(128, 128, 0, 1);
 };
 
 enum : unsigned { SITE_Q = 0x201, SITE_KVF = 0x202, SITE_KVE = 0x203, SITE_S = 0x204, SITE_P = 0x205,
@@ -124,12 +130,12 @@ __device__ __forceinline__ float exp2_fma(float x) {
 #define WD_EXP2_EMU_PER8 1   // of every 8 exponentials, this many run on the FMA pipe
 #endif
 
-template <int NQ, int NSEG>
-__global__ void __launch_bounds__(Cfg<NQ, NSEG>::THREADS, 1)
+template <int NQ, int NSEG, typename TI>
+__global__ void __launch_bounds__(Cfg<NQ, NSEG, TI>::THREADS, 1)
 k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK0,
           const __grid_constant__ CUtensorMap tmV0, const __grid_constant__ CUtensorMap tmK1,
           const __grid_constant__ CUtensorMap tmV1, const Params p) {
-  using C = Cfg<NQ, NSEG>;
+  using C = Cfg<NQ, NSEG, TI>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
@@ -348,7 +354,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         }
         tmem_wait_st();
       }
-      // P = exp2(s * scale - m) as packed bf16 pairs into TMEM over this warp's
+      // P = exp2(s * scale - m) as packed pairs (operand type) into TMEM over this warp's
       // own S columns: chunk c of 16 keys -> 8 columns at 8c (masked keys hold
       // -inf, so their exponential is 0)
       float2 rs2 = make_float2(0.f, 0.f);
@@ -364,7 +370,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           const float e0 = ((k & 7) >= 8 - WD_EXP2_EMU_PER8) ? exp2_fma(arg.x) : ex2(arg.x);
           const float e1 = (((k + 1) & 7) >= 8 - WD_EXP2_EMU_PER8) ? exp2_fma(arg.y) : ex2(arg.y);
           rs2 = fadd2(rs2, make_float2(e0, e1));
-          pk[k >> 1] = pack_bf16x2(e0, e1);
+          pk[k >> 1] = C::HALF ? pack_f16x2(e0, e1) : pack_bf16x2(e0, e1);
         }
         tmem_st8(s_addr + c * 8, pk);
         if (SPLIT == 1 && c == CH - 1) {   // keys 0-63 of P are written: release the first half of P V
@@ -435,10 +441,10 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 }  // namespace tca
 
 // ------------------------------------------------------------------ host side
-// 3D bf16 tensor map over [batches, rows, cols] (cols contiguous, row stride
+// 3D tensor map (bf16 or IEEE half elements) over [batches, rows, cols] (cols contiguous, row stride
 // `rs` elements, batch stride `bs` elements); box = 64 cols x 128 rows x 1.
-static wd_status make_tmap_3d(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int64_t batches,
-                              int64_t rs, int64_t bs) {
+static wd_status make_tmap_3d(CUtensorMap* m, CUtensorMapDataType type, const void* base, int64_t cols, int64_t rows,
+                              int64_t batches, int64_t rs, int64_t bs) {
   auto fn = encode_fn();
   if (!fn) { set_error("cuTensorMapEncodeTiled unavailable"); return WD_ERR_CUDA; }
   if (batches > 1 && (bs * 2) % 16) { set_error("attention: batch stride not 16-byte aligned"); return WD_ERR_ALIGN; }
@@ -448,36 +454,37 @@ static wd_status make_tmap_3d(CUtensorMap* m, const void* base, int64_t cols, in
                            static_cast<cuuint64_t>(batches > 1 ? bs : rs * rows) * 2};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+  CUresult r = fn(m, type, 3, const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) { set_error("cuTensorMapEncodeTiled (3d) failed (%d)", static_cast<int>(r)); return WD_ERR_CUDA; }
   return WD_OK;
 }
 
-template <int NQ, int NSEG>
+template <int NQ, int NSEG, typename TI>
 static wd_status launch_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk0, const CUtensorMap& tv0,
                                 const CUtensorMap& tk1, const CUtensorMap& tv1, const tca::Params& p, int batch,
                                 int heads, cudaStream_t st) {
-  using C = tca::Cfg<NQ, NSEG>;
+  using C = tca::Cfg<NQ, NSEG, TI>;
   static bool attr[16] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr[dev & 15]) {
-    cudaFuncSetAttribute(tca::k_attn_tc<NQ, NSEG>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaFuncSetAttribute(tca::k_attn_tc<NQ, NSEG, TI>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     attr[dev & 15] = true;
   }
   dim3 grid((p.Lq + tca::BQ * NQ - 1) / (tca::BQ * NQ), heads, batch);
   Trace tr(NSEG == 2 ? KC_ATTN_CROSS : KC_ATTN_SELF, st);
-  tca::k_attn_tc<NQ, NSEG><<<grid, C::THREADS, C::SMEM, st>>>(tq, tk0, tv0, tk1, tv1, p);
+  tca::k_attn_tc<NQ, NSEG, TI><<<grid, C::THREADS, C::SMEM, st>>>(tq, tk0, tv0, tk1, tv1, p);
   return launch_status("attention_tc");
 }
 
 // The q/k/v pointers of AttnArgs may point into the middle of a row (the
 // fused q|k|v buffer); the tensor maps start at the row's first element that
 // is 16-byte aligned (the pointer itself) and use the row stride as extent.
-wd_status attention_tc(const AttnArgs<bf16>& a, cudaStream_t st) {
-  if (a.dh != tca::DH) return attention_simt<bf16>(a, st);
+template <typename TI>
+static wd_status attention_tc_t(const AttnArgs<TI, bf16>& a, cudaStream_t st) {
+  if (a.dh != tca::DH) return attention_simt<TI, bf16>(a, st);
   if (a.n1 <= 0 || (a.k2 && a.n2 <= 0)) { set_error("attention: empty key segment"); return WD_ERR_SHAPE; }
   const int D = a.heads * a.dh;
   auto al = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; };
@@ -486,12 +493,14 @@ wd_status attention_tc(const AttnArgs<bf16>& a, cudaStream_t st) {
     set_error("attention_tc: operands must be 16-byte aligned with row strides multiple of 8");
     return WD_ERR_ALIGN;
   }
+  const CUtensorMapDataType ty =
+      std::is_same<TI, f16>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap tq, tk0, tv0, tk1, tv1;
   // Each map covers D columns from its own base pointer.
-  WD_TRY(make_tmap_3d(&tq, a.q, D, a.Lq, a.batch, a.q_rs, a.q_rs * a.Lq));
+  WD_TRY(make_tmap_3d(&tq, ty, a.q, D, a.Lq, a.batch, a.q_rs, a.q_rs * a.Lq));
   const int64_t b1 = a.kv1_bs ? a.batch : 1;
-  WD_TRY(make_tmap_3d(&tk0, a.k1, D, a.n1, b1, a.kv1_rs, a.kv1_bs));
-  WD_TRY(make_tmap_3d(&tv0, a.v1, D, a.n1, b1, a.kv1_rs, a.kv1_bs));
+  WD_TRY(make_tmap_3d(&tk0, ty, a.k1, D, a.n1, b1, a.kv1_rs, a.kv1_bs));
+  WD_TRY(make_tmap_3d(&tv0, ty, a.v1, D, a.n1, b1, a.kv1_rs, a.kv1_bs));
   tca::Params p{};
   p.Lq = a.Lq;
   p.seg[0] = tca::Seg{a.n1, a.kv1_bs == 0};
@@ -500,12 +509,15 @@ wd_status attention_tc(const AttnArgs<bf16>& a, cudaStream_t st) {
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(a.dh));
   if (a.k2) {
     const int64_t b2 = a.kv2_bs ? a.batch : 1;
-    WD_TRY(make_tmap_3d(&tk1, a.k2, D, a.n2, b2, a.kv2_rs, a.kv2_bs));
-    WD_TRY(make_tmap_3d(&tv1, a.v2, D, a.n2, b2, a.kv2_rs, a.kv2_bs));
+    WD_TRY(make_tmap_3d(&tk1, ty, a.k2, D, a.n2, b2, a.kv2_rs, a.kv2_bs));
+    WD_TRY(make_tmap_3d(&tv1, ty, a.v2, D, a.n2, b2, a.kv2_rs, a.kv2_bs));
     p.seg[1] = tca::Seg{a.n2, a.kv2_bs == 0};
-    return launch_attn_tc<1, 2>(tq, tk0, tv0, tk1, tv1, p, a.batch, a.heads, st);
+    return launch_attn_tc<1, 2, TI>(tq, tk0, tv0, tk1, tv1, p, a.batch, a.heads, st);
   }
-  return launch_attn_tc<2, 1>(tq, tk0, tv0, tk0, tv0, p, a.batch, a.heads, st);
+  return launch_attn_tc<2, 1, TI>(tq, tk0, tv0, tk0, tv0, p, a.batch, a.heads, st);
 }
+
+wd_status attention_tc(const AttnArgs<bf16, bf16>& a, cudaStream_t st) { return attention_tc_t<bf16>(a, st); }
+wd_status attention_tc(const AttnArgs<f16, bf16>& a, cudaStream_t st) { return attention_tc_t<f16>(a, st); }
 
 }  // namespace wd

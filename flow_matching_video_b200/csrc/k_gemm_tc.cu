@@ -1,6 +1,7 @@
 // k_gemm_tc.cu — bf16 GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA)
 // with the epilogues of the DiT block fused in: bias, bias+GELU, bias then
-// gate * (.) added into the fp32 residual stream, fp32 store, unpatchify.
+// gate * (.) added into the fp32 residual stream, fp32 store, IEEE half store
+// (cross-attention operands), unpatchify.
 //
 // C[m, n] = sum_k A[m, k] * B[n, k]: A = activations [M, K], B = a Linear
 // weight [N, K]; both K-major, loaded by TMA into 128-byte-swizzled shared
@@ -27,7 +28,7 @@ constexpr int BM = 128, BK = 64;
 #endif
 constexpr int EPI_WG = WD_GEMM_EPI_WG;
 #ifndef WD_GEMM_RESID_PIPE
-#define WD_GEMM_RESID_PIPE 0   // residual epilogue loads one chunk ahead
+#define WD_GEMM_RESID_PIPE 1   // residual epilogue loads one chunk ahead
 #endif
 #ifndef WD_GEMM_RESID_PREFETCH
 #define WD_GEMM_RESID_PREFETCH 0   // producer prefetches each tile's fp32 residual block into L2
@@ -74,6 +75,13 @@ __device__ __forceinline__ void epilogue32(const Epi& ep, int64_t m, int n, cons
     for (int j = 0; j < 4; ++j) {
       dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
                           pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+    }
+  } else if constexpr (MODE == EPI_STORE_F16) {
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<f16*>(ep.out) + m * ep.ldo + n);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      dst[j] = make_uint4(pack_f16x2(v[8 * j], v[8 * j + 1]), pack_f16x2(v[8 * j + 2], v[8 * j + 3]),
+                          pack_f16x2(v[8 * j + 4], v[8 * j + 5]), pack_f16x2(v[8 * j + 6], v[8 * j + 7]));
     }
   } else if constexpr (MODE == EPI_F32) {
     float4* dst = reinterpret_cast<float4*>(static_cast<float*>(ep.out) + m * ep.ldo + n);
@@ -347,6 +355,7 @@ static wd_status dispatch_mode(int mode, const CUtensorMap& ta, const CUtensorMa
     case EPI_F32: return launch_tc<BN, EPI_F32>(ta, tb, ep, M, N, K, st);
     case EPI_RESID: return launch_tc<BN, EPI_RESID>(ta, tb, ep, M, N, K, st);
     case EPI_UNPATCH: return launch_tc<BN, EPI_UNPATCH>(ta, tb, ep, M, N, K, st);
+    case EPI_STORE_F16: return launch_tc<BN, EPI_STORE_F16>(ta, tb, ep, M, N, K, st);
   }
   set_error("gemm_tc: bad epilogue %d", mode);
   return WD_ERR_ARG;

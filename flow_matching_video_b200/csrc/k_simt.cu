@@ -20,6 +20,7 @@ __device__ __forceinline__ void epi_one(int mode, const Epi& ep, int64_t m, int 
       break;
     }
     case EPI_UNPATCH: static_cast<float*>(ep.out)[unpatch_index(ep, m, n)] = v; break;
+    case EPI_STORE_F16: static_cast<f16*>(ep.out)[m * ep.ldo + n] = __float2half_rn(v); break;
   }
 }
 
@@ -89,8 +90,8 @@ template wd_status gemm_simt<bf16>(int, int, int, const bf16*, int64_t, const bf
 // 64-key tiles through shared memory with an online softmax (exp2, log2(e)/
 // sqrt(dh) folded into q).  A second key/value segment, when present, gets its
 // own softmax and is added after normalisation ("图解 Wan2.1 I2V" 5.4).
-template <typename T, int DH>
-__global__ void __launch_bounds__(256) k_attn_simt(AttnArgs<T> a, float qscale) {
+template <typename T, typename TO, int DH>
+__global__ void __launch_bounds__(256) k_attn_simt(AttnArgs<T, TO> a, float qscale) {
   constexpr int BQ = 64, BK = 64, P = 68, CW = DH / 16;
   extern __shared__ __align__(16) float sm[];
   float* Qt = sm;               // [DH][P]  q transposed
@@ -191,40 +192,41 @@ __global__ void __launch_bounds__(256) k_attn_simt(AttnArgs<T> a, float qscale) 
   for (int i = 0; i < 4; ++i) {
     const int l = q0 + ty * 4 + i;
     if (l >= a.Lq) continue;
-    T* dst = a.o + (static_cast<int64_t>(b) * a.Lq + l) * a.o_rs + h * DH + tx * CW;
+    TO* dst = a.o + (static_cast<int64_t>(b) * a.Lq + l) * a.o_rs + h * DH + tx * CW;
 #pragma unroll
-    for (int c = 0; c < CW; ++c) dst[c] = from_f<T>(out[i][c]);
+    for (int c = 0; c < CW; ++c) dst[c] = from_f<TO>(out[i][c]);
   }
 }
 
-template <typename T, int DH>
-static wd_status launch_attn_simt(const AttnArgs<T>& a, cudaStream_t st) {
+template <typename T, typename TO, int DH>
+static wd_status launch_attn_simt(const AttnArgs<T, TO>& a, cudaStream_t st) {
   const size_t smem = (2 * DH * 68 + 64 * DH + 64 * 68) * sizeof(float);
   static bool attr_set[16] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr_set[dev & 15]) {
-    cudaFuncSetAttribute(k_attn_simt<T, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaFuncSetAttribute(k_attn_simt<T, TO, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     attr_set[dev & 15] = true;
   }
   dim3 grid((a.Lq + 63) / 64, a.heads, a.batch);
   const float qscale = 1.4426950408889634f / sqrtf(static_cast<float>(DH));
   Trace tr(a.k2 ? KC_ATTN_CROSS : KC_ATTN_SELF, st);
-  k_attn_simt<T, DH><<<grid, 256, smem, st>>>(a, qscale);
+  k_attn_simt<T, TO, DH><<<grid, 256, smem, st>>>(a, qscale);
   return launch_status("attention_simt");
 }
 
-template <typename T>
-wd_status attention_simt(const AttnArgs<T>& a, cudaStream_t st) {
+template <typename T, typename TO>
+wd_status attention_simt(const AttnArgs<T, TO>& a, cudaStream_t st) {
   if (a.n1 <= 0 || (a.k2 && a.n2 <= 0)) { set_error("attention: empty key segment"); return WD_ERR_SHAPE; }
   switch (a.dh) {
-    case 32: return launch_attn_simt<T, 32>(a, st);
-    case 64: return launch_attn_simt<T, 64>(a, st);
-    case 128: return launch_attn_simt<T, 128>(a, st);
+    case 32: return launch_attn_simt<T, TO, 32>(a, st);
+    case 64: return launch_attn_simt<T, TO, 64>(a, st);
+    case 128: return launch_attn_simt<T, TO, 128>(a, st);
     default: set_error("attention: head dim %d not supported (32, 64, 128)", a.dh); return WD_ERR_SHAPE;
   }
 }
-template wd_status attention_simt<float>(const AttnArgs<float>&, cudaStream_t);
-template wd_status attention_simt<bf16>(const AttnArgs<bf16>&, cudaStream_t);
+template wd_status attention_simt<float, float>(const AttnArgs<float, float>&, cudaStream_t);
+template wd_status attention_simt<bf16, bf16>(const AttnArgs<bf16, bf16>&, cudaStream_t);
+template wd_status attention_simt<f16, bf16>(const AttnArgs<f16, bf16>&, cudaStream_t);
 
 }  // namespace wd

@@ -106,13 +106,19 @@ static wd_status gemm(int M, int N, int K, const void* A, int64_t lda, const voi
   return gemm_simt<T>(M, N, K, static_cast<const T*>(A), lda, static_cast<const T*>(B), ldb, mode, ep, st);
 }
 
-template <typename T>
-static wd_status attention(const AttnArgs<T>& a, cudaStream_t st) {
-  if constexpr (sizeof(T) == 2) {
+template <typename TI, typename TO>
+static wd_status attention(const AttnArgs<TI, TO>& a, cudaStream_t st) {
+  if constexpr (sizeof(TI) == 2) {
     if (!(g_debug_flags & 2u) && a.dh == 128) return attention_tc(a, st);
   }
-  return attention_simt<T>(a, st);
+  return attention_simt<TI, TO>(a, st);
 }
+
+// Element type of the cross-attention operands (qc and the K/V cache): IEEE
+// half on the bf16 path, where the text cross-attention's sharp softmax
+// amplifies operand rounding; the activation type otherwise.
+template <typename T> struct CrossT { using type = T; static constexpr int store = EPI_STORE; };
+template <> struct CrossT<bf16> { using type = f16; static constexpr int store = EPI_STORE_F16; };
 
 static Epi epi(void* out, int64_t ldo, const float* bias, const float* ga = nullptr, const float* gb = nullptr) {
   Epi e{};
@@ -143,14 +149,15 @@ static wd_status block_forward_t(const wd_dims* d, const wd_block_weights* w, co
   const int rms = d->norm == WD_NORM_RMS;
   const float* mod = w->mod;
   // cross K/V cache parts
-  const size_t es = sizeof(T);
+  using CT = typename CrossT<T>::type;
+  const size_t es = sizeof(CT);
   const char* kvp = static_cast<const char*>(kv);
   const size_t n_img_b = up256(static_cast<size_t>(d->n_img) * D * es);
   const size_t n_txt_b = up256(static_cast<size_t>(batch) * d->n_txt * D * es);
-  const T* k_img = reinterpret_cast<const T*>(kvp);
-  const T* v_img = reinterpret_cast<const T*>(kvp + n_img_b);
-  const T* k_txt = reinterpret_cast<const T*>(kvp + 2 * n_img_b);
-  const T* v_txt = reinterpret_cast<const T*>(kvp + 2 * n_img_b + n_txt_b);
+  const CT* k_img = reinterpret_cast<const CT*>(kvp);
+  const CT* v_img = reinterpret_cast<const CT*>(kvp + n_img_b);
+  const CT* k_txt = reinterpret_cast<const CT*>(kvp + 2 * n_img_b);
+  const CT* v_txt = reinterpret_cast<const CT*>(kvp + 2 * n_img_b + n_txt_b);
 
   // 1. h = norm(X)(1 + scale1) + shift1
   WD_TRY(norm_rows<T>(d, X, rows, e0, mod, e0 + D, mod + D, nullptr, nullptr, rms, Bf, st));
@@ -162,27 +169,27 @@ static wd_status block_forward_t(const wd_dims* d, const wd_block_weights* w, co
   WD_TRY(qknorm_rope<T>(A, rows, *d, w->g_q, w->g_k, ws.rope, st));
   // 4. full self-attention -> o
   {
-    AttnArgs<T> a{};
+    AttnArgs<T, T> a{};
     a.q = A; a.q_rs = 3 * D;
     a.k1 = A + D; a.v1 = A + 2 * D; a.kv1_rs = 3 * D; a.kv1_bs = L * 3 * D; a.n1 = static_cast<int>(L);
     a.o = Bf; a.o_rs = D;
     a.batch = batch; a.Lq = static_cast<int>(L); a.heads = d->heads; a.dh = dh;
-    WD_TRY(attention<T>(a, st));
+    WD_TRY(attention(a, st));
   }
   // 5. X += gate1 * (o Wo^T + b)
   WD_TRY(gemm<T>(M, D, D, Bf, D, w->o_w, D, EPI_RESID, epi(X, D, w->o_b, e0 + 2 * D, mod + 2 * D), st));
   // 6. hc = LN_affine(X);  7. qc = hc Wcq^T + b
   WD_TRY(norm_rows<T>(d, X, rows, nullptr, nullptr, nullptr, nullptr, w->cn_g, w->cn_b, 0, Bf, st));
-  WD_TRY(gemm<T>(M, D, D, Bf, D, w->cq_w, D, EPI_STORE, epi(A, D, w->cq_b), st));
+  WD_TRY(gemm<T>(M, D, D, Bf, D, w->cq_w, D, CrossT<T>::store, epi(A, D, w->cq_b), st));
   // 8. oc = attn(qc, K_img, V_img) + attn(qc, K_txt, V_txt)
   {
-    AttnArgs<T> a{};
-    a.q = A; a.q_rs = D;
+    AttnArgs<CT, T> a{};
+    a.q = reinterpret_cast<const CT*>(A); a.q_rs = D;
     a.k1 = k_img; a.v1 = v_img; a.kv1_rs = D; a.kv1_bs = 0; a.n1 = d->n_img;
     a.k2 = k_txt; a.v2 = v_txt; a.kv2_rs = D; a.kv2_bs = static_cast<int64_t>(d->n_txt) * D; a.n2 = d->n_txt;
     a.o = Bf; a.o_rs = D;
     a.batch = batch; a.Lq = static_cast<int>(L); a.heads = d->heads; a.dh = dh;
-    WD_TRY(attention<T>(a, st));
+    WD_TRY(attention(a, st));
   }
   // 9. X += oc Wco^T + b
   WD_TRY(gemm<T>(M, D, D, Bf, D, w->co_w, D, EPI_RESID, epi(X, D, w->co_b), st));
@@ -350,7 +357,7 @@ wd_status wd_cross_kv(const wd_dims* d, const wd_block_weights* w, const void* c
   WD_NEED(kv);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int D = d->D;
-  const size_t es = esize(d);
+  const size_t es = esize(d);   // context and K/V cache elements: 2 bytes (bf16 / IEEE half) or 4 (fp32)
   const char* p = static_cast<const char*>(ctx);
   const void* ctx_txt = p;
   const void* ctx_img = p + up256(static_cast<size_t>(batch) * d->n_txt * D * es);
@@ -359,10 +366,11 @@ wd_status wd_cross_kv(const wd_dims* d, const wd_block_weights* w, const void* c
   void *k_img = q, *v_img = q + ni, *k_txt = q + 2 * ni, *v_txt = q + 2 * ni + nt;
   const int Mt = batch * d->n_txt;
   if (d->dtype == WD_BF16) {
-    WD_TRY(gemm<bf16>(d->n_img, D, D, ctx_img, D, w->cki_w, D, EPI_STORE, epi(k_img, D, w->cki_b), st));
-    WD_TRY(gemm<bf16>(d->n_img, D, D, ctx_img, D, w->cvi_w, D, EPI_STORE, epi(v_img, D, w->cvi_b), st));
-    WD_TRY(gemm<bf16>(Mt, D, D, ctx_txt, D, w->ck_w, D, EPI_STORE, epi(k_txt, D, w->ck_b), st));
-    WD_TRY(gemm<bf16>(Mt, D, D, ctx_txt, D, w->cv_w, D, EPI_STORE, epi(v_txt, D, w->cv_b), st));
+    // stored as IEEE half: the cross-attention operands of the bf16 path
+    WD_TRY(gemm<bf16>(d->n_img, D, D, ctx_img, D, w->cki_w, D, EPI_STORE_F16, epi(k_img, D, w->cki_b), st));
+    WD_TRY(gemm<bf16>(d->n_img, D, D, ctx_img, D, w->cvi_w, D, EPI_STORE_F16, epi(v_img, D, w->cvi_b), st));
+    WD_TRY(gemm<bf16>(Mt, D, D, ctx_txt, D, w->ck_w, D, EPI_STORE_F16, epi(k_txt, D, w->ck_b), st));
+    WD_TRY(gemm<bf16>(Mt, D, D, ctx_txt, D, w->cv_w, D, EPI_STORE_F16, epi(v_txt, D, w->cv_b), st));
   } else {
     WD_TRY(gemm<float>(d->n_img, D, D, ctx_img, D, w->cki_w, D, EPI_STORE, epi(k_img, D, w->cki_b), st));
     WD_TRY(gemm<float>(d->n_img, D, D, ctx_img, D, w->cvi_w, D, EPI_STORE, epi(v_img, D, w->cvi_b), st));
@@ -438,11 +446,15 @@ wd_status wd_unpatchify(const wd_dims* d, const wd_head_weights* w, const float*
 
 // ---------------------------------------------------------------- building blocks (tested one by one)
 // C = epilogue(A[M,K] B[N,K]^T) with the epilogue codes of the block
-// (0 store, 1 GELU, 2 fp32 store, 3 gated residual add into fp32 out).
+// (0 store, 1 GELU, 2 fp32 store, 3 gated residual add into fp32 out,
+// 5 IEEE half store, bf16 inputs only).
 wd_status wd_gemm(int dtype, int M, int N, int K, const void* A, const void* B, const float* bias, int epilogue,
                   void* out, const float* gate_a, const float* gate_b, wd_stream stream) {
   WD_NEED(A); WD_NEED(B); WD_NEED(out); WD_OPT(bias); WD_OPT(gate_a); WD_OPT(gate_b);
-  if (epilogue < 0 || epilogue > 3) { set_error("epilogue %d", epilogue); return WD_ERR_ARG; }
+  if (epilogue < 0 || epilogue > 5 || epilogue == EPI_UNPATCH || (epilogue == EPI_STORE_F16 && dtype != WD_BF16)) {
+    set_error("epilogue %d (dtype %d)", epilogue, dtype);
+    return WD_ERR_ARG;
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Epi ep = epi(out, N, bias, gate_a, gate_b);
   if (dtype == WD_BF16) return gemm<bf16>(M, N, K, A, K, B, K, epilogue, ep, st);
@@ -453,7 +465,8 @@ wd_status wd_gemm(int dtype, int M, int N, int K, const void* A, const void* B, 
 
 // O[b, l, h*dh:(h+1)*dh] = softmax(q k^T / sqrt(dh)) v  (+ second segment).
 // q [batch, Lq, heads*dh]; k1/v1 [batch or 1 (kv1_shared), n1, heads*dh];
-// k2/v2 likewise or NULL; o [batch, Lq, heads*dh].
+// k2/v2 likewise or NULL; o [batch, Lq, heads*dh] (bf16 when the operands
+// are IEEE half).
 wd_status wd_attention(int dtype, int batch, int Lq, int heads, int dh, const void* q, const void* k1, const void* v1,
                        int n1, int kv1_shared, const void* k2, const void* v2, int n2, int kv2_shared, void* o,
                        wd_stream stream) {
@@ -468,16 +481,22 @@ wd_status wd_attention(int dtype, int batch, int Lq, int heads, int dh, const vo
     return a;
   };
   if (dtype == WD_BF16) {
-    AttnArgs<bf16> a{};
+    AttnArgs<bf16, bf16> a{};
     a.q = static_cast<const bf16*>(q); a.k1 = static_cast<const bf16*>(k1); a.v1 = static_cast<const bf16*>(v1);
     a.k2 = static_cast<const bf16*>(k2); a.v2 = static_cast<const bf16*>(v2); a.o = static_cast<bf16*>(o);
-    return attention<bf16>(fill(a), st);
+    return attention(fill(a), st);
+  }
+  if (dtype == WD_F16) {
+    AttnArgs<f16, bf16> a{};
+    a.q = static_cast<const f16*>(q); a.k1 = static_cast<const f16*>(k1); a.v1 = static_cast<const f16*>(v1);
+    a.k2 = static_cast<const f16*>(k2); a.v2 = static_cast<const f16*>(v2); a.o = static_cast<bf16*>(o);
+    return attention(fill(a), st);
   }
   if (dtype == WD_F32) {
-    AttnArgs<float> a{};
+    AttnArgs<float, float> a{};
     a.q = static_cast<const float*>(q); a.k1 = static_cast<const float*>(k1); a.v1 = static_cast<const float*>(v1);
     a.k2 = static_cast<const float*>(k2); a.v2 = static_cast<const float*>(v2); a.o = static_cast<float*>(o);
-    return attention<float>(fill(a), st);
+    return attention(fill(a), st);
   }
   set_error("dtype %d", dtype);
   return WD_ERR_DTYPE;

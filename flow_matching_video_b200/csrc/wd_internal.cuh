@@ -2,9 +2,11 @@
 // translation unit: wd_lib.cu includes every kernel file).
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 #include <cstdio>
 #include <string>
 
@@ -14,6 +16,7 @@
 namespace wd {
 
 using bf16 = __nv_bfloat16;
+using f16 = __half;
 
 // ------------------------------------------------------------------ errors
 void set_error(const char* fmt, ...);
@@ -44,12 +47,18 @@ struct Trace {
 template <typename T> __device__ __forceinline__ float to_f(T v);
 template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f<bf16>(bf16 v) { return __bfloat162float(v); }
+template <> __device__ __forceinline__ float to_f<f16>(f16 v) { return __half2float(v); }
 template <typename T> __device__ __forceinline__ T from_f(float v);
 template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ bf16 from_f<bf16>(float v) { return __float2bfloat16_rn(v); }
+template <> __device__ __forceinline__ f16 from_f<f16>(float v) { return __float2half_rn(v); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
@@ -69,6 +78,7 @@ enum EpiMode : int {
   EPI_F32 = 2,        // out[m, n] = v                        (out fp32)
   EPI_RESID = 3,      // out[m, n] += g[n] * v, g = ga + gb   (out fp32 residual, in place)
   EPI_UNPATCH = 4,    // unpatchify scatter of v into [B, 16, T, H, W] fp32
+  EPI_STORE_F16 = 5,  // out[m, n] = v                        (out IEEE half: cross-attention operands)
 };
 
 struct Epi {
@@ -101,17 +111,21 @@ wd_status gemm_tc(int M, int N, int K, const bf16* A, int64_t lda, const bf16* B
 
 // Multi-head attention O = softmax(Q K^T / sqrt(dh)) V per (batch, head),
 // optionally summed with a second, independently normalised key/value
-// segment (the decoupled image/text cross-attention).
-template <typename T>
+// segment (the decoupled image/text cross-attention).  TI is the type of
+// q, k and v; TO the type of o (the bf16 path's cross-attention reads IEEE
+// half operands and writes bf16).
+template <typename TI, typename TO = TI>
 struct AttnArgs {
-  const T* q; int64_t q_rs;                    // q row (b, l): q + (b*Lq + l)*q_rs + h*dh
-  const T* k1; const T* v1; int64_t kv1_rs; int64_t kv1_bs; int n1;
-  const T* k2; const T* v2; int64_t kv2_rs; int64_t kv2_bs; int n2;   // k2 == null: one segment
-  T* o; int64_t o_rs;
+  const TI* q; int64_t q_rs;                   // q row (b, l): q + (b*Lq + l)*q_rs + h*dh
+  const TI* k1; const TI* v1; int64_t kv1_rs; int64_t kv1_bs; int n1;
+  const TI* k2; const TI* v2; int64_t kv2_rs; int64_t kv2_bs; int n2;   // k2 == null: one segment
+  TO* o; int64_t o_rs;
   int batch, Lq, heads, dh;
 };
-template <typename T>
-wd_status attention_simt(const AttnArgs<T>& a, cudaStream_t st);
-wd_status attention_tc(const AttnArgs<bf16>& a, cudaStream_t st);
+template <typename TI, typename TO>
+wd_status attention_simt(const AttnArgs<TI, TO>& a, cudaStream_t st);
+// Tensor-core attention (dh = 128; other head sizes go to attention_simt).
+wd_status attention_tc(const AttnArgs<bf16, bf16>& a, cudaStream_t st);
+wd_status attention_tc(const AttnArgs<f16, bf16>& a, cudaStream_t st);
 
 }  // namespace wd

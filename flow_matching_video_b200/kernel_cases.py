@@ -27,15 +27,19 @@ def bf(*shape):
     return torch.randn(*shape, device="cuda").to(torch.bfloat16)
 
 
+def hf(*shape):
+    return torch.randn(*shape, device="cuda").to(torch.float16)
+
+
 def make_case(name: str, B: int):
     rows = B * L
     if name == "attn_self":
         q, k, v, o = bf(B, L, D), bf(B, L, D), bf(B, L, D), torch.empty(B, L, D, device="cuda", dtype=torch.bfloat16)
         return (lambda: wd.wd_attention(wd.WD_BF16, B, L, H, 128, q, k, v, L, 0, o)), 4.0 * B * L * L * D, "FLOP"
-    if name == "attn_cross":
-        q, o = bf(B, L, D), torch.empty(B, L, D, device="cuda", dtype=torch.bfloat16)
-        ki, vi, kt, vt = bf(NI, D), bf(NI, D), bf(B, NT, D), bf(B, NT, D)
-        return (lambda: wd.wd_attention(wd.WD_BF16, B, L, H, 128, q, ki, vi, NI, 1, o, kt, vt, NT, 0),
+    if name == "attn_cross":   # IEEE half operands, bf16 output, as in the block
+        q, o = hf(B, L, D), torch.empty(B, L, D, device="cuda", dtype=torch.bfloat16)
+        ki, vi, kt, vt = hf(NI, D), hf(NI, D), hf(B, NT, D), hf(B, NT, D)
+        return (lambda: wd.wd_attention(wd.WD_F16, B, L, H, 128, q, ki, vi, NI, 1, o, kt, vt, NT, 0),
                 4.0 * B * L * (NI + NT) * D, "FLOP")
     gemms = {"gemm_qkv": (3 * D, D, wd.EPI_STORE), "gemm_o": (D, D, wd.EPI_RESID),
              "gemm_ffn1": (F, D, wd.EPI_GELU), "gemm_ffn2": (D, F, wd.EPI_RESID)}

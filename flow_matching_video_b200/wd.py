@@ -17,9 +17,9 @@ if not os.path.exists(LIB_PATH):
     raise ImportError(f"libwd.so not built ({LIB_PATH}); run `python -m flow_matching_video_b200.build`")
 _lib = C.CDLL(LIB_PATH)
 
-WD_F32, WD_BF16 = 0, 1
+WD_F32, WD_BF16, WD_F16 = 0, 1, 2
 WD_NORM_LAYER, WD_NORM_RMS = 0, 1
-EPI_STORE, EPI_GELU, EPI_F32, EPI_RESID = 0, 1, 2, 3
+EPI_STORE, EPI_GELU, EPI_F32, EPI_RESID, EPI_STORE_F16 = 0, 1, 2, 3, 5
 STATUS = {0: "WD_OK", 1: "WD_ERR_ARG", 2: "WD_ERR_SHAPE", 3: "WD_ERR_DTYPE", 4: "WD_ERR_ALIGN",
           5: "WD_ERR_WORKSPACE", 6: "WD_ERR_CUDA", 7: "WD_ERR_TIMEOUT", 8: "WD_ERR_UNSUPPORTED"}
 

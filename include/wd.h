@@ -53,7 +53,10 @@ typedef enum {
   WD_ERR_UNSUPPORTED = 8  /* feature not built for this configuration     */
 } wd_status;
 
-typedef enum { WD_F32 = 0, WD_BF16 = 1 } wd_dtype;
+/* WD_F16 (IEEE half) is not a model dtype: it names the cross-attention
+ * operands of the WD_BF16 path (the K/V cache and the cross queries) and the
+ * operand type accepted by wd_attention. */
+typedef enum { WD_F32 = 0, WD_BF16 = 1, WD_F16 = 2 } wd_dtype;
 typedef enum { WD_NORM_LAYER = 0, WD_NORM_RMS = 1 } wd_norm;
 
 /* Model and video dimensions.  D = model width, heads x (D/heads) attention
@@ -137,7 +140,9 @@ size_t wd_ctx_bytes(const wd_dims* d, int batch);
 
 /* Bytes of ONE block's cross-attention K/V cache written by wd_cross_kv:
  * k_img [n_img,D], v_img [n_img,D], k_txt [batch,n_txt,D], v_txt [batch,n_txt,D]
- * in that order, dtype elements, each part starting on a 256-byte boundary. */
+ * in that order, each part starting on a 256-byte boundary.  Elements are
+ * fp32 for WD_F32 and IEEE half for WD_BF16 (the text cross-attention softmax
+ * is sharp, so its operands keep 11 significant bits rather than 8). */
 size_t wd_kv_bytes(const wd_dims* d, int batch);
 
 /* ------------------------------------------------------------------ the path */
@@ -181,7 +186,8 @@ wd_status wd_patch_embed(const wd_dims* d, const float* x_t, const float* y, con
  * ([I2V] 5.2-5.5): adaLN-modulated full 3D self-attention with QK-RMSNorm and
  * 3D RoPE, gate1 residual; decoupled image/text cross-attention, plain
  * residual; adaLN-modulated GELU FFN, gate2 residual.  e0 [6,D] fp32 from
- * wd_time_mod; kv from wd_cross_kv for this block. */
+ * wd_time_mod; kv from wd_cross_kv for this block.  On the WD_BF16 path the
+ * cross-attention queries are stored as IEEE half, like the K/V cache. */
 wd_status wd_block_forward(const wd_dims* d, const wd_block_weights* w, const float* e0,
                            const void* kv, int batch, float* X, void* ws, size_t ws_bytes,
                            wd_stream stream);
@@ -234,7 +240,8 @@ wd_status wd_patch_embed_noalloc(const wd_dims* d, const float* x_t, const float
  * NULL.  epilogue 0: out [M,N] = v in dtype; 1: out = GELU(v) (erf form,
  * [I2V] 5.5) in dtype; 2: out = v in fp32; 3: out [M,N] fp32 += g*v with
  * g = gate_a + gate_b (either may be NULL; both NULL means 1) — the gated
- * residual of [I2V] 5.2.  bf16 runs on the tcgen05 tensor cores (N a
+ * residual of [I2V] 5.2; 5 (WD_BF16 only): out = v in IEEE half (the
+ * cross-attention operands).  bf16 runs on the tcgen05 tensor cores (N a
  * multiple of 64, K a multiple of 8), fp32 on the CUDA cores. */
 wd_status wd_gemm(int dtype, int M, int N, int K, const void* A, const void* B, const float* bias, int epilogue,
                   void* out, const float* gate_a, const float* gate_b, wd_stream stream);
@@ -243,7 +250,10 @@ wd_status wd_gemm(int dtype, int M, int N, int K, const void* A, const void* B, 
  * head h, o = softmax(q k1^T / sqrt(dh)) v1 [+ softmax(q k2^T / sqrt(dh)) v2].
  * q, o [batch, Lq, heads*dh]; k1, v1 [batch, n1, heads*dh] or, with
  * kv1_shared != 0, [n1, heads*dh] shared by the batch; k2/v2 likewise, or
- * NULL for one segment.  dh in {32, 64, 128}. */
+ * NULL for one segment.  dh in {32, 64, 128}.  dtype WD_F32: all fp32;
+ * WD_BF16: all bf16; WD_F16: q, k, v IEEE half and o bf16 (the bf16 path's
+ * cross-attention).  The probabilities enter the P V product in the operand
+ * type (bf16 or half), with fp32 softmax statistics and accumulation. */
 wd_status wd_attention(int dtype, int batch, int Lq, int heads, int dh, const void* q, const void* k1, const void* v1,
                        int n1, int kv1_shared, const void* k2, const void* v2, int n2, int kv2_shared, void* o,
                        wd_stream stream);

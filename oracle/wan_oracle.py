@@ -16,8 +16,9 @@ Every function cites the passage of the source pages it follows:
 Where the pages are silent the oracle takes the plainest reading; each one is
 marked "Reading:" below.  Storage rounding: with ``rnd=True`` the oracle rounds
 to bfloat16 (round-to-nearest-even) at exactly the points where the GPU path
-stores a bf16 tensor (GEMM operands, q/k/v, attention outputs, FFN hidden, the
-cross-attention K/V cache), so a bf16 run is compared with the same function.
+stores a bf16 tensor (GEMM operands, q/k/v, attention outputs, FFN hidden),
+and to IEEE half where it stores a half tensor (the cross-attention queries
+and K/V cache), so a bf16 run is compared with the same function.
 Parity pins: see tests/test_oracle_*.py.  Functions whose full output no page
 pins ("parity unpinned"): dit_forward / block_forward values beyond the
 invariants (AdaLN-Zero identity, attention and RoPE special cases) checked in
@@ -47,8 +48,31 @@ def bf16(a) -> np.ndarray:
     return np.ldexp(np.rint(m * 256.0) / 256.0, e)
 
 
+def fp16(a) -> np.ndarray:
+    """Round to the nearest IEEE binary16 value, ties to even.
+
+    Normal halves keep 11 significant bits: for a = m * 2**e (|m| in
+    [0.5, 1)) the spacing is 2**(e - 11).  Below 2**-14 the spacing stays at
+    2**-24 (subnormals).  Results above the largest finite half, 65504, are
+    infinite.
+    Reading: the pages fix no precision; the bf16 model keeps its
+    cross-attention operands (cross queries and the K/V cache) in IEEE half,
+    because the text cross-attention softmax is sharp (scores of several
+    units) and amplifies the rounding of its operands.
+    """
+    a = np.asarray(a, dtype=F64)
+    _, e = np.frexp(a)
+    q = np.maximum(e - 11, -24)
+    r = np.ldexp(np.rint(np.ldexp(a, -q)), q)
+    return np.where(np.abs(r) > 65504.0, np.copysign(np.inf, a), r)
+
+
 def _st(a, rnd: bool):
     return bf16(a) if rnd else np.asarray(a, dtype=F64)
+
+
+def _st16(a, rnd: bool):
+    return fp16(a) if rnd else np.asarray(a, dtype=F64)
 
 
 # ---------------------------------------------------------------- shapes
@@ -273,10 +297,10 @@ def cross_kv(w: dict, blk: int, ctx_txt, ctx_img, rnd: bool = False):
     Linear_k / Linear_v, the image branch its own k_img / v_img."""
     p = f"blk{blk}."
     return dict(
-        k_txt=_st(linear(ctx_txt, w[p + "ck.w"], w[p + "ck.b"]), rnd),
-        v_txt=_st(linear(ctx_txt, w[p + "cv.w"], w[p + "cv.b"]), rnd),
-        k_img=_st(linear(ctx_img, w[p + "cki.w"], w[p + "cki.b"]), rnd),
-        v_img=_st(linear(ctx_img, w[p + "cvi.w"], w[p + "cvi.b"]), rnd),
+        k_txt=_st16(linear(ctx_txt, w[p + "ck.w"], w[p + "ck.b"]), rnd),
+        v_txt=_st16(linear(ctx_txt, w[p + "cv.w"], w[p + "cv.b"]), rnd),
+        k_img=_st16(linear(ctx_img, w[p + "cki.w"], w[p + "cki.b"]), rnd),
+        v_img=_st16(linear(ctx_img, w[p + "cvi.w"], w[p + "cvi.b"]), rnd),
     )
 
 
@@ -328,7 +352,7 @@ def block_forward(X, e0, w: dict, blk: int, kv: dict, dims, rnd: bool = False, r
         xr = x[rows] + gate1 * linear(o, w[p + "o.w"], w[p + "o.b"])
         # ---- decoupled cross-attention (not modulated, not gated)
         hc = _st(layer_norm(xr, eps, w[p + "cn.g"], w[p + "cn.b"]), rnd)
-        qc = _st(linear(hc, w[p + "cq.w"], w[p + "cq.b"]), rnd).reshape(len(rows), nh, dh)
+        qc = _st16(linear(hc, w[p + "cq.w"], w[p + "cq.b"]), rnd).reshape(len(rows), nh, dh)
         kt, vt = kv["k_txt"][b], kv["v_txt"][b]
         ki, vi = kv["k_img"], kv["v_img"]
         o_img = attention(qc, ki.reshape(-1, nh, dh), vi.reshape(-1, nh, dh))

@@ -112,14 +112,16 @@ GEMM_SHAPES = [(300, 192, 72), (128, 256, 64), (1000, 384, 1536), (257, 64, 144)
 
 U32 = 2.0 ** -24          # fp32 unit roundoff
 BF16_HALF_ULP = 2.0 ** -8 # bf16 round-to-nearest: |round(v) - v| <= 2^-8 |v|
+F16_HALF_ULP = 2.0 ** -11 # IEEE half, normal range: |round(v) - v| <= 2^-11 |v|
+F16_SUB = 2.0 ** -25      # IEEE half below 2^-14: |round(v) - v| <= 2^-25
 
 
 def _gemm_case(wd, dtype, M, N, K, epi, seed=0):
     """Run one GEMM and return (got, exact, bound): an elementwise error bound
     derived from the arithmetic.  Accumulating K products in fp32 in any order
     errs by at most K*u*sum|a_k b_k| (u = 2^-24; doubled to allow truncating
-    adders); a bf16 store adds at most half an ulp, 2^-8 |v|; GELU has slope
-    below 1.13."""
+    adders); a bf16 store adds at most half an ulp, 2^-8 |v| (an IEEE half
+    store 2^-11 |v|, or 2^-25 below 2^-14); GELU has slope below 1.13."""
     rng = np.random.default_rng(seed + M + N + K + epi)
     A = rng.standard_normal((M, K)).astype(np.float32)
     B = (rng.standard_normal((N, K)) * 0.05).astype(np.float32)
@@ -138,14 +140,17 @@ def _gemm_case(wd, dtype, M, N, K, epi, seed=0):
         want = X0 + g * acc
         bound = np.abs(g) * acc_err + 2 * U32 * (np.abs(X0) + np.abs(g * acc))
     else:
-        out = torch.empty((M, N), device="cuda", dtype=torch.float32 if epi == wd.EPI_F32 else tdt)
+        odt = {wd.EPI_F32: torch.float32, wd.EPI_STORE_F16: torch.float16}.get(epi, tdt)
+        out = torch.empty((M, N), device="cuda", dtype=odt)
         if epi == wd.EPI_GELU:
             want = O.gelu(acc)
             bound = 1.13 * acc_err + 1e-6 * (np.abs(want) + 1.0)
         else:
             want = acc
             bound = acc_err + U32 * np.abs(want)
-        if epi != wd.EPI_F32 and is_bf:
+        if epi == wd.EPI_STORE_F16:
+            bound = bound * (1 + F16_HALF_ULP) + F16_HALF_ULP * np.abs(want) + F16_SUB
+        elif epi != wd.EPI_F32 and is_bf:
             bound = bound * (1 + BF16_HALF_ULP) + BF16_HALF_ULP * np.abs(want)
     wd.wd_gemm(dtype, M, N, K, dev(A, tdt), dev(B, tdt), dev(bias), epi, out,
                dev(ga) if epi == wd.EPI_RESID else None, dev(gb) if epi == wd.EPI_RESID else None)
@@ -177,10 +182,18 @@ def test_gemm_f32_cuda_cores(wd, M, N, K, epi):
     assert rel(got, want) < TOL_F32
 
 
-def test_gemm_bf16_simt_reference_kernel(wd):
+@pytest.mark.parametrize("M,N,K", [(2 * 512, 1536, 1536), (257, 5120, 5120), (97, 64, 144)])
+def test_gemm_bf16_half_store(wd, M, N, K):
+    """Epilogue 5: the cross-attention operands stored as IEEE half."""
+    got, want, bound = _gemm_case(wd, wd.WD_BF16, M, N, K, wd.EPI_STORE_F16)
+    assert_within(got, want, bound)
+
+
+@pytest.mark.parametrize("epi", [0, 5])
+def test_gemm_bf16_simt_reference_kernel(wd, epi):
     wd.wd_set_debug_flags(1)
     try:
-        got, want, bound = _gemm_case(wd, wd.WD_BF16, 300, 192, 72, 0)
+        got, want, bound = _gemm_case(wd, wd.WD_BF16, 300, 192, 72, epi)
     finally:
         wd.wd_set_debug_flags(0)
     assert_within(got, want, bound)
@@ -202,10 +215,11 @@ ATTN_CASES = [  # batch, Lq, heads, dh, n1, shared1, n2, shared2
 
 def _attn_case(wd, dtype, b, Lq, h, dh, n1, s1, n2, s2, seed=0):
     """Run one attention and return (got, exact, bound).  The exact value is
-    the oracle's attention on the same (bf16-representable) inputs, unrounded.
+    the oracle's attention on the same (representable) inputs, unrounded.
     Bound: a bf16 output store errs by at most 2^-8 |o|; probabilities stored
-    as bf16 before the P V product err by at most 2^-8 p each, which moves o
-    by at most 2^-8 * softmax(q k^T) |v| (doubled for the fp32 sums and ex2)."""
+    in the operand type before the P V product err by at most u p each
+    (u = 2^-8 for bf16, 2^-11 for IEEE half), which moves o by at most
+    u * softmax(q k^T) |v| (doubled for the fp32 sums and ex2)."""
     rng = np.random.default_rng(seed + Lq + n1 + n2 + dh)
     D = h * dh
     q = rng.standard_normal((b, Lq, D)).astype(np.float32)
@@ -215,13 +229,13 @@ def _attn_case(wd, dtype, b, Lq, h, dh, n1, s1, n2, s2, seed=0):
     if n2:
         k2 = rng.standard_normal(((1 if s2 else b), n2, D)).astype(np.float32)
         v2 = rng.standard_normal(((1 if s2 else b), n2, D)).astype(np.float32)
-    is_bf = dtype == wd.WD_BF16
-    if is_bf:
-        q, k1, v1 = bf(q), bf(k1), bf(v1)
-        if n2:
-            k2, v2 = bf(k2), bf(v2)
-    tdt = torch.bfloat16 if is_bf else torch.float32
-    o = torch.empty((b, Lq, D), device="cuda", dtype=tdt)
+    is_bf, is_half = dtype == wd.WD_BF16, dtype == wd.WD_F16
+    rnd = bf if is_bf else (lambda a: a.astype(np.float16).astype(np.float32)) if is_half else (lambda a: a)
+    q, k1, v1 = rnd(q), rnd(k1), rnd(v1)
+    if n2:
+        k2, v2 = rnd(k2), rnd(v2)
+    tdt = torch.bfloat16 if is_bf else torch.float16 if is_half else torch.float32
+    o = torch.empty((b, Lq, D), device="cuda", dtype=torch.bfloat16 if is_half else tdt)
     wd.wd_attention(dtype, b, Lq, h, dh, dev(q, tdt), dev(k1, tdt), dev(v1, tdt), n1, s1, o,
                     dev(k2, tdt) if n2 else None, dev(v2, tdt) if n2 else None, n2, s2)
     wd.wd_check()
@@ -239,8 +253,9 @@ def _attn_case(wd, dtype, b, Lq, h, dh, n1, s1, n2, s2, seed=0):
             ra = ra + O.attention(qq, kk.reshape(n, h, dh), np.abs(vv).reshape(n, h, dh))
         want[bb] = r.reshape(Lq, D)
         pv_abs[bb] = ra.reshape(Lq, D)
-    if is_bf:
-        bound = BF16_HALF_ULP * np.abs(want) + 2 * BF16_HALF_ULP * pv_abs + 1e-6
+    if is_bf or is_half:
+        u_p = BF16_HALF_ULP if is_bf else F16_HALF_ULP
+        bound = BF16_HALF_ULP * np.abs(want) + 2 * u_p * pv_abs + 1e-6
     else:
         bound = 1e-5 * (np.abs(want) + pv_abs)
     return host(o), want, bound
@@ -253,16 +268,24 @@ def test_attention_bf16(wd, case):
 
 
 @pytest.mark.parametrize("case", ATTN_CASES)
+def test_attention_half_operands(wd, case):
+    """IEEE half q/k/v (and P), bf16 output: the bf16 model's cross-attention."""
+    got, want, bound = _attn_case(wd, wd.WD_F16, *case)
+    assert_within(got, want, bound)
+
+
+@pytest.mark.parametrize("case", ATTN_CASES)
 def test_attention_f32(wd, case):
     got, want, bound = _attn_case(wd, wd.WD_F32, *case)
     assert_within(got, want, bound)
     assert rel(got, want) < TOL_F32
 
 
-def test_attention_bf16_simt_reference_kernel(wd):
+@pytest.mark.parametrize("half", [0, 1])
+def test_attention_bf16_simt_reference_kernel(wd, half):
     wd.wd_set_debug_flags(2)
     try:
-        got, want, bound = _attn_case(wd, wd.WD_BF16, 2, 130, 3, 128, 257, 1, 512, 0)
+        got, want, bound = _attn_case(wd, wd.WD_F16 if half else wd.WD_BF16, 2, 130, 3, 128, 257, 1, 512, 0)
     finally:
         wd.wd_set_debug_flags(0)
     assert_within(got, want, bound)

@@ -113,19 +113,23 @@ def test_small_bf16_forward(mods):
 
 # ------------------------------------------------------------------ single bf16 blocks on sampled rows
 def _block_parity(mods, wl, n_rows, tau):
+    """Patch embedding (every element), then one block on sampled rows.  The
+    block's inputs X_in and e0 come from the oracle (rounded to fp32, the
+    residual stream's storage type) and are handed to both sides."""
     model, wd = mods
     net, w, x, txt, y, d = setup(mods, wl, blocks=[0])
     B, L, D = wl.batch, d.L, d.D
     x_t = np.stack([x["x0"]] * B)
+    X_in = O.patch_embed(x_t, O.build_cond_y(x["img_lat"]), w["pe.w"], w["pe.b"], rnd=True)
     # patch embedding (full size, every element)
-    wd.wd_time_mod(net.cd, net.time_w, tau, net.e, net.e0)
     wd.wd_patch_embed(net.cd, dev(x_t), y, net.w["pe.w"], net.w["pe.b"], B, net.X, net.ws)
     wd.wd_check()
-    X_in = host(net.X)
-    want_pe = O.patch_embed(x_t, O.build_cond_y(x["img_lat"]), w["pe.w"], w["pe.b"], rnd=True)
-    assert rel(X_in, want_pe) < TOL_BF16
-    e0 = host(net.e0)
-    # one block
+    assert rel(host(net.X), X_in) < TOL_BF16
+    # one block, from the oracle's X_in and e0
+    X_in = X_in.astype(np.float32).astype(np.float64)
+    e0 = O.time_mod(w, tau, D)[1].astype(np.float32).astype(np.float64)
+    net.X.copy_(dev(X_in))
+    net.e0.copy_(dev(e0))
     wd.wd_block_forward(net.cd, net.block_w[0], net.e0, net.kv[0], B, net.X, net.ws)
     wd.wd_check()
     X_out = host(net.X)

@@ -36,6 +36,23 @@ def test_bf16_round_matches_torch_conversion():
     np.testing.assert_array_equal(O.bf16(a), want)
 
 
+def test_fp16_round_matches_numpy_half():
+    # normals, subnormals (|a| < 2**-14), overflow to infinity (> 65504)
+    a = RNG.standard_normal(20000) * np.exp(RNG.uniform(-25, 12, 20000))
+    # exact ties halfway between neighbouring halves, both parities of the kept bit
+    h = RNG.integers(1, 0x7BFF, 4000, dtype=np.uint16)
+    lo = h.view(np.float16).astype(np.float64)
+    hi = (h + 1).view(np.float16).astype(np.float64)
+    ties = (lo + hi) / 2
+    a = np.concatenate([a, ties, -ties, [0.0, -0.0, 65504.0, 65519.0, 65520.0, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -26]])
+    with np.errstate(over="ignore"):
+        want = a.astype(np.float16).astype(np.float64)
+    np.testing.assert_array_equal(O.fp16(a), want)
+    # ties go to the even neighbour
+    even = np.where(h % 2 == 0, lo, hi)
+    np.testing.assert_array_equal(O.fp16(ties), even)
+
+
 # ------------------------------------------------------------------ shapes printed on the pages
 def test_key_numbers():
     k = GOLD["key_numbers"]
