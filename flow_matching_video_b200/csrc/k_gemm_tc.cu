@@ -27,12 +27,6 @@ constexpr int BM = 128, BK = 64;
 #define WD_GEMM_EPI_WG 1   // epilogue warpgroups; each takes an equal share of the tile's columns
 #endif
 constexpr int EPI_WG = WD_GEMM_EPI_WG;
-#ifndef WD_GEMM_RESID_PIPE
-#define WD_GEMM_RESID_PIPE 1   // residual epilogue loads one chunk ahead
-#endif
-#ifndef WD_GEMM_RESID_PREFETCH
-#define WD_GEMM_RESID_PREFETCH 0   // producer prefetches each tile's fp32 residual block into L2
-#endif
 constexpr int THREADS = 64 + 128 * EPI_WG;
 
 template <int BN>
@@ -43,7 +37,11 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  // gated residual: per epilogue warp two 32 x 32 fp32 staging tiles for the TMA reduce-add
+  static constexpr int RESID_STAGE_BYTES = 32 * 32 * 4;
+  static constexpr int STG_BYTES = 4 * EPI_WG * 2 * RESID_STAGE_BYTES;
+  static constexpr int smem(int mode) { return 1024 + STAGES * STAGE_BYTES + (mode == EPI_RESID ? STG_BYTES : 0) + BAR_BYTES; }
+  static_assert(1024 + STAGES * STAGE_BYTES + STG_BYTES + BAR_BYTES <= 232448, "shared memory budget of one CTA exceeded");
   static constexpr uint32_t IDESC = idesc_bf16(BM, BN, 0, 0);
 };
 
@@ -53,8 +51,7 @@ enum : unsigned { SITE_EMPTY = 0x101, SITE_FULL = 0x102, SITE_TFULL = 0x103, SIT
 // ------------------------------------------------------------------ epilogue on 32 columns
 // One thread = one output row m; columns n .. n+31 come from the accumulator.
 template <int MODE>
-__device__ __forceinline__ void epilogue32(const Epi& ep, int64_t m, int n, const uint32_t (&r)[32],
-                                           const float4 (&xres)[8]) {
+__device__ __forceinline__ void epilogue32(const Epi& ep, int64_t m, int n, const uint32_t (&r)[32]) {
   float v[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
@@ -87,23 +84,6 @@ __device__ __forceinline__ void epilogue32(const Epi& ep, int64_t m, int n, cons
     float4* dst = reinterpret_cast<float4*>(static_cast<float*>(ep.out) + m * ep.ldo + n);
 #pragma unroll
     for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-  } else if constexpr (MODE == EPI_RESID) {
-    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(ep.out) + m * ep.ldo + n);
-    const bool gated = ep.gate_a || ep.gate_b;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float4 g = make_float4(1.f, 1.f, 1.f, 1.f);
-      if (gated) {
-        const float4 ga = ep.gate_a ? __ldg(reinterpret_cast<const float4*>(ep.gate_a + n + 4 * j))
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 gb = ep.gate_b ? __ldg(reinterpret_cast<const float4*>(ep.gate_b + n + 4 * j))
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-        g = make_float4(ga.x + gb.x, ga.y + gb.y, ga.z + gb.z, ga.w + gb.w);
-      }
-      float4 x = xres[j];
-      x.x += g.x * v[4 * j]; x.y += g.y * v[4 * j + 1]; x.z += g.z * v[4 * j + 2]; x.w += g.w * v[4 * j + 3];
-      dst[j] = x;
-    }
   } else {   // EPI_UNPATCH
     float* out = static_cast<float*>(ep.out);
 #pragma unroll
@@ -121,7 +101,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::STAGES * C::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+  float* stg = reinterpret_cast<float*>(sB + C::STAGES * C::B_BYTES);   // 1024-byte aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES + (MODE == EPI_RESID ? C::STG_BYTES : 0));
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;   // [2]
   uint64_t* tempty = tfull + 2;          // [2]
@@ -157,9 +138,6 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       bool ok = true;
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
         const int m0 = (t / n_tiles) * BM, n0 = (t % n_tiles) * BN;
-        // the epilogue of this tile reads and rewrites X[m0:m0+128, n0:n0+BN]
-        // one mainloop from now: have it in L2 by then
-        if (MODE == EPI_RESID && WD_GEMM_RESID_PREFETCH) tma_prefetch_l2_2d(&tmX, n0, m0);
         for (int k = 0; k < k_iters; ++k) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, SITE_EMPTY)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
@@ -214,46 +192,56 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     const int c_begin = ((warp - 2) >> 2) * COLS;
     int acc = 0;
     uint32_t acc_phase = 0;
+    [[maybe_unused]] uint32_t chunk = 0;   // residual staging tiles used so far (alternating)
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
       const int m0 = (t / n_tiles) * BM, n0 = (t % n_tiles) * BN;
       if (!mbar_wait_warp(&tfull[acc], acc_phase, SITE_TFULL)) break;
       tc_fence_after();
       const int64_t m = m0 + q * 32 + lane;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
-      if constexpr (MODE == EPI_RESID && WD_GEMM_RESID_PIPE) {
-        // residual loads run one 32-column chunk ahead of the TMEM reads
-        const float4* row_x = reinterpret_cast<const float4*>(static_cast<float*>(ep.out) + m * ep.ldo + n0);
-        float4 xres[2][8];
-        if (m < M) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) xres[0][j] = row_x[c_begin / 4 + j];
-        }
-#pragma unroll
-        for (int c = c_begin, i = 0; c < c_begin + COLS; c += 32, ++i) {
-          if (c + 32 < c_begin + COLS && m < M) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) xres[(i + 1) & 1][j] = row_x[(c + 32) / 4 + j];
-          }
+      if constexpr (MODE == EPI_RESID) {
+        // X[m, n] += g[n] * v through the TMA: this warp's 32 rows x 32 columns
+        // go to a 128-byte-swizzled staging tile (row `lane`, 16-byte chunk j
+        // at chunk j ^ (lane & 7)), then one lane reduces the tile into X in
+        // L2, so no residual load waits in the SM.
+        const bool gated = ep.gate_a || ep.gate_b;
+#pragma unroll 1
+        for (int c = c_begin; c < c_begin + COLS; c += 32) {
           uint32_t r[32];
           tmem_ld32(tbase + c, r);
+          float* tile = stg + ((warp - 2) * 2 + (chunk & 1)) * (32 * 32);
+          if (lane == 0) bulk_wait_group_read<1>();   // the reduce that last read this tile is done with it
+          __syncwarp();
           tmem_wait_ld();
-          if (m < M) epilogue32<MODE>(ep, m, n0 + c, r, xres[i & 1]);
+          float4* row = reinterpret_cast<float4*>(tile + lane * 32);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int n = n0 + c + 4 * j;
+            float4 g = make_float4(1.f, 1.f, 1.f, 1.f);
+            if (gated) {
+              const float4 ga = ep.gate_a ? __ldg(reinterpret_cast<const float4*>(ep.gate_a + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
+              const float4 gb = ep.gate_b ? __ldg(reinterpret_cast<const float4*>(ep.gate_b + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
+              g = make_float4(ga.x + gb.x, ga.y + gb.y, ga.z + gb.z, ga.w + gb.w);
+            }
+            const float4 bb = ep.bias ? __ldg(reinterpret_cast<const float4*>(ep.bias + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            row[j ^ (lane & 7)] = make_float4(g.x * (__uint_as_float(r[4 * j]) + bb.x), g.y * (__uint_as_float(r[4 * j + 1]) + bb.y),
+                                              g.z * (__uint_as_float(r[4 * j + 2]) + bb.z), g.w * (__uint_as_float(r[4 * j + 3]) + bb.w));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && m0 + q * 32 < M) {   // rows past M inside the box are skipped by the TMA
+            tma_reduce_add_2d(tile, &tmX, n0 + c, m0 + q * 32);
+            bulk_commit_group();
+          }
+          ++chunk;
         }
       } else {
 #pragma unroll 1
         for (int c = c_begin; c < c_begin + COLS; c += 32) {
-          float4 xres[8];
-          if constexpr (MODE == EPI_RESID) {   // residual loads in flight while TMEM is read
-            if (m < M) {
-              const float4* src = reinterpret_cast<const float4*>(static_cast<float*>(ep.out) + m * ep.ldo + n0 + c);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) xres[j] = src[j];
-            }
-          }
           uint32_t r[32];
           tmem_ld32(tbase + c, r);
           tmem_wait_ld();
-          if (m < M) epilogue32<MODE>(ep, m, n0 + c, r, xres);
+          if (m < M) epilogue32<MODE>(ep, m, n0 + c, r);
         }
       }
       tc_fence_before();
@@ -261,6 +249,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       if (lane == 0) mbar_arrive(&tempty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (MODE == EPI_RESID && lane == 0) bulk_wait_group<0>();   // reductions performed before exit
   }
 
   tc_fence_before();
@@ -309,8 +298,8 @@ static int sm_count() {
   return cnt[dev & 15];
 }
 
-// 2D fp32 tensor map over the residual stream [rows, cols], box BN x 128, no swizzle
-// (used only for L2 prefetches).
+// 2D fp32 tensor map over the residual stream [rows, cols], box_cols x box_rows,
+// 128-byte swizzle (box_cols = 32: one 128-byte row per box row).
 static wd_status make_tmap_f32(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_cols,
                                int box_rows) {
   auto fn = encode_fn();
@@ -320,7 +309,7 @@ static wd_status make_tmap_f32(CUtensorMap* m, const void* base, int64_t rows, i
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t es[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) { set_error("cuTensorMapEncodeTiled (f32) failed (%d)", static_cast<int>(r)); return WD_ERR_CUDA; }
   return WD_OK;
@@ -334,15 +323,15 @@ static wd_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const E
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr[dev & 15]) {
-    cudaFuncSetAttribute(tcg::k_gemm_tc<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaFuncSetAttribute(tcg::k_gemm_tc<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::smem(MODE));
     attr[dev & 15] = true;
   }
   const int tiles = ((M + tcg::BM - 1) / tcg::BM) * (N / BN);
   const int grid = tiles < sm_count() ? tiles : sm_count();
   CUtensorMap tx = ta;   // unused unless the epilogue adds into the fp32 residual
-  if (MODE == EPI_RESID) WD_TRY(make_tmap_f32(&tx, ep.out, M, N, ep.ldo, BN, tcg::BM));
+  if (MODE == EPI_RESID) WD_TRY(make_tmap_f32(&tx, ep.out, M, N, ep.ldo, 32, 32));
   Trace tr(KC_GEMM, st);
-  tcg::k_gemm_tc<BN, MODE><<<grid, tcg::THREADS, C::SMEM, st>>>(ta, tb, tx, ep, M, N, K);
+  tcg::k_gemm_tc<BN, MODE><<<grid, tcg::THREADS, C::smem(MODE), st>>>(ta, tb, tx, ep, M, N, K);
   return launch_status("gemm_tc");
 }
 
