@@ -22,7 +22,10 @@
 //                    units; the final 1/l keeps the result exact), then the
 //                    normalised output written out.
 // With NQ = 2 the two tiles ping-pong: while one tile's warps run their
-// softmax, the tensor cores compute the other tile's P V and next S.
+// softmax, the tensor cores compute the other tile's P V and next S.  With
+// two key segments (one Q tile: its O and O' take half of TMEM) S is double
+// buffered instead: S of block n + 1 is computed while the softmax works on
+// block n, and P V of block n runs while it works on block n + 1.
 #include "wd_internal.cuh"
 
 namespace wd {
@@ -58,9 +61,16 @@ struct Cfg {
   static constexpr int SMEM = 1024 + BAR_OFF + 512;
   static_assert(SMEM <= 232448, "shared memory budget of one CTA exceeded (reduce WD_ATTN_RING)");
   static constexpr int TMEM_COLS = 512;
-  // TMEM columns: S_t, O_t (per tile); with two segments one tile has O and O'
-  __host__ __device__ static constexpr int s_col(int t) { return NSEG == 1 ? t * 256 : 0; }
-  __host__ __device__ static constexpr int o_col(int t, int seg) { return NSEG == 1 ? t * 256 + 128 : 128 + 128 * seg; }
+  // TMEM columns.  One segment: S_t, O_t per tile (two tiles).  Two segments
+  // (one tile): O and O' in the middle and two S buffers, so that S of block
+  // n + 1 is computed while the softmax works on block n.
+  static constexpr bool DB = NSEG == 2;   // double-buffered S
+  static_assert(!DB || NQ == 1, "two key segments use one Q tile");
+  static constexpr int NBUF = DB ? 2 : NQ;   // S/P buffers (and their barriers)
+  __host__ __device__ static constexpr int buf(int t, int n) { return DB ? (n & 1) : t; }
+  __host__ __device__ static constexpr uint32_t par(int n) { return DB ? ((n >> 1) & 1u) : (n & 1u); }
+  __host__ __device__ static constexpr int s_col(int t, int n) { return DB ? ((n & 1) ? 384 : 0) : t * 256; }
+  __host__ __device__ static constexpr int o_col(int t, int seg) { return DB ? 128 + 128 * seg : t * 256 + 128; }
   // Q K^T: both K-major; P V: P from TMEM, V MN-major (dh contiguous).  P is
   // held in the operands' type (A and B of one MMA share their type).
   static constexpr bool HALF = std::is_same<TI, f16>::value;
@@ -142,10 +152,11 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   uint64_t* q_full = bars;                 // 1
   uint64_t* kv_full = bars + 1;            // RING
   uint64_t* kv_empty = kv_full + RING;     // RING
-  uint64_t* s_full = kv_empty + RING;      // NQ
-  uint64_t* p_full = s_full + NQ;          // NQ: all of P_t written
-  uint64_t* p_half = p_full + NQ;          // NQ: keys 0-63 of P_t written
-  uint64_t* o_done = p_half + NQ;          // NQ
+  uint64_t* s_full = kv_empty + RING;      // NBUF
+  uint64_t* p_full = s_full + C::NBUF;     // NBUF: all of P written
+  uint64_t* p_half = p_full + C::NBUF;     // NBUF: keys 0-63 of P written
+  uint64_t* pv_done = p_half + C::NBUF;    // NBUF: P V of the block in that buffer completed (double buffering)
+  uint64_t* o_done = pv_done + C::NBUF;    // NQ
   uint64_t* tdone = o_done + NQ;           // 1
   uint64_t* mx_bar = tdone + 1;            // NQ x 4: the two warps of a lane quarter swap row maxima
   uint64_t* fin_bar = mx_bar + 4 * NQ;     // NQ x 4: ... and their row sums at the end
@@ -165,12 +176,13 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < RING; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
-    for (int t = 0; t < NQ; ++t) {
-      mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], C::SM_WARPS);
-      mbar_init(&p_half[t], C::SM_WARPS);
-      mbar_init(&o_done[t], 1);
+    for (int i = 0; i < C::NBUF; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], C::SM_WARPS);
+      mbar_init(&p_half[i], C::SM_WARPS);
+      mbar_init(&pv_done[i], 1);
     }
+    for (int t = 0; t < NQ; ++t) mbar_init(&o_done[t], 1);
     mbar_init(tdone, 1);
     for (int i = 0; i < 4 * NQ; ++i) { mbar_init(&mx_bar[i], 2); mbar_init(&fin_bar[i], 2); }
     fence_mbar_init();
@@ -222,21 +234,22 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       tc_fence_after();
       const uint32_t q0 = smem_u32(smem + C::Q_OFF);
       const uint32_t r0 = smem_u32(smem + C::RING_OFF);
-      // P_t V_j for block n-1 of tile t
+      // P_t V_j for block n of tile t
       auto issue_pv = [&](int t, int n) -> bool {
         const int vseq = 2 * n + 1, vslot = vseq % RING;
         const int sg = n < nb0 ? 0 : 1;
         const int first = (n == 0) || (n == nb0);
+        const int bi = C::buf(t, n);
         const uint32_t d = tmem + C::o_col(t, sg);
-        const uint32_t pa = tmem + C::s_col(t), vb = r0 + vslot * TILE_BYTES;
+        const uint32_t pa = tmem + C::s_col(t, n), vb = r0 + vslot * TILE_BYTES;
         // With one softmax warp per lane quarter, P arrives in two halves (keys
         // 0-63, then 64-127): the first four k-steps start as soon as the first
         // half is in TMEM.
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           if (SPLIT == 1 || half == 0) {
-            uint64_t* bar = (SPLIT == 1 && half == 0) ? &p_half[t] : &p_full[t];
-            if (!MMA_WAIT(bar, n & 1u, SITE_P)) return false;
+            uint64_t* bar = (SPLIT == 1 && half == 0) ? &p_half[bi] : &p_full[bi];
+            if (!MMA_WAIT(bar, C::par(n), SITE_P)) return false;
           }
           if (half == 0 && !MMA_WAIT(&kv_full[vslot], (vseq / RING) & 1u, SITE_KVF)) return false;
           tc_fence_after();
@@ -250,33 +263,60 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     (!first || kk) ? 1u : 0u);
           }
         }
+        if (C::DB) umma_commit(&pv_done[bi]);
         if (t == NQ - 1) umma_commit(&kv_empty[vslot]);
         return true;
       };
-      for (int n = 0; n < NB && ok; ++n) {
-        const int kseq = 2 * n, kslot = kseq % RING;
-        for (int t = 0; t < NQ && ok; ++t) {
-          // P_t V of the previous block first: it needs only P_t and that V tile,
-          // not the next K tile.
-          if (n > 0 && !issue_pv(t, n - 1)) { ok = false; break; }
-          if (t == 0) {
-            if (!MMA_WAIT(&kv_full[kslot], (kseq / RING) & 1u, SITE_KVF)) { ok = false; break; }
-            tc_fence_after();
-          }
-          const uint32_t d = tmem + C::s_col(t);
-          const uint32_t qa = q0 + t * TILE_BYTES, kb = r0 + kslot * TILE_BYTES;
+      // S_t = Q_t K_n^T into tile t's S buffer for block n (K tile already waited for)
+      auto issue_s = [&](int t, int n) {
+        const int kslot = (2 * n) % RING;
+        const uint32_t d = tmem + C::s_col(t, n);
+        const uint32_t qa = q0 + t * TILE_BYTES, kb = r0 + kslot * TILE_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-            umma_ss(d, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), C::IDESC_S, kk ? 1u : 0u);
-          }
-          umma_commit(&s_full[t]);
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+          umma_ss(d, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), C::IDESC_S, kk ? 1u : 0u);
         }
-        if (ok) umma_commit(&kv_empty[kslot]);
-      }
-      for (int t = 0; t < NQ && ok; ++t) {
-        if (!issue_pv(t, NB - 1)) { ok = false; break; }
-        umma_commit(&o_done[t]);
+        umma_commit(&s_full[C::buf(t, n)]);
+      };
+      auto wait_k = [&](int n) -> bool {
+        const int kseq = 2 * n;
+        if (!MMA_WAIT(&kv_full[kseq % RING], (kseq / RING) & 1u, SITE_KVF)) return false;
+        tc_fence_after();
+        return true;
+      };
+      if constexpr (C::DB) {
+        // One tile, two S buffers: S of blocks 0 and 1 first; then per block
+        // P V, and S of the block two ahead into the buffer that P V has read.
+        for (int n = 0; n < 2 && n < NB && ok; ++n) {
+          if (!wait_k(n)) { ok = false; break; }
+          issue_s(0, n);
+          umma_commit(&kv_empty[(2 * n) % RING]);
+        }
+        for (int n = 0; n < NB && ok; ++n) {
+          if (!issue_pv(0, n)) { ok = false; break; }
+          if (n + 2 < NB) {
+            if (!wait_k(n + 2)) { ok = false; break; }
+            issue_s(0, n + 2);
+            umma_commit(&kv_empty[(2 * (n + 2)) % RING]);
+          }
+        }
+        if (ok) umma_commit(&o_done[0]);
+      } else {
+        for (int n = 0; n < NB && ok; ++n) {
+          for (int t = 0; t < NQ && ok; ++t) {
+            // P_t V of the previous block first: it needs only P_t and that V tile,
+            // not the next K tile.
+            if (n > 0 && !issue_pv(t, n - 1)) { ok = false; break; }
+            if (t == 0 && !wait_k(n)) { ok = false; break; }
+            issue_s(t, n);
+          }
+          if (ok) umma_commit(&kv_empty[(2 * n) % RING]);
+        }
+        for (int t = 0; t < NQ && ok; ++t) {
+          if (!issue_pv(t, NB - 1)) { ok = false; break; }
+          umma_commit(&o_done[t]);
+        }
       }
       umma_commit(tdone);
       mbar_wait(tdone, 0, SITE_DRAIN);
@@ -291,7 +331,6 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const int quarter = warp & 3;          // TMEM lanes this warp may access
     const int r = quarter * 32 + lane;     // query row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t s_addr = tmem + lane_base + C::s_col(t) + hc * COLS;
     [[maybe_unused]] uint64_t* my_mx = &mx_bar[t * 4 + quarter];
     float m = -INFINITY, l = 0.f, l_first = 0.f;
     bool ok = true;
@@ -299,7 +338,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       const int sg = n < nb0 ? 0 : 1;
       const bool first = (n == 0) || (n == nb0);
       if (NSEG == 2 && n == nb0) { l_first = l; m = -INFINITY; l = 0.f; }
-      if (!SM_WAIT(&s_full[t], n & 1u, SITE_S)) { ok = false; break; }
+      const int bi = C::buf(t, n);
+      const uint32_t s_addr = tmem + lane_base + C::s_col(t, n) + hc * COLS;
+      if (!SM_WAIT(&s_full[bi], C::par(n), SITE_S)) { ok = false; break; }
       tc_fence_after();
       // keys of this block that exist, counted from this warp's first column
       const int valid = (sg ? nk1 : nk0) - (n - (sg ? nb0 : 0)) * BKV - hc * COLS;
@@ -339,9 +380,13 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       m = m_new;
       const float neg_m = -m;
       // O_t *= alpha on this warp's output columns for rows whose reference
-      // max moved, before any of this block's P V can start (P V of the previous
-      // block has completed: its commit precedes the S commit waited on above)
+      // max moved, before any of this block's P V can start.  With one S
+      // buffer per tile, P V of the previous block has completed (its commit
+      // precedes the S commit waited on above); with two, S of this block was
+      // issued before that P V, so wait for it.
       if (__any_sync(0xffffffffu, grow) && !first) {
+        if (C::DB && !mbar_wait_warp(&pv_done[C::buf(t, n - 1)], C::par(n - 1), SITE_O)) { ok = false; break; }
+        if (C::DB) tc_fence_after();
         const uint32_t o_addr = tmem + lane_base + C::o_col(t, sg) + hc * COLS;
 #pragma unroll 1
         for (int c = 0; c < CH; ++c) {
@@ -377,14 +422,14 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&p_half[t]);
+          if (lane == 0) mbar_arrive(&p_half[bi]);
         }
       }
       tmem_wait_st();
       l = l * alpha + (rs2.x + rs2.y);     // this warp's share of the row sum
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[t]);
+      if (lane == 0) mbar_arrive(&p_full[bi]);
     }
     // ---------------------------------------------------------- epilogue
     if (SPLIT == 2 && ok) {
