@@ -320,6 +320,7 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return 0
     pk = peaks()
+    wbytes = sum(t.numel() * t.element_size() for t in weights.values())
     flops = step_flops(d, B)
     tflops = flops / (ms / 1e3) / 1e12
     # roofline of the dominant kernel (self-attention), timed live with events
@@ -341,12 +342,15 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "video": "81 frames 480x832", "latent": [16, d.T, d.H, d.W],
+        "config": {"workload": wl.name, "video": f"{4 * (d.T - 1) + 1} frames {8 * d.H}x{8 * d.W}",
+                   "latent": [16, d.T, d.H, d.W],
                    "tokens": d.L, "batch": B, "blocks": d.blocks, "D": d.D, "heads": d.heads, "ffn": d.ffn,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "no flush: per-step working set (3.1 GB weights, 0.4 GB residual stream) exceeds L2"},
+                   "l2": (f"no flush: per-step working set ({wbytes / 1e9:.1f} GB weights, "
+                          f"{net.X.numel() * 4 / 1e9:.1f} GB residual stream) exceeds L2")},
         "tflops": tflops, "pct_bf16_peak": tflops / pk["bf16_tflops"],
         "pct_bf16_peak_sustained": tflops / peak_s, "s_per_step": ms / 1e3,
+        "s_per_video_latent": ms / 1e3 * wl.steps,   # the workload's Euler steps of one video
         "e2e": {"value": value_e2e, "unit": "tokens/s",
                 "h2d_bytes_per_step": x_host.numel() * 4, "d2h_bytes_per_step": out_host.numel() * 4},
         "gpu_launches": launches,
