@@ -509,7 +509,7 @@ static wd_status make_tmap_3d(CUtensorMap* m, CUtensorMapDataType type, const vo
 template <int NQ, int NSEG, typename TI>
 static wd_status launch_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk0, const CUtensorMap& tv0,
                                 const CUtensorMap& tk1, const CUtensorMap& tv1, const tca::Params& p, int batch,
-                                int heads, cudaStream_t st) {
+                                int heads, bool cross, cudaStream_t st) {
   using C = tca::Cfg<NQ, NSEG, TI>;
   static bool attr[16] = {};
   int dev = 0;
@@ -519,7 +519,7 @@ static wd_status launch_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk0, c
     attr[dev & 15] = true;
   }
   dim3 grid((p.Lq + tca::BQ * NQ - 1) / (tca::BQ * NQ), heads, batch);
-  Trace tr(NSEG == 2 ? KC_ATTN_CROSS : KC_ATTN_SELF, st);
+  Trace tr(cross ? KC_ATTN_CROSS : KC_ATTN_SELF, st);
   tca::k_attn_tc<NQ, NSEG, TI><<<grid, C::THREADS, C::SMEM, st>>>(tq, tk0, tv0, tk1, tv1, p);
   return launch_status("attention_tc");
 }
@@ -557,9 +557,9 @@ static wd_status attention_tc_t(const AttnArgs<TI, bf16>& a, cudaStream_t st) {
     WD_TRY(make_tmap_3d(&tk1, ty, a.k2, D, a.n2, b2, a.kv2_rs, a.kv2_bs));
     WD_TRY(make_tmap_3d(&tv1, ty, a.v2, D, a.n2, b2, a.kv2_rs, a.kv2_bs));
     p.seg[1] = tca::Seg{a.n2, a.kv2_bs == 0};
-    return launch_attn_tc<1, 2, TI>(tq, tk0, tv0, tk1, tv1, p, a.batch, a.heads, st);
+    return launch_attn_tc<1, 2, TI>(tq, tk0, tv0, tk1, tv1, p, a.batch, a.heads, a.cross, st);
   }
-  return launch_attn_tc<2, 1, TI>(tq, tk0, tv0, tk0, tv0, p, a.batch, a.heads, st);
+  return launch_attn_tc<2, 1, TI>(tq, tk0, tv0, tk0, tv0, p, a.batch, a.heads, a.cross, st);
 }
 
 wd_status attention_tc(const AttnArgs<bf16, bf16>& a, cudaStream_t st) { return attention_tc_t<bf16>(a, st); }

@@ -210,7 +210,7 @@ static wd_status launch_attn_simt(const AttnArgs<T, TO>& a, cudaStream_t st) {
   }
   dim3 grid((a.Lq + 63) / 64, a.heads, a.batch);
   const float qscale = 1.4426950408889634f / sqrtf(static_cast<float>(DH));
-  Trace tr(a.k2 ? KC_ATTN_CROSS : KC_ATTN_SELF, st);
+  Trace tr(a.cross ? KC_ATTN_CROSS : KC_ATTN_SELF, st);
   k_attn_simt<T, TO, DH><<<grid, 256, smem, st>>>(a, qscale);
   return launch_status("attention_simt");
 }

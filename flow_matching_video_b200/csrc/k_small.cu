@@ -301,19 +301,20 @@ wd_status qknorm_rope(T* qkv, int64_t rows, const wd_dims& d, const float* gq, c
 
 // ============================================================ patch gather
 // a[m, k] for m = b*L + l and k = c*4 + kh*2 + kw: the (1,2,2) receptive field
-// of token l in the 36-channel input concat(x_t[16], y[20])
-// ("图解 Wan2.1 I2V" 4.2 and 5.1); y is shared by the batch.
+// of token l in the 36-channel input concat(x_t[16], y[20]) (K = 144,
+// "图解 Wan2.1 I2V" 4.2 and 5.1; y is shared by the batch), or in x_t alone
+// for the text-to-video model (K = 64, section 9 of the same page).
 template <typename T>
 __global__ void __launch_bounds__(256) k_patch_gather(const float* __restrict__ xt, const float* __restrict__ y, int B,
-                                                      int Tn, int H, int W, T* __restrict__ a) {
+                                                      int Tn, int H, int W, int K, T* __restrict__ a) {
   const int Hp = H / 2, Wp = W / 2;
   const int64_t L = static_cast<int64_t>(Tn) * Hp * Wp;
-  const int64_t n = static_cast<int64_t>(B) * L * 144;
+  const int64_t n = static_cast<int64_t>(B) * L * K;
   const int64_t HW = static_cast<int64_t>(H) * W, plane = Tn * HW;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int k = static_cast<int>(i % 144);
-    const int64_t m = i / 144;
+    const int k = static_cast<int>(i % K);
+    const int64_t m = i / K;
     const int64_t b = m / L;
     const int l = static_cast<int>(m - b * L);
     const int x = l % Wp, yy = (l / Wp) % Hp, f = l / (Wp * Hp);

@@ -52,7 +52,8 @@ static wd_status check_dims(const wd_dims* d) {
     set_error("latent grid T=%d H=%d W=%d (T<=256, H and W even)", d->T, d->H, d->W);
     return WD_ERR_SHAPE;
   }
-  if (d->n_txt <= 0 || d->n_img <= 0 || d->c_txt <= 0 || d->c_img <= 0 || (d->c_txt % 8) || (d->c_img % 8)) {
+  // n_img = 0 selects the text-to-video model (no image branch, c_img unused)
+  if (d->n_txt <= 0 || d->n_img < 0 || d->c_txt <= 0 || (d->c_txt % 8) || (d->n_img > 0 && (d->c_img <= 0 || d->c_img % 8))) {
     set_error("context sizes n_txt=%d c_txt=%d n_img=%d c_img=%d", d->n_txt, d->c_txt, d->n_img, d->c_img);
     return WD_ERR_SHAPE;
   }
@@ -67,6 +68,9 @@ static wd_status check_batch(int batch) {
 
 static int64_t tokens(const wd_dims* d) { return static_cast<int64_t>(d->T) * (d->H / 2) * (d->W / 2); }
 static size_t esize(const wd_dims* d) { return d->dtype == WD_BF16 ? 2 : 4; }
+// Patch width of the patch embedding: 36 input channels x (1,2,2) for the
+// image-to-video model, 16 x (1,2,2) for the text-to-video model (n_img = 0).
+static int patch_k(const wd_dims* d) { return d->n_img > 0 ? 144 : 64; }
 static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Workspace layout (each part 256-byte aligned):
@@ -185,8 +189,13 @@ static wd_status block_forward_t(const wd_dims* d, const wd_block_weights* w, co
   {
     AttnArgs<CT, T> a{};
     a.q = reinterpret_cast<const CT*>(A); a.q_rs = D;
-    a.k1 = k_img; a.v1 = v_img; a.kv1_rs = D; a.kv1_bs = 0; a.n1 = d->n_img;
-    a.k2 = k_txt; a.v2 = v_txt; a.kv2_rs = D; a.kv2_bs = static_cast<int64_t>(d->n_txt) * D; a.n2 = d->n_txt;
+    a.cross = true;
+    if (d->n_img > 0) {
+      a.k1 = k_img; a.v1 = v_img; a.kv1_rs = D; a.kv1_bs = 0; a.n1 = d->n_img;
+      a.k2 = k_txt; a.v2 = v_txt; a.kv2_rs = D; a.kv2_bs = static_cast<int64_t>(d->n_txt) * D; a.n2 = d->n_txt;
+    } else {   // text-to-video: one stream, text keys only ("图解 Wan2.1 I2V" 9)
+      a.k1 = k_txt; a.v1 = v_txt; a.kv1_rs = D; a.kv1_bs = static_cast<int64_t>(d->n_txt) * D; a.n1 = d->n_txt;
+    }
     a.o = Bf; a.o_rs = D;
     a.batch = batch; a.Lq = static_cast<int>(L); a.heads = d->heads; a.dh = dh;
     WD_TRY(attention(a, st));
@@ -320,9 +329,9 @@ wd_status wd_context_embed(const wd_dims* d, const wd_ctx_weights* w, const void
   WD_TRY(check_batch(batch));
   if (!w) { set_error("ctx weights NULL"); return WD_ERR_ARG; }
   WD_NEED(w->txt1_w); WD_NEED(w->txt1_b); WD_NEED(w->txt2_w); WD_NEED(w->txt2_b);
-  WD_NEED(w->img1_w); WD_NEED(w->img1_b); WD_NEED(w->img2_w); WD_NEED(w->img2_b);
+  const bool img = d->n_img > 0;   // the text-to-video model has no CLIP branch
+  if (img) { WD_NEED(w->img1_w); WD_NEED(w->img1_b); WD_NEED(w->img2_w); WD_NEED(w->img2_b); WD_NEED(clip); }
   WD_NEED(txt);
-  WD_NEED(clip);
   WD_NEED(ctx);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int D = d->D;
@@ -335,13 +344,17 @@ wd_status wd_context_embed(const wd_dims* d, const wd_ctx_weights* w, const void
   if (d->dtype == WD_BF16) {
     WD_TRY(gemm<bf16>(Mt, D, d->c_txt, txt, d->c_txt, w->txt1_w, d->c_txt, EPI_GELU, epi(hid, D, w->txt1_b), st));
     WD_TRY(gemm<bf16>(Mt, D, D, hid, D, w->txt2_w, D, EPI_STORE, epi(ctx_txt, D, w->txt2_b), st));
-    WD_TRY(gemm<bf16>(d->n_img, D, d->c_img, clip, d->c_img, w->img1_w, d->c_img, EPI_GELU, epi(hid, D, w->img1_b), st));
-    WD_TRY(gemm<bf16>(d->n_img, D, D, hid, D, w->img2_w, D, EPI_STORE, epi(ctx_img, D, w->img2_b), st));
+    if (img) {
+      WD_TRY(gemm<bf16>(d->n_img, D, d->c_img, clip, d->c_img, w->img1_w, d->c_img, EPI_GELU, epi(hid, D, w->img1_b), st));
+      WD_TRY(gemm<bf16>(d->n_img, D, D, hid, D, w->img2_w, D, EPI_STORE, epi(ctx_img, D, w->img2_b), st));
+    }
   } else {
     WD_TRY(gemm<float>(Mt, D, d->c_txt, txt, d->c_txt, w->txt1_w, d->c_txt, EPI_GELU, epi(hid, D, w->txt1_b), st));
     WD_TRY(gemm<float>(Mt, D, D, hid, D, w->txt2_w, D, EPI_STORE, epi(ctx_txt, D, w->txt2_b), st));
-    WD_TRY(gemm<float>(d->n_img, D, d->c_img, clip, d->c_img, w->img1_w, d->c_img, EPI_GELU, epi(hid, D, w->img1_b), st));
-    WD_TRY(gemm<float>(d->n_img, D, D, hid, D, w->img2_w, D, EPI_STORE, epi(ctx_img, D, w->img2_b), st));
+    if (img) {
+      WD_TRY(gemm<float>(d->n_img, D, d->c_img, clip, d->c_img, w->img1_w, d->c_img, EPI_GELU, epi(hid, D, w->img1_b), st));
+      WD_TRY(gemm<float>(d->n_img, D, D, hid, D, w->img2_w, D, EPI_STORE, epi(ctx_img, D, w->img2_b), st));
+    }
   }
   return WD_OK;
 }
@@ -352,7 +365,8 @@ wd_status wd_cross_kv(const wd_dims* d, const wd_block_weights* w, const void* c
   WD_TRY(check_batch(batch));
   if (!w) { set_error("block weights NULL"); return WD_ERR_ARG; }
   WD_NEED(w->ck_w); WD_NEED(w->ck_b); WD_NEED(w->cv_w); WD_NEED(w->cv_b);
-  WD_NEED(w->cki_w); WD_NEED(w->cki_b); WD_NEED(w->cvi_w); WD_NEED(w->cvi_b);
+  const bool img = d->n_img > 0;   // the text-to-video model has text keys and values only
+  if (img) { WD_NEED(w->cki_w); WD_NEED(w->cki_b); WD_NEED(w->cvi_w); WD_NEED(w->cvi_b); }
   WD_NEED(ctx);
   WD_NEED(kv);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -367,13 +381,17 @@ wd_status wd_cross_kv(const wd_dims* d, const wd_block_weights* w, const void* c
   const int Mt = batch * d->n_txt;
   if (d->dtype == WD_BF16) {
     // stored as IEEE half: the cross-attention operands of the bf16 path
-    WD_TRY(gemm<bf16>(d->n_img, D, D, ctx_img, D, w->cki_w, D, EPI_STORE_F16, epi(k_img, D, w->cki_b), st));
-    WD_TRY(gemm<bf16>(d->n_img, D, D, ctx_img, D, w->cvi_w, D, EPI_STORE_F16, epi(v_img, D, w->cvi_b), st));
+    if (img) {
+      WD_TRY(gemm<bf16>(d->n_img, D, D, ctx_img, D, w->cki_w, D, EPI_STORE_F16, epi(k_img, D, w->cki_b), st));
+      WD_TRY(gemm<bf16>(d->n_img, D, D, ctx_img, D, w->cvi_w, D, EPI_STORE_F16, epi(v_img, D, w->cvi_b), st));
+    }
     WD_TRY(gemm<bf16>(Mt, D, D, ctx_txt, D, w->ck_w, D, EPI_STORE_F16, epi(k_txt, D, w->ck_b), st));
     WD_TRY(gemm<bf16>(Mt, D, D, ctx_txt, D, w->cv_w, D, EPI_STORE_F16, epi(v_txt, D, w->cv_b), st));
   } else {
-    WD_TRY(gemm<float>(d->n_img, D, D, ctx_img, D, w->cki_w, D, EPI_STORE, epi(k_img, D, w->cki_b), st));
-    WD_TRY(gemm<float>(d->n_img, D, D, ctx_img, D, w->cvi_w, D, EPI_STORE, epi(v_img, D, w->cvi_b), st));
+    if (img) {
+      WD_TRY(gemm<float>(d->n_img, D, D, ctx_img, D, w->cki_w, D, EPI_STORE, epi(k_img, D, w->cki_b), st));
+      WD_TRY(gemm<float>(d->n_img, D, D, ctx_img, D, w->cvi_w, D, EPI_STORE, epi(v_img, D, w->cvi_b), st));
+    }
     WD_TRY(gemm<float>(Mt, D, D, ctx_txt, D, w->ck_w, D, EPI_STORE, epi(k_txt, D, w->ck_b), st));
     WD_TRY(gemm<float>(Mt, D, D, ctx_txt, D, w->cv_w, D, EPI_STORE, epi(v_txt, D, w->cv_b), st));
   }
@@ -384,21 +402,23 @@ wd_status wd_patch_embed(const wd_dims* d, const float* x_t, const float* y, con
                          float* X, void* ws, size_t ws_bytes, wd_stream stream) {
   WD_TRY(check_dims(d));
   WD_TRY(check_batch(batch));
-  WD_NEED(x_t); WD_NEED(y); WD_NEED(w); WD_NEED(b); WD_NEED(X); WD_NEED(ws);
+  WD_NEED(x_t); WD_NEED(w); WD_NEED(b); WD_NEED(X); WD_NEED(ws);
+  if (d->n_img > 0) { WD_NEED(y); } else { WD_OPT(y); }
   const Ws L = ws_layout(d, batch, ws);
   if (ws_bytes < L.bytes) { set_error("workspace %zu < %zu bytes", ws_bytes, L.bytes); return WD_ERR_WORKSPACE; }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t rows = batch * tokens(d);
-  const int64_t n = rows * 144;
+  const int K = patch_k(d);
+  const int64_t n = rows * K;
   const unsigned grid = static_cast<unsigned>((n + 255) / 256 < 65536 ? (n + 255) / 256 : 65536);
   if (d->dtype == WD_BF16) {
-    { Trace tr(KC_SMALL, st); k_patch_gather<bf16><<<grid, 256, 0, st>>>(x_t, y, batch, d->T, d->H, d->W, static_cast<bf16*>(L.b)); }
+    { Trace tr(KC_SMALL, st); k_patch_gather<bf16><<<grid, 256, 0, st>>>(x_t, y, batch, d->T, d->H, d->W, K, static_cast<bf16*>(L.b)); }
     WD_TRY(launch_status("patch_gather"));
-    WD_TRY(gemm<bf16>(static_cast<int>(rows), d->D, 144, L.b, 144, w, 144, EPI_F32, epi(X, d->D, b), st));
+    WD_TRY(gemm<bf16>(static_cast<int>(rows), d->D, K, L.b, K, w, K, EPI_F32, epi(X, d->D, b), st));
   } else {
-    { Trace tr(KC_SMALL, st); k_patch_gather<float><<<grid, 256, 0, st>>>(x_t, y, batch, d->T, d->H, d->W, static_cast<float*>(L.b)); }
+    { Trace tr(KC_SMALL, st); k_patch_gather<float><<<grid, 256, 0, st>>>(x_t, y, batch, d->T, d->H, d->W, K, static_cast<float*>(L.b)); }
     WD_TRY(launch_status("patch_gather"));
-    WD_TRY(gemm<float>(static_cast<int>(rows), d->D, 144, L.b, 144, w, 144, EPI_F32, epi(X, d->D, b), st));
+    WD_TRY(gemm<float>(static_cast<int>(rows), d->D, K, L.b, K, w, K, EPI_F32, epi(X, d->D, b), st));
   }
   return WD_OK;
 }
@@ -475,6 +495,7 @@ wd_status wd_attention(int dtype, int batch, int Lq, int heads, int dh, const vo
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t D = static_cast<int64_t>(heads) * dh;
   auto fill = [&](auto a) {
+    a.cross = k2 != nullptr;
     a.q_rs = D; a.kv1_rs = D; a.kv1_bs = kv1_shared ? 0 : n1 * D; a.n1 = n1;
     a.kv2_rs = D; a.kv2_bs = kv2_shared ? 0 : n2 * D; a.n2 = k2 ? n2 : 0;
     a.o_rs = D; a.batch = batch; a.Lq = Lq; a.heads = heads; a.dh = dh;

@@ -121,6 +121,7 @@ struct AttnArgs {
   const TI* k2; const TI* v2; int64_t kv2_rs; int64_t kv2_bs; int n2;   // k2 == null: one segment
   TO* o; int64_t o_rs;
   int batch, Lq, heads, dh;
+  bool cross;                                  // counted as cross-attention in the launch trace
 };
 template <typename TI, typename TO>
 wd_status attention_simt(const AttnArgs<TI, TO>& a, cudaStream_t st);

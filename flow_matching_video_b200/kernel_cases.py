@@ -3,9 +3,10 @@
     python -m flow_matching_video_b200.kernel_cases CASE [--batch B] [--iters N] [--warmup W]
 
 CASE is one of attn_self, attn_cross, gemm_qkv, gemm_o, gemm_ffn1, gemm_ffn2,
-norm, qknorm_rope, euler.  Shapes are those of one block of the 30-block
-480p/81-frame model (L = 32760 tokens per sample, D = 1536, 12 heads x 128,
-FFN 8960, 257 image + 512 text keys).  Inputs are seeded random values; the
+euler, euler_hbm (the norm and RoPE kernels are timed inside the step).
+Shapes are those of one block of the 30-block 480p/81-frame model (L = 32760
+tokens per sample, D = 1536, 12 heads x 128, FFN 8960, 257 image + 512 text
+keys); euler_hbm streams 2^26 elements so that every launch reads HBM.  Inputs are seeded random values; the
 case prints the mean device time per launch (CUDA events) and the
 algorithmic FLOPs or bytes per launch.
 """
@@ -52,8 +53,10 @@ def make_case(name: str, B: int):
                                    g if epi == wd.EPI_RESID else None)), 2.0 * rows * N * K, "FLOP"
     d = synth.Dims(D=D, heads=H, ffn=F, blocks=1, T=21, H=60, W=104, n_txt=NT, c_txt=4096, n_img=NI,
                    c_img=1280, dtype="bf16")
-    if name == "euler":
-        n = 16 * 21 * 60 * 104
+    if name in ("euler", "euler_hbm"):
+        # euler: the step's latent (33.5 MB, L2-resident between launches);
+        # euler_hbm: 2^26 elements (1.07 GB of traffic), so every launch streams HBM
+        n = 16 * 21 * 60 * 104 if name == "euler" else 1 << 26
         x, vc, vu = (torch.randn(n, device="cuda") for _ in range(3))
         return (lambda: wd.wd_euler_cfg_step(x, vc, vu, 5.0, 1 / 12)), 16.0 * n, "B"
     raise SystemExit(f"unknown case {name}")

@@ -1,9 +1,12 @@
-"""Device-side Wan2.1-style I2V DiT built on the libwd C ABI.
+"""Device-side Wan2.1-style DiT built on the libwd C ABI.
 
 Holds the weights and buffers in device memory (torch tensors) and sequences
 the entry points of libwd for one denoising forward and one CFG Euler step
-("图解 Wan2.1 I2V" section 7).  Every arithmetic step runs in libwd's kernels;
-this module only allocates, fills structs of pointers and calls.
+("图解 Wan2.1 I2V" section 7), for the image-to-video model and its
+text-to-video counterpart (section 9 of that page: n_img = 0), and the
+two-expert timestep MoE sampler of Wan2.2 ("Wan（通义万相）..." 7.2).  Every
+arithmetic step runs in libwd's kernels; this module only allocates, fills
+structs of pointers and calls.
 """
 from __future__ import annotations
 
@@ -44,13 +47,16 @@ def random_weights_on_device(wl: synth.Workload, device) -> dict:
 
     g("t1.w", (D, synth.T_EMB)); g("t1.b", (D,)); g("t2.w", (D, D)); g("t2.b", (D,))
     g("tp.w", (6 * D, D)); g("tp.b", (6 * D,))
-    g("pe.w", (D, synth.PATCH_K), td); g("pe.b", (D,))
+    g("pe.w", (D, d.patch_k), td); g("pe.b", (D,))
     g("txt1.w", (D, d.c_txt), td); g("txt1.b", (D,)); g("txt2.w", (D, D), td); g("txt2.b", (D,))
-    g("img1.w", (D, d.c_img), td); g("img1.b", (D,)); g("img2.w", (D, D), td); g("img2.b", (D,))
+    if not d.t2v:
+        g("img1.w", (D, d.c_img), td); g("img1.b", (D,)); g("img2.w", (D, D), td); g("img2.b", (D,))
     for i in range(d.blocks):
         p = f"blk{i}."
         for nm, shp in (("qkv", (3 * D, D)), ("o", (D, D)), ("cq", (D, D)), ("ck", (D, D)), ("cv", (D, D)),
                         ("cki", (D, D)), ("cvi", (D, D)), ("co", (D, D)), ("f1", (F, D)), ("f2", (D, F))):
+            if d.t2v and nm in ("cki", "cvi"):
+                continue
             g(p + nm + ".w", shp, td)
             g(p + nm + ".b", (shp[0],))
         g(p + "gq", (D,), mean=1.0); g(p + "gk", (D,), mean=1.0)
@@ -63,14 +69,17 @@ def random_weights_on_device(wl: synth.Workload, device) -> dict:
 class DiT:
     """The DiT of one workload on one device, with its buffers for `batch` rows."""
 
-    def __init__(self, dims: synth.Dims, weights: dict, batch: int, device="cuda"):
+    def __init__(self, dims: synth.Dims, weights: dict, batch: int, device="cuda", buffers_from: "DiT" = None):
+        """buffers_from: another DiT of the same dims and batch whose workspace,
+        residual stream and output buffers this one shares (the experts of a
+        timestep MoE run one at a time); the context and K/V cache stay per model."""
         self.dims = dims
         self.cd = wd.make_dims(dims)
         self.batch = batch
         self.device = torch.device(device)
         self.w = weights
         self.tdtype = _tdtype(dims)
-        p = lambda k: self.w[k].data_ptr()
+        p = lambda k: self.w[k].data_ptr() if k in self.w else 0   # image weights: none for text-to-video
         self.time_w = wd.wd_time_weights(*(p(k) for k in ("t1.w", "t1.b", "t2.w", "t2.b", "tp.w", "tp.b")))
         self.ctx_w = wd.wd_ctx_weights(*(p(k) for k in ("txt1.w", "txt1.b", "txt2.w", "txt2.b",
                                                         "img1.w", "img1.b", "img2.w", "img2.b")))
@@ -84,10 +93,15 @@ class DiT:
         self.head_w = wd.wd_head_weights(p("head.mod"), p("head.w"), p("head.b"))
         L, D = dims.L, dims.D
         dev = self.device
-        self.ws = torch.empty(wd.wd_workspace_bytes(self.cd, batch), dtype=torch.uint8, device=dev)
         self.ctx = torch.empty(wd.wd_ctx_bytes(self.cd, batch), dtype=torch.uint8, device=dev)
         kvb = wd.wd_kv_bytes(self.cd, batch)
         self.kv = torch.empty((dims.blocks, kvb), dtype=torch.uint8, device=dev)
+        if buffers_from is not None:
+            assert buffers_from.dims == dims and buffers_from.batch == batch
+            src = buffers_from
+            self.ws, self.X, self.e, self.e0, self.v = src.ws, src.X, src.e, src.e0, src.v
+            return
+        self.ws = torch.empty(wd.wd_workspace_bytes(self.cd, batch), dtype=torch.uint8, device=dev)
         self.X = torch.empty((batch, L, D), dtype=torch.float32, device=dev)
         self.e = torch.empty(D, dtype=torch.float32, device=dev)
         self.e0 = torch.empty((6, D), dtype=torch.float32, device=dev)
@@ -99,15 +113,17 @@ class DiT:
         wd.wd_build_cond_y(self.cd, img_lat, y, known_frames)
         return y
 
-    def prepare_context(self, txt: torch.Tensor, clip: torch.Tensor):
-        """txt [batch, n_txt, c_txt], clip [n_img, c_img] in the storage type."""
+    def prepare_context(self, txt: torch.Tensor, clip: torch.Tensor = None):
+        """txt [batch, n_txt, c_txt], clip [n_img, c_img] in the storage type
+        (None for the text-to-video model)."""
         wd.wd_context_embed(self.cd, self.ctx_w, txt, clip, self.batch, self.ctx)
         for i in range(self.dims.blocks):
             wd.wd_cross_kv(self.cd, self.block_w[i], self.ctx, self.batch, self.kv[i])
 
     # -------------------------------------------------------------- per step
     def forward(self, x_t: torch.Tensor, y: torch.Tensor, tau: float, stream=None) -> torch.Tensor:
-        """v = DiT(concat(x_t, y), tau) for x_t [batch, 16, T, H, W]; returns self.v."""
+        """v = DiT(concat(x_t, y), tau) for x_t [batch, 16, T, H, W]; returns self.v.
+        y is None for the text-to-video model."""
         wd.wd_time_mod(self.cd, self.time_w, tau, self.e, self.e0, stream)
         wd.wd_patch_embed(self.cd, x_t, y, self.w["pe.w"], self.w["pe.b"], self.batch, self.X, self.ws, stream)
         for i in range(self.dims.blocks):
@@ -124,3 +140,26 @@ class DiT:
         wd.wd_euler_cfg_step(xb[0], v[0], v[1], cfg_scale, dt, stream=stream)
         xb[1].copy_(xb[0])
         return xb
+
+
+class MoE:
+    """Timestep-level mixture of two experts of one architecture (Wan2.2,
+    "Wan（通义万相）..." 7.2): every CFG Euler step runs the high-noise expert
+    while the noise level tau / 1000 exceeds t_moe, the low-noise expert from
+    there on.  The experts share their device buffers."""
+
+    def __init__(self, dims: synth.Dims, w_high: dict, w_low: dict, t_moe: float, batch: int = 2, device="cuda"):
+        self.high = DiT(dims, w_high, batch, device)
+        self.low = DiT(dims, w_low, batch, device, buffers_from=self.high)
+        self.t_moe = t_moe
+
+    def prepare_context(self, txt: torch.Tensor, clip: torch.Tensor = None):
+        self.high.prepare_context(txt, clip)
+        self.low.prepare_context(txt, clip)
+
+    def expert(self, tau: float) -> DiT:
+        return self.high if tau / 1000.0 > self.t_moe else self.low
+
+    def cfg_euler_step(self, xb: torch.Tensor, y: torch.Tensor, tau: float, dt: float, cfg_scale: float,
+                       stream=None):
+        return self.expert(tau).cfg_euler_step(xb, y, tau, dt, cfg_scale, stream)

@@ -25,6 +25,7 @@ LATENT_C = 16          # VAE latent channels
 MASK_C = 4             # mask channels (VAE temporal stride)
 IN_C = LATENT_C + MASK_C + LATENT_C   # 36-channel DiT input
 PATCH_K = IN_C * 1 * 2 * 2            # 144 values per (1,2,2) patch
+PATCH_K_T2V = LATENT_C * 1 * 2 * 2    # 64: the text-to-video model embeds x_t alone
 OUT_P = LATENT_C * 1 * 2 * 2          # 64 head outputs per token
 T_EMB = 256            # sinusoidal timestep embedding width
 WEIGHT_STD = 0.02
@@ -64,6 +65,15 @@ class Dims:
         return self.T * self.Hp * self.Wp
 
     @property
+    def t2v(self) -> bool:
+        """Text-to-video model ("图解 Wan2.1 I2V" section 9): no image branch."""
+        return self.n_img == 0
+
+    @property
+    def patch_k(self) -> int:
+        return PATCH_K_T2V if self.t2v else PATCH_K
+
+    @property
     def F_pix(self) -> int:
         """Pixel frames that a latent of T frames encodes: T = 1 + (F-1)/4."""
         return 4 * (self.T - 1) + 1
@@ -78,6 +88,7 @@ class Workload:
     steps: int = 1      # Euler steps of the sampler
     cfg_scale: float = 5.0
     txt_valid: tuple = (512, 512)   # text rows >= n_valid are zero; n_valid ~ U[lo, hi]
+    t_moe: float = None   # two experts (timestep MoE): the high-noise one while the noise level exceeds t_moe
 
 
 # The five workloads: a tiny fp32 model, one bf16 block at 480p/17 frames,
@@ -107,7 +118,24 @@ SMALL_BF16 = Workload("small-bf16-dh128-L105",
                            n_img=9, c_img=32, dtype="bf16"),
                       batch=2, seed=1012, steps=1, txt_valid=(5, 24))
 
-WORKLOADS = {w.name: w for w in (TINY, BLOCK_480P17, STACK_480P81, WIDE_720P81, SAMPLE_480P81, SMALL_BF16)}
+# Text-to-video counterparts ("图解 Wan2.1 I2V" section 9: 16 input channels, text-only
+# cross-attention, no CLIP branch), and the two-expert timestep MoE sampler of
+# Wan2.2 ("Wan（通义万相）..." 7.2) on the tiny model.
+TINY_T2V = replace(TINY, name="tiny-fp32-2blk-L32-t2v", dims=replace(TINY.dims, n_img=0, c_img=0), seed=1021)
+SMALL_BF16_T2V = replace(SMALL_BF16, name="small-bf16-dh128-L105-t2v", dims=replace(SMALL_BF16.dims, n_img=0, c_img=0),
+                         seed=1022)
+STACK_480P81_T2V = replace(STACK_480P81, name="bf16-30blk-D1536-L32760-t2v-cfg",
+                           dims=replace(STACK_480P81.dims, n_img=0, c_img=0), seed=1023)
+TINY_MOE = replace(TINY, name="tiny-fp32-2blk-L32-moe", seed=1031, steps=4, t_moe=0.6)
+
+WORKLOADS = {w.name: w for w in (TINY, BLOCK_480P17, STACK_480P81, WIDE_720P81, SAMPLE_480P81, SMALL_BF16,
+                                 TINY_T2V, SMALL_BF16_T2V, STACK_480P81_T2V, TINY_MOE)}
+
+
+def experts(wl: Workload):
+    """(high-noise, low-noise) expert workloads of a timestep-MoE sampler: the
+    same shapes and inputs, weights from separate seeds."""
+    return replace(wl, seed=wl.seed), replace(wl, seed=wl.seed + 500)
 
 
 def stream(seed: int, name: str) -> np.random.Generator:
@@ -148,22 +176,25 @@ def model_weights(wl: Workload, blocks=None) -> dict:
     w["tp.w"] = normal(s, "tp.w", (6 * D, D), std)
     w["tp.b"] = normal(s, "tp.b", (6 * D,), std)
     # patch embedding Conv3d(36, D, (1,2,2)) flattened to [D, 36*1*2*2]
-    w["pe.w"] = normal(s, "pe.w", (D, PATCH_K), std, dtype=dt)
+    w["pe.w"] = normal(s, "pe.w", (D, d.patch_k), std, dtype=dt)
     w["pe.b"] = normal(s, "pe.b", (D,), std)
-    # text and CLIP projections
+    # text and CLIP projections (the text-to-video model has no CLIP branch)
     w["txt1.w"] = normal(s, "txt1.w", (D, d.c_txt), std, dtype=dt)
     w["txt1.b"] = normal(s, "txt1.b", (D,), std)
     w["txt2.w"] = normal(s, "txt2.w", (D, D), std, dtype=dt)
     w["txt2.b"] = normal(s, "txt2.b", (D,), std)
-    w["img1.w"] = normal(s, "img1.w", (D, d.c_img), std, dtype=dt)
-    w["img1.b"] = normal(s, "img1.b", (D,), std)
-    w["img2.w"] = normal(s, "img2.w", (D, D), std, dtype=dt)
-    w["img2.b"] = normal(s, "img2.b", (D,), std)
+    if not d.t2v:
+        w["img1.w"] = normal(s, "img1.w", (D, d.c_img), std, dtype=dt)
+        w["img1.b"] = normal(s, "img1.b", (D,), std)
+        w["img2.w"] = normal(s, "img2.w", (D, D), std, dtype=dt)
+        w["img2.b"] = normal(s, "img2.b", (D,), std)
+    mats = (("qkv", (3 * D, D)), ("o", (D, D)), ("cq", (D, D)), ("ck", (D, D)), ("cv", (D, D)),
+            ("cki", (D, D)), ("cvi", (D, D)), ("co", (D, D)), ("f1", (F, D)), ("f2", (D, F)))
     for i in (range(d.blocks) if blocks is None else blocks):
         p = f"blk{i}."
-        for nm, shp in (("qkv", (3 * D, D)), ("o", (D, D)), ("cq", (D, D)), ("ck", (D, D)),
-                        ("cv", (D, D)), ("cki", (D, D)), ("cvi", (D, D)), ("co", (D, D)),
-                        ("f1", (F, D)), ("f2", (D, F))):
+        for nm, shp in mats:
+            if d.t2v and nm in ("cki", "cvi"):
+                continue
             w[p + nm + ".w"] = normal(s, p + nm + ".w", shp, std, dtype=dt)
             w[p + nm + ".b"] = normal(s, p + nm + ".b", (shp[0],), std)
         w[p + "gq"] = normal(s, p + "gq", (D,), std, mean=1.0)
@@ -189,7 +220,8 @@ def inputs(wl: Workload) -> dict:
     txt[n_valid:] = 0.0
     x["txt"] = txt
     x["txt_valid"] = n_valid
-    x["clip"] = normal(s, "clip", (d.n_img, d.c_img), dtype=d.dtype)
+    if not d.t2v:
+        x["clip"] = normal(s, "clip", (d.n_img, d.c_img), dtype=d.dtype)
     return x
 
 

@@ -63,8 +63,12 @@ typedef enum { WD_NORM_LAYER = 0, WD_NORM_RMS = 1 } wd_norm;
  * heads, ffn = FFN hidden width, blocks = DiT blocks; T, H, W = latent frames,
  * height and width (H, W even); the token grid is T x H/2 x W/2 and the token
  * count L = T*(H/2)*(W/2) ([I2V] 5.1).  n_txt x c_txt text tokens (umT5,
- * [I2V] 3.1), n_img x c_img CLIP tokens ([I2V] 3.2).  norm selects the adaLN
- * norm (LayerNorm without affine by default, [I2V] 5.2); eps its epsilon. */
+ * [I2V] 3.1), n_img x c_img CLIP tokens ([I2V] 3.2).  n_img = 0 selects the
+ * text-to-video model of [I2V] 9: 16 input channels (x_t alone, no y), no CLIP
+ * projection, and a single-stream cross-attention over the text tokens only;
+ * c_img and every image weight are then unused (may be 0 / NULL).  norm
+ * selects the adaLN norm (LayerNorm without affine by default, [I2V] 5.2); eps
+ * its epsilon. */
 typedef struct {
   int D, heads, ffn, blocks;
   int T, H, W;
@@ -159,13 +163,15 @@ wd_status wd_build_cond_y(const wd_dims* d, const float* img_lat, const int* kno
  * txt [batch, n_txt, c_txt] and clip [n_img, c_img] in dtype (the CFG
  * unconditional row carries zeroed text, [I2V] Q5).  ctx receives
  * wd_ctx_bytes(d, batch) bytes: ctx_txt [batch,n_txt,D], ctx_img [n_img,D]
- * (dtype), then scratch. */
+ * (dtype), then scratch.  With n_img = 0 there is no CLIP input (clip and the
+ * img weights may be NULL). */
 wd_status wd_context_embed(const wd_dims* d, const wd_ctx_weights* w, const void* txt,
                            const void* clip, int batch, void* ctx, wd_stream stream);
 
 /* One block's cross-attention keys and values from the context written by
  * wd_context_embed ([I2V] 5.4: text uses Linear_k/Linear_v, image its own
- * k_img/v_img).  kv receives wd_kv_bytes(d, batch) bytes. */
+ * k_img/v_img).  kv receives wd_kv_bytes(d, batch) bytes.  With n_img = 0
+ * only the text keys and values are written (their parts start at 0). */
 wd_status wd_cross_kv(const wd_dims* d, const wd_block_weights* w, const void* ctx, int batch,
                       void* kv, wd_stream stream);
 
@@ -177,7 +183,9 @@ wd_status wd_time_mod(const wd_dims* d, const wd_time_weights* w, float tau, flo
 /* Patch embedding of concat(x_t, y) ([I2V] 4.2, 5.1): Conv3d(36, D, (1,2,2),
  * stride (1,2,2)) as a GEMM.  x_t [batch,16,T,H,W] fp32, y [20,T,H,W] fp32
  * shared by the batch, w [D,144] (Conv3d weight [D,36,1,2,2] flattened) in
- * dtype, b [D] fp32 -> X [batch, L, D] fp32, token l = (f*(H/2)+y)*(W/2)+x. */
+ * dtype, b [D] fp32 -> X [batch, L, D] fp32, token l = (f*(H/2)+y)*(W/2)+x.
+ * Text-to-video (n_img = 0, [I2V] 9): Conv3d(16, D, ...) of x_t alone, w
+ * [D,64], y unused (may be NULL). */
 wd_status wd_patch_embed(const wd_dims* d, const float* x_t, const float* y, const void* w,
                          const float* b, int batch, float* X, void* ws, size_t ws_bytes,
                          wd_stream stream);

@@ -271,11 +271,15 @@ def unpatchify(p, T: int, Hp: int, Wp: int, C: int = 16):
 def patch_embed(x_t, y, w_pe, b_pe, rnd: bool = False):
     """tokens = Conv3d(36, D, (1,2,2), stride (1,2,2))(concat(x_t, y)) as a GEMM
     ([I2V] 4.2 for the 36-channel concat, 5.1 for the patchify).
-    x_t [B,16,T,H,W]; y [20,T,H,W] shared by the batch -> [B, L, D]."""
+    x_t [B,16,T,H,W]; y [20,T,H,W] shared by the batch -> [B, L, D].
+    y None: the text-to-video model, Conv3d(16, D, ...) of x_t alone ([I2V] 9)."""
     x_t = np.asarray(x_t, F64)
     B = x_t.shape[0]
-    yb = np.broadcast_to(np.asarray(y, F64)[None], (B,) + np.shape(y))
-    x_in = np.concatenate([x_t, yb], axis=1)
+    if y is None:
+        x_in = x_t
+    else:
+        yb = np.broadcast_to(np.asarray(y, F64)[None], (B,) + np.shape(y))
+        x_in = np.concatenate([x_t, yb], axis=1)
     return linear(_st(patchify(x_in), rnd), w_pe, b_pe)
 
 
@@ -283,10 +287,13 @@ def patch_embed(x_t, y, w_pe, b_pe, rnd: bool = False):
 def context_embed(w: dict, txt, clip, rnd: bool = False):
     """Text MLP [n_txt, c_txt] -> [n_txt, D] and CLIP MLPProj [n_img, c_img] ->
     [n_img, D] ([I2V] 7 steps 1-2).  txt is [B, n_txt, c_txt] (the
-    unconditional row carries zeroed text, [I2V] Q5); clip is [n_img, c_img].
+    unconditional row carries zeroed text, [I2V] Q5); clip is [n_img, c_img],
+    or None for the text-to-video model, which has no CLIP branch ([I2V] 9).
     Reading: each MLP is Linear -> GELU -> Linear with biases."""
     t = _st(gelu(linear(txt, w["txt1.w"], w["txt1.b"])), rnd)
     ctx_txt = _st(linear(t, w["txt2.w"], w["txt2.b"]), rnd)
+    if clip is None:
+        return ctx_txt, None
     i = _st(gelu(linear(clip, w["img1.w"], w["img1.b"])), rnd)
     ctx_img = _st(linear(i, w["img2.w"], w["img2.b"]), rnd)
     return ctx_txt, ctx_img
@@ -294,14 +301,15 @@ def context_embed(w: dict, txt, clip, rnd: bool = False):
 
 def cross_kv(w: dict, blk: int, ctx_txt, ctx_img, rnd: bool = False):
     """Per-block cross-attention keys/values of [I2V] 5.4: the text branch uses
-    Linear_k / Linear_v, the image branch its own k_img / v_img."""
+    Linear_k / Linear_v, the image branch its own k_img / v_img.  ctx_img None
+    (text-to-video, [I2V] 9): text keys and values only."""
     p = f"blk{blk}."
-    return dict(
-        k_txt=_st16(linear(ctx_txt, w[p + "ck.w"], w[p + "ck.b"]), rnd),
-        v_txt=_st16(linear(ctx_txt, w[p + "cv.w"], w[p + "cv.b"]), rnd),
-        k_img=_st16(linear(ctx_img, w[p + "cki.w"], w[p + "cki.b"]), rnd),
-        v_img=_st16(linear(ctx_img, w[p + "cvi.w"], w[p + "cvi.b"]), rnd),
-    )
+    kv = dict(k_txt=_st16(linear(ctx_txt, w[p + "ck.w"], w[p + "ck.b"]), rnd),
+              v_txt=_st16(linear(ctx_txt, w[p + "cv.w"], w[p + "cv.b"]), rnd))
+    if ctx_img is not None:
+        kv["k_img"] = _st16(linear(ctx_img, w[p + "cki.w"], w[p + "cki.b"]), rnd)
+        kv["v_img"] = _st16(linear(ctx_img, w[p + "cvi.w"], w[p + "cvi.b"]), rnd)
+    return kv
 
 
 # ---------------------------------------------------------------- one DiT block
@@ -354,10 +362,13 @@ def block_forward(X, e0, w: dict, blk: int, kv: dict, dims, rnd: bool = False, r
         hc = _st(layer_norm(xr, eps, w[p + "cn.g"], w[p + "cn.b"]), rnd)
         qc = _st16(linear(hc, w[p + "cq.w"], w[p + "cq.b"]), rnd).reshape(len(rows), nh, dh)
         kt, vt = kv["k_txt"][b], kv["v_txt"][b]
-        ki, vi = kv["k_img"], kv["v_img"]
-        o_img = attention(qc, ki.reshape(-1, nh, dh), vi.reshape(-1, nh, dh))
         o_txt = attention(qc, kt.reshape(-1, nh, dh), vt.reshape(-1, nh, dh))
-        oc = _st((o_img + o_txt).reshape(len(rows), D), rnd)
+        if "k_img" in kv:
+            ki, vi = kv["k_img"], kv["v_img"]
+            o_img = attention(qc, ki.reshape(-1, nh, dh), vi.reshape(-1, nh, dh))
+            oc = _st((o_img + o_txt).reshape(len(rows), D), rnd)
+        else:   # text-to-video: single-stream cross-attention ([I2V] 9)
+            oc = _st(o_txt.reshape(len(rows), D), rnd)
         xr = xr + linear(oc, w[p + "co.w"], w[p + "co.b"])
         # ---- gated FFN
         h2 = _st(adaln_modulate(xr, shift2, scale2, eps, dims.norm), rnd)
@@ -426,9 +437,10 @@ def sample(x0, img_lat, w: dict, txt, clip, dims, steps: int, cfg_scale: float,
     `steps` CFG Euler steps.  The cond row sees the text, the uncond row zeroed
     text with CLIP and y kept ([I2V] Q5).  ``model(x, tau)`` (optional) stands
     in for the DiT and returns (v_c, v_u).  Returns the final latent and the
-    per-step velocities."""
+    per-step velocities.  img_lat and clip None: the text-to-video model
+    ([I2V] 9), which has no y and no CLIP context."""
     if model is None:
-        y = build_cond_y(img_lat, known_pixel_frames)
+        y = None if img_lat is None else build_cond_y(img_lat, known_pixel_frames)
         txt2 = np.stack([np.asarray(txt, F64), np.zeros_like(txt, dtype=F64)])
         ctx_txt, ctx_img = context_embed(w, txt2, clip, rnd)
         kvs = [cross_kv(w, i, ctx_txt, ctx_img, rnd) for i in range(dims.blocks)]
@@ -443,3 +455,38 @@ def sample(x0, img_lat, w: dict, txt, clip, dims, steps: int, cfg_scale: float,
         trace.append((v_c, v_u))
         x = euler_cfg_step(x, v_c, v_u, cfg_scale, dt)
     return x, trace
+
+
+def expert_for(noise_level: float, t_moe: float) -> str:
+    """Timestep-level MoE of Wan2.2 ([WAN] 7.2): the high-noise expert while the
+    noise level exceeds the boundary t_moe, the low-noise expert from there on.
+    Reading: the page's t in this passage is the noise level (high noise first,
+    in the order of denoising), here 1 - t_k = tau / 1000; its rule for t_moe
+    (SNR(t_moe) = SNR_min / 2) is garbled and cannot be evaluated as printed
+    (SNR_min is 0 at pure noise), so t_moe is a parameter."""
+    return "high" if noise_level > t_moe else "low"
+
+
+def sample_moe(x0, img_lat, w_high: dict, w_low: dict, txt, clip, dims, steps: int, cfg_scale: float,
+               t_moe: float, rnd: bool = False):
+    """The sampler of `sample` with two experts of the same architecture
+    ([WAN] 7.2): each Euler step evaluates the expert that `expert_for` picks
+    for that step's noise level; each expert has its own context projections
+    and cross-attention keys and values.  Returns the final latent, the
+    per-step velocities and the expert used at each step."""
+    y = None if img_lat is None else build_cond_y(img_lat)
+    txt2 = np.stack([np.asarray(txt, F64), np.zeros_like(txt, dtype=F64)])
+    kvs = {}
+    for name, w in (("high", w_high), ("low", w_low)):
+        ctx_txt, ctx_img = context_embed(w, txt2, clip, rnd)
+        kvs[name] = [cross_kv(w, i, ctx_txt, ctx_img, rnd) for i in range(dims.blocks)]
+    ws = {"high": w_high, "low": w_low}
+    x = np.asarray(x0, F64)
+    trace, used = [], []
+    for t, dt, tau in schedule(steps):
+        name = expert_for(tau / 1000.0, t_moe)
+        v = dit_forward(np.stack([x, x]), y, tau, ws[name], kvs[name], dims, rnd)
+        trace.append((v[0], v[1]))
+        used.append(name)
+        x = euler_cfg_step(x, v[0], v[1], cfg_scale, dt)
+    return x, trace, used

@@ -69,6 +69,24 @@ def test_invalid_dims_rejected(wd):
     d.dtype = 9
     assert wd.wd_workspace_bytes(d, 2) == 0
     assert wd.wd_workspace_bytes(wd.make_dims(synth.TINY.dims), 0) == 0
+    d = wd.make_dims(synth.TINY.dims)
+    d.n_img = -1           # negative image token count
+    assert wd.wd_workspace_bytes(d, 2) == 0
+    d = wd.make_dims(synth.TINY.dims)
+    d.c_img = 0            # an image branch needs a CLIP width
+    assert wd.wd_workspace_bytes(d, 2) == 0
+    # n_img = 0 is the text-to-video model: valid, and its K/V cache holds text only
+    d = wd.make_dims(synth.TINY_T2V.dims)
+    assert wd.wd_workspace_bytes(d, 2) > 0
+    assert wd.wd_kv_bytes(d, 2) == 2 * (2 * 16 * 128 * 4)
+
+
+def test_patch_embed_needs_y_only_for_image_to_video(wd):
+    lib = wd.lib()
+    args = (0x1000, None, 0x3000, 0x4000, 2, 0x5000, 0x6000, 16, None)   # y = NULL, tiny workspace
+    assert lib.wd_patch_embed(C.byref(wd.make_dims(synth.TINY.dims)), *args) == 1          # WD_ERR_ARG
+    assert "y is NULL" in wd.wd_last_error()
+    assert lib.wd_patch_embed(C.byref(wd.make_dims(synth.TINY_T2V.dims)), *args) == 5      # workspace check next
 
 
 def test_null_and_misaligned_pointers_rejected_before_launch(wd):

@@ -56,12 +56,16 @@ def setup(mods, wl, blocks=None):
     net = model.DiT(d, dw, wl.batch)
     tdt = net.tdtype
     txt = np.stack([x["txt"], np.zeros_like(x["txt"])]) if wl.batch == 2 else x["txt"][None]
+    if d.t2v:   # text-to-video: no CLIP context, no y
+        net.prepare_context(dev(txt, tdt))
+        return net, w, x, txt, None, d
     net.prepare_context(dev(txt, tdt), dev(x["clip"], tdt))
     y = net.build_cond_y(dev(x["img_lat"]))
     return net, w, x, txt, y, d
 
 
 def oracle_context(w, txt, clip, d, rnd):
+    clip = None if d.t2v else clip
     ctx_t, ctx_i = O.context_embed(w, txt, clip, rnd)
     return [O.cross_kv(w, i, ctx_t, ctx_i, rnd) for i in range(d.blocks)]
 
@@ -189,3 +193,66 @@ def test_head_unpatchify_bf16_480p81(mods):
     wd.wd_unpatchify(net.cd, net.head_w, net.e, 2, net.X, net.v, net.ws)
     wd.wd_check()
     assert rel(host(net.v), O.head_unpatchify(X, e, w, d, rnd=True)) < TOL_BF16
+
+
+# ------------------------------------------------------------------ text-to-video model and timestep MoE
+def test_tiny_fp32_t2v_sampler(mods):
+    """Text-to-video ("图解 Wan2.1 I2V" 9): 16-channel patch embedding, text-only
+    cross-attention; the whole 2-step CFG sampler, every element."""
+    model, wd = mods
+    wl = synth.TINY_T2V
+    net, w, x, txt, y, d = setup(mods, wl)
+    assert y is None
+    xb = dev(np.stack([x["x0"], x["x0"]]))
+    vs = []
+    for t, dt, tau in O.schedule(wl.steps):
+        net.cfg_euler_step(xb, None, tau, dt, wl.cfg_scale)
+        vs.append(host(net.v))
+    wd.wd_check()
+    want_x, trace = O.sample(x["x0"], None, w, x["txt"], None, d, wl.steps, wl.cfg_scale, rnd=False)
+    for (vc, vu), got in zip(trace, vs):
+        assert rel(got[0], vc) < TOL_F32
+        assert rel(got[1], vu) < TOL_F32
+    assert rel(host(xb[0]), want_x) < TOL_F32
+
+
+def test_small_bf16_t2v_forward(mods):
+    """Text-to-video at bf16 with 128-wide heads and a ragged grid: the
+    tensor-core GEMMs (K = 64 patch embedding) and the single-stream half
+    cross-attention kernel."""
+    wl = synth.SMALL_BF16_T2V
+    net, w, x, txt, y, d = setup(mods, wl)
+    xb = np.stack([x["x0"], x["x0"]])
+    v = host(net.forward(dev(xb), None, 612.5))
+    kvs = oracle_context(w, txt, None, d, True)
+    want = O.dit_forward(xb, None, 612.5, w, kvs, d, True)
+    assert rel(v, want) < TOL_BF16
+
+
+def test_tiny_fp32_moe_sampler(mods):
+    """Two-expert timestep MoE ("Wan（通义万相）..." 7.2): 4 CFG Euler steps, the
+    high-noise expert at noise levels 1 and 0.75, the low-noise one at 0.5 and
+    0.25; every element of every velocity and of the final latent."""
+    model, wd = mods
+    wl = synth.TINY_MOE
+    d = wl.dims
+    w_hi, w_lo = (synth.model_weights(e) for e in synth.experts(wl))
+    x = synth.inputs(wl)
+    moe = model.MoE(d, model.weights_to_device(w_hi, d, "cuda"), model.weights_to_device(w_lo, d, "cuda"), wl.t_moe)
+    txt = np.stack([x["txt"], np.zeros_like(x["txt"])])
+    moe.prepare_context(dev(txt), dev(x["clip"]))
+    y = moe.high.build_cond_y(dev(x["img_lat"]))
+    xb = dev(np.stack([x["x0"], x["x0"]]))
+    used, vs = [], []
+    for t, dt, tau in O.schedule(wl.steps):
+        used.append("high" if moe.expert(tau) is moe.high else "low")
+        moe.cfg_euler_step(xb, y, tau, dt, wl.cfg_scale)
+        vs.append(host(moe.high.v))   # the experts share their output buffer
+    wd.wd_check()
+    want_x, trace, want_used = O.sample_moe(x["x0"], x["img_lat"], w_hi, w_lo, x["txt"], x["clip"], d, wl.steps,
+                                            wl.cfg_scale, wl.t_moe)
+    assert used == want_used == ["high", "high", "low", "low"]
+    for (vc, vu), got in zip(trace, vs):
+        assert rel(got[0], vc) < TOL_F32
+        assert rel(got[1], vu) < TOL_F32
+    assert rel(host(xb[0]), want_x) < TOL_F32

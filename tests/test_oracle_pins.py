@@ -455,3 +455,87 @@ def test_tiny_sampler_runs_and_guidance_matters():
     assert np.abs(vc - vu).max() > 1e-6          # zeroed text changes the prediction
     np.testing.assert_allclose(xf, O.euler_cfg_step(O.euler_cfg_step(x["x0"], *trace[0], 5.0, 0.5),
                                                     *trace[1], 5.0, 0.5), atol=1e-14)
+
+
+# ------------------------------------------------------------------ text-to-video model ([I2V] 9)
+def test_t2v_patch_embed_is_conv3d_of_16_channels():
+    B, T, H, W, D = 2, 3, 6, 8, 10
+    x_t = RNG.standard_normal((B, 16, T, H, W))
+    w = RNG.standard_normal((D, 16, 1, 2, 2))
+    b = RNG.standard_normal(D)
+    got = O.patch_embed(x_t, None, w.reshape(D, 64), b)
+    ref = TF.conv3d(T64(x_t), T64(w), T64(b), stride=(1, 2, 2)).numpy()
+    np.testing.assert_allclose(got, ref.reshape(B, D, -1).transpose(0, 2, 1), atol=1e-12)
+
+
+def test_t2v_block_is_i2v_block_without_image_values():
+    # with V_img = 0 the image stream adds nothing, so the dual cross-attention
+    # of the image-to-video block reduces to the single text stream
+    d, w, kv, X = _tiny()
+    e0 = RNG.standard_normal((6, d.D))
+    w = dict(w, **{"blk0.cvi.w": np.zeros_like(w["blk0.cvi.w"]), "blk0.cvi.b": np.zeros(d.D)})
+    txt = RNG.standard_normal((2, d.n_txt, d.c_txt))
+    clip = RNG.standard_normal((d.n_img, d.c_img))
+    ctx_t, ctx_i = O.context_embed(w, txt, clip)
+    kv_i2v = O.cross_kv(w, 0, ctx_t, ctx_i)
+    assert np.all(kv_i2v["v_img"] == 0)
+    kv_t2v = O.cross_kv(w, 0, ctx_t, None)
+    assert set(kv_t2v) == {"k_txt", "v_txt"}
+    np.testing.assert_allclose(O.block_forward(X, e0, w, 0, kv_t2v, d), O.block_forward(X, e0, w, 0, kv_i2v, d),
+                               atol=1e-12)
+    # ... and the image stream does matter when its values are not zero
+    w2 = dict(w, **{"blk0.cvi.b": np.ones(d.D)})
+    kv2 = O.cross_kv(w2, 0, ctx_t, ctx_i)
+    assert np.abs(O.block_forward(X, e0, w2, 0, kv2, d) - O.block_forward(X, e0, w2, 0, kv_t2v, d)).max() > 1e-3
+
+
+def test_t2v_context_has_no_clip_branch():
+    w = synth.model_weights(synth.TINY_T2V)
+    assert "img1.w" not in w and "blk0.cki.w" not in w and w["pe.w"].shape == (128, 64)
+    txt = RNG.standard_normal((2, 16, 64))
+    ctx_t, ctx_i = O.context_embed(w, txt, None)
+    assert ctx_i is None and ctx_t.shape == (2, 16, 128)
+
+
+def test_t2v_tiny_sampler_runs_and_guidance_matters():
+    wl = synth.TINY_T2V
+    w = synth.model_weights(wl)
+    x = synth.inputs(wl)
+    xf, trace = O.sample(x["x0"], None, w, x["txt"], None, wl.dims, wl.steps, wl.cfg_scale)
+    assert xf.shape == (16, 2, 8, 8) and np.all(np.isfinite(xf))
+    assert np.abs(trace[0][0] - trace[0][1]).max() > 1e-6
+
+
+# ------------------------------------------------------------------ timestep MoE ([WAN] 7.2)
+def test_moe_expert_choice_follows_noise_level():
+    assert O.expert_for(1.0, 0.6) == "high" and O.expert_for(0.61, 0.6) == "high"
+    assert O.expert_for(0.6, 0.6) == "low" and O.expert_for(0.25, 0.6) == "low"
+    # on the 4-step grid the noise levels are 1, 0.75, 0.5, 0.25
+    assert [O.expert_for(tau / 1000.0, 0.6) for _, _, tau in O.schedule(4)] == ["high", "high", "low", "low"]
+
+
+def _moe_inputs():
+    wl = synth.TINY_MOE
+    w_hi, w_lo = (synth.model_weights(e) for e in synth.experts(wl))
+    return wl, w_hi, w_lo, synth.inputs(wl)
+
+
+def test_moe_with_one_expert_throughout_is_the_plain_sampler():
+    wl, w_hi, w_lo, x = _moe_inputs()
+    args = (x["txt"], x["clip"], wl.dims, wl.steps, wl.cfg_scale)
+    x_lo, _, used = O.sample_moe(x["x0"], x["img_lat"], w_hi, w_lo, *args, t_moe=1.0)
+    assert used == ["low"] * wl.steps
+    np.testing.assert_array_equal(x_lo, O.sample(x["x0"], x["img_lat"], w_lo, *args)[0])
+    x_hi, _, used = O.sample_moe(x["x0"], x["img_lat"], w_hi, w_lo, *args, t_moe=-1.0)
+    assert used == ["high"] * wl.steps
+    np.testing.assert_array_equal(x_hi, O.sample(x["x0"], x["img_lat"], w_hi, *args)[0])
+
+
+def test_moe_with_identical_experts_is_the_plain_sampler_and_the_switch_matters():
+    wl, w_hi, w_lo, x = _moe_inputs()
+    args = (x["txt"], x["clip"], wl.dims, wl.steps, wl.cfg_scale)
+    x_same, _, used = O.sample_moe(x["x0"], x["img_lat"], w_hi, w_hi, *args, t_moe=wl.t_moe)
+    assert used == ["high", "high", "low", "low"]
+    np.testing.assert_array_equal(x_same, O.sample(x["x0"], x["img_lat"], w_hi, *args)[0])
+    x_moe, _, _ = O.sample_moe(x["x0"], x["img_lat"], w_hi, w_lo, *args, t_moe=wl.t_moe)
+    assert np.abs(x_moe - x_same).max() > 1e-3
