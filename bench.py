@@ -56,7 +56,7 @@ def block_flops(d) -> dict:
 
 def step_flops(d, batch) -> float:
     f = block_flops(d)
-    extra = 2.0 * d.L * 144 * d.D + 2.0 * d.L * d.D * 64      # patch embedding + head
+    extra = 2.0 * d.L * d.patch_k * d.D + 2.0 * d.L * d.D * 64      # patch embedding + head
     return batch * (d.blocks * sum(f.values()) + extra)
 
 
@@ -118,9 +118,10 @@ class OracleSample:
         self.d1 = replace(wl.dims, blocks=1)
         self.w = synth.model_weights(wl, blocks=[0])
         x = synth.inputs(wl)
-        self.X = O.patch_embed(x["x0"][None], O.build_cond_y(x["img_lat"]), self.w["pe.w"], self.w["pe.b"], rnd=True)
+        y = None if wl.dims.t2v else O.build_cond_y(x["img_lat"])
+        self.X = O.patch_embed(x["x0"][None], y, self.w["pe.w"], self.w["pe.b"], rnd=True)
         _, self.e0 = O.time_mod(self.w, 1000.0, self.d1.D)
-        ctx_t, ctx_i = O.context_embed(self.w, x["txt"][None], x["clip"], rnd=True)
+        ctx_t, ctx_i = O.context_embed(self.w, x["txt"][None], None if wl.dims.t2v else x["clip"], rnd=True)
         self.kv = O.cross_kv(self.w, 0, ctx_t, ctx_i, rnd=True)
         # first call pays allocation and BLAS start-up; not part of any rate
         self.block(self.np.arange(8))
@@ -234,13 +235,21 @@ def run_ours(args, rank, world, local_rank):
     B = wl.batch
     torch.manual_seed(0)
     weights = model.random_weights_on_device(wl, dev)
-    net = model.DiT(d, weights, B, dev)
+    if args.cfg_cache is not None:   # the sampler with the CFG cache: late steps run the conditional row alone
+        runner = model.CfgCache(d, weights, args.cfg_cache, dev)
+        net = runner.pair
+    else:
+        runner = net = model.DiT(d, weights, B, dev)
     x = synth.inputs(replace(wl, seed=wl.seed + 7919 * rank))   # an independent video per rank
     tdt = net.tdtype
     txt2 = torch.from_numpy(np.stack([x["txt"], np.zeros_like(x["txt"])])).to(dev, tdt)
-    clip = torch.from_numpy(x["clip"]).to(dev, tdt)
-    net.prepare_context(txt2, clip)
-    y = net.build_cond_y(torch.from_numpy(x["img_lat"]).to(dev))
+    if d.t2v:   # text-to-video: no CLIP context and no y
+        runner.prepare_context(txt2)
+        y = None
+    else:
+        clip = torch.from_numpy(x["clip"]).to(dev, tdt)
+        runner.prepare_context(txt2, clip)
+        y = net.build_cond_y(torch.from_numpy(x["img_lat"]).to(dev))
     x_host = torch.from_numpy(x["x0"]).pin_memory()
     out_host = torch.empty_like(x_host).pin_memory()
     xb = torch.empty((2,) + tuple(x_host.shape), device=dev)
@@ -252,7 +261,7 @@ def run_ours(args, rank, world, local_rank):
 
     def step(i):
         _, dt, tau = sched[i % n_sched]
-        net.cfg_euler_step(xb, y, tau, dt, wl.cfg_scale)
+        runner.cfg_euler_step(xb, y, tau, dt, wl.cfg_scale)
 
     def barrier():
         if world > 1:
@@ -322,6 +331,12 @@ def run_ours(args, rank, world, local_rank):
     pk = peaks()
     wbytes = sum(t.numel() * t.element_size() for t in weights.values())
     flops = step_flops(d, B)
+    cache_note = None
+    if args.cfg_cache is not None:
+        # timed steps that ran only the conditional row do half the work of a CFG step
+        fresh = sum(1 for i in range(args.steps) if sched[(args.warmup + i) % n_sched][2] / 1000.0 > args.cfg_cache)
+        flops *= (fresh + 0.5 * (args.steps - fresh)) / args.steps
+        cache_note = {"t_cfg": args.cfg_cache, "steps_with_both_rows": fresh, "steps_conditional_only": args.steps - fresh}
     tflops = flops / (ms / 1e3) / 1e12
     # roofline of the dominant kernel (self-attention), timed live with events
     n_att, ms_att = tr["attn_self"]
@@ -361,6 +376,7 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": traffic_for("attn_self", os.path.join(ROOT, "flow_matching_video_b200", "csrc",
                                                                       "k_attn_tc.cu"))},
         "kernel_time_share": share,
+        **({"cfg_cache": cache_note} if cache_note else {}),
         "clocks": clk,
     }
     if cpu is not None:
@@ -377,6 +393,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cfg-cache", type=float, default=None, metavar="T",
+                    help="sample with the CFG cache: steps at noise level <= T reuse the last unconditional velocity")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -163,3 +163,42 @@ class MoE:
     def cfg_euler_step(self, xb: torch.Tensor, y: torch.Tensor, tau: float, dt: float, cfg_scale: float,
                        stream=None):
         return self.expert(tau).cfg_euler_step(xb, y, tau, dt, cfg_scale, stream)
+
+
+class CfgCache:
+    """CFG cache ("Wan（通义万相）..." 5.3, skip the unconditional path in the late
+    steps): while the noise level tau / 1000 exceeds t_cfg a step evaluates both
+    rows; from the first step at or below it only the conditional row runs
+    (a batch-1 model on the same weights, with its own K/V cache of the
+    conditional text) and the CFG combination reuses the last unconditional
+    velocity computed."""
+
+    def __init__(self, dims: synth.Dims, weights: dict, t_cfg: float, device="cuda"):
+        self.pair = DiT(dims, weights, 2, device)
+        self.cond = DiT(dims, weights, 1, device)
+        self.t_cfg = t_cfg
+        self.v_u = torch.empty((16, dims.T, dims.H, dims.W), dtype=torch.float32, device=self.pair.device)
+        self.have_v_u = False
+
+    def prepare_context(self, txt: torch.Tensor, clip: torch.Tensor = None):
+        """txt [2, n_txt, c_txt] (row 0 the text, row 1 zeroed)."""
+        self.pair.prepare_context(txt, clip)
+        self.cond.prepare_context(txt[:1].contiguous(), clip)
+        self.have_v_u = False
+
+    def fresh(self, tau: float) -> bool:
+        return not self.have_v_u or tau / 1000.0 > self.t_cfg
+
+    def cfg_euler_step(self, xb: torch.Tensor, y: torch.Tensor, tau: float, dt: float, cfg_scale: float,
+                       stream=None):
+        """xb [2, 16, T, H, W] as for DiT.cfg_euler_step."""
+        if self.fresh(tau):
+            v = self.pair.forward(xb, y, tau, stream)
+            self.v_u.copy_(v[1])
+            self.have_v_u = True
+            v_c = v[0]
+        else:
+            v_c = self.cond.forward(xb[:1], y, tau, stream)[0]
+        wd.wd_euler_cfg_step(xb[0], v_c, self.v_u, cfg_scale, dt, stream=stream)
+        xb[1].copy_(xb[0])
+        return xb

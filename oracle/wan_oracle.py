@@ -490,3 +490,32 @@ def sample_moe(x0, img_lat, w_high: dict, w_low: dict, txt, clip, dims, steps: i
         used.append(name)
         x = euler_cfg_step(x, v[0], v[1], cfg_scale, dt)
     return x, trace, used
+
+
+def sample_cfg_cache(x0, img_lat, w: dict, txt, clip, dims, steps: int, cfg_scale: float, t_cfg: float,
+                     rnd: bool = False):
+    """The sampler of `sample` with the CFG cache of [WAN] 5.3 ("skip the
+    unconditional path in the late steps").  Reading: while the noise level
+    tau / 1000 exceeds t_cfg both rows are evaluated; from the first step at or
+    below it only the conditional row is, and the CFG combination reuses the
+    last unconditional velocity computed.  Returns the final latent, the
+    per-step (v_c, v_u) actually combined, and per step whether v_u was fresh."""
+    y = None if img_lat is None else build_cond_y(img_lat)
+    txt2 = np.stack([np.asarray(txt, F64), np.zeros_like(txt, dtype=F64)])
+    ctx_txt, ctx_img = context_embed(w, txt2, clip, rnd)
+    kvs = [cross_kv(w, i, ctx_txt, ctx_img, rnd) for i in range(dims.blocks)]
+    kvs_c = [cross_kv(w, i, ctx_txt[:1], ctx_img, rnd) for i in range(dims.blocks)]   # the conditional row alone
+    x = np.asarray(x0, F64)
+    trace, fresh = [], []
+    v_u = None
+    for t, dt, tau in schedule(steps):
+        if v_u is None or tau / 1000.0 > t_cfg:
+            v = dit_forward(np.stack([x, x]), y, tau, w, kvs, dims, rnd)
+            v_c, v_u = v[0], v[1]
+            fresh.append(True)
+        else:
+            v_c = dit_forward(x[None], y, tau, w, kvs_c, dims, rnd)[0]
+            fresh.append(False)
+        trace.append((v_c, v_u))
+        x = euler_cfg_step(x, v_c, v_u, cfg_scale, dt)
+    return x, trace, fresh

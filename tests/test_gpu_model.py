@@ -256,3 +256,27 @@ def test_tiny_fp32_moe_sampler(mods):
         assert rel(got[0], vc) < TOL_F32
         assert rel(got[1], vu) < TOL_F32
     assert rel(host(xb[0]), want_x) < TOL_F32
+
+
+def test_tiny_fp32_cfg_cache_sampler(mods):
+    """CFG cache ("Wan（通义万相）..." 5.3): 4 steps, the unconditional velocity
+    computed at noise levels 1 and 0.75 and reused at 0.5 and 0.25, where only
+    the conditional row runs (batch 1); every element of the final latent."""
+    model, wd = mods
+    wl = synth.TINY_MOE
+    d = wl.dims
+    w = synth.model_weights(wl)
+    x = synth.inputs(wl)
+    cc = model.CfgCache(d, model.weights_to_device(w, d, "cuda"), t_cfg=0.5)
+    cc.prepare_context(dev(np.stack([x["txt"], np.zeros_like(x["txt"])])), dev(x["clip"]))
+    y = cc.pair.build_cond_y(dev(x["img_lat"]))
+    xb = dev(np.stack([x["x0"], x["x0"]]))
+    fresh = []
+    for t, dt, tau in O.schedule(wl.steps):
+        fresh.append(cc.fresh(tau))
+        cc.cfg_euler_step(xb, y, tau, dt, wl.cfg_scale)
+    wd.wd_check()
+    want_x, _, want_fresh = O.sample_cfg_cache(x["x0"], x["img_lat"], w, x["txt"], x["clip"], d, wl.steps,
+                                                wl.cfg_scale, 0.5)
+    assert fresh == want_fresh == [True, True, False, False]
+    assert rel(host(xb[0]), want_x) < TOL_F32

@@ -539,3 +539,43 @@ def test_moe_with_identical_experts_is_the_plain_sampler_and_the_switch_matters(
     np.testing.assert_array_equal(x_same, O.sample(x["x0"], x["img_lat"], w_hi, *args)[0])
     x_moe, _, _ = O.sample_moe(x["x0"], x["img_lat"], w_hi, w_lo, *args, t_moe=wl.t_moe)
     assert np.abs(x_moe - x_same).max() > 1e-3
+
+
+# ------------------------------------------------------------------ CFG cache ([WAN] 5.3)
+def test_cfg_cache_never_taken_is_the_plain_sampler():
+    wl = synth.TINY_MOE   # 4 steps: noise levels 1, 0.75, 0.5, 0.25
+    w = synth.model_weights(wl)
+    x = synth.inputs(wl)
+    args = (x["txt"], x["clip"], wl.dims, wl.steps, wl.cfg_scale)
+    xc, _, fresh = O.sample_cfg_cache(x["x0"], x["img_lat"], w, *args, t_cfg=0.0)
+    assert fresh == [True] * 4
+    np.testing.assert_array_equal(xc, O.sample(x["x0"], x["img_lat"], w, *args)[0])
+
+
+def test_cfg_cache_reuses_the_last_unconditional_velocity():
+    wl = synth.TINY_MOE
+    w = synth.model_weights(wl)
+    x = synth.inputs(wl)
+    args = (x["txt"], x["clip"], wl.dims, wl.steps, wl.cfg_scale)
+    xc, trace, fresh = O.sample_cfg_cache(x["x0"], x["img_lat"], w, *args, t_cfg=0.5)
+    assert fresh == [True, True, False, False]
+    assert trace[2][1] is trace[1][1] and trace[3][1] is trace[1][1]
+    # the conditional row computed alone is the conditional row of the batch of two
+    x_after2 = O.euler_cfg_step(O.euler_cfg_step(x["x0"], *trace[0], wl.cfg_scale, 0.25), *trace[1], wl.cfg_scale, 0.25)
+    v_pair = O.dit_forward(np.stack([x_after2, x_after2]), O.build_cond_y(x["img_lat"]), 500.0, w,
+                           [O.cross_kv(w, i, *O.context_embed(w, np.stack([x["txt"], 0 * x["txt"]]), x["clip"]))
+                            for i in range(wl.dims.blocks)], wl.dims)
+    np.testing.assert_allclose(trace[2][0], v_pair[0], atol=1e-12)
+    # and it changes the result relative to fresh CFG
+    assert np.abs(xc - O.sample(x["x0"], x["img_lat"], w, *args)[0]).max() > 1e-6
+
+
+def test_cfg_cache_is_exact_at_guidance_scale_one():
+    # s = 1: v = v_c whatever v_u is, so caching v_u changes nothing
+    wl = synth.TINY_MOE
+    w = synth.model_weights(wl)
+    x = synth.inputs(wl)
+    args = (x["txt"], x["clip"], wl.dims, wl.steps, 1.0)
+    xc, _, fresh = O.sample_cfg_cache(x["x0"], x["img_lat"], w, *args, t_cfg=0.6)
+    assert fresh == [True, True, False, False]
+    np.testing.assert_allclose(xc, O.sample(x["x0"], x["img_lat"], w, *args)[0], atol=1e-12)
