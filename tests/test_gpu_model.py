@@ -6,7 +6,11 @@
 * one bf16 block at 480p/17 frames (L=7800) and at 480p/81 frames
   (L=32760, batch 2 — the benchmark's launch configuration), on sampled token
   rows that the oracle computes exactly (keys/values still cover all tokens),
-  including the last rows of the ragged final tile.  Tolerance 2e-2.
+  including the last rows of the ragged final tile.  Tolerance 2e-2;
+* the wide 720p block, the 12-step sampler of the full 30-block model on a
+  short grid, head + unpatchify;
+* the text-to-video model (tiny sampler, small bf16 forward, 480p block), the
+  two-expert timestep MoE sampler and the CFG-cache sampler.
 """
 import numpy as np
 import pytest
@@ -124,7 +128,7 @@ def _block_parity(mods, wl, n_rows, tau):
     net, w, x, txt, y, d = setup(mods, wl, blocks=[0])
     B, L, D = wl.batch, d.L, d.D
     x_t = np.stack([x["x0"]] * B)
-    X_in = O.patch_embed(x_t, O.build_cond_y(x["img_lat"]), w["pe.w"], w["pe.b"], rnd=True)
+    X_in = O.patch_embed(x_t, None if d.t2v else O.build_cond_y(x["img_lat"]), w["pe.w"], w["pe.b"], rnd=True)
     # patch embedding (full size, every element)
     wd.wd_patch_embed(net.cd, dev(x_t), y, net.w["pe.w"], net.w["pe.b"], B, net.X, net.ws)
     wd.wd_check()
@@ -153,6 +157,11 @@ def test_block_bf16_480p17(mods):
 
 def test_block_bf16_480p81_batch2(mods):
     _block_parity(mods, synth.STACK_480P81, 192, 1000.0)
+
+
+def test_block_bf16_480p81_t2v_batch2(mods):
+    # text-to-video: 16-channel patch embedding, single-stream text cross-attention
+    _block_parity(mods, synth.STACK_480P81_T2V, 192, 900.0)
 
 
 def test_block_bf16_720p81_wide_batch2(mods):

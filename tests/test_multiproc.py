@@ -51,3 +51,64 @@ def test_single_rank_is_local():
     import bench
     ms, value = bench.reduce_over_ranks(400.0, 1000.0, 1)
     assert ms == 400.0 and value == pytest.approx(2500.0)
+
+
+# ------------------------------------------------------------------ CFG split over two ranks
+class _StandInModel:
+    """A deterministic batch-1 velocity field for the exchange test: the text
+    row and the zeroed-text row differ, as the DiT's do."""
+
+    def __init__(self, text_row: bool):
+        self.text_row = text_row
+
+    def forward(self, x1, y, tau):
+        import torch
+        base = torch.sin(x1 * 1.7 + tau / 1000.0)
+        return base + (0.3 * torch.cos(x1) if self.text_row else 0.0)
+
+
+def _euler(x, v_c, v_u, s, dt):
+    x += dt * (v_u + s * (v_c - v_u))
+
+
+def _cfg_rank(rank, world, port, x0, steps, out):
+    import torch
+    import torch.distributed as dist
+    from flow_matching_video_b200.cfg_split import CfgSplit
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        split = CfgSplit(_StandInModel(text_row=(rank == 0)), euler=_euler)
+        x = x0.clone()
+        for k in range(steps):
+            split.cfg_euler_step(x, None, 1000.0 * (1 - k / steps), 1.0 / steps, 5.0)
+        out[rank] = x.numpy()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_cfg_split_two_gloo_ranks_match_the_single_process_step():
+    import numpy as np
+    import torch
+    steps = 3
+    x0 = torch.randn(16, 2, 4, 6, dtype=torch.float64, generator=torch.Generator().manual_seed(3))
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_cfg_rank, args=(r, 2, port, x0, steps, out)) for r in range(2)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=120)
+        assert all(p.exitcode == 0 for p in procs)
+        x0_, x1_ = out[0], out[1]
+    # both ranks hold the same latent ...
+    np.testing.assert_array_equal(x0_, x1_)
+    # ... equal to the CFG Euler steps taken in one process with both rows
+    cond, uncond = _StandInModel(True), _StandInModel(False)
+    x = x0.clone()
+    for k in range(steps):
+        tau = 1000.0 * (1 - k / steps)
+        _euler(x, cond.forward(x[None], None, tau)[0], uncond.forward(x[None], None, tau)[0], 5.0, 1.0 / steps)
+    np.testing.assert_allclose(x0_, x.numpy(), rtol=0, atol=1e-15)
