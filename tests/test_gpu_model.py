@@ -143,7 +143,7 @@ def _block_parity(mods, wl, n_rows, tau):
     X_out = host(net.X)
     rng = np.random.default_rng(L)
     rows = np.unique(np.concatenate([rng.choice(L, n_rows, replace=False), np.arange(L - 70, L), [0]]))
-    kvs = oracle_context(w, txt, x["clip"], d, True)
+    kvs = oracle_context(w, txt, x.get("clip"), d, True)
     want = O.block_forward(X_in, e0, w, 0, kvs[0], d, rnd=True, rows=rows)
     got = X_out[:, rows]
     assert rel(got, want) < TOL_BF16
