@@ -43,6 +43,7 @@ struct Cfg {
   static constexpr int smem(int mode) { return 1024 + STAGES * STAGE_BYTES + (mode == EPI_RESID ? STG_BYTES : 0) + BAR_BYTES; }
   static_assert(1024 + STAGES * STAGE_BYTES + STG_BYTES + BAR_BYTES <= 232448, "shared memory budget of one CTA exceeded");
   static constexpr uint32_t IDESC = idesc_bf16(BM, BN, 0, 0);
+  static constexpr uint32_t IDESC_F8 = idesc_e4m3(BM, BN, 0, 0);
 };
 
 // Wait-site ids recorded in the device error word on a timeout.
@@ -55,6 +56,14 @@ __device__ __forceinline__ void epilogue32(const Epi& ep, int64_t m, int n, cons
   float v[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+  if (ep.sa) {   // FP8 operands: acc * (sa[m] * sb[n])
+    const float sm = ep.sa[m];
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      const float4 b = __ldg(reinterpret_cast<const float4*>(ep.sb + n + j));
+      v[j] *= sm * b.x; v[j + 1] *= sm * b.y; v[j + 2] *= sm * b.z; v[j + 3] *= sm * b.w;
+    }
+  }
   if (ep.bias) {
 #pragma unroll
     for (int j = 0; j < 32; j += 4) {
@@ -92,7 +101,7 @@ __device__ __forceinline__ void epilogue32(const Epi& ep, int64_t m, int n, cons
 }
 
 // ------------------------------------------------------------------ kernel
-template <int BN, int MODE>
+template <int BN, int MODE, bool F8>
 __global__ void __launch_bounds__(THREADS, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
           const __grid_constant__ CUtensorMap tmX, const Epi ep, int M, int N, int K) {
@@ -113,7 +122,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   const int n_tiles = N / BN;
   const int m_tiles = (M + BM - 1) / BM;
   const int tiles = m_tiles * n_tiles;
-  const int k_iters = (K + BK - 1) / BK;
+  constexpr int KS = F8 ? 2 * BK : BK;   // K elements per 128-byte stage row
+  const int k_iters = (K + KS - 1) / KS;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -141,8 +151,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         for (int k = 0; k < k_iters; ++k) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, SITE_EMPTY)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-          tma_load_2d(sA + stage * C::A_BYTES, &tmA, k * BK, m0, &full[stage]);
-          tma_load_2d(sB + stage * C::B_BYTES, &tmB, k * BK, n0, &full[stage]);
+          tma_load_2d(sA + stage * C::A_BYTES, &tmA, k * KS, m0, &full[stage]);
+          tma_load_2d(sB + stage * C::B_BYTES, &tmB, k * KS, n0, &full[stage]);
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -169,9 +179,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            umma_ss(d, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), C::IDESC,
-                    (k | kk) != 0);
+          for (int kk = 0; kk < BK / 16; ++kk) {   // 32 bytes of K per MMA: 16 bf16 or 32 e4m3 elements
+            if constexpr (F8)
+              umma_ss_f8(d, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), C::IDESC_F8,
+                         (k | kk) != 0);
+            else
+              umma_ss(d, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), C::IDESC,
+                      (k | kk) != 0);
           }
           umma_commit(&empty[stage]);   // frees the smem slot once these MMAs have read it
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -224,8 +238,14 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
               g = make_float4(ga.x + gb.x, ga.y + gb.y, ga.z + gb.z, ga.w + gb.w);
             }
             const float4 bb = ep.bias ? __ldg(reinterpret_cast<const float4*>(ep.bias + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
-            row[j ^ (lane & 7)] = make_float4(g.x * (__uint_as_float(r[4 * j]) + bb.x), g.y * (__uint_as_float(r[4 * j + 1]) + bb.y),
-                                              g.z * (__uint_as_float(r[4 * j + 2]) + bb.z), g.w * (__uint_as_float(r[4 * j + 3]) + bb.w));
+            float4 a = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                   __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+            if (ep.sa) {   // FP8 operands: acc * (sa[m] * sb[n])
+              const float sm = m < M ? ep.sa[m] : 0.f;
+              const float4 sb = __ldg(reinterpret_cast<const float4*>(ep.sb + n));
+              a.x *= sm * sb.x; a.y *= sm * sb.y; a.z *= sm * sb.z; a.w *= sm * sb.w;
+            }
+            row[j ^ (lane & 7)] = make_float4(g.x * (a.x + bb.x), g.y * (a.y + bb.y), g.z * (a.z + bb.z), g.w * (a.w + bb.w));
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -273,17 +293,19 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2D bf16 tensor map over a row-major [rows, cols] matrix with row stride
-// `ld` elements; box = box_cols x box_rows, 128-byte swizzle.
+// 2D tensor map over a row-major [rows, cols] matrix of bf16 (or, with
+// one_byte, e4m3 codes as uint8) with row stride `ld` elements; box =
+// box_cols x box_rows, 128-byte swizzle.
 static wd_status make_tmap_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
-                                int box_cols, int box_rows) {
+                                int box_cols, int box_rows, bool one_byte = false) {
   auto fn = encode_fn();
   if (!fn) { set_error("cuTensorMapEncodeTiled unavailable"); return WD_ERR_CUDA; }
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * (one_byte ? 1 : 2)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t es[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+  CUresult r = fn(m, one_byte ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) { set_error("cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r)); return WD_ERR_CUDA; }
@@ -315,7 +337,7 @@ static wd_status make_tmap_f32(CUtensorMap* m, const void* base, int64_t rows, i
   return WD_OK;
 }
 
-template <int BN, int MODE>
+template <int BN, int MODE, bool F8 = false>
 static wd_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const Epi& ep, int M, int N, int K,
                            cudaStream_t st) {
   using C = tcg::Cfg<BN>;
@@ -323,7 +345,7 @@ static wd_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const E
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr[dev & 15]) {
-    cudaFuncSetAttribute(tcg::k_gemm_tc<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::smem(MODE));
+    cudaFuncSetAttribute(tcg::k_gemm_tc<BN, MODE, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::smem(MODE));
     attr[dev & 15] = true;
   }
   const int tiles = ((M + tcg::BM - 1) / tcg::BM) * (N / BN);
@@ -331,7 +353,7 @@ static wd_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const E
   CUtensorMap tx = ta;   // unused unless the epilogue adds into the fp32 residual
   if (MODE == EPI_RESID) WD_TRY(make_tmap_f32(&tx, ep.out, M, N, ep.ldo, 32, 32));
   Trace tr(KC_GEMM, st);
-  tcg::k_gemm_tc<BN, MODE><<<grid, tcg::THREADS, C::smem(MODE), st>>>(ta, tb, tx, ep, M, N, K);
+  tcg::k_gemm_tc<BN, MODE, F8><<<grid, tcg::THREADS, C::smem(MODE), st>>>(ta, tb, tx, ep, M, N, K);
   return launch_status("gemm_tc");
 }
 
@@ -376,6 +398,38 @@ wd_status gemm_tc(int M, int N, int K, const bf16* A, int64_t lda, const bf16* B
     case 128: return dispatch_mode<128>(mode, ta, tb, ep, M, N, K, st);
     default: return dispatch_mode<64>(mode, ta, tb, ep, M, N, K, st);
   }
+}
+
+// e4m3 operands: N a multiple of 256 (one tile width), K and the row strides
+// multiples of 16 bytes; the block's GEMMs all have that shape.
+wd_status gemm_tc_fp8(int M, int N, int K, const uint8_t* A, int64_t lda, const uint8_t* B, int64_t ldb, int mode,
+                      const Epi& ep, cudaStream_t st) {
+  if (M <= 0 || N <= 0 || K <= 0) { set_error("gemm_fp8: empty shape %d x %d x %d", M, N, K); return WD_ERR_SHAPE; }
+  if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B)) & 15u) {
+    set_error("gemm_fp8: operands must be 16-byte aligned");
+    return WD_ERR_ALIGN;
+  }
+  if ((lda % 16) || (ldb % 16) || (K % 16)) {
+    set_error("gemm_fp8: K=%d, lda=%lld, ldb=%lld must be multiples of 16", K, (long long)lda, (long long)ldb);
+    return WD_ERR_SHAPE;
+  }
+  if (N % 256) { set_error("gemm_fp8: N=%d must be a multiple of 256", N); return WD_ERR_SHAPE; }
+  if (!ep.sa || !ep.sb) { set_error("gemm_fp8: row and column scales are required"); return WD_ERR_ARG; }
+  if (ep.ldo % 8 || (reinterpret_cast<uintptr_t>(ep.out) & 15u)) {
+    set_error("gemm_fp8: output must be 16-byte aligned with ldo %% 8 == 0");
+    return WD_ERR_ALIGN;
+  }
+  CUtensorMap ta, tb;
+  WD_TRY(make_tmap_bf16(&ta, A, M, K, lda, 2 * tcg::BK, tcg::BM, true));
+  WD_TRY(make_tmap_bf16(&tb, B, N, K, ldb, 2 * tcg::BK, 256, true));
+  switch (mode) {
+    case EPI_STORE: return launch_tc<256, EPI_STORE, true>(ta, tb, ep, M, N, K, st);
+    case EPI_GELU: return launch_tc<256, EPI_GELU, true>(ta, tb, ep, M, N, K, st);
+    case EPI_F32: return launch_tc<256, EPI_F32, true>(ta, tb, ep, M, N, K, st);
+    case EPI_RESID: return launch_tc<256, EPI_RESID, true>(ta, tb, ep, M, N, K, st);
+  }
+  set_error("gemm_fp8: bad epilogue %d", mode);
+  return WD_ERR_ARG;
 }
 
 }  // namespace wd

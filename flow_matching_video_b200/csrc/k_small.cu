@@ -1,7 +1,10 @@
 // k_small.cu — the bandwidth-bound and latency-bound kernels of the step:
 // conditioning y, CFG Euler update, shared time MLP, adaLN norm+modulate,
-// QK-RMSNorm + 3D RoPE, and the patch gather feeding the patch-embed GEMM.
+// QK-RMSNorm + 3D RoPE, the patch gather feeding the patch-embed GEMM, and
+// the per-row e4m3 quantisation feeding the FP8 GEMM.
 #include "wd_internal.cuh"
+
+#include <cuda_fp8.h>
 
 namespace wd {
 
@@ -324,5 +327,67 @@ __global__ void __launch_bounds__(256) k_patch_gather(const float* __restrict__ 
     a[i] = from_f<T>(v);
   }
 }
+
+
+// ============================================================ e4m3 row quantisation
+// One warp per row: amax over the row, scale = amax / 448 (IEEE division), then
+// q = e4m3(x / scale) with round-to-nearest-even and saturation at +-448 (the
+// FP8 GEMM of "Wan（通义万相）..." 5.3 with per-token / per-channel scales).
+// Each lane converts 8 consecutive elements per pass; K is a multiple of 8.
+template <typename T>
+__global__ void __launch_bounds__(256) k_quant_rows_e4m3(const T* __restrict__ x, int rows, int K,
+                                                          uint8_t* __restrict__ q, float* __restrict__ scale) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const T* xr = x + static_cast<int64_t>(row) * K;
+  auto load8 = [&](int k, float (&v)[8]) {
+    if constexpr (sizeof(T) == 2) {
+      const uint4 u = *reinterpret_cast<const uint4*>(xr + k);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = unpack_bf16x2(w[i]);
+        v[2 * i] = f.x; v[2 * i + 1] = f.y;
+      }
+    } else {
+      const float4 a = *reinterpret_cast<const float4*>(xr + k), b = *reinterpret_cast<const float4*>(xr + k + 4);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+  };
+  float amax = 0.f;
+  for (int k = 8 * lane; k < K; k += 256) {
+    float v[8];
+    load8(k, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+  uint8_t* qr = q + static_cast<int64_t>(row) * K;
+  for (int k = 8 * lane; k < K; k += 256) {
+    float v[8];
+    load8(k, v);
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t c = __nv_cvt_float_to_fp8(__fdiv_rn(v[i], s), __NV_SATFINITE, __NV_E4M3);
+      w[i >> 2] |= c << (8 * (i & 3));
+    }
+    *reinterpret_cast<uint2*>(qr + k) = make_uint2(w[0], w[1]);
+  }
+  if (lane == 0) scale[row] = s;
+}
+
+template <typename T>
+wd_status quant_rows_e4m3(int rows, int K, const T* x, uint8_t* q, float* scale, cudaStream_t st) {
+  if (rows <= 0 || K <= 0 || K % 8) { set_error("quant_rows: rows=%d, K=%d (K a multiple of 8)", rows, K); return WD_ERR_SHAPE; }
+  const int64_t threads = static_cast<int64_t>(rows) * 32;
+  Trace tr(KC_SMALL, st);
+  k_quant_rows_e4m3<T><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(x, rows, K, q, scale);
+  return launch_status("quant_rows_e4m3");
+}
+template wd_status quant_rows_e4m3<bf16>(int, int, const bf16*, uint8_t*, float*, cudaStream_t);
+template wd_status quant_rows_e4m3<float>(int, int, const float*, uint8_t*, float*, cudaStream_t);
 
 }  // namespace wd

@@ -483,6 +483,28 @@ wd_status wd_gemm(int dtype, int M, int N, int K, const void* A, const void* B, 
   return WD_ERR_DTYPE;
 }
 
+// Per-row e4m3 quantisation and the FP8 GEMM ("Wan（通义万相）..." 5.3).
+wd_status wd_quant_rows_e4m3(int dtype, int rows, int K, const void* x, void* q, float* scale, wd_stream stream) {
+  WD_NEED(x); WD_NEED(q); WD_NEED(scale);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == WD_BF16) return quant_rows_e4m3<bf16>(rows, K, static_cast<const bf16*>(x), static_cast<uint8_t*>(q), scale, st);
+  if (dtype == WD_F32) return quant_rows_e4m3<float>(rows, K, static_cast<const float*>(x), static_cast<uint8_t*>(q), scale, st);
+  set_error("dtype %d", dtype);
+  return WD_ERR_DTYPE;
+}
+
+wd_status wd_gemm_fp8(int M, int N, int K, const void* Aq, const float* sa, const void* Bq, const float* sb,
+                      const float* bias, int epilogue, void* out, const float* gate_a, const float* gate_b,
+                      wd_stream stream) {
+  WD_NEED(Aq); WD_NEED(sa); WD_NEED(Bq); WD_NEED(sb); WD_NEED(out); WD_OPT(bias); WD_OPT(gate_a); WD_OPT(gate_b);
+  if (epilogue < 0 || epilogue > EPI_RESID) { set_error("gemm_fp8: epilogue %d (0-3)", epilogue); return WD_ERR_ARG; }
+  Epi ep = epi(out, N, bias, gate_a, gate_b);
+  ep.sa = sa;
+  ep.sb = sb;
+  return gemm_tc_fp8(M, N, K, static_cast<const uint8_t*>(Aq), K, static_cast<const uint8_t*>(Bq), K, epilogue, ep,
+                     static_cast<cudaStream_t>(stream));
+}
+
 // O[b, l, h*dh:(h+1)*dh] = softmax(q k^T / sqrt(dh)) v  (+ second segment).
 // q [batch, Lq, heads*dh]; k1/v1 [batch or 1 (kv1_shared), n1, heads*dh];
 // k2/v2 likewise or NULL; o [batch, Lq, heads*dh] (bf16 when the operands

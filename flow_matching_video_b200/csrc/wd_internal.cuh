@@ -88,6 +88,8 @@ struct Epi {
   const float* gate_a;    // EPI_RESID: gate = gate_a[n] + gate_b[n]; both null -> 1
   const float* gate_b;
   int T, Hp, Wp, L;       // EPI_UNPATCH geometry
+  const float* sa;        // FP8 GEMM: acc[m, n] is scaled by sa[m] * sb[n] before the bias; null otherwise
+  const float* sb;
 };
 
 // Unpatchify address of GEMM element (row m = b*L + l, column n = c*4+kh*2+kw).
@@ -108,6 +110,13 @@ wd_status gemm_simt(int M, int N, int K, const T* A, int64_t lda, const T* B, in
 // Tensor-core (tcgen05 + TMA) bf16 GEMM.
 wd_status gemm_tc(int M, int N, int K, const bf16* A, int64_t lda, const bf16* B, int64_t ldb, int mode,
                   const Epi& ep, cudaStream_t st);
+// The same with e4m3 operands (one byte each; lda, ldb in elements = bytes) and the
+// scales ep.sa[M], ep.sb[N] applied to the fp32 accumulator.
+wd_status gemm_tc_fp8(int M, int N, int K, const uint8_t* A, int64_t lda, const uint8_t* B, int64_t ldb, int mode,
+                      const Epi& ep, cudaStream_t st);
+// Per-row e4m3 quantisation: scale[r] = amax_r / 448, q[r, k] = e4m3(x[r, k] / scale[r]).
+template <typename T>
+wd_status quant_rows_e4m3(int rows, int K, const T* x, uint8_t* q, float* scale, cudaStream_t st);
 
 // Multi-head attention O = softmax(Q K^T / sqrt(dh)) V per (batch, head),
 // optionally summed with a second, independently normalised key/value

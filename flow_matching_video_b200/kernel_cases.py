@@ -3,12 +3,13 @@
     python -m flow_matching_video_b200.kernel_cases CASE [--batch B] [--iters N] [--warmup W]
 
 CASE is one of attn_self, attn_cross, gemm_qkv, gemm_o, gemm_ffn1, gemm_ffn2,
-euler, euler_hbm (the norm and RoPE kernels are timed inside the step).
+euler, euler_hbm, gemm_fp8_qkv, gemm_fp8_o, gemm_fp8_ffn1, gemm_fp8_ffn2,
+quant_ffn_hidden (the norm and RoPE kernels are timed inside the step).
 Shapes are those of one block of the 30-block 480p/81-frame model (L = 32760
 tokens per sample, D = 1536, 12 heads x 128, FFN 8960, 257 image + 512 text
-keys); euler_hbm streams 2^26 elements so that every launch reads HBM.  Inputs are seeded random values; the
-case prints the mean device time per launch (CUDA events) and the
-algorithmic FLOPs or bytes per launch.
+keys); euler_hbm streams 2^26 elements so that every launch reads HBM.
+Inputs are seeded random values; the case prints the mean device time per
+launch (CUDA events) and the algorithmic FLOPs or bytes per launch.
 """
 from __future__ import annotations
 
@@ -51,6 +52,23 @@ def make_case(name: str, B: int):
         g = torch.zeros(N, device="cuda")
         return (lambda: wd.wd_gemm(wd.WD_BF16, rows, N, K, A, W, bias, epi, out,
                                    g if epi == wd.EPI_RESID else None)), 2.0 * rows * N * K, "FLOP"
+    fp8 = {"gemm_fp8_qkv": (3 * D, D, wd.EPI_STORE), "gemm_fp8_o": (D, D, wd.EPI_RESID),
+           "gemm_fp8_ffn1": (F, D, wd.EPI_GELU), "gemm_fp8_ffn2": (D, F, wd.EPI_RESID)}
+    if name in fp8:   # e4m3 operands with per-row scales; FLOPs counted as for the bf16 GEMM
+        N, K, epi = fp8[name]
+        A, W = bf(rows, K), bf(N, K) * 0.02
+        qa, sa = torch.empty((rows, K), dtype=torch.uint8, device="cuda"), torch.empty(rows, device="cuda")
+        qw, sw = torch.empty((N, K), dtype=torch.uint8, device="cuda"), torch.empty(N, device="cuda")
+        wd.wd_quant_rows_e4m3(wd.WD_BF16, rows, K, A, qa, sa)
+        wd.wd_quant_rows_e4m3(wd.WD_BF16, N, K, W, qw, sw)
+        bias, g = torch.zeros(N, device="cuda"), torch.zeros(N, device="cuda")
+        out = torch.zeros(rows, N, device="cuda", dtype=torch.float32 if epi == wd.EPI_RESID else torch.bfloat16)
+        return (lambda: wd.wd_gemm_fp8(rows, N, K, qa, sa, qw, sw, bias, epi, out,
+                                       g if epi == wd.EPI_RESID else None)), 2.0 * rows * N * K, "FLOP"
+    if name == "quant_ffn_hidden":   # the FFN hidden activations [B*L, 8960] bf16 -> e4m3 + row scales
+        x = bf(rows, F)
+        q, sc = torch.empty((rows, F), dtype=torch.uint8, device="cuda"), torch.empty(rows, device="cuda")
+        return (lambda: wd.wd_quant_rows_e4m3(wd.WD_BF16, rows, F, x, q, sc)), 3.0 * rows * F + 4.0 * rows, "B"
     d = synth.Dims(D=D, heads=H, ffn=F, blocks=1, T=21, H=60, W=104, n_txt=NT, c_txt=4096, n_img=NI,
                    c_img=1280, dtype="bf16")
     if name in ("euler", "euler_hbm"):

@@ -70,6 +70,8 @@ SIGNATURES = {
     "wd_euler_cfg_step": (_I, [_P, _P, _P, _F, _F, _S, _P]),
     "wd_gemm": (_I, [_I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P]),
     "wd_attention": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P, _I, _I, _P, _P]),
+    "wd_quant_rows_e4m3": (_I, [_I, _I, _I, _P, _P, _P, _P]),
+    "wd_gemm_fp8": (_I, [_I, _I, _I, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P]),
     "wd_set_debug_flags": (None, [C.c_uint]),
     "wd_trace_enable": (None, [_I]),
     "wd_trace_read": (_I, [C.POINTER(C.c_int64), C.POINTER(C.c_double)]),
@@ -185,6 +187,15 @@ def wd_euler_cfg_step(x, v_cond, v_uncond, cfg_scale: float, dt: float, n=None, 
     n = x.numel() if n is None else n
     _ok(_lib.wd_euler_cfg_step(_p(x), _p(v_cond), _p(v_uncond), float(cfg_scale), float(dt), n, _stream(stream)),
         "wd_euler_cfg_step")
+
+
+def wd_quant_rows_e4m3(dtype, rows, K, x, q, scale, stream=None):
+    _ok(_lib.wd_quant_rows_e4m3(dtype, rows, K, _p(x), _p(q), _p(scale), _stream(stream)), "wd_quant_rows_e4m3")
+
+
+def wd_gemm_fp8(M, N, K, Aq, sa, Bq, sb, bias, epilogue, out, gate_a=None, gate_b=None, stream=None):
+    _ok(_lib.wd_gemm_fp8(M, N, K, _p(Aq), _p(sa), _p(Bq), _p(sb), _p(bias), epilogue, _p(out), _p(gate_a),
+                         _p(gate_b), _stream(stream)), "wd_gemm_fp8")
 
 
 def wd_gemm(dtype, M, N, K, A, B, bias, epilogue, out, gate_a=None, gate_b=None, stream=None):

@@ -266,6 +266,29 @@ wd_status wd_attention(int dtype, int batch, int Lq, int heads, int dh, const vo
                        int n1, int kv1_shared, const void* k2, const void* v2, int n2, int kv2_shared, void* o,
                        wd_stream stream);
 
+/* FP8 building blocks ([WAN] 5.3: FP8 GEMM with per-token activation and
+ * per-channel weight scales).  No counterpart is wired into wd_block_forward:
+ * the block runs bf16; these are the next step's kernels, exposed to be
+ * checked and measured on their own. */
+
+/* Per-row e4m3 quantisation: for each row r of x [rows, K] (dtype WD_BF16 or
+ * WD_F32, K a multiple of 8), scale[r] = max_k |x[r,k]| / 448 (1 for an
+ * all-zero row, fp32, IEEE division) and q[r,k] = e4m3(x[r,k] / scale[r])
+ * (one byte per element, round-to-nearest-even, saturating at +-448), so that
+ * x ~ scale[r] * q.  For a Linear weight [out, in] the rows are the output
+ * channels. */
+wd_status wd_quant_rows_e4m3(int dtype, int rows, int K, const void* x, void* q, float* scale, wd_stream stream);
+
+/* FP8 GEMM on the tcgen05 tensor cores (kind::f8f6f4): with
+ * v[m,n] = sa[m] * sb[n] * sum_k Aq[m,k] Bq[n,k] + bias[n] (fp32 accumulation),
+ * the epilogues of wd_gemm: 0 out bf16 = v, 1 out bf16 = GELU(v), 2 out fp32
+ * = v, 3 out fp32 += (gate_a + gate_b) * v.  Aq [M,K] and Bq [N,K] e4m3 from
+ * wd_quant_rows_e4m3, sa [M], sb [N] their scales; N a multiple of 256, K a
+ * multiple of 16; out [M,N]. */
+wd_status wd_gemm_fp8(int M, int N, int K, const void* Aq, const float* sa, const void* Bq, const float* sb,
+                      const float* bias, int epilogue, void* out, const float* gate_a, const float* gate_b,
+                      wd_stream stream);
+
 /* ------------------------------------------------------------------ tracing
  * Every kernel launch is counted by class.  With timing enabled, each launch
  * is also bracketed by two CUDA events recorded on its own stream, so the

@@ -519,3 +519,41 @@ def sample_cfg_cache(x0, img_lat, w: dict, txt, clip, dims, steps: int, cfg_scal
         trace.append((v_c, v_u))
         x = euler_cfg_step(x, v_c, v_u, cfg_scale, dt)
     return x, trace, fresh
+
+
+# ---------------------------------------------------------------- FP8 building blocks ([WAN] 5.3)
+E4M3_MAX = 448.0
+
+
+def e4m3(a) -> np.ndarray:
+    """Round to the nearest float8 e4m3 value (1 sign, 4 exponent bits with
+    bias 7, 3 mantissa bits, no infinities), ties to even, saturating at +-448.
+    Normal values keep 4 significant bits: for a = m * 2**e (|m| in [0.5, 1))
+    the spacing is 2**(e - 4); below 2**-6 it stays 2**-9 (subnormals)."""
+    a = np.asarray(a, dtype=F64)
+    _, e = np.frexp(a)
+    q = np.maximum(e - 4, -9)
+    r = np.ldexp(np.rint(np.ldexp(a, -q)), q)
+    return np.clip(r, -E4M3_MAX, E4M3_MAX)
+
+
+def quant_rows_e4m3(x):
+    """Per-row (per-token, or per-output-channel for a weight) FP8 quantisation
+    of [WAN] 5.3 "FP8 GEMM": scale_r = amax_r / 448 and q = e4m3(x / scale_r), so
+    that x ~ scale_r * q.  Reading: the scale and the quotient are computed in
+    fp32 (IEEE division, the precision the kernel uses, so both sides take the
+    same rounding decisions); an all-zero row gets scale 1.
+    Returns (q [rows, K] float64 holding e4m3 values, scale [rows] float32)."""
+    x = np.asarray(x, dtype=np.float32)
+    amax = np.abs(x).max(axis=1)
+    scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    y = (x / scale[:, None]).astype(np.float32)
+    return e4m3(y), scale
+
+
+def gemm_fp8(qa, sa, qb, sb, bias=None):
+    """C[m, n] = sa[m] * sb[n] * sum_k qa[m, k] qb[n, k] (+ bias[n]): the FP8 GEMM
+    with per-row scales of both operands, products and sums in float64."""
+    acc = np.asarray(qa, F64) @ np.asarray(qb, F64).T
+    out = acc * np.asarray(sa, F64)[:, None] * np.asarray(sb, F64)[None, :]
+    return out + np.asarray(bias, F64) if bias is not None else out

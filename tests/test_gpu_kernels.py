@@ -289,3 +289,70 @@ def test_attention_bf16_simt_reference_kernel(wd, half):
     finally:
         wd.wd_set_debug_flags(0)
     assert_within(got, want, bound)
+
+
+# ------------------------------------------------------------------ FP8 building blocks ("Wan（通义万相）..." 5.3)
+def _e4m3_bytes(vals):
+    """e4m3 values (float64, exactly representable) -> their one-byte codes."""
+    return torch.from_numpy(np.ascontiguousarray(vals)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+@pytest.mark.parametrize("rows,K,dtype", [(257, 1536, "bf16"), (3, 8, "bf16"), (130, 8960, "bf16"), (64, 136, "f32")])
+def test_quant_rows_e4m3_bit_exact(wd, rows, K, dtype):
+    rng = np.random.default_rng(rows + K)
+    x = (rng.standard_normal((rows, K)) * np.exp(rng.uniform(-4, 4, (rows, 1)))).astype(np.float32)
+    x[min(1, rows - 1)] = 0.0                                    # an all-zero row
+    if dtype == "bf16":
+        x = bf(x).astype(np.float32)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    q = torch.empty((rows, K), dtype=torch.uint8, device="cuda")
+    s = torch.empty(rows, dtype=torch.float32, device="cuda")
+    wd.wd_quant_rows_e4m3(wd.WD_BF16 if dtype == "bf16" else wd.WD_F32, rows, K, dev(x, tdt), q, s)
+    wd.wd_check()
+    want_q, want_s = O.quant_rows_e4m3(x)
+    np.testing.assert_array_equal(s.cpu().numpy(), want_s)
+    np.testing.assert_array_equal(q.cpu().numpy(), _e4m3_bytes(want_q))
+
+
+FP8_SHAPES = [(300, 256, 128), (2000, 1536, 1536), (1000, 8960, 1536), (513, 1536, 8960), (129, 4608, 64)]
+
+
+@pytest.mark.parametrize("M,N,K", FP8_SHAPES)
+@pytest.mark.parametrize("epi", [0, 1, 2, 3])
+def test_gemm_fp8_tensor_cores(wd, M, N, K, epi):
+    """Operands quantised on the GPU (checked against the oracle's codes), then the
+    e4m3 GEMM against the oracle's scaled product of the same codes.  Bound: the
+    products of two e4m3 codes are exact in fp32, so the accumulation errs by at
+    most 2K u sum|qa qb|; scaling and bias add 3 u |v|; a bf16 store 2^-8 |v|."""
+    rng = np.random.default_rng(M + N + K + epi)
+    A = bf(rng.standard_normal((M, K))).astype(np.float32)
+    B = bf(rng.standard_normal((N, K)) * 0.05).astype(np.float32)
+    bias = rng.standard_normal(N).astype(np.float32) * 0.1
+    ga, gb = rng.standard_normal(N).astype(np.float32), rng.standard_normal(N).astype(np.float32) * 0.1
+    qa, sa = (torch.empty((M, K), dtype=torch.uint8, device="cuda"), torch.empty(M, device="cuda"))
+    qb, sb = (torch.empty((N, K), dtype=torch.uint8, device="cuda"), torch.empty(N, device="cuda"))
+    wd.wd_quant_rows_e4m3(wd.WD_BF16, M, K, dev(A, torch.bfloat16), qa, sa)
+    wd.wd_quant_rows_e4m3(wd.WD_BF16, N, K, dev(B, torch.bfloat16), qb, sb)
+    oqa, osa = O.quant_rows_e4m3(A)
+    oqb, osb = O.quant_rows_e4m3(B)
+    np.testing.assert_array_equal(qa.cpu().numpy(), _e4m3_bytes(oqa))
+    np.testing.assert_array_equal(qb.cpu().numpy(), _e4m3_bytes(oqb))
+    v = O.gemm_fp8(oqa, osa, oqb, osb, bias)
+    s2 = np.abs(osa.astype(np.float64))[:, None] * np.abs(osb.astype(np.float64))[None, :]
+    acc_err = 2.0 * K * U32 * (np.abs(oqa) @ np.abs(oqb).T) * s2 + 3 * U32 * (np.abs(v) + np.abs(bias))
+    if epi == 3:
+        X0 = rng.standard_normal((M, N)).astype(np.float32)
+        out = dev(X0)
+        g = ga.astype(np.float64) + gb
+        want = X0 + g * v
+        bound = np.abs(g) * acc_err + 2 * U32 * (np.abs(X0) + np.abs(g * v))
+    else:
+        out = torch.empty((M, N), device="cuda", dtype=torch.float32 if epi == 2 else torch.bfloat16)
+        want = O.gelu(v) if epi == 1 else v
+        bound = (1.13 if epi == 1 else 1.0) * acc_err + U32 * np.abs(want) + 1e-6 * (epi == 1)
+        if epi != 2:
+            bound = bound * (1 + BF16_HALF_ULP) + BF16_HALF_ULP * np.abs(want)
+    wd.wd_gemm_fp8(M, N, K, qa, sa, qb, sb, dev(bias), epi, out, dev(ga) if epi == 3 else None,
+                   dev(gb) if epi == 3 else None)
+    wd.wd_check()
+    assert_within(host(out), want, bound)

@@ -579,3 +579,43 @@ def test_cfg_cache_is_exact_at_guidance_scale_one():
     xc, _, fresh = O.sample_cfg_cache(x["x0"], x["img_lat"], w, *args, t_cfg=0.6)
     assert fresh == [True, True, False, False]
     np.testing.assert_allclose(xc, O.sample(x["x0"], x["img_lat"], w, *args)[0], atol=1e-12)
+
+
+# ------------------------------------------------------------------ FP8 building blocks ([WAN] 5.3)
+def test_e4m3_round_matches_torch_conversion():
+    a = RNG.standard_normal(20000) * np.exp(RNG.uniform(-14, 7, 20000))
+    a = a[np.abs(a) <= 448.0]                      # torch's e4m3fn turns overflow into NaN; saturation is pinned below
+    # exact ties between neighbouring e4m3 values, both parities
+    codes = np.arange(1, 0x7E, dtype=np.uint8)     # positive finite codes below 448
+    vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    ties = (vals[:-1] + vals[1:]) / 2
+    a = np.concatenate([a, ties, -ties, [0.0, -0.0, 448.0, 2.0 ** -9, 2.0 ** -10, 3 * 2.0 ** -10]])
+    want = torch.from_numpy(a).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.e4m3(a), want)
+    # saturation at the largest finite value
+    np.testing.assert_array_equal(O.e4m3([464.0, 1e6, -500.0]), [448.0, 448.0, -448.0])
+
+
+def test_quant_rows_reconstructs_within_half_an_e4m3_step():
+    x = (RNG.standard_normal((64, 300)) * np.exp(RNG.uniform(-3, 3, (64, 1)))).astype(np.float32)
+    x[5] = 0.0                                      # an all-zero row
+    q, s = O.quant_rows_e4m3(x)
+    assert s.dtype == np.float32 and s[5] == 1.0 and np.all(q[5] == 0)
+    assert np.all(np.abs(q).max(axis=1)[np.arange(64) != 5] == 448.0)   # each row's amax maps to 448
+    err = np.abs(q * s[:, None].astype(np.float64) - x)
+    # |x/s - q| <= half a step of the e4m3 grid at |x/s| (2^-4 relative, or 2^-10 absolute below 2^-6),
+    # plus the fp32 rounding of x / s
+    y = np.abs(x / s[:, None])
+    step = np.maximum(2.0 ** (np.floor(np.log2(np.maximum(y, 2.0 ** -6))) - 3), 2.0 ** -9)
+    assert np.all(err <= (step / 2 + y * 2.0 ** -23) * s[:, None] + 1e-30)
+
+
+def test_gemm_fp8_is_the_scaled_integer_dot_product():
+    # e4m3 values times 2^9 are integers: the GEMM of the codes is an exact integer product
+    qa = O.e4m3(RNG.standard_normal((7, 64)) * 20)
+    qb = O.e4m3(RNG.standard_normal((5, 64)) * 20)
+    ia, ib = (qa * 512).astype(np.int64), (qb * 512).astype(np.int64)
+    assert np.all(ia == qa * 512) and np.all(ib == qb * 512)
+    sa, sb, bias = RNG.uniform(0.5, 2, 7), RNG.uniform(0.5, 2, 5), RNG.standard_normal(5)
+    want = (ia @ ib.T).astype(np.float64) / 512 ** 2 * sa[:, None] * sb[None, :] + bias
+    np.testing.assert_allclose(O.gemm_fp8(qa, sa, qb, sb, bias), want, rtol=1e-15, atol=1e-12)
