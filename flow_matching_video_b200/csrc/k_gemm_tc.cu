@@ -7,11 +7,11 @@
 // weight [N, K]; both K-major, loaded by TMA into 128-byte-swizzled shared
 // memory tiles of 64 K-elements.
 //
-// CTA = 2 + 4 * EPI_WG warps, persistent over output tiles of 128 x BN:
+// CTA = 2 + 4 * epi_wg warps, persistent over output tiles of 128 x BN:
 //   warp 0     TMA producer (one lane): STAGES-deep ring of (A, B) tiles
 //   warp 1     TMEM owner + MMA issuer (one lane): 128 x BN x 16 UMMAs,
 //              accumulating in one of two TMEM buffers
-//   warps 2..  epilogue, EPI_WG warpgroups: each warp reads its 32-lane
+//   warps 2..  epilogue, epi_wg warpgroups: each warp reads its 32-lane
 //              quarter of the accumulator for its warpgroup's share of the
 //              columns (tcgen05.ld), applies the epilogue and stores; they
 //              release the TMEM buffer so the next tile's MMAs overlap it.
@@ -23,11 +23,11 @@ namespace wd {
 namespace tcg {
 
 constexpr int BM = 128, BK = 64;
-#ifndef WD_GEMM_EPI_WG
-#define WD_GEMM_EPI_WG 1   // epilogue warpgroups; each takes an equal share of the tile's columns
-#endif
-constexpr int EPI_WG = WD_GEMM_EPI_WG;
-constexpr int THREADS = 64 + 128 * EPI_WG;
+// Epilogue warpgroups per mode, each taking an equal share of a tile's columns:
+// two for the GELU epilogue (erf per element; with e4m3 operands it outlasts
+// the MMAs of a tile), one otherwise.
+template <int MODE> __host__ __device__ constexpr int epi_wg() { return MODE == EPI_GELU ? 2 : 1; }
+template <int MODE> __host__ __device__ constexpr int threads() { return 64 + 128 * epi_wg<MODE>(); }
 
 template <int BN>
 struct Cfg {
@@ -39,7 +39,7 @@ struct Cfg {
   static constexpr int BAR_BYTES = 256;
   // gated residual: per epilogue warp two 32 x 32 fp32 staging tiles for the TMA reduce-add
   static constexpr int RESID_STAGE_BYTES = 32 * 32 * 4;
-  static constexpr int STG_BYTES = 4 * EPI_WG * 2 * RESID_STAGE_BYTES;
+  static constexpr int STG_BYTES = 4 * 2 * RESID_STAGE_BYTES;
   static constexpr int smem(int mode) { return 1024 + STAGES * STAGE_BYTES + (mode == EPI_RESID ? STG_BYTES : 0) + BAR_BYTES; }
   static_assert(1024 + STAGES * STAGE_BYTES + STG_BYTES + BAR_BYTES <= 232448, "shared memory budget of one CTA exceeded");
   static constexpr uint32_t IDESC = idesc_bf16(BM, BN, 0, 0);
@@ -102,7 +102,7 @@ __device__ __forceinline__ void epilogue32(const Epi& ep, int64_t m, int n, cons
 
 // ------------------------------------------------------------------ kernel
 template <int BN, int MODE, bool F8>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(threads<MODE>(), 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
           const __grid_constant__ CUtensorMap tmX, const Epi ep, int M, int N, int K) {
   using C = Cfg<BN>;
@@ -127,7 +127,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 4 * EPI_WG); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 4 * epi_wg<MODE>()); }
     mbar_init(tdone, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -202,7 +202,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   } else {
     // ---------------------------------------------------------- epilogue warps
     const int q = warp & 3;   // TMEM lane quarter this warp may access
-    constexpr int COLS = BN / EPI_WG;
+    constexpr int COLS = BN / epi_wg<MODE>();
     const int c_begin = ((warp - 2) >> 2) * COLS;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -353,7 +353,7 @@ static wd_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const E
   CUtensorMap tx = ta;   // unused unless the epilogue adds into the fp32 residual
   if (MODE == EPI_RESID) WD_TRY(make_tmap_f32(&tx, ep.out, M, N, ep.ldo, 32, 32));
   Trace tr(KC_GEMM, st);
-  tcg::k_gemm_tc<BN, MODE, F8><<<grid, tcg::THREADS, C::smem(MODE), st>>>(ta, tb, tx, ep, M, N, K);
+  tcg::k_gemm_tc<BN, MODE, F8><<<grid, tcg::threads<MODE>(), C::smem(MODE), st>>>(ta, tb, tx, ep, M, N, K);
   return launch_status("gemm_tc");
 }
 
