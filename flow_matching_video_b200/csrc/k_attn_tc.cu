@@ -96,22 +96,9 @@ struct Params {
   float scale_log2;
 };
 
-#ifndef WD_ATTN_POLL_NS
-#define WD_ATTN_POLL_NS 0    // > 0: the MMA thread and the softmax warps poll their barriers with this sleep
-#endif
-#ifndef WD_ATTN_WAIT_HINT_NS
-#define WD_ATTN_WAIT_HINT_NS 0   // > 0: suspend-time hint for the MMA thread's and softmax warps' try_wait
-#endif
-#if WD_ATTN_POLL_NS > 0
-#define MMA_WAIT(bar, par, site) mbar_wait_poll(bar, par, site, WD_ATTN_POLL_NS)
-#define SM_WAIT(bar, par, site) __all_sync(0xffffffffu, mbar_wait_poll(bar, par, site, WD_ATTN_POLL_NS))
-#elif WD_ATTN_WAIT_HINT_NS > 0
-#define MMA_WAIT(bar, par, site) mbar_wait_hint(bar, par, site, WD_ATTN_WAIT_HINT_NS)
-#define SM_WAIT(bar, par, site) __all_sync(0xffffffffu, mbar_wait_hint(bar, par, site, WD_ATTN_WAIT_HINT_NS))
-#else
+// Bounded waits: the MMA thread alone, the softmax warps as whole warps.
 #define MMA_WAIT(bar, par, site) mbar_wait(bar, par, site)
 #define SM_WAIT(bar, par, site) mbar_wait_warp(bar, par, site)
-#endif
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
