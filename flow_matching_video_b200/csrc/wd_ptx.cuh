@@ -1,6 +1,7 @@
 // wd_ptx.cuh — thin inline-PTX wrappers for sm_100a: mbarriers, TMA tiled
-// loads, tcgen05 (TMEM allocation, UMMA issue/commit, TMEM loads) and the
-// bounded waits every pipeline in this library uses.
+// loads and reduce-adds, tcgen05 (TMEM allocation, UMMA issue/commit for
+// bf16 / half / e4m3 operands, TMEM loads and stores) and the bounded waits
+// every pipeline in this library uses.
 //
 // Every wait is bounded: a wait that has not completed after WD_WAIT_NS of
 // %globaltimer time records `site` in the device error word (first writer
