@@ -116,3 +116,13 @@ def test_product_path_has_no_oracle_import():
             if f.endswith((".py", ".cu", ".cuh")):
                 src = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert not re.search(r"(from|import)\s+oracle|wan_oracle|liboracle", src), f
+
+
+def test_binding_fails_loudly_without_the_library():
+    """The product path has no fallback: the binding, run as if it sat in a
+    directory without libwd.so, refuses to import (no file is written)."""
+    path = os.path.join(ROOT, "flow_matching_video_b200", "wd.py")
+    src = open(path, encoding="utf-8").read()
+    fake = os.path.join(ROOT, "no_such_directory", "wd.py")
+    with pytest.raises(ImportError, match="libwd.so not built"):
+        exec(compile(src, path, "exec"), {"__name__": "wd_without_lib", "__file__": fake})
