@@ -33,8 +33,11 @@ def up_to_date() -> bool:
 def build(verbose: bool = False, force: bool = False) -> str:
     if not force and up_to_date():
         return OUT
+    # a temporary name per process, renamed into place atomically: ranks that
+    # start together never write into one file, and a loader never sees half a file
+    tmp = f"{OUT}.{os.getpid()}.tmp"
     cmd = [NVCC, "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
-           "-Xcompiler", "-fPIC", "-shared", "-o", OUT + ".tmp", os.path.join(SRC, "wd_lib.cu")]
+           "-Xcompiler", "-fPIC", "-shared", "-o", tmp, os.path.join(SRC, "wd_lib.cu")]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -43,7 +46,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
         raise RuntimeError("nvcc failed building libwd.so")
     if verbose:
         sys.stderr.write(r.stderr)
-    os.replace(OUT + ".tmp", OUT)
+    os.replace(tmp, OUT)
     return OUT
 
 
