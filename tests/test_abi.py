@@ -126,3 +126,20 @@ def test_binding_fails_loudly_without_the_library():
     fake = os.path.join(ROOT, "no_such_directory", "wd.py")
     with pytest.raises(ImportError, match="libwd.so not built"):
         exec(compile(src, path, "exec"), {"__name__": "wd_without_lib", "__file__": fake})
+
+
+def test_empty_sizes_are_a_no_op_or_rejected_before_launch(wd):
+    lib = wd.lib()
+    # an empty latent: nothing to update, nothing launched
+    assert lib.wd_euler_cfg_step(0x1000, 0x2000, 0x3000, 5.0, 0.5, 0, None) == 0
+    # attention without queries or keys, GEMMs without rows: WD_ERR_SHAPE, before any CUDA call
+    assert lib.wd_attention(1, 1, 0, 1, 128, 0x1000, 0x2000, 0x3000, 8, 0, None, None, 0, 0, 0x4000, None) == 2
+    assert lib.wd_attention(1, 1, 8, 1, 128, 0x1000, 0x2000, 0x3000, 0, 0, None, None, 0, 0, 0x4000, None) == 2
+    assert lib.wd_attention(2, 1, 8, 1, 128, 0x1000, 0x2000, 0x3000, 8, 1, 0x5000, 0x6000, 0, 0, 0x4000, None) == 2
+    assert lib.wd_gemm(1, 0, 64, 64, 0x1000, 0x2000, None, 0, 0x3000, None, None, None) == 2
+    assert lib.wd_gemm_fp8(0, 256, 64, 0x1000, 0x2000, 0x3000, 0x4000, None, 0, 0x5000, None, None, None) == 2
+    assert lib.wd_quant_rows_e4m3(1, 0, 64, 0x1000, 0x2000, 0x3000, None) == 2
+    assert lib.wd_quant_rows_e4m3(1, 4, 12, 0x1000, 0x2000, 0x3000, None) == 2    # K not a multiple of 8
+    # the FP8 GEMM's shape rules: N a multiple of 256, scales required
+    assert lib.wd_gemm_fp8(8, 128, 64, 0x1000, 0x2000, 0x3000, 0x4000, None, 0, 0x5000, None, None, None) == 2
+    assert lib.wd_gemm_fp8(8, 256, 64, 0x1000, None, 0x3000, 0x4000, None, 0, 0x5000, None, None, None) == 1
