@@ -619,3 +619,20 @@ def test_gemm_fp8_is_the_scaled_integer_dot_product():
     sa, sb, bias = RNG.uniform(0.5, 2, 7), RNG.uniform(0.5, 2, 5), RNG.standard_normal(5)
     want = (ia @ ib.T).astype(np.float64) / 512 ** 2 * sa[:, None] * sb[None, :] + bias
     np.testing.assert_allclose(O.gemm_fp8(qa, sa, qb, sb, bias), want, rtol=1e-15, atol=1e-12)
+
+
+# ------------------------------------------------------------------ rounding invariants (property-based)
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+_floats = st.floats(min_value=-6e4, max_value=6e4, allow_nan=False, allow_infinity=False, width=64)
+
+
+@settings(max_examples=300, deadline=None)
+@given(st.lists(_floats, min_size=2, max_size=64))
+def test_rounding_functions_are_idempotent_monotone_and_odd(xs):
+    x = np.sort(np.asarray(xs))
+    for fn in (O.bf16, O.fp16, O.e4m3):
+        r = fn(x)
+        np.testing.assert_array_equal(fn(r), r)                 # values of the format round to themselves
+        assert np.all(np.diff(r) >= 0)                          # order is kept
+        np.testing.assert_array_equal(fn(-x), -r)               # odd
