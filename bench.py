@@ -385,6 +385,19 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+def launch_ranks(n: int) -> int:
+    """Re-run this command as n ranks of torch.distributed.run on this node
+    (rendezvous on 127.0.0.1), bounded by a timeout; rank 0 prints the line."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = ["timeout", "-k", "60", "3600", sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -398,9 +411,18 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # one process per GPU: start the ranks under torch.distributed.run and wait for them
+        return launch_ranks(args.gpus)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if world != args.gpus:
+        sys.stderr.write(f"bench.py: --gpus {args.gpus} but the launcher started {world} rank(s); "
+                         f"give the launcher --nproc-per-node {args.gpus}\n")
+        return 2
     if args.impl == "reference":
         return run_reference(args, rank)
     if world > 1:

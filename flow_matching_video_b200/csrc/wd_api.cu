@@ -47,6 +47,12 @@ static wd_status check_dims(const wd_dims* d) {
   const int dh = d->D / d->heads;
   if (dh != 32 && dh != 64 && dh != 128) { set_error("head dim %d unsupported (32, 64, 128)", dh); return WD_ERR_SHAPE; }
   if (d->D % 128) { set_error("D=%d must be a multiple of 128", d->D); return WD_ERR_SHAPE; }
+  // The bf16 model runs its attention on the tensor cores, which take 128-wide heads only;
+  // other widths would fall back to the CUDA-core kernel, so a model asking for them is refused.
+  if (d->dtype == WD_BF16 && dh != 128) {
+    set_error("bf16 model: head dim %d has no tensor-core attention (128 only)", dh);
+    return WD_ERR_UNSUPPORTED;
+  }
   if (d->ffn <= 0 || d->ffn % 64) { set_error("ffn=%d must be a positive multiple of 64", d->ffn); return WD_ERR_SHAPE; }
   if (d->T <= 0 || d->T > 256 || d->H <= 0 || d->W <= 0 || (d->H & 1) || (d->W & 1)) {
     set_error("latent grid T=%d H=%d W=%d (T<=256, H and W even)", d->T, d->H, d->W);
@@ -220,6 +226,7 @@ const char* wd_last_error(void) { return g_msg; }
 const char* wd_version(void) { return "libwd 0.1 sm_100a"; }
 
 void wd_set_debug_flags(unsigned flags) { g_debug_flags = flags; }
+unsigned wd_debug_flags(void) { return g_debug_flags; }
 
 wd_status wd_check(wd_stream stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

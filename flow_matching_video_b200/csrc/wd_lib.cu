@@ -7,3 +7,4 @@
 #include "k_attn_tc.cu"
 #include "wd_api.cu"
 #include "wd_noalloc.cu"
+#include "wd_testing.cu"

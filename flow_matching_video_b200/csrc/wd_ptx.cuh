@@ -58,17 +58,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Wait until the phase with the given parity has completed.  Bounded.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned site) {
+// Wait until the phase with the given parity has completed, for at most
+// limit_ns of %globaltimer time; on running out, record `site` and return false.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, unsigned site, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0 && globaltimer_ns() - t0 > WD_WAIT_NS) {
+    if ((i & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) {
       record_error(site);
       return false;
     }
   }
+}
+// The same with the library's limit (WD_WAIT_NS): every pipeline wait.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned site) {
+  return mbar_wait_limit(bar, parity, site, WD_WAIT_NS);
 }
 
 // Bounded wait taken by all 32 lanes of a warp; the result is warp-uniform, so

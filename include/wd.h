@@ -223,9 +223,12 @@ wd_status wd_euler_cfg_step(float* x, const float* v_cond, const float* v_uncond
  * this library, WD_NOALLOC_PATCH_SCRATCH_BYTES large, which every GPU that
  * loads the library reserves until the process exits.
  * - Same arguments and results as wd_patch_embed, minus the workspace.
- * - Sizes beyond the array (batch * L * 144 * element size bytes, i.e. more
- *   than 174762 token rows in bf16 or 87381 in fp32) return WD_ERR_WORKSPACE
- *   before any launch.
+ * - The scratch takes batch * L * K * element-size bytes, with K = 144 for
+ *   the image-to-video model (36 channels x 2 x 2) and K = 64 for the
+ *   text-to-video model (16 x 2 x 2): at most 174762 token rows in bf16 or
+ *   87381 in fp32 for image-to-video, 393216 in bf16 or 196608 in fp32 for
+ *   text-to-video.  Larger requests return WD_ERR_WORKSPACE before any
+ *   launch.
  * - The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
  *   before capturing the stream into a graph.
@@ -261,7 +264,12 @@ wd_status wd_gemm(int dtype, int M, int N, int K, const void* A, const void* B, 
  * NULL for one segment.  dh in {32, 64, 128}.  dtype WD_F32: all fp32;
  * WD_BF16: all bf16; WD_F16: q, k, v IEEE half and o bf16 (the bf16 path's
  * cross-attention).  The probabilities enter the P V product in the operand
- * type (bf16 or half), with fp32 softmax statistics and accumulation. */
+ * type (bf16 or half), with fp32 softmax statistics and accumulation.
+ * Kernels: bf16 and half with dh = 128 run on the tcgen05 tensor cores; bf16
+ * and half with dh = 32 or 64, and every fp32 call, run on the CUDA cores
+ * (a reference kernel, far slower).  A WD_BF16 model (wd_dims) with heads of
+ * any width but 128 is refused with WD_ERR_UNSUPPORTED, so the model path
+ * never takes the CUDA-core attention. */
 wd_status wd_attention(int dtype, int batch, int Lq, int heads, int dh, const void* q, const void* k1, const void* v1,
                        int n1, int kv1_shared, const void* k2, const void* v2, int n2, int kv2_shared, void* o,
                        wd_stream stream);
@@ -289,6 +297,28 @@ wd_status wd_gemm_fp8(int M, int N, int K, const void* Aq, const float* sa, cons
                       const float* bias, int epilogue, void* out, const float* gate_a, const float* gate_b,
                       wd_stream stream);
 
+/* ------------------------------------------------------------------ test hooks
+ * Two entry points that exist only so that tests can reach pieces of the
+ * kernels no output of the path exposes on its own.  Not part of the step. */
+
+/* Evaluates, for each of the n fp32 values x[i], the three 2^x of the
+ * attention kernels' world: y_fma[i] = the FMA-pipe 2^x that the softmax of
+ * the tensor-core attention uses for some of its exponentials (range
+ * reduction to x = j + f, |f| <= 1/2, a degree-3 polynomial in f with a
+ * stated relative error below 7.5e-5, inputs below -125 clamped to -125),
+ * y_mufu[i] = the MUFU approximation ex2.approx.ftz.f32 used for the rest,
+ * y_lib[i] = CUDA's exp2f.  All device arrays of n floats; n > 0. */
+wd_status wd_test_exp2(const float* x, float* y_fma, float* y_mufu, float* y_lib, int64_t n, wd_stream stream);
+
+/* Launches one warp that waits on an mbarrier phase nothing completes, with
+ * the library's bounded wait given a limit of limit_ns (at most 100 ms, not
+ * the pipelines' 2 s).  When the limit runs out the wait records `site`
+ * (non-zero) in the device error word and the kernel returns; out[0] (device
+ * int) receives 1 if the wait saw completion, 0 if it ran out.  A following
+ * wd_check(stream) then returns WD_ERR_TIMEOUT naming the site and clears
+ * the word, as it does for a pipeline wait that ran out. */
+wd_status wd_test_wait_timeout(uint64_t limit_ns, unsigned site, int* out, wd_stream stream);
+
 /* ------------------------------------------------------------------ tracing
  * Every kernel launch is counted by class.  With timing enabled, each launch
  * is also bracketed by two CUDA events recorded on its own stream, so the
@@ -304,8 +334,11 @@ void wd_trace_enable(int on);
 wd_status wd_trace_read(int64_t* launches, double* total_ms);
 
 /* Debugging aid: bit 0 routes bf16 GEMMs, bit 1 bf16 attention, to the
- * CUDA-core kernels instead of the tensor-core ones.  Process-wide. */
+ * CUDA-core kernels instead of the tensor-core ones.  Process-wide, for
+ * tests only: while a bit is set every call of the library runs at CUDA-core
+ * speed.  wd_debug_flags() returns the bits in force (0 by default). */
 void wd_set_debug_flags(unsigned flags);
+unsigned wd_debug_flags(void);
 
 #ifdef __cplusplus
 }

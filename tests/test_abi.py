@@ -143,3 +143,19 @@ def test_empty_sizes_are_a_no_op_or_rejected_before_launch(wd):
     # the FP8 GEMM's shape rules: N a multiple of 256, scales required
     assert lib.wd_gemm_fp8(8, 128, 64, 0x1000, 0x2000, 0x3000, 0x4000, None, 0, 0x5000, None, None, None) == 2
     assert lib.wd_gemm_fp8(8, 256, 64, 0x1000, None, 0x3000, 0x4000, None, 0, 0x5000, None, None, None) == 1
+
+
+def test_bf16_model_needs_128_wide_heads(wd):
+    """The bf16 model's attention runs on the tensor cores (128-wide heads);
+    any other width is refused rather than run on the CUDA cores."""
+    lib = wd.lib()
+    d = wd.make_dims(synth.SMALL_BF16.dims)
+    d.heads = 4                                   # D = 256 -> 64-wide heads
+    assert wd.wd_workspace_bytes(d, 2) == 0
+    bw = wd.wd_block_weights(*([0x1000] * len(wd.BLOCK_FIELDS)))
+    assert lib.wd_block_forward(C.byref(d), C.byref(bw), 0x2000, 0x3000, 2, 0x4000, 0x5000, 1 << 30, None) == 8
+    assert "head dim 64" in wd.wd_last_error()
+    # the fp32 model keeps its CUDA-core path for any supported width
+    d = wd.make_dims(synth.TINY.dims)
+    assert wd.wd_workspace_bytes(d, 2) > 0
+    assert wd.wd_debug_flags() == 0

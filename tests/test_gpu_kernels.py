@@ -356,3 +356,47 @@ def test_gemm_fp8_tensor_cores(wd, M, N, K, epi):
                    dev(gb) if epi == 3 else None)
     wd.wd_check()
     assert_within(host(out), want, bound)
+
+
+# ------------------------------------------------------------------ the softmax's 2^x and the bounded waits
+def test_exp2_fma_within_its_stated_bound(wd):
+    """The FMA-pipe 2^x of the attention softmax, on a dense grid over
+    [-130, 0] plus every half-integer (where the range reduction's rounding
+    switches the integer part) and its float32 neighbours: relative error at
+    most 7.5e-5 against float64 2^x, the bound its polynomial was fitted to;
+    inputs below -125 give 2^-125 within the same bound.  The MUFU ex2 and
+    CUDA's exp2f are checked beside it."""
+    halves = np.arange(-130.0, 0.5, 0.5, dtype=np.float32)
+    x = np.concatenate([np.linspace(-130.0, 0.0, 2_000_001, dtype=np.float32), halves,
+                        np.nextafter(halves, np.float32(1)), np.nextafter(halves, np.float32(-200)),
+                        np.float32([-1e-30, -1e-7, -0.0, -125.0, -125.5, -126.0, -1000.0])]).astype(np.float32)
+    gx = dev(x)
+    outs = [torch.empty_like(gx) for _ in range(3)]
+    wd.wd_test_exp2(gx, *outs)
+    wd.wd_check()
+    y_fma, y_mufu, y_lib = (o.cpu().numpy().astype(np.float64) for o in outs)
+    x64 = x.astype(np.float64)
+    ref = np.exp2(np.maximum(x64, -125.0))
+    r_fma = np.abs(y_fma / ref - 1.0)
+    assert r_fma.max() <= 7.5e-5, (r_fma.max(), x[r_fma.argmax()])
+    in_range = x64 >= -125.0
+    exact = np.exp2(x64[in_range])
+    assert np.abs(y_lib[in_range] / exact - 1.0).max() <= 2.0 ** -22          # exp2f: 2 ulp
+    assert np.abs(y_mufu[in_range] / exact - 1.0).max() <= 2.0 ** -20         # far below a bf16 half-ulp
+    assert np.abs(y_fma[in_range] / y_lib[in_range] - 1.0).max() <= 7.5e-5 + 2.0 ** -22
+
+
+def test_bounded_wait_runs_out_reports_and_recovers(wd):
+    """A wait that nothing completes, with a 1 ms limit: the kernel returns,
+    wd_check reports WD_ERR_TIMEOUT with the site and clears the error word,
+    the next wd_check is clean, and the library keeps working (a GEMM then
+    meets its bound)."""
+    out = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    wd.wd_check()
+    wd.wd_test_wait_timeout(1_000_000, 0x9A1, out)
+    assert wd.wd_check_status() == 7
+    assert "0x9a1" in wd.wd_last_error()
+    assert int(out.item()) == 0
+    assert wd.wd_check_status() == 0
+    got, want, bound = _gemm_case(wd, wd.WD_BF16, 300, 192, 72, 3)
+    assert_within(got, want, bound)

@@ -54,9 +54,13 @@ def setup(mods, wl, blocks=None):
     d = wl.dims
     w = synth.model_weights(wl, blocks=blocks)
     x = synth.inputs(wl)
+    wdev = w
     if blocks is not None:
         d = synth.Dims(**{**d.__dict__, "blocks": len(blocks)})
-    dw = model.weights_to_device(w, d, "cuda")
+        # the device model numbers its blocks 0.. in the order given
+        ren = {f"blk{b}.": f"blk{j}." for j, b in enumerate(blocks)}
+        wdev = {next((ren[p] + k[len(p):] for p in ren if k.startswith(p)), k): v for k, v in w.items()}
+    dw = model.weights_to_device(wdev, d, "cuda")
     net = model.DiT(d, dw, wl.batch)
     tdt = net.tdtype
     txt = np.stack([x["txt"], np.zeros_like(x["txt"])]) if wl.batch == 2 else x["txt"][None]
@@ -120,12 +124,27 @@ def test_small_bf16_forward(mods):
 
 
 # ------------------------------------------------------------------ single bf16 blocks on sampled rows
-def _block_parity(mods, wl, n_rows, tau):
+# Against the oracle WITHOUT storage rounding (rnd=False: every intermediate in
+# float64), a bf16 run also carries the rounding of the tensors it stores in
+# bf16 / half, which the pages do not fix.  Measured on the CPU, the rounded
+# and unrounded oracles differ by 0.5 % of the RMS on a block's output and by
+# 1.2 % on its contribution (480p/17 frames); the bound for the GPU against
+# the unrounded oracle is the bf16 bar for the GPU's own arithmetic plus as
+# much again for that storage rounding.
+TOL_BF16_UNROUNDED = 2 * TOL_BF16
+
+
+def _block_parity(mods, wl, n_rows, tau, block=0, deep=None):
     """Patch embedding (every element), then one block on sampled rows.  The
     block's inputs X_in and e0 come from the oracle (rounded to fp32, the
-    residual stream's storage type) and are handed to both sides."""
+    residual stream's storage type) and are handed to both sides.  `block`
+    picks which block of the workload's model (its own seeded weights);
+    `deep` = (channel offset std, per-element std) adds a seeded synthetic
+    drift to X_in, standing in for the residual stream deep in the stack.
+    The output is compared with the oracle that mirrors the GPU's storage
+    rounding (bar TOL_BF16) and, reported and bounded, with the unrounded one."""
     model, wd = mods
-    net, w, x, txt, y, d = setup(mods, wl, blocks=[0])
+    net, w, x, txt, y, d = setup(mods, wl, blocks=[block])   # the device model's block 0 = this block
     B, L, D = wl.batch, d.L, d.D
     x_t = np.stack([x["x0"]] * B)
     X_in = O.patch_embed(x_t, None if d.t2v else O.build_cond_y(x["img_lat"]), w["pe.w"], w["pe.b"], rnd=True)
@@ -133,6 +152,9 @@ def _block_parity(mods, wl, n_rows, tau):
     wd.wd_patch_embed(net.cd, dev(x_t), y, net.w["pe.w"], net.w["pe.b"], B, net.X, net.ws)
     wd.wd_check()
     assert rel(host(net.X), X_in) < TOL_BF16
+    if deep is not None:
+        g = np.random.default_rng(1000 + block)
+        X_in = X_in + g.standard_normal(D) * deep[0] + g.standard_normal(X_in.shape) * deep[1]
     # one block, from the oracle's X_in and e0
     X_in = X_in.astype(np.float32).astype(np.float64)
     e0 = O.time_mod(w, tau, D)[1].astype(np.float32).astype(np.float64)
@@ -143,12 +165,23 @@ def _block_parity(mods, wl, n_rows, tau):
     X_out = host(net.X)
     rng = np.random.default_rng(L)
     rows = np.unique(np.concatenate([rng.choice(L, n_rows, replace=False), np.arange(L - 70, L), [0]]))
-    kvs = oracle_context(w, txt, x.get("clip"), d, True)
-    want = O.block_forward(X_in, e0, w, 0, kvs[0], d, rnd=True, rows=rows)
+    w_blk = w
+    d_blk = synth.Dims(**{**d.__dict__, "blocks": block + 1})
     got = X_out[:, rows]
-    assert rel(got, want) < TOL_BF16
+    errs = {}
+    for rnd in (True, False):
+        ctx_t, ctx_i = O.context_embed(w_blk, txt, None if d.t2v else x["clip"], rnd)
+        kv = O.cross_kv(w_blk, block, ctx_t, ctx_i, rnd)
+        want = O.block_forward(X_in, e0, w_blk, block, kv, d_blk, rnd=rnd, rows=rows)
+        errs[rnd] = (rel(got, want), rel(got - X_in[:, rows], want - X_in[:, rows]))
+    print(f"\n[{wl.name} block {block}{' deep' if deep else ''}] max|gpu-oracle|/rms: X_out {errs[True][0]:.3e}, "
+          f"contribution {errs[True][1]:.3e}; against the unrounded oracle: X_out {errs[False][0]:.3e}, "
+          f"contribution {errs[False][1]:.3e}; rms(X_in) {np.sqrt((X_in ** 2).mean()):.3f}")
+    assert errs[True][0] < TOL_BF16
     # the block's own contribution, judged on its own scale
-    assert rel(got - X_in[:, rows], want - X_in[:, rows]) < TOL_BF16
+    assert errs[True][1] < TOL_BF16
+    assert errs[False][0] < TOL_BF16_UNROUNDED
+    assert errs[False][1] < TOL_BF16_UNROUNDED
 
 
 def test_block_bf16_480p17(mods):
@@ -162,6 +195,47 @@ def test_block_bf16_480p81_batch2(mods):
 def test_block_bf16_480p81_t2v_batch2(mods):
     # text-to-video: 16-channel patch embedding, single-stream text cross-attention
     _block_parity(mods, synth.STACK_480P81_T2V, 192, 900.0)
+
+
+@pytest.mark.parametrize("block,deep", [(15, (0.55, 0.41)), (29, (0.76, 0.55))])
+def test_block_bf16_480p81_deep_blocks_batch2(mods, block, deep):
+    """Blocks 15 and 29 of the 30-block stack (their own weights), at the
+    benchmark's launch configuration (L = 32760, batch 2), on a residual
+    stream with the magnitude it has that deep: the oracle's own 30-block
+    stack of this model (short grid, T = 2, 8 x 8 latent) takes the stream
+    from RMS 0.24 after the patch embedding to 0.72 before block 15 and 0.97
+    before block 29, mostly as a per-channel offset shared by all tokens (RMS
+    0.55 and 0.76).  X_in is the patch embedding plus a seeded offset per
+    channel and per-element noise of those sizes, the same array on both
+    sides (the GPU's own deep stream is not handed to the oracle: no oracle
+    input comes from the CUDA path)."""
+    _block_parity(mods, synth.STACK_480P81, 192, 350.0, block=block, deep=deep)
+
+
+def test_stack_480p81_full_forward_is_deterministic(mods):
+    """The whole 30-block forward at L = 32760, batch 2 (device-drawn
+    weights), run twice: the residual stream and the velocity agree bit for
+    bit (every output element is written by one tile, no atomics), and they
+    are finite."""
+    model, wd = mods
+    wl = synth.STACK_480P81
+    d = wl.dims
+    w = model.random_weights_on_device(wl, torch.device("cuda"))
+    net = model.DiT(d, w, wl.batch)
+    x = synth.inputs(wl)
+    txt = np.stack([x["txt"], np.zeros_like(x["txt"])])
+    net.prepare_context(dev(txt, torch.bfloat16), dev(x["clip"], torch.bfloat16))
+    y = net.build_cond_y(dev(x["img_lat"]))
+    xb = dev(np.stack([x["x0"], x["x0"]]))
+    outs = []
+    for _ in range(2):
+        v = net.forward(xb, y, 1000.0)
+        wd.wd_check()
+        outs.append((net.X.clone(), v.clone()))
+    (X1, v1), (X2, v2) = outs
+    assert torch.isfinite(X1).all() and torch.isfinite(v1).all()
+    assert torch.equal(X1, X2) and torch.equal(v1, v2)
+    assert float(v1.float().pow(2).mean().sqrt()) > 0
 
 
 def test_block_bf16_720p81_wide_batch2(mods):

@@ -1,0 +1,316 @@
+"""More pins of the CPU oracle: the pieces of a block and of the sampler that
+the other pin file checks only with a branch switched off.
+
+* the token grid against the Conv3d output grid ("图解 Wan2.1 I2V" 5.1);
+* the self-attention branch of a block with several tokens: adaLN, the fused
+  projection, QK-RMSNorm over the full width D, the head split, 3D RoPE as a
+  complex rotation per segment with positions from the token grid, and
+  softmax attention — restated with torch (float64) and compared with the
+  oracle ("图解 Wan2.1 I2V" 5.2, 5.3 (1) and (2));
+* the cross-attention keys: each stream's keys come from its own weights
+  (zero image key weights make the image stream the mean of its values),
+  "图解 Wan2.1 I2V" 5.4;
+* the text MLP and the CLIP MLPProj against torch ("图解 Wan2.1 I2V" 7);
+* the sampler's unconditional row: zeroed text, CLIP and y unchanged
+  ("图解 Wan2.1 I2V" Q5).
+
+Each pin is also run against oracles with a plausible mistake planted
+(monkeypatched on the CPU, for the length of one test): the token grid with
+rows and columns swapped, RMSNorm per head instead of over D, a RoPE turning
+the wrong way or reading the wrong coordinate, the text and image key weights
+swapped, the unconditional row keeping its text.  The pin must fail on each.
+"""
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as TF
+
+from oracle import wan_oracle as O
+from flow_matching_video_b200 import synth
+
+RNG = np.random.default_rng(11)
+
+
+def T64(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64))
+
+
+def _tiny(T=2, H=4, W=6, D=48, heads=2, ffn=40, seed=99):
+    """A tiny fp64 model whose token grid has T, H/2 and W/2 all different
+    (2 x 2 x 3), so a swapped axis changes the positions."""
+    d = synth.Dims(D=D, heads=heads, ffn=ffn, blocks=1, T=T, H=H, W=W, n_txt=5, c_txt=12,
+                   n_img=4, c_img=10, dtype="f32")
+    wl = synth.Workload("pin", d, batch=2, seed=seed)
+    w = {k: v.astype(np.float64) for k, v in synth.model_weights(wl).items()}
+    for k in list(w):                      # larger weights so that every term matters
+        if k.endswith(".w"):
+            w[k] = w[k] * 10
+    txt = RNG.standard_normal((2, d.n_txt, d.c_txt))
+    clip = RNG.standard_normal((d.n_img, d.c_img))
+    X = RNG.standard_normal((2, d.L, D))
+    return d, w, txt, clip, X
+
+
+def _gated(w, D, g1, g2):
+    """e0 and block weights such that gate1 = g1, gate2 = g2 exactly."""
+    e0 = RNG.standard_normal((6, D))
+    mod = w["blk0.mod"].copy()
+    mod[2] = g1 - e0[2]
+    mod[5] = g2 - e0[5]
+    return e0, dict(w, **{"blk0.mod": mod})
+
+
+# ------------------------------------------------------------------ token grid
+def conv3d_token_grid(T, H, W):
+    """(frame, row, column) of every token, read off a torch Conv3d with the
+    patch embedding's kernel and stride (1, 2, 2) whose input channels carry
+    each voxel's own coordinates; the tokens are the flattened output grid
+    ("图解 Wan2.1 I2V" 5.1)."""
+    f, yy, xx = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    x_in = T64(np.stack([f, yy, xx]))[None]                # [1, 3, T, H, W]
+    wgt = torch.zeros(3, 3, 1, 2, 2, dtype=torch.float64)
+    for c in range(3):
+        wgt[c, c, 0, 0, 0] = 1.0                           # each patch's top-left voxel
+    out = TF.conv3d(x_in, wgt, stride=(1, 2, 2))           # [1, 3, T, H/2, W/2]
+    tok = out.flatten(2)[0].T.numpy()                      # [L, 3] in token order
+    return tok[:, 0].astype(int), (tok[:, 1] // 2).astype(int), (tok[:, 2] // 2).astype(int)
+
+
+def _grid_mismatch(T, H, W):
+    want = conv3d_token_grid(T, H, W)
+    got = O.grid_positions(T, H // 2, W // 2)
+    return sum(int(np.any(np.asarray(g) != np.asarray(wv))) for g, wv in zip(got, want))
+
+
+def test_grid_positions_are_the_conv3d_output_grid():
+    for T, H, W in [(2, 4, 6), (3, 10, 14), (1, 2, 8), (5, 6, 4)]:
+        assert _grid_mismatch(T, H, W) == 0
+    # the same map as unravelling the token index over (T, H/2, W/2)
+    f, y, x = np.unravel_index(np.arange(3 * 5 * 7), (3, 5, 7))
+    np.testing.assert_array_equal(np.stack(O.grid_positions(3, 5, 7)), np.stack([f, y, x]))
+
+
+def test_grid_pin_catches_swapped_rows_and_columns(monkeypatch):
+    orig = O.grid_positions
+
+    def swapped(T, Hp, Wp):   # rows and columns exchanged
+        f, y, x = orig(T, Wp, Hp)
+        return f, x, y
+    monkeypatch.setattr(O, "grid_positions", swapped)
+    assert _grid_mismatch(2, 4, 6) > 0
+
+
+# ------------------------------------------------------------------ self-attention branch
+def rope_complex(x, pos, dh):
+    """3D RoPE as complex multiplication ("图解 Wan2.1 I2V" 5.3 (2)): each head
+    of x [B, L, h, dh] is cut into frame / row / column segments of
+    dh - 4(dh//6), 2(dh//6), 2(dh//6) channels; in segment s the channel pairs
+    (2j, 2j+1) form the complex number z_j, multiplied by
+    exp(i * p_s * 10000^(-2j/d_s)) with p_s the token's coordinate on axis s."""
+    sizes = (dh - 4 * (dh // 6), 2 * (dh // 6), 2 * (dh // 6))
+    out, off = [], 0
+    for size, p in zip(sizes, pos):
+        seg = x[..., off:off + size]
+        z = torch.view_as_complex(seg.reshape(*seg.shape[:-1], size // 2, 2).contiguous())
+        j = torch.arange(size // 2, dtype=torch.float64)
+        theta = T64(p)[:, None] * torch.pow(torch.tensor(10000.0, dtype=torch.float64), -2.0 * j / size)
+        rot = torch.polar(torch.ones_like(theta), theta)[None, :, None, :]   # [1, L, 1, size/2]
+        out.append(torch.view_as_real(z * rot).reshape(seg.shape))
+        off += size
+    return torch.cat(out, dim=-1)
+
+
+def self_branch_torch(X, e0, w, d):
+    """X + gate1 * Linear_o(attention) of one block, restated with torch:
+    h = LayerNorm(X)(1 + scale1) + shift1; [q k v] = Linear_qkv(h);
+    q, k = RMSNorm over D with gains; heads split; RoPE; SDPA; Linear_o."""
+    B, L, D, h, dh = X.shape[0], d.L, d.D, d.heads, d.dh
+    mod = e0 + w["blk0.mod"]
+    Xt = T64(X)
+    hh = TF.layer_norm(Xt, (D,), eps=d.eps) * (1 + T64(mod[1])) + T64(mod[0])
+    q, k, v = TF.linear(hh, T64(w["blk0.qkv.w"]), T64(w["blk0.qkv.b"])).split(D, dim=-1)
+    q = TF.rms_norm(q, (D,), weight=T64(w["blk0.gq"]), eps=d.eps)
+    k = TF.rms_norm(k, (D,), weight=T64(w["blk0.gk"]), eps=d.eps)
+    pos = conv3d_token_grid(d.T, d.H, d.W)
+    heads = lambda t: t.reshape(B, L, h, dh)
+    q, k, v = rope_complex(heads(q), pos, dh), rope_complex(heads(k), pos, dh), heads(v)
+    o = TF.scaled_dot_product_attention(q.transpose(1, 2), k.transpose(1, 2), v.transpose(1, 2))
+    o = o.transpose(1, 2).reshape(B, L, D)
+    return (Xt + T64(mod[2]) * TF.linear(o, T64(w["blk0.o.w"]), T64(w["blk0.o.b"]))).numpy()
+
+
+def _self_branch_error():
+    d, w, txt, clip, X = _tiny()
+    e0, w = _gated(w, d.D, 0.8, 0.0)
+    # cross-attention output projection zero: the block is X + the self-attention branch
+    w = dict(w, **{"blk0.co.w": np.zeros_like(w["blk0.co.w"]), "blk0.co.b": np.zeros(d.D)})
+    ctx_t, ctx_i = O.context_embed(w, txt, clip)
+    kv = O.cross_kv(w, 0, ctx_t, ctx_i)
+    got = O.block_forward(X, e0, w, 0, kv, d)
+    want = self_branch_torch(X, e0, w, d)
+    # the branch moves X by far more than the comparison's bound
+    assert np.abs(want - X).max() > 1.0
+    return float(np.abs(got - want).max())
+
+
+def test_block_self_attention_branch_against_torch_restatement():
+    assert _self_branch_error() < 1e-10
+
+
+def test_self_attention_pin_catches_swapped_grid_axes(monkeypatch):
+    orig = O.grid_positions
+
+    def swapped(T, Hp, Wp):
+        f, y, x = orig(T, Wp, Hp)
+        return f, x, y
+    monkeypatch.setattr(O, "grid_positions", swapped)
+    assert _self_branch_error() > 1e-3
+
+
+def test_self_attention_pin_catches_rms_norm_per_head(monkeypatch):
+    def per_head(x, eps, gamma=None, dh=24):   # the tiny model's head width
+        x = np.asarray(x, np.float64)
+        s = x.reshape(*x.shape[:-1], -1, dh)
+        y = (s / np.sqrt((s * s).mean(axis=-1, keepdims=True) + eps)).reshape(x.shape)
+        return y * gamma if gamma is not None else y
+    monkeypatch.setattr(O, "rms_norm", per_head)
+    assert _self_branch_error() > 1e-3
+
+
+def test_self_attention_pin_catches_rope_turning_the_wrong_way(monkeypatch):
+    orig = O.rope_3d
+    monkeypatch.setattr(O, "rope_3d", lambda x, pf, py, px: orig(x, -np.asarray(pf), -np.asarray(py), -np.asarray(px)))
+    assert _self_branch_error() > 1e-3
+
+
+def test_self_attention_pin_catches_rope_reading_the_wrong_coordinate(monkeypatch):
+    orig = O.rope_3d
+    monkeypatch.setattr(O, "rope_3d", lambda x, pf, py, px: orig(x, pf, px, py))
+    assert _self_branch_error() > 1e-3
+
+
+def test_self_attention_pin_catches_rope_on_values(monkeypatch):
+    # the oracle's branch with RoPE also applied to v: attention of (q, k, R v)
+    orig_att = O.attention
+    d = _tiny()[0]
+    pf, py, px = conv3d_token_grid(d.T, d.H, d.W)
+
+    def att(q, k, v):
+        if v.shape[0] == d.L:   # self-attention (cross keys are fewer than L here)
+            v = O.rope_3d(v, pf, py, px)
+        return orig_att(q, k, v)
+    monkeypatch.setattr(O, "attention", att)
+    assert _self_branch_error() > 1e-3
+
+
+# ------------------------------------------------------------------ cross-attention keys and values
+def _cross_setup():
+    d, w, txt, clip, X = _tiny()
+    ctx_t, ctx_i = O.context_embed(w, txt, clip)
+    qc = RNG.standard_normal((7, d.heads, d.dh)) * 3
+    return d, w, ctx_t, ctx_i, qc
+
+
+def _cross_kv_errors(cross_kv):
+    """With the image key weight zero, every image key is the bias, so the
+    image stream of every query is the mean of the image values (and the text
+    keys are unchanged); with the text key weight zero the text stream is the
+    mean of the text values.  Returns the largest deviation."""
+    d, w, ctx_t, ctx_i, qc = _cross_setup()
+    nh, dh = d.heads, d.dh
+    sp = lambda a: np.asarray(a).reshape(-1, nh, dh)
+    errs = []
+    full = cross_kv(w, 0, ctx_t, ctx_i)
+    # the text keys and values of the full weights against torch
+    kt = TF.linear(T64(ctx_t), T64(w["blk0.ck.w"]), T64(w["blk0.ck.b"])).numpy()
+    vi = TF.linear(T64(ctx_i), T64(w["blk0.cvi.w"]), T64(w["blk0.cvi.b"])).numpy()
+    errs += [np.abs(full["k_txt"] - kt).max(), np.abs(full["v_img"] - vi).max()]
+    wz = dict(w, **{"blk0.cki.w": np.zeros_like(w["blk0.cki.w"])})
+    z = cross_kv(wz, 0, ctx_t, ctx_i)
+    o_img = O.attention(qc, sp(z["k_img"]), sp(z["v_img"]))
+    errs.append(np.abs(o_img - sp(z["v_img"]).mean(axis=0)[None]).max())
+    errs.append(np.abs(z["k_txt"] - full["k_txt"]).max())
+    wz = dict(w, **{"blk0.ck.w": np.zeros_like(w["blk0.ck.w"])})
+    z = cross_kv(wz, 0, ctx_t, ctx_i)
+    o_txt = O.attention(qc, sp(z["k_txt"][0]), sp(z["v_txt"][0]))
+    errs.append(np.abs(o_txt - sp(z["v_txt"][0]).mean(axis=0)[None]).max())
+    errs.append(np.abs(z["k_img"] - full["k_img"]).max())
+    return float(max(errs))
+
+
+def test_cross_kv_each_stream_keys_from_its_own_weights():
+    assert _cross_kv_errors(O.cross_kv) < 1e-10
+
+
+def test_cross_kv_pin_catches_swapped_key_weights():
+    def swapped(w, blk, ctx_txt, ctx_img, rnd=False):
+        p = f"blk{blk}."
+        w2 = dict(w, **{p + "ck.w": w[p + "cki.w"], p + "ck.b": w[p + "cki.b"],
+                        p + "cki.w": w[p + "ck.w"], p + "cki.b": w[p + "ck.b"]})
+        return O.cross_kv(w2, blk, ctx_txt, ctx_img, rnd)
+    assert _cross_kv_errors(swapped) > 1e-3
+
+
+# ------------------------------------------------------------------ context MLPs
+def test_text_and_clip_mlps_against_torch():
+    d, w, txt, clip, _ = _tiny()
+    ctx_t, ctx_i = O.context_embed(w, txt, clip)
+    mlp = lambda x, a, b: TF.linear(TF.gelu(TF.linear(T64(x), T64(w[a + ".w"]), T64(w[a + ".b"]))),
+                                    T64(w[b + ".w"]), T64(w[b + ".b"])).numpy()
+    np.testing.assert_allclose(ctx_t, mlp(txt, "txt1", "txt2"), atol=1e-11)
+    np.testing.assert_allclose(ctx_i, mlp(clip, "img1", "img2"), atol=1e-11)
+    assert ctx_i.shape == (d.n_img, d.D) and ctx_t.shape == (2, d.n_txt, d.D)
+
+
+# ------------------------------------------------------------------ the sampler's two rows
+def _sampler_inputs_seen(monkeypatch):
+    """Run the tiny sampler and record what the context MLPs and the DiT see."""
+    wl = synth.TINY
+    d = wl.dims
+    w = synth.model_weights(wl)
+    x = synth.inputs(wl)
+    seen = {"ctx": [], "fwd": []}
+    orig_ctx, orig_fwd = O.context_embed, O.dit_forward
+
+    def ctx(w_, txt, clip, rnd=False):
+        seen["ctx"].append((np.array(txt), None if clip is None else np.array(clip)))
+        return orig_ctx(w_, txt, clip, rnd)
+
+    def fwd(x_t, y, tau, w_, kvs, dims, rnd=False):
+        seen["fwd"].append((np.array(x_t), None if y is None else np.array(y)))
+        return orig_fwd(x_t, y, tau, w_, kvs, dims, rnd)
+    monkeypatch.setattr(O, "context_embed", ctx)
+    monkeypatch.setattr(O, "dit_forward", fwd)
+    O.sample(x["x0"], x["img_lat"], w, x["txt"], x["clip"], d, wl.steps, wl.cfg_scale)
+    return x, seen
+
+
+def _unconditional_row_ok(x, seen):
+    (txt2, clip), = seen["ctx"]
+    y_want = O.build_cond_y(x["img_lat"])
+    ok = txt2.shape[0] == 2 and np.array_equal(txt2[0], x["txt"]) and not np.any(txt2[1])
+    ok &= np.array_equal(clip, x["clip"])              # CLIP is kept for the unconditional row
+    for xb, y in seen["fwd"]:
+        ok &= xb.shape[0] == 2 and np.array_equal(xb[0], xb[1])   # both rows see the same latent
+        ok &= y is not None and np.array_equal(y, y_want)          # and the same y
+    return bool(ok) and len(seen["fwd"]) == synth.TINY.steps
+
+
+def test_sampler_unconditional_row_zeroes_only_the_text(monkeypatch):
+    x, seen = _sampler_inputs_seen(monkeypatch)
+    assert np.any(x["txt"])
+    assert _unconditional_row_ok(x, seen)
+
+
+def test_unconditional_row_pin_catches_a_row_that_keeps_its_text(monkeypatch):
+    orig_stack = np.stack
+    txt_shape = synth.inputs(synth.TINY)["txt"].shape
+
+    def keep_text(arrs, *a, **k):     # sample() builds [txt, 0]; plant [txt, txt]
+        arrs = list(arrs)
+        if len(arrs) == 2 and np.shape(arrs[0]) == txt_shape and not np.any(arrs[1]):
+            arrs[1] = arrs[0]
+        return orig_stack(arrs, *a, **k)
+    monkeypatch.setattr(O.np, "stack", keep_text)
+    x, seen = _sampler_inputs_seen(monkeypatch)
+    assert not _unconditional_row_ok(x, seen)
