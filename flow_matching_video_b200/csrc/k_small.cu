@@ -215,12 +215,14 @@ __global__ void k_rope_table(float2* tab, int T, int Hp, int Wp, int dh) {
 // ============================================================ QK-RMSNorm + 3D RoPE
 // In place on the fused projection buffer qkv [rows, 3D]: q = cols [0, D),
 // k = cols [D, 2D).  q <- RoPE(RMSNorm_D(q) * g_q), k likewise
-// ("图解 Wan2.1 I2V" 5.3 (1) and (2)).  One warp per (row, q|k); each lane
-// owns NC chunks of 4 channels (2 rotation pairs), so the row sits in
-// registers between the norm and the rotation.
+// ("图解 Wan2.1 I2V" 5.3 (1) and (2)).  The rows are batch x n_tok tokens of a
+// slice that starts at token tok0 of the sequence (the whole sequence: tok0
+// = 0, n_tok = L), so row r holds token tok0 + r % n_tok.  One warp per
+// (row, q|k); each lane owns NC chunks of 4 channels (2 rotation pairs), so
+// the row sits in registers between the norm and the rotation.
 template <typename T, int NC>
-__global__ void __launch_bounds__(256) k_qknorm_rope(T* qkv, int64_t rows, int D, int dh, int L, int Hp, int Wp,
-                                                     int T_, const float* __restrict__ gq,
+__global__ void __launch_bounds__(256) k_qknorm_rope(T* qkv, int64_t rows, int D, int dh, int n_tok, int tok0, int Hp,
+                                                     int Wp, int T_, const float* __restrict__ gq,
                                                      const float* __restrict__ gk, const float2* __restrict__ tab,
                                                      float eps) {
   const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -248,7 +250,7 @@ __global__ void __launch_bounds__(256) k_qknorm_rope(T* qkv, int64_t rows, int D
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float r = rsqrtf(ss / D + eps);
-  const int l = static_cast<int>(row % L);
+  const int l = tok0 + static_cast<int>(row % n_tok);   // the token's index in the whole sequence
   const int px = l % Wp, py = (l / Wp) % Hp, pf = l / (Wp * Hp);
   const int half = dh / 2;
   const int s6 = dh / 6, dT = dh - 4 * s6, dH = 2 * s6;
@@ -278,13 +280,13 @@ __global__ void __launch_bounds__(256) k_qknorm_rope(T* qkv, int64_t rows, int D
 
 template <typename T>
 wd_status qknorm_rope(T* qkv, int64_t rows, const wd_dims& d, const float* gq, const float* gk, const float2* tab,
-                      cudaStream_t st) {
+                      int64_t n_tok, int64_t tok0, cudaStream_t st) {
   const int D = d.D, dh = D / d.heads;
-  const int L = d.T * (d.H / 2) * (d.W / 2);
   const unsigned grid = static_cast<unsigned>((2 * rows * 32 + 255) / 256);
+  const int nt = static_cast<int>(n_tok), t0 = static_cast<int>(tok0);
   Trace tr(KC_ROPE, st);
-#define WD_QKR(NC)                                                                                       \
-  k_qknorm_rope<T, NC><<<grid, 256, 0, st>>>(qkv, rows, D, dh, L, d.H / 2, d.W / 2, d.T, gq, gk, tab, d.eps); \
+#define WD_QKR(NC)                                                                                            \
+  k_qknorm_rope<T, NC><<<grid, 256, 0, st>>>(qkv, rows, D, dh, nt, t0, d.H / 2, d.W / 2, d.T, gq, gk, tab, d.eps); \
   break;
   switch (D / 128) {
     case 1: WD_QKR(1)

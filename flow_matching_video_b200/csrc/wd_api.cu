@@ -148,11 +148,54 @@ static wd_status norm_rows(const wd_dims* d, const float* x, int64_t rows, const
 }
 
 // ------------------------------------------------------------------ block forward
+// One block is three pieces, in this order, all on the same stream:
+//   block_qkv_t        h = norm1(X)(1 + scale1) + shift1, q|k|v = h Wqkv^T + b,
+//                      QK-RMSNorm + 3D RoPE in place (rows: a token slice)
+//   self_attention_t   o = softmax(q k^T / sqrt(dh)) v over the whole sequence
+//   block_post_t       X += gate1 (o Wo^T + b), the cross-attention, the FFN
+//                      (rows: a token slice; every step here is row-local or
+//                      reads only the context's keys and values)
+// wd_block_forward runs them on the whole sequence with its workspace; the
+// split entry points run them one by one (token slices for sequence
+// parallelism, reused attention outputs for the attention cache).
+
 template <typename T>
-static wd_status block_forward_t(const wd_dims* d, const wd_block_weights* w, const float* e0, const void* kv,
-                                 int batch, float* X, const Ws& ws, cudaStream_t st) {
+static wd_status block_qkv_t(const wd_dims* d, const wd_block_weights* w, const float* e0, int batch, int64_t tok0,
+                             int64_t n_tok, const float* X, T* qkv, const Ws& ws, cudaStream_t st) {
+  const int D = d->D, dh = D / d->heads;
+  const int64_t rows = batch * n_tok;
+  T* Bf = static_cast<T*>(ws.b);
+  const float* mod = w->mod;
+  // 1. h = norm(X)(1 + scale1) + shift1
+  WD_TRY(norm_rows<T>(d, X, rows, e0, mod, e0 + D, mod + D, nullptr, nullptr, d->norm == WD_NORM_RMS, Bf, st));
+  // 2. q|k|v = h Wqkv^T + b
+  WD_TRY(gemm<T>(static_cast<int>(rows), 3 * D, D, Bf, D, w->qkv_w, D, EPI_STORE, epi(qkv, 3 * D, w->qkv_b), st));
+  // 3. QK-RMSNorm + 3D RoPE in place (the cos/sin table lives in the workspace; it is
+  //    rebuilt here because the library cannot assume the caller left it intact)
+  { Trace tr(KC_SMALL, st); k_rope_table<<<64, 256, 0, st>>>(ws.rope, d->T, d->H / 2, d->W / 2, dh); }
+  WD_TRY(launch_status("rope_table"));
+  return qknorm_rope<T>(qkv, rows, *d, w->g_q, w->g_k, ws.rope, n_tok, tok0, st);
+}
+
+// Full self-attention over the fused projection buffer qkv [batch, L, 3 * heads * dh]
+// (q of `heads` heads, then k, then v) -> o [batch, L, heads * dh].
+template <typename T>
+static wd_status self_attention_t(const wd_dims* d, int batch, int heads, const T* qkv, T* o, cudaStream_t st) {
+  const int dh = d->D / d->heads, Dh = heads * dh;
+  const int64_t L = tokens(d);
+  AttnArgs<T, T> a{};
+  a.q = qkv; a.q_rs = 3 * Dh;
+  a.k1 = qkv + Dh; a.v1 = qkv + 2 * Dh; a.kv1_rs = 3 * Dh; a.kv1_bs = L * 3 * Dh; a.n1 = static_cast<int>(L);
+  a.o = o; a.o_rs = Dh;
+  a.batch = batch; a.Lq = static_cast<int>(L); a.heads = heads; a.dh = dh;
+  return attention(a, st);
+}
+
+template <typename T>
+static wd_status block_post_t(const wd_dims* d, const wd_block_weights* w, const float* e0, const void* kv, int batch,
+                              int64_t n_tok, const T* o, float* X, const Ws& ws, cudaStream_t st) {
   const int D = d->D, F = d->ffn, dh = D / d->heads;
-  const int64_t L = tokens(d), rows = batch * L;
+  const int64_t rows = batch * n_tok;
   const int M = static_cast<int>(rows);
   T* A = static_cast<T*>(ws.a);
   T* Bf = static_cast<T*>(ws.b);
@@ -169,25 +212,8 @@ static wd_status block_forward_t(const wd_dims* d, const wd_block_weights* w, co
   const CT* k_txt = reinterpret_cast<const CT*>(kvp + 2 * n_img_b);
   const CT* v_txt = reinterpret_cast<const CT*>(kvp + 2 * n_img_b + n_txt_b);
 
-  // 1. h = norm(X)(1 + scale1) + shift1
-  WD_TRY(norm_rows<T>(d, X, rows, e0, mod, e0 + D, mod + D, nullptr, nullptr, rms, Bf, st));
-  // 2. q|k|v = h Wqkv^T + b
-  WD_TRY(gemm<T>(M, 3 * D, D, Bf, D, w->qkv_w, D, EPI_STORE, epi(A, 3 * D, w->qkv_b), st));
-  // 3. QK-RMSNorm + 3D RoPE in place
-  { Trace tr(KC_SMALL, st); k_rope_table<<<64, 256, 0, st>>>(ws.rope, d->T, d->H / 2, d->W / 2, dh); }
-  WD_TRY(launch_status("rope_table"));
-  WD_TRY(qknorm_rope<T>(A, rows, *d, w->g_q, w->g_k, ws.rope, st));
-  // 4. full self-attention -> o
-  {
-    AttnArgs<T, T> a{};
-    a.q = A; a.q_rs = 3 * D;
-    a.k1 = A + D; a.v1 = A + 2 * D; a.kv1_rs = 3 * D; a.kv1_bs = L * 3 * D; a.n1 = static_cast<int>(L);
-    a.o = Bf; a.o_rs = D;
-    a.batch = batch; a.Lq = static_cast<int>(L); a.heads = d->heads; a.dh = dh;
-    WD_TRY(attention(a, st));
-  }
   // 5. X += gate1 * (o Wo^T + b)
-  WD_TRY(gemm<T>(M, D, D, Bf, D, w->o_w, D, EPI_RESID, epi(X, D, w->o_b, e0 + 2 * D, mod + 2 * D), st));
+  WD_TRY(gemm<T>(M, D, D, o, D, w->o_w, D, EPI_RESID, epi(X, D, w->o_b, e0 + 2 * D, mod + 2 * D), st));
   // 6. hc = LN_affine(X);  7. qc = hc Wcq^T + b
   WD_TRY(norm_rows<T>(d, X, rows, nullptr, nullptr, nullptr, nullptr, w->cn_g, w->cn_b, 0, Bf, st));
   WD_TRY(gemm<T>(M, D, D, Bf, D, w->cq_w, D, CrossT<T>::store, epi(A, D, w->cq_b), st));
@@ -203,7 +229,7 @@ static wd_status block_forward_t(const wd_dims* d, const wd_block_weights* w, co
       a.k1 = k_txt; a.v1 = v_txt; a.kv1_rs = D; a.kv1_bs = static_cast<int64_t>(d->n_txt) * D; a.n1 = d->n_txt;
     }
     a.o = Bf; a.o_rs = D;
-    a.batch = batch; a.Lq = static_cast<int>(L); a.heads = d->heads; a.dh = dh;
+    a.batch = batch; a.Lq = static_cast<int>(n_tok); a.heads = d->heads; a.dh = dh;
     WD_TRY(attention(a, st));
   }
   // 9. X += oc Wco^T + b
@@ -213,6 +239,17 @@ static wd_status block_forward_t(const wd_dims* d, const wd_block_weights* w, co
   WD_TRY(gemm<T>(M, F, D, Bf, D, w->f1_w, D, EPI_GELU, epi(A, F, w->f1_b), st));
   WD_TRY(gemm<T>(M, D, F, A, F, w->f2_w, F, EPI_RESID, epi(X, D, w->f2_b, e0 + 5 * D, mod + 5 * D), st));
   return WD_OK;
+}
+
+template <typename T>
+static wd_status block_forward_t(const wd_dims* d, const wd_block_weights* w, const float* e0, const void* kv,
+                                 int batch, float* X, const Ws& ws, cudaStream_t st) {
+  const int64_t L = tokens(d);
+  T* A = static_cast<T*>(ws.a);
+  T* Bf = static_cast<T*>(ws.b);
+  WD_TRY(block_qkv_t<T>(d, w, e0, batch, 0, L, X, A, ws, st));          // q|k|v -> bufA
+  WD_TRY(self_attention_t<T>(d, batch, d->heads, A, Bf, st));           // o -> bufB
+  return block_post_t<T>(d, w, e0, kv, batch, L, Bf, X, ws, st);
 }
 
 }  // namespace wd
@@ -445,6 +482,61 @@ wd_status wd_block_forward(const wd_dims* d, const wd_block_weights* w, const fl
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d->dtype == WD_BF16) return block_forward_t<bf16>(d, w, e0, kv, batch, X, L, st);
   return block_forward_t<float>(d, w, e0, kv, batch, X, L, st);
+}
+
+// The three pieces of wd_block_forward, callable one by one.
+static wd_status check_slice(const wd_dims* d, int64_t tok0, int64_t n_tok) {
+  const int64_t L = tokens(d);
+  if (n_tok <= 0 || tok0 < 0 || tok0 + n_tok > L) {
+    set_error("token slice [%lld, %lld) outside the sequence [0, %lld)", (long long)tok0, (long long)(tok0 + n_tok),
+              (long long)L);
+    return WD_ERR_SHAPE;
+  }
+  return WD_OK;
+}
+
+wd_status wd_block_qkv(const wd_dims* d, const wd_block_weights* w, const float* e0, int batch, int64_t tok0,
+                       int64_t n_tok, const float* X, void* qkv, void* ws, size_t ws_bytes, wd_stream stream) {
+  WD_TRY(check_dims(d));
+  WD_TRY(check_batch(batch));
+  WD_TRY(check_slice(d, tok0, n_tok));
+  if (!w) { set_error("block weights NULL"); return WD_ERR_ARG; }
+  WD_NEED(w->qkv_w); WD_NEED(w->qkv_b); WD_NEED(w->g_q); WD_NEED(w->g_k); WD_NEED(w->mod);
+  WD_NEED(e0); WD_NEED(X); WD_NEED(qkv); WD_NEED(ws);
+  const Ws L = ws_layout(d, batch, ws);
+  if (ws_bytes < L.bytes) { set_error("workspace %zu < %zu bytes", ws_bytes, L.bytes); return WD_ERR_WORKSPACE; }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d->dtype == WD_BF16) return block_qkv_t<bf16>(d, w, e0, batch, tok0, n_tok, X, static_cast<bf16*>(qkv), L, st);
+  return block_qkv_t<float>(d, w, e0, batch, tok0, n_tok, X, static_cast<float*>(qkv), L, st);
+}
+
+wd_status wd_block_self_attention(const wd_dims* d, int batch, int heads, const void* qkv, void* o, wd_stream stream) {
+  WD_TRY(check_dims(d));
+  WD_TRY(check_batch(batch));
+  if (heads <= 0 || heads > d->heads) { set_error("heads=%d (1..%d)", heads, d->heads); return WD_ERR_SHAPE; }
+  WD_NEED(qkv); WD_NEED(o);
+  if (batch * tokens(d) > 0x7fffffff) { set_error("too many rows"); return WD_ERR_SHAPE; }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d->dtype == WD_BF16)
+    return self_attention_t<bf16>(d, batch, heads, static_cast<const bf16*>(qkv), static_cast<bf16*>(o), st);
+  return self_attention_t<float>(d, batch, heads, static_cast<const float*>(qkv), static_cast<float*>(o), st);
+}
+
+wd_status wd_block_post(const wd_dims* d, const wd_block_weights* w, const float* e0, const void* kv, int batch,
+                        int64_t n_tok, const void* o, float* X, void* ws, size_t ws_bytes, wd_stream stream) {
+  WD_TRY(check_dims(d));
+  WD_TRY(check_batch(batch));
+  WD_TRY(check_slice(d, 0, n_tok));
+  if (!w) { set_error("block weights NULL"); return WD_ERR_ARG; }
+  WD_NEED(w->o_w); WD_NEED(w->o_b); WD_NEED(w->cn_g); WD_NEED(w->cn_b); WD_NEED(w->cq_w); WD_NEED(w->cq_b);
+  WD_NEED(w->co_w); WD_NEED(w->co_b); WD_NEED(w->f1_w); WD_NEED(w->f1_b); WD_NEED(w->f2_w); WD_NEED(w->f2_b);
+  WD_NEED(w->mod);
+  WD_NEED(e0); WD_NEED(kv); WD_NEED(o); WD_NEED(X); WD_NEED(ws);
+  const Ws L = ws_layout(d, batch, ws);
+  if (ws_bytes < L.bytes) { set_error("workspace %zu < %zu bytes", ws_bytes, L.bytes); return WD_ERR_WORKSPACE; }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d->dtype == WD_BF16) return block_post_t<bf16>(d, w, e0, kv, batch, n_tok, static_cast<const bf16*>(o), X, L, st);
+  return block_post_t<float>(d, w, e0, kv, batch, n_tok, static_cast<const float*>(o), X, L, st);
 }
 
 wd_status wd_unpatchify(const wd_dims* d, const wd_head_weights* w, const float* e, int batch, const float* X, float* v,

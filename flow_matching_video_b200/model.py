@@ -202,3 +202,61 @@ class CfgCache:
         wd.wd_euler_cfg_step(xb[0], v_c, self.v_u, cfg_scale, dt, stream=stream)
         xb[1].copy_(xb[0])
         return xb
+
+
+class AttnCache:
+    """Attention cache ("Wan（通义万相）..." 5.3, reuse attention outputs across
+    steps): each block's self-attention output o (the input of its output
+    projection) is kept per block and batch row.  A step recomputes it while
+    nothing is stored, while its noise level tau / 1000 exceeds t_attn, and
+    otherwise once `interval` steps have passed since the last recomputation;
+    the steps in between skip each block's norm, q/k/v projection, QK-norm,
+    RoPE and self-attention and run only wd_block_post on the stored o.
+    Memory: blocks x batch x L x D elements of the storage type (6 GB for the
+    30-block 480p model at batch 2)."""
+
+    def __init__(self, dims: synth.Dims, weights: dict, t_attn: float, interval: int, batch: int = 2,
+                 device="cuda"):
+        if interval < 1:
+            raise ValueError("interval must be >= 1")
+        self.net = DiT(dims, weights, batch, device)
+        self.t_attn, self.interval = t_attn, interval
+        net = self.net
+        self.o = torch.empty((dims.blocks, batch, dims.L, dims.D), dtype=net.tdtype, device=net.device)
+        self.qkv = torch.empty((batch, dims.L, 3 * dims.D), dtype=net.tdtype, device=net.device)
+        self.step = 0
+        self.last_fresh = None
+
+    def prepare_context(self, txt: torch.Tensor, clip: torch.Tensor = None):
+        self.net.prepare_context(txt, clip)
+        self.step, self.last_fresh = 0, None
+
+    def fresh(self, tau: float) -> bool:
+        return (self.last_fresh is None or tau / 1000.0 > self.t_attn
+                or self.step - self.last_fresh >= self.interval)
+
+    def forward(self, x_t: torch.Tensor, y: torch.Tensor, tau: float, stream=None) -> torch.Tensor:
+        """One forward; recomputes or reuses the attention outputs as fresh(tau) says."""
+        net, d = self.net, self.net.dims
+        fresh = self.fresh(tau)
+        wd.wd_time_mod(net.cd, net.time_w, tau, net.e, net.e0, stream)
+        wd.wd_patch_embed(net.cd, x_t, y, net.w["pe.w"], net.w["pe.b"], net.batch, net.X, net.ws, stream)
+        for i in range(d.blocks):
+            if fresh:
+                wd.wd_block_qkv(net.cd, net.block_w[i], net.e0, net.batch, 0, d.L, net.X, self.qkv, net.ws, stream)
+                wd.wd_block_self_attention(net.cd, net.batch, d.heads, self.qkv, self.o[i], stream)
+            wd.wd_block_post(net.cd, net.block_w[i], net.e0, net.kv[i], net.batch, d.L, self.o[i], net.X, net.ws,
+                             stream)
+        wd.wd_unpatchify(net.cd, net.head_w, net.e, net.batch, net.X, net.v, net.ws, stream)
+        if fresh:
+            self.last_fresh = self.step
+        self.step += 1
+        return net.v
+
+    def cfg_euler_step(self, xb: torch.Tensor, y: torch.Tensor, tau: float, dt: float, cfg_scale: float,
+                       stream=None):
+        """xb [2, 16, T, H, W] as for DiT.cfg_euler_step."""
+        v = self.forward(xb, y, tau, stream)
+        wd.wd_euler_cfg_step(xb[0], v[0], v[1], cfg_scale, dt, stream=stream)
+        xb[1].copy_(xb[0])
+        return xb

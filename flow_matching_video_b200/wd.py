@@ -66,6 +66,9 @@ SIGNATURES = {
     "wd_patch_embed": (_I, [_PD, _P, _P, _P, _P, _I, _P, _P, _S, _P]),
     "wd_patch_embed_noalloc": (_I, [_PD, _P, _P, _P, _P, _I, _P, _P]),
     "wd_block_forward": (_I, [_PD, C.POINTER(wd_block_weights), _P, _P, _I, _P, _P, _S, _P]),
+    "wd_block_qkv": (_I, [_PD, C.POINTER(wd_block_weights), _P, _I, _L, _L, _P, _P, _P, _S, _P]),
+    "wd_block_self_attention": (_I, [_PD, _I, _I, _P, _P, _P]),
+    "wd_block_post": (_I, [_PD, C.POINTER(wd_block_weights), _P, _P, _I, _L, _P, _P, _P, _S, _P]),
     "wd_unpatchify": (_I, [_PD, C.POINTER(wd_head_weights), _P, _I, _P, _P, _P, _S, _P]),
     "wd_euler_cfg_step": (_I, [_P, _P, _P, _F, _F, _S, _P]),
     "wd_gemm": (_I, [_I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P]),
@@ -179,6 +182,21 @@ def wd_patch_embed_noalloc(dims, x_t, y, w, b, batch, X, stream=None):
 def wd_block_forward(dims, w: wd_block_weights, e0, kv, batch, X, ws, stream=None):
     _ok(_lib.wd_block_forward(C.byref(dims), C.byref(w), _p(e0), _p(kv), batch, _p(X), _p(ws),
                               ws.numel() * ws.element_size(), _stream(stream)), "wd_block_forward")
+
+
+def wd_block_qkv(dims, w: wd_block_weights, e0, batch, tok0, n_tok, X, qkv, ws, stream=None):
+    _ok(_lib.wd_block_qkv(C.byref(dims), C.byref(w), _p(e0), batch, tok0, n_tok, _p(X), _p(qkv), _p(ws),
+                          ws.numel() * ws.element_size(), _stream(stream)), "wd_block_qkv")
+
+
+def wd_block_self_attention(dims, batch, heads, qkv, o, stream=None):
+    _ok(_lib.wd_block_self_attention(C.byref(dims), batch, heads, _p(qkv), _p(o), _stream(stream)),
+        "wd_block_self_attention")
+
+
+def wd_block_post(dims, w: wd_block_weights, e0, kv, batch, n_tok, o, X, ws, stream=None):
+    _ok(_lib.wd_block_post(C.byref(dims), C.byref(w), _p(e0), _p(kv), batch, n_tok, _p(o), _p(X), _p(ws),
+                           ws.numel() * ws.element_size(), _stream(stream)), "wd_block_post")
 
 
 def wd_unpatchify(dims, w: wd_head_weights, e, batch, X, v, ws, stream=None):

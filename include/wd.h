@@ -200,6 +200,38 @@ wd_status wd_block_forward(const wd_dims* d, const wd_block_weights* w, const fl
                            const void* kv, int batch, float* X, void* ws, size_t ws_bytes,
                            wd_stream stream);
 
+/* The three pieces of wd_block_forward, callable one by one on the same
+ * workspace (wd_workspace_bytes(d, batch) bytes), for sequence parallelism
+ * (each GPU holds a slice of the tokens, [WAN] 5.2) and for the attention
+ * cache (a later step reuses a block's attention output, [WAN] 5.3).  Run in
+ * order on one token slice, wd_block_qkv (slice), wd_block_self_attention
+ * (whole sequence) and wd_block_post (slice) give wd_block_forward's result
+ * bit for bit: they launch the same kernels on the same rows.
+ *
+ * wd_block_qkv: for the n_tok tokens starting at token tok0 of the sequence
+ * (0 <= tok0, tok0 + n_tok <= L) and every sample of the batch,
+ * h = norm(X)(1 + scale1) + shift1, [q k v] = h Wqkv^T + b, then q, k <-
+ * RoPE3D(RMSNorm_D(.) g) with each token's (frame, row, column) taken from
+ * its place tok0 + i in the whole grid ([I2V] 5.2, 5.3 (1), (2)).
+ * X [batch, n_tok, D] fp32 (read only); qkv [batch, n_tok, 3D] in dtype
+ * (q, then k, then v of all heads).  The workspace serves as scratch. */
+wd_status wd_block_qkv(const wd_dims* d, const wd_block_weights* w, const float* e0, int batch, int64_t tok0,
+                       int64_t n_tok, const float* X, void* qkv, void* ws, size_t ws_bytes, wd_stream stream);
+
+/* Full non-causal self-attention over the whole sequence for `heads` heads
+ * (1 <= heads <= d->heads; fewer than all when the heads are split across
+ * GPUs): qkv [batch, L, 3 * heads * dh] in dtype, laid out as q of the
+ * heads, then k, then v; o [batch, L, heads * dh] in dtype ([I2V] 5.3). */
+wd_status wd_block_self_attention(const wd_dims* d, int batch, int heads, const void* qkv, void* o, wd_stream stream);
+
+/* The rest of the block for n_tok tokens of every sample (1 <= n_tok <= L):
+ * X += gate1 (o Wo^T + b); X += Linear_co(decoupled cross-attention of
+ * Linear_cq(LN_affine(X)) over kv); X += gate2 FFN(norm(X)(1 + scale2) +
+ * shift2) ([I2V] 5.2-5.5).  o [batch, n_tok, D] in dtype (the attention
+ * output of these tokens), X [batch, n_tok, D] fp32 in place. */
+wd_status wd_block_post(const wd_dims* d, const wd_block_weights* w, const float* e0, const void* kv, int batch,
+                        int64_t n_tok, const void* o, float* X, void* ws, size_t ws_bytes, wd_stream stream);
+
 /* Head and unpatchify ([I2V] 5.5): z = LN(X)(1 + e + mod[1]) + e + mod[0],
  * p = z w^T + b, v[b,c,f,2y+kh,2x+kw] = p[b, l, c*4+kh*2+kw].
  * X [batch,L,D] fp32, e [D] fp32 -> v [batch,16,T,H,W] fp32. */

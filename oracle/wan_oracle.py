@@ -313,68 +313,109 @@ def cross_kv(w: dict, blk: int, ctx_txt, ctx_img, rnd: bool = False):
 
 
 # ---------------------------------------------------------------- one DiT block
-def block_forward(X, e0, w: dict, blk: int, kv: dict, dims, rnd: bool = False, rows=None):
-    """One DiT block ([I2V] 5.2-5.5), order self-attention -> cross -> FFN.
+def _mod(e0, w: dict, blk: int):
+    """mod = e0 + b_i, rows (shift1, scale1, gate1, shift2, scale2, gate2) ([WAN] 2.5)."""
+    return np.asarray(e0, F64) + np.asarray(w[f"blk{blk}.mod"], F64)
 
-    X [B, L, D] residual stream; e0 [6, D]; kv from cross_kv (k_txt/v_txt
-    [B, n_txt, D], k_img/v_img [n_img, D]).  ``rows`` (optional index array)
-    computes the output only for those token rows of every sample; keys and
-    values still cover all L tokens, so the result is exact for those rows.
 
-    mod = e0 + b_i                                    ([WAN] 2.5)
-    h   = norm(X)(1 + scale1) + shift1                ([I2V] 5.2)
-    q,k = RMSNorm(Linear_q/k h), v = Linear_v h       ([I2V] 5.3 (1))
-    q,k = RoPE3D(q), RoPE3D(k)                        ([I2V] 5.3 (2))
-    X  += gate1 * Linear_o(attn(q, k, v))             ([I2V] 5.2, 5.3)
-    X  += Linear_co(attn(qc, K_img, V_img) + attn(qc, K_txt, V_txt)),
-          qc = Linear_cq(LN_affine(X))                ([I2V] 5.4; no adaLN, no gate)
-    X  += gate2 * Linear_2(GELU(Linear_1(norm(X)(1+scale2)+shift2)))   ([I2V] 5.5)
-    Readings: QK-RMSNorm over the full width D with learned gains, before the
-    head split; the cross-attention input gets a LayerNorm with affine gains.
-    """
+def block_qkv(x, e0, w: dict, blk: int, dims, tok, rnd: bool = False, want=("q", "k", "v")):
+    """The projections of the self-attention for some tokens of one sample
+    ([I2V] 5.2, 5.3 (1) and (2)): x [n, D] are the residual-stream rows of the
+    tokens whose sequence indices are `tok` [n];
+    h = norm(x)(1 + scale1) + shift1, [q k v] = Linear_qkv(h) (the fused
+    projection's rows q; k; v), q and k RMS-normalised over the full width D
+    with their gains, split into heads and rotated by the 3D RoPE at each
+    token's (frame, row, column) in the grid; v split into heads.
+    Returns {name: [n, heads, dh]} for the names in `want`.
+    Reading: QK-RMSNorm over D before the head split (the page's
+    RMSNorm(Linear_q(x)))."""
     p = f"blk{blk}."
     D, nh, dh, eps = dims.D, dims.heads, dims.dh, dims.eps
-    X = np.asarray(X, F64)
-    B, L, _ = X.shape
-    rows = np.arange(L) if rows is None else np.asarray(rows)
-    mod = np.asarray(e0, F64) + np.asarray(w[p + "mod"], F64)
-    shift1, scale1, gate1, shift2, scale2, gate2 = mod
-    pf, py, px = grid_positions(dims.T, dims.Hp, dims.Wp)
+    shift1, scale1 = _mod(e0, w, blk)[:2]
+    tok = np.asarray(tok)
+    n = len(tok)
+    pf, py, px = (a[tok] for a in grid_positions(dims.T, dims.Hp, dims.Wp))
+    h = _st(adaln_modulate(x, shift1, scale1, eps, dims.norm), rnd)
+    wqkv, bqkv = w[p + "qkv.w"], w[p + "qkv.b"]
+    out = {}
+    for j, name in enumerate(("q", "k", "v")):
+        if name not in want:
+            continue
+        a = _st(linear(h, wqkv[j * D:(j + 1) * D], bqkv[j * D:(j + 1) * D]), rnd)
+        if name == "v":
+            out[name] = a.reshape(n, nh, dh)
+        else:
+            a = rms_norm(a, eps, w[p + ("gq" if name == "q" else "gk")]).reshape(n, nh, dh)
+            out[name] = _st(rope_3d(a, pf, py, px), rnd)
+    return out
 
-    out = np.empty((B, len(rows), D))
+
+def block_self_attention(X, e0, w: dict, blk: int, dims, rnd: bool = False, rows=None):
+    """The attention output o of a block's self-attention for the token rows
+    `rows` of every sample (default all): o = softmax(q k^T / sqrt(dh)) v per
+    head over all L keys, heads concatenated -> [B, len(rows), D], the input of
+    Linear_o ([I2V] 5.3).  Keys and values cover every token, so the rows are
+    exact."""
+    X = np.asarray(X, F64)
+    B, L, D = X.shape
+    rows = np.arange(L) if rows is None else np.asarray(rows)
+    o = np.empty((B, len(rows), D))
     for b in range(B):
-        x = X[b]
-        # ---- self-attention (keys and values need every token)
-        h = _st(adaln_modulate(x, shift1, scale1, eps, dims.norm), rnd)
-        wqkv, bqkv = w[p + "qkv.w"], w[p + "qkv.b"]
-        # the fused projection's rows (q; k; v); q is needed only for the requested rows
-        q = _st(linear(h[rows], wqkv[:D], bqkv[:D]), rnd)
-        k = _st(linear(h, wqkv[D:2 * D], bqkv[D:2 * D]), rnd)
-        v = _st(linear(h, wqkv[2 * D:], bqkv[2 * D:]), rnd)
-        q = rms_norm(q, eps, w[p + "gq"]).reshape(len(rows), nh, dh)
-        k = rms_norm(k, eps, w[p + "gk"]).reshape(L, nh, dh)
-        q = _st(rope_3d(q, pf[rows], py[rows], px[rows]), rnd)
-        k = _st(rope_3d(k, pf, py, px), rnd)
-        v = v.reshape(L, nh, dh)
-        o = _st(attention(q, k, v).reshape(len(rows), D), rnd)
-        xr = x[rows] + gate1 * linear(o, w[p + "o.w"], w[p + "o.b"])
+        kv = block_qkv(X[b], e0, w, blk, dims, np.arange(L), rnd, want=("k", "v"))
+        q = block_qkv(X[b][rows], e0, w, blk, dims, rows, rnd, want=("q",))["q"]
+        o[b] = _st(attention(q, kv["k"], kv["v"]).reshape(len(rows), D), rnd)
+    return o
+
+
+def block_after_attention(Xr, o, e0, w: dict, blk: int, kv: dict, dims, rnd: bool = False):
+    """The rest of the block for some token rows, given their self-attention
+    output o [B, n, D] and their residual-stream rows Xr [B, n, D]
+    ([I2V] 5.2-5.5):
+    X  += gate1 * Linear_o(o)
+    X  += Linear_co(attn(qc, K_img, V_img) + attn(qc, K_txt, V_txt)),
+          qc = Linear_cq(LN_affine(X))                (no adaLN, no gate)
+    X  += gate2 * Linear_2(GELU(Linear_1(norm(X)(1+scale2)+shift2)))
+    Reading: the cross-attention input gets a LayerNorm with affine gains."""
+    p = f"blk{blk}."
+    D, nh, dh, eps = dims.D, dims.heads, dims.dh, dims.eps
+    Xr = np.asarray(Xr, F64)
+    B, n, _ = Xr.shape
+    shift1, scale1, gate1, shift2, scale2, gate2 = _mod(e0, w, blk)
+    out = np.empty((B, n, D))
+    for b in range(B):
+        xr = Xr[b] + gate1 * linear(o[b], w[p + "o.w"], w[p + "o.b"])
         # ---- decoupled cross-attention (not modulated, not gated)
         hc = _st(layer_norm(xr, eps, w[p + "cn.g"], w[p + "cn.b"]), rnd)
-        qc = _st16(linear(hc, w[p + "cq.w"], w[p + "cq.b"]), rnd).reshape(len(rows), nh, dh)
+        qc = _st16(linear(hc, w[p + "cq.w"], w[p + "cq.b"]), rnd).reshape(n, nh, dh)
         kt, vt = kv["k_txt"][b], kv["v_txt"][b]
         o_txt = attention(qc, kt.reshape(-1, nh, dh), vt.reshape(-1, nh, dh))
         if "k_img" in kv:
             ki, vi = kv["k_img"], kv["v_img"]
             o_img = attention(qc, ki.reshape(-1, nh, dh), vi.reshape(-1, nh, dh))
-            oc = _st((o_img + o_txt).reshape(len(rows), D), rnd)
+            oc = _st((o_img + o_txt).reshape(n, D), rnd)
         else:   # text-to-video: single-stream cross-attention ([I2V] 9)
-            oc = _st(o_txt.reshape(len(rows), D), rnd)
+            oc = _st(o_txt.reshape(n, D), rnd)
         xr = xr + linear(oc, w[p + "co.w"], w[p + "co.b"])
         # ---- gated FFN
         h2 = _st(adaln_modulate(xr, shift2, scale2, eps, dims.norm), rnd)
         u = _st(gelu(linear(h2, w[p + "f1.w"], w[p + "f1.b"])), rnd)
         out[b] = xr + gate2 * linear(u, w[p + "f2.w"], w[p + "f2.b"])
     return out
+
+
+def block_forward(X, e0, w: dict, blk: int, kv: dict, dims, rnd: bool = False, rows=None):
+    """One DiT block ([I2V] 5.2-5.5), order self-attention -> cross -> FFN:
+    block_self_attention, then block_after_attention.
+
+    X [B, L, D] residual stream; e0 [6, D]; kv from cross_kv (k_txt/v_txt
+    [B, n_txt, D], k_img/v_img [n_img, D]).  ``rows`` (optional index array)
+    computes the output only for those token rows of every sample; keys and
+    values still cover all L tokens, so the result is exact for those rows.
+    """
+    X = np.asarray(X, F64)
+    rows = np.arange(X.shape[1]) if rows is None else np.asarray(rows)
+    o = block_self_attention(X, e0, w, blk, dims, rnd, rows)
+    return block_after_attention(X[:, rows], o, e0, w, blk, kv, dims, rnd)
 
 
 # ---------------------------------------------------------------- head
@@ -390,12 +431,22 @@ def head_unpatchify(X, e, w: dict, dims, rnd: bool = False):
 
 
 # ---------------------------------------------------------------- whole DiT
-def dit_forward(x_t, y, tau: float, w: dict, kvs: list, dims, rnd: bool = False):
-    """v = DiT(concat(x_t, y), tau, context) for a batch ([I2V] 5, 7)."""
+def dit_forward(x_t, y, tau: float, w: dict, kvs: list, dims, rnd: bool = False, attn=None):
+    """v = DiT(concat(x_t, y), tau, context) for a batch ([I2V] 5, 7).
+    attn (optional, the attention cache of [WAN] 5.3): a dict with "o", a
+    list holding per block the self-attention output o [B, L, D] last
+    computed, and "reuse": when true every block takes its stored o instead of
+    computing its self-attention; otherwise each block's o is computed and
+    stored there."""
     e, e0 = time_mod(w, tau, dims.D)
     X = patch_embed(x_t, y, w["pe.w"], w["pe.b"], rnd)
     for i in range(dims.blocks):
-        X = block_forward(X, e0, w, i, kvs[i], dims, rnd)
+        if attn is None:
+            X = block_forward(X, e0, w, i, kvs[i], dims, rnd)
+            continue
+        if not attn["reuse"]:
+            attn["o"][i] = block_self_attention(X, e0, w, i, dims, rnd)
+        X = block_after_attention(X, attn["o"][i], e0, w, i, kvs[i], dims, rnd)
     return head_unpatchify(X, e, w, dims, rnd)
 
 
@@ -518,6 +569,46 @@ def sample_cfg_cache(x0, img_lat, w: dict, txt, clip, dims, steps: int, cfg_scal
             fresh.append(False)
         trace.append((v_c, v_u))
         x = euler_cfg_step(x, v_c, v_u, cfg_scale, dt)
+    return x, trace, fresh
+
+
+def attn_cache_fresh(k: int, noise_level: float, last_fresh, t_attn: float, interval: int) -> bool:
+    """Whether step k recomputes the self-attention under the attention cache
+    of [WAN] 5.3 ("reuse attention outputs across steps").  Reading: a step
+    recomputes while nothing is stored, while its noise level exceeds t_attn
+    (the early steps, where the latent changes fastest), and otherwise once
+    `interval` steps have passed since the last recomputation; the steps in
+    between reuse.  interval = 1 never reuses."""
+    return last_fresh is None or noise_level > t_attn or k - last_fresh >= interval
+
+
+def sample_attn_cache(x0, img_lat, w: dict, txt, clip, dims, steps: int, cfg_scale: float, t_attn: float,
+                      interval: int, rnd: bool = False):
+    """The sampler of `sample` with the attention cache of [WAN] 5.3.
+    Reading: what is reused is each block's self-attention output o (the
+    input of its output projection), per block and per batch row; on a
+    reusing step each block skips its norm, q/k/v projection, QK-norm, RoPE
+    and self-attention and takes the o stored at the last recomputing step,
+    while the gated output projection (with this step's gate), the
+    cross-attention and the FFN run as usual.  Returns the final latent, the
+    per-step velocities and per step whether it recomputed."""
+    y = None if img_lat is None else build_cond_y(img_lat)
+    txt2 = np.stack([np.asarray(txt, F64), np.zeros_like(txt, dtype=F64)])
+    ctx_txt, ctx_img = context_embed(w, txt2, clip, rnd)
+    kvs = [cross_kv(w, i, ctx_txt, ctx_img, rnd) for i in range(dims.blocks)]
+    cache = {"o": [None] * dims.blocks, "reuse": False}
+    x = np.asarray(x0, F64)
+    trace, fresh = [], []
+    last = None
+    for k, (t, dt, tau) in enumerate(schedule(steps)):
+        f = attn_cache_fresh(k, tau / 1000.0, last, t_attn, interval)
+        if f:
+            last = k
+        cache["reuse"] = not f
+        v = dit_forward(np.stack([x, x]), y, tau, w, kvs, dims, rnd, attn=cache)
+        trace.append((v[0], v[1]))
+        fresh.append(f)
+        x = euler_cfg_step(x, v[0], v[1], cfg_scale, dt)
     return x, trace, fresh
 
 

@@ -363,3 +363,85 @@ def test_tiny_fp32_cfg_cache_sampler(mods):
                                                 wl.cfg_scale, 0.5)
     assert fresh == want_fresh == [True, True, False, False]
     assert rel(host(xb[0]), want_x) < TOL_F32
+
+
+# ------------------------------------------------------------------ the block in pieces: sequence parallelism, attention cache
+def test_block_pieces_equal_the_fused_block_bit_for_bit(mods):
+    """wd_block_qkv + wd_block_self_attention + wd_block_post on the whole
+    sequence launch the same kernels on the same rows as wd_block_forward:
+    identical output (480p/81 frames, batch 2)."""
+    model, wd = mods
+    wl = synth.STACK_480P81
+    net, w, x, txt, y, d = setup(mods, wl, blocks=[0])
+    B = wl.batch
+    rng = np.random.default_rng(3)
+    X0 = dev(rng.standard_normal((B, d.L, d.D)) * 0.5)
+    net.e0.copy_(dev(O.time_mod(w, 800.0, d.D)[1]))
+    net.X.copy_(X0)
+    wd.wd_block_forward(net.cd, net.block_w[0], net.e0, net.kv[0], B, net.X, net.ws)
+    want = net.X.clone()
+    X = X0.clone()
+    qkv = torch.empty((B, d.L, 3 * d.D), dtype=torch.bfloat16, device="cuda")
+    o = torch.empty((B, d.L, d.D), dtype=torch.bfloat16, device="cuda")
+    wd.wd_block_qkv(net.cd, net.block_w[0], net.e0, B, 0, d.L, X, qkv, net.ws)
+    wd.wd_block_self_attention(net.cd, B, d.heads, qkv, o)
+    wd.wd_block_post(net.cd, net.block_w[0], net.e0, net.kv[0], B, d.L, o, X, net.ws)
+    wd.wd_check()
+    assert torch.equal(X, want)
+    assert float((want - X0).abs().max()) > 0.1
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_ulysses_ranks_emulated_on_one_gpu_equal_the_fused_block(mods, world):
+    """Head-sharded sequence parallelism ("Wan（通义万相）..." 5.2, inner level):
+    `world` ranks, run one after the other on this GPU with the all-to-all done
+    by copies (no rank waits for another), each holding a token slice, through
+    the real orchestration of seq_parallel and libwd's split entry points; the
+    gathered residual stream equals wd_block_forward's bit for bit
+    (480p/81 frames, batch 2: 32760 tokens, 12 heads)."""
+    model, wd = mods
+    from flow_matching_video_b200 import seq_parallel as SP
+    wl = synth.STACK_480P81
+    net, w, x, txt, y, d = setup(mods, wl, blocks=[0])
+    B = wl.batch
+    rng = np.random.default_rng(4)
+    X0 = dev(rng.standard_normal((B, d.L, d.D)) * 0.5)
+    net.e0.copy_(dev(O.time_mod(w, 600.0, d.D)[1]))
+    net.X.copy_(X0)
+    wd.wd_block_forward(net.cd, net.block_w[0], net.e0, net.kv[0], B, net.X, net.ws)
+    want = net.X.clone()
+    ops = SP.LibwdOps(net)
+    blocks = [SP.UlyssesBlock(ops, r, world, d.L, d.heads) for r in range(world)]
+    X_locals = [X0[:, b.tok0:b.tok0 + b.n].contiguous() for b in blocks]
+    SP.block_in_one_process(blocks, X_locals, 0)
+    wd.wd_check()
+    assert torch.equal(torch.cat(X_locals, dim=1), want)
+
+
+def test_tiny_fp32_attention_cache_sampler(mods):
+    """Attention cache ("Wan（通义万相）..." 5.3): 4 steps with t_attn = 0.6 and
+    interval 2, so the self-attention is computed at noise levels 1, 0.75 and
+    0.25 and reused at 0.5; every element of every velocity and of the final
+    latent against the oracle's sampler with the same cache (1e-4)."""
+    model, wd = mods
+    wl = synth.TINY_MOE
+    d = wl.dims
+    w = synth.model_weights(wl)
+    x = synth.inputs(wl)
+    ac = model.AttnCache(d, model.weights_to_device(w, d, "cuda"), t_attn=0.6, interval=2)
+    ac.prepare_context(dev(np.stack([x["txt"], np.zeros_like(x["txt"])])), dev(x["clip"]))
+    y = ac.net.build_cond_y(dev(x["img_lat"]))
+    xb = dev(np.stack([x["x0"], x["x0"]]))
+    fresh, vs = [], []
+    for t, dt, tau in O.schedule(wl.steps):
+        fresh.append(ac.fresh(tau))
+        ac.cfg_euler_step(xb, y, tau, dt, wl.cfg_scale)
+        vs.append(host(ac.net.v))
+    wd.wd_check()
+    want_x, trace, want_fresh = O.sample_attn_cache(x["x0"], x["img_lat"], w, x["txt"], x["clip"], d, wl.steps,
+                                                    wl.cfg_scale, 0.6, 2)
+    assert fresh == want_fresh == [True, True, False, True]
+    for (vc, vu), got in zip(trace, vs):
+        assert rel(got[0], vc) < TOL_F32
+        assert rel(got[1], vu) < TOL_F32
+    assert rel(host(xb[0]), want_x) < TOL_F32

@@ -314,3 +314,68 @@ def test_unconditional_row_pin_catches_a_row_that_keeps_its_text(monkeypatch):
     monkeypatch.setattr(O.np, "stack", keep_text)
     x, seen = _sampler_inputs_seen(monkeypatch)
     assert not _unconditional_row_ok(x, seen)
+
+
+# ------------------------------------------------------------------ attention cache ("Wan（通义万相）..." 5.3)
+def test_attention_cache_decisions():
+    # noise levels 1, 0.75, 0.5, 0.25 of a 4-step schedule
+    levels = [1.0, 0.75, 0.5, 0.25]
+
+    def pattern(t_attn, interval):
+        last, out = None, []
+        for k, lv in enumerate(levels):
+            f = O.attn_cache_fresh(k, lv, last, t_attn, interval)
+            last = k if f else last
+            out.append(f)
+        return out
+    assert pattern(0.6, 2) == [True, True, False, True]
+    assert pattern(0.6, 1) == [True] * 4           # interval 1 never reuses
+    assert pattern(0.0, 3) == [True] * 4           # every noise level above 0: always recompute
+    assert pattern(1.0, 4) == [True, False, False, False]
+
+
+def test_attention_cache_never_taken_is_the_plain_sampler():
+    wl = synth.TINY_MOE                            # the tiny model, 4 steps
+    d, w, x = wl.dims, synth.model_weights(wl), synth.inputs(wl)
+    want, trace = O.sample(x["x0"], x["img_lat"], w, x["txt"], x["clip"], d, wl.steps, wl.cfg_scale)
+    got, trace2, fresh = O.sample_attn_cache(x["x0"], x["img_lat"], w, x["txt"], x["clip"], d, wl.steps,
+                                             wl.cfg_scale, t_attn=0.6, interval=1)
+    assert fresh == [True] * 4
+    np.testing.assert_array_equal(got, want)
+
+
+def test_attention_cache_reuse_is_exact_at_the_step_that_filled_it():
+    """A forward that reuses the stored attention outputs at the same latent
+    and noise level as the forward that stored them gives the same velocity;
+    at another latent it differs from a fresh forward (the cache is used)."""
+    d, w, txt, clip, X = _tiny()
+    d = synth.Dims(**{**d.__dict__, "blocks": 1})
+    ctx_t, ctx_i = O.context_embed(w, txt, clip)
+    kvs = [O.cross_kv(w, 0, ctx_t, ctx_i)]
+    img = RNG.standard_normal((16, d.T, d.H, d.W))
+    y = O.build_cond_y(img)
+    xt = RNG.standard_normal((2, 16, d.T, d.H, d.W))
+    cache = {"o": [None], "reuse": False}
+    v_fresh = O.dit_forward(xt, y, 600.0, w, kvs, d, attn=cache)
+    np.testing.assert_array_equal(v_fresh, O.dit_forward(xt, y, 600.0, w, kvs, d))
+    cache["reuse"] = True
+    np.testing.assert_array_equal(O.dit_forward(xt, y, 600.0, w, kvs, d, attn=cache), v_fresh)
+    xt2 = xt + RNG.standard_normal(xt.shape)
+    assert np.abs(O.dit_forward(xt2, y, 600.0, w, kvs, d, attn=cache) - O.dit_forward(xt2, y, 600.0, w, kvs, d)).max() > 1e-3
+
+
+def test_attention_cache_pin_catches_a_cache_that_is_never_read(monkeypatch):
+    """Planted mistake: the reusing step recomputes anyway.  Then the 4-step
+    sampler with reuse equals the plain sampler, which the real cache does not."""
+    wl = synth.TINY_MOE
+    d, w, x = wl.dims, synth.model_weights(wl), synth.inputs(wl)
+    plain, _ = O.sample(x["x0"], x["img_lat"], w, x["txt"], x["clip"], d, wl.steps, wl.cfg_scale)
+    real, _, fresh = O.sample_attn_cache(x["x0"], x["img_lat"], w, x["txt"], x["clip"], d, wl.steps, wl.cfg_scale,
+                                         t_attn=0.6, interval=2)
+    assert fresh == [True, True, False, True]
+    assert np.abs(real - plain).max() > 1e-6
+    orig = O.dit_forward
+    monkeypatch.setattr(O, "dit_forward", lambda *a, attn=None, **k: orig(*a, **k))
+    broken, _, _ = O.sample_attn_cache(x["x0"], x["img_lat"], w, x["txt"], x["clip"], d, wl.steps, wl.cfg_scale,
+                                       t_attn=0.6, interval=2)
+    np.testing.assert_array_equal(broken, plain)
