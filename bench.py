@@ -233,35 +233,61 @@ def run_ours(args, rank, world, local_rank):
     wl = synth.WORKLOADS[args.workload]
     d = wl.dims
     B = wl.batch
+    mode = "cfg-split" if args.cfg_split else ("ulysses" if args.seq_parallel else "replicas")
+    if mode == "cfg-split" and world != 2:
+        raise SystemExit("--cfg-split runs one video's two CFG rows on exactly two GPUs (--gpus 2)")
     torch.manual_seed(0)
     weights = model.random_weights_on_device(wl, dev)
-    if args.cfg_cache is not None:   # the sampler with the CFG cache: late steps run the conditional row alone
-        runner = model.CfgCache(d, weights, args.cfg_cache, dev)
-        net = runner.pair
+    # replicas: an independent video per rank; the split modes: one video shared by all ranks
+    x = synth.inputs(replace(wl, seed=wl.seed + 7919 * rank) if mode == "replicas" else wl)
+    tdt = torch.bfloat16 if d.dtype == "bf16" else torch.float32
+    txt = torch.from_numpy(np.stack([x["txt"], np.zeros_like(x["txt"])])).to(dev, tdt)
+    clip = None if d.t2v else torch.from_numpy(x["clip"]).to(dev, tdt)
+    attn_cache = None
+    if mode == "cfg-split":
+        # rank 0 evaluates the text row, rank 1 the zeroed-text row, each with a batch-1 model
+        from flow_matching_video_b200.cfg_split import CfgSplit
+        net = model.DiT(d, weights, 1, dev)
+        net.prepare_context(txt[rank:rank + 1].contiguous(), clip)
+        runner = CfgSplit(net)
+        rows_local = 1
+    elif mode == "ulysses":
+        from flow_matching_video_b200.seq_parallel import SeqParallelDiT
+        net = model.DiT(d, weights, B, dev)
+        net.prepare_context(txt, clip)
+        runner = SeqParallelDiT(net, rank, world)
+        rows_local = B / world       # each rank carries 1/world of the tokens through the blocks
     else:
-        runner = net = model.DiT(d, weights, B, dev)
-    x = synth.inputs(replace(wl, seed=wl.seed + 7919 * rank))   # an independent video per rank
-    tdt = net.tdtype
-    txt2 = torch.from_numpy(np.stack([x["txt"], np.zeros_like(x["txt"])])).to(dev, tdt)
-    if d.t2v:   # text-to-video: no CLIP context and no y
-        runner.prepare_context(txt2)
-        y = None
-    else:
-        clip = torch.from_numpy(x["clip"]).to(dev, tdt)
-        runner.prepare_context(txt2, clip)
-        y = net.build_cond_y(torch.from_numpy(x["img_lat"]).to(dev))
+        if args.cfg_cache is not None:   # the sampler with the CFG cache: late steps run the conditional row alone
+            runner = model.CfgCache(d, weights, args.cfg_cache, dev)
+            net = runner.pair
+        elif args.attn_cache is not None:   # the sampler with the attention cache
+            t_attn, interval = args.attn_cache
+            runner = attn_cache = model.AttnCache(d, weights, t_attn, int(interval), B, dev)
+            net = runner.net
+        else:
+            runner = net = model.DiT(d, weights, B, dev)
+        runner.prepare_context(txt, clip)
+        rows_local = B
+    y = None if d.t2v else net.build_cond_y(torch.from_numpy(x["img_lat"]).to(dev))
     x_host = torch.from_numpy(x["x0"]).pin_memory()
     out_host = torch.empty_like(x_host).pin_memory()
-    xb = torch.empty((2,) + tuple(x_host.shape), device=dev)
-    xb[0].copy_(x_host)
-    xb[1].copy_(x_host)
+    n_rows = 1 if mode == "cfg-split" else 2
+    xb = torch.empty((n_rows,) + tuple(x_host.shape), device=dev)
+    xb.copy_(x_host.expand_as(xb))
     n_sched = 12
     sched = [(k / n_sched, 1.0 / n_sched, 1000.0 * (1 - k / n_sched)) for k in range(n_sched)]
     stream = torch.cuda.current_stream(dev)
+    fresh_steps = []   # attention cache: whether each timed step recomputed the attention
 
     def step(i):
         _, dt, tau = sched[i % n_sched]
-        runner.cfg_euler_step(xb, y, tau, dt, wl.cfg_scale)
+        if attn_cache is not None:
+            fresh_steps.append(attn_cache.fresh(tau))
+        if mode == "cfg-split":
+            runner.cfg_euler_step(xb[0], y, tau, dt, wl.cfg_scale)
+        else:
+            runner.cfg_euler_step(xb, y, tau, dt, wl.cfg_scale)
 
     def barrier():
         if world > 1:
@@ -292,8 +318,9 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     clk = clocks.stop()
     wd.wd_check()
-    tokens_step = B * d.L * d.blocks
+    tokens_step = rows_local * d.L * d.blocks
     ms, value = reduce_over_ranks(e0.elapsed_time(e1) / args.steps, tokens_step, world, dev)
+    timed_fresh = list(fresh_steps[args.warmup:args.warmup + args.steps])
 
     # ------------------------------------------------ the same steps again with per-launch events
     # (kernel shares, launch count and the live roofline; kept out of the timed region above)
@@ -316,7 +343,8 @@ def run_ours(args, rank, world, local_rank):
     h0.record(stream)
     for i in range(args.steps):
         xb[0].copy_(x_host, non_blocking=True)
-        xb[1].copy_(xb[0])
+        if n_rows == 2:
+            xb[1].copy_(xb[0])
         step(i)
         out_host.copy_(xb[0], non_blocking=True)
     h1.record(stream)
@@ -330,18 +358,26 @@ def run_ours(args, rank, world, local_rank):
         return 0
     pk = peaks()
     wbytes = sum(t.numel() * t.element_size() for t in weights.values())
-    flops = step_flops(d, B)
+    # the whole job's algorithmic work per step: one CFG step (both rows) per video
+    flops = step_flops(d, B) * (world if mode == "replicas" else 1)
     cache_note = None
     if args.cfg_cache is not None:
         # timed steps that ran only the conditional row do half the work of a CFG step
         fresh = sum(1 for i in range(args.steps) if sched[(args.warmup + i) % n_sched][2] / 1000.0 > args.cfg_cache)
         flops *= (fresh + 0.5 * (args.steps - fresh)) / args.steps
         cache_note = {"t_cfg": args.cfg_cache, "steps_with_both_rows": fresh, "steps_conditional_only": args.steps - fresh}
+    if attn_cache is not None:
+        # a reusing step skips, per block and row, the q/k/v projection and the self-attention
+        reuse = sum(1 for f in timed_fresh if not f)
+        skipped = B * d.blocks * (2.0 * d.L * d.D * 3 * d.D + block_flops(d)["attn_self"])
+        flops -= skipped * reuse / args.steps
+        cache_note = {"t_attn": attn_cache.t_attn, "interval": attn_cache.interval,
+                      "steps_recomputing": len(timed_fresh) - reuse, "steps_reusing": reuse}
     tflops = flops / (ms / 1e3) / 1e12
     # roofline of the dominant kernel (self-attention), timed live with events
     n_att, ms_att = tr["attn_self"]
     avg_att = ms_att / max(n_att, 1)
-    att_flops = B * block_flops(d)["attn_self"]
+    att_flops = (1 if mode == "cfg-split" else B) * block_flops(d)["attn_self"] / (world if mode == "ulysses" else 1)
     achieved = att_flops / (avg_att / 1e3) / 1e12
     peak_s = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
     share = {k: round(v[1] / max(sum(u[1] for u in tr.values()), 1e-9), 4) for k, v in tr.items()}
@@ -355,12 +391,15 @@ def run_ours(args, rank, world, local_rank):
                "detail": det}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak" if mode == "replicas" else "strong",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "video": f"{4 * (d.T - 1) + 1} frames {8 * d.H}x{8 * d.W}",
                    "latent": [16, d.T, d.H, d.W],
                    "tokens": d.L, "batch": B, "blocks": d.blocks, "D": d.D, "heads": d.heads, "ffn": d.ffn,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "parallelism": ("single GPU" if world == 1 and mode == "replicas" else
+                                   {"replicas": f"replicas x{world}", "cfg-split": "CFG rows split over 2 GPUs",
+                                    "ulysses": f"Ulysses sequence parallel x{world}"}[mode]),
                    "l2": (f"no flush: per-step working set ({wbytes / 1e9:.1f} GB weights, "
                           f"{net.X.numel() * 4 / 1e9:.1f} GB residual stream) exceeds L2")},
         "tflops": tflops, "pct_bf16_peak": tflops / pk["bf16_tflops"],
@@ -376,7 +415,7 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": traffic_for("attn_self", os.path.join(ROOT, "flow_matching_video_b200", "csrc",
                                                                       "k_attn_tc.cu"))},
         "kernel_time_share": share,
-        **({"cfg_cache": cache_note} if cache_note else {}),
+        **({("attn_cache" if attn_cache is not None else "cfg_cache"): cache_note} if cache_note else {}),
         "clocks": clk,
     }
     if cpu is not None:
@@ -408,6 +447,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cfg-cache", type=float, default=None, metavar="T",
                     help="sample with the CFG cache: steps at noise level <= T reuse the last unconditional velocity")
+    ap.add_argument("--attn-cache", type=float, nargs=2, default=None, metavar=("T", "INTERVAL"),
+                    help="sample with the attention cache: at noise level <= T recompute the self-attention every "
+                         "INTERVAL steps and reuse each block's last output in between")
+    ap.add_argument("--cfg-split", action="store_true",
+                    help="one video on two GPUs: rank 0 the text row, rank 1 the zeroed-text row (--gpus 2)")
+    ap.add_argument("--seq-parallel", action="store_true",
+                    help="one video on all GPUs: the blocks under head-sharded (Ulysses) sequence parallelism")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

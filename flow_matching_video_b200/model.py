@@ -204,6 +204,23 @@ class CfgCache:
         return xb
 
 
+def forward_reusing_attention(net: DiT, x_t, y, tau: float, o: torch.Tensor, qkv: torch.Tensor, fresh: bool,
+                              stream=None) -> torch.Tensor:
+    """A forward of `net` whose blocks either compute their self-attention
+    output into o[i] (fresh) or take it from there: o [blocks, net.batch, L, D]
+    and qkv [net.batch, L, 3D] in the storage type (qkv is scratch)."""
+    d = net.dims
+    wd.wd_time_mod(net.cd, net.time_w, tau, net.e, net.e0, stream)
+    wd.wd_patch_embed(net.cd, x_t, y, net.w["pe.w"], net.w["pe.b"], net.batch, net.X, net.ws, stream)
+    for i in range(d.blocks):
+        if fresh:
+            wd.wd_block_qkv(net.cd, net.block_w[i], net.e0, net.batch, 0, d.L, net.X, qkv, net.ws, stream)
+            wd.wd_block_self_attention(net.cd, net.batch, d.heads, qkv, o[i], stream)
+        wd.wd_block_post(net.cd, net.block_w[i], net.e0, net.kv[i], net.batch, d.L, o[i], net.X, net.ws, stream)
+    wd.wd_unpatchify(net.cd, net.head_w, net.e, net.batch, net.X, net.v, net.ws, stream)
+    return net.v
+
+
 class AttnCache:
     """Attention cache ("Wan（通义万相）..." 5.3, reuse attention outputs across
     steps): each block's self-attention output o (the input of its output
@@ -237,26 +254,61 @@ class AttnCache:
 
     def forward(self, x_t: torch.Tensor, y: torch.Tensor, tau: float, stream=None) -> torch.Tensor:
         """One forward; recomputes or reuses the attention outputs as fresh(tau) says."""
-        net, d = self.net, self.net.dims
         fresh = self.fresh(tau)
-        wd.wd_time_mod(net.cd, net.time_w, tau, net.e, net.e0, stream)
-        wd.wd_patch_embed(net.cd, x_t, y, net.w["pe.w"], net.w["pe.b"], net.batch, net.X, net.ws, stream)
-        for i in range(d.blocks):
-            if fresh:
-                wd.wd_block_qkv(net.cd, net.block_w[i], net.e0, net.batch, 0, d.L, net.X, self.qkv, net.ws, stream)
-                wd.wd_block_self_attention(net.cd, net.batch, d.heads, self.qkv, self.o[i], stream)
-            wd.wd_block_post(net.cd, net.block_w[i], net.e0, net.kv[i], net.batch, d.L, self.o[i], net.X, net.ws,
-                             stream)
-        wd.wd_unpatchify(net.cd, net.head_w, net.e, net.batch, net.X, net.v, net.ws, stream)
+        v = forward_reusing_attention(self.net, x_t, y, tau, self.o, self.qkv, fresh, stream)
         if fresh:
             self.last_fresh = self.step
         self.step += 1
-        return net.v
+        return v
 
     def cfg_euler_step(self, xb: torch.Tensor, y: torch.Tensor, tau: float, dt: float, cfg_scale: float,
                        stream=None):
         """xb [2, 16, T, H, W] as for DiT.cfg_euler_step."""
         v = self.forward(xb, y, tau, stream)
         wd.wd_euler_cfg_step(xb[0], v[0], v[1], cfg_scale, dt, stream=stream)
+        xb[1].copy_(xb[0])
+        return xb
+
+
+class DiffusionCache:
+    """The attention cache and the CFG cache together ("Wan（通义万相）..." 5.3,
+    "diffusion cache"): while the noise level exceeds t_cfg both rows run
+    (batch 2), afterwards the conditional row alone (batch 1) with the last
+    unconditional velocity reused; in either case each block's self-attention
+    output is recomputed or reused by the attention cache's rule (t_attn,
+    interval; one step counter).  A conditional-only step reads and writes the
+    conditional row's stored outputs."""
+
+    def __init__(self, dims: synth.Dims, weights: dict, t_cfg: float, t_attn: float, interval: int, device="cuda"):
+        self.cfg = CfgCache(dims, weights, t_cfg, device)
+        self.attn = AttnCache.__new__(AttnCache)   # the rule and the buffers, on the pair model
+        self.attn.net, self.attn.t_attn, self.attn.interval = self.cfg.pair, t_attn, interval
+        net = self.cfg.pair
+        self.attn.o = torch.empty((dims.blocks, 2, dims.L, dims.D), dtype=net.tdtype, device=net.device)
+        self.attn.qkv = torch.empty((2, dims.L, 3 * dims.D), dtype=net.tdtype, device=net.device)
+        self.attn.step, self.attn.last_fresh = 0, None
+        # the conditional row's slices of the buffers (contiguous per block)
+        self.o_cond = [self.attn.o[i, :1] for i in range(dims.blocks)]
+
+    def prepare_context(self, txt: torch.Tensor, clip: torch.Tensor = None):
+        self.cfg.prepare_context(txt, clip)
+        self.attn.step, self.attn.last_fresh = 0, None
+
+    def cfg_euler_step(self, xb: torch.Tensor, y: torch.Tensor, tau: float, dt: float, cfg_scale: float,
+                       stream=None):
+        """xb [2, 16, T, H, W] as for DiT.cfg_euler_step."""
+        cc, ac = self.cfg, self.attn
+        fresh = ac.fresh(tau)
+        if cc.fresh(tau):
+            v = forward_reusing_attention(cc.pair, xb, y, tau, ac.o, ac.qkv, fresh, stream)
+            cc.v_u.copy_(v[1])
+            cc.have_v_u = True
+            v_c = v[0]
+        else:
+            v_c = forward_reusing_attention(cc.cond, xb[:1], y, tau, self.o_cond, ac.qkv[:1], fresh, stream)[0]
+        if fresh:
+            ac.last_fresh = ac.step
+        ac.step += 1
+        wd.wd_euler_cfg_step(xb[0], v_c, cc.v_u, cfg_scale, dt, stream=stream)
         xb[1].copy_(xb[0])
         return xb

@@ -190,3 +190,13 @@ class SeqParallelDiT:
         net.X.copy_(self._gather.permute(1, 0, 2, 3).reshape(net.X.shape))
         wd.wd_unpatchify(net.cd, net.head_w, net.e, net.batch, net.X, net.v, net.ws)
         return net.v
+
+    def cfg_euler_step(self, xb: torch.Tensor, y, tau: float, dt: float, cfg_scale: float) -> torch.Tensor:
+        """One CFG Euler step on xb [2, 16, T, H, W] (row 0 the text row, row 1
+        the zeroed-text row; the model's context was prepared so): every rank
+        ends with the same updated latent in both rows."""
+        from . import wd
+        v = self.forward(xb, y, tau)
+        wd.wd_euler_cfg_step(xb[0], v[0], v[1], cfg_scale, dt)
+        xb[1].copy_(xb[0])
+        return xb

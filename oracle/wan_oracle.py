@@ -612,6 +612,45 @@ def sample_attn_cache(x0, img_lat, w: dict, txt, clip, dims, steps: int, cfg_sca
     return x, trace, fresh
 
 
+def sample_diffusion_cache(x0, img_lat, w: dict, txt, clip, dims, steps: int, cfg_scale: float, t_cfg: float,
+                           t_attn: float, interval: int, rnd: bool = False):
+    """The sampler with both caches of [WAN] 5.3 at once (its "diffusion
+    cache"): the CFG cache's rule picks whether a step runs both rows or the
+    conditional row alone (reusing the last unconditional velocity); the
+    attention cache's rule (one step counter) picks whether the blocks
+    recompute their self-attention outputs or reuse them.  Reading: a
+    conditional-only step reads and writes the stored outputs of the
+    conditional row.  Returns the final latent and per step (both rows?,
+    attention recomputed?)."""
+    y = None if img_lat is None else build_cond_y(img_lat)
+    txt2 = np.stack([np.asarray(txt, F64), np.zeros_like(txt, dtype=F64)])
+    ctx_txt, ctx_img = context_embed(w, txt2, clip, rnd)
+    kvs = [cross_kv(w, i, ctx_txt, ctx_img, rnd) for i in range(dims.blocks)]
+    kvs_c = [cross_kv(w, i, ctx_txt[:1], ctx_img, rnd) for i in range(dims.blocks)]
+    o = [None] * dims.blocks              # per block [2, L, D]: row 0 conditional, row 1 unconditional
+    x = np.asarray(x0, F64)
+    v_u, last, decisions = None, None, []
+    for k, (t, dt, tau) in enumerate(schedule(steps)):
+        both = v_u is None or tau / 1000.0 > t_cfg
+        fresh = attn_cache_fresh(k, tau / 1000.0, last, t_attn, interval)
+        if fresh:
+            last = k
+        if both:
+            cache = {"o": o, "reuse": not fresh}
+            v = dit_forward(np.stack([x, x]), y, tau, w, kvs, dims, rnd, attn=cache)
+            v_c, v_u = v[0], v[1]
+        else:
+            cache = {"o": [None if a is None else a[:1] for a in o], "reuse": not fresh}
+            v_c = dit_forward(x[None], y, tau, w, kvs_c, dims, rnd, attn=cache)[0]
+            for i in range(dims.blocks):
+                if o[i] is None:
+                    o[i] = np.zeros((2,) + cache["o"][i].shape[1:])
+                o[i][:1] = cache["o"][i]
+        decisions.append((both, fresh))
+        x = euler_cfg_step(x, v_c, v_u, cfg_scale, dt)
+    return x, decisions
+
+
 # ---------------------------------------------------------------- FP8 building blocks ([WAN] 5.3)
 E4M3_MAX = 448.0
 

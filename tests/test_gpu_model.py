@@ -445,3 +445,28 @@ def test_tiny_fp32_attention_cache_sampler(mods):
         assert rel(got[0], vc) < TOL_F32
         assert rel(got[1], vu) < TOL_F32
     assert rel(host(xb[0]), want_x) < TOL_F32
+
+
+def test_tiny_fp32_diffusion_cache_sampler(mods):
+    """Both caches of "Wan（通义万相）..." 5.3 together: 4 steps with t_cfg = 0.5,
+    t_attn = 0.6, interval 2 — both rows with fresh attention at noise levels
+    1 and 0.75, the conditional row alone reusing its stored attention outputs
+    at 0.5 and recomputing them at 0.25; every element of the final latent (1e-4)."""
+    model, wd = mods
+    wl = synth.TINY_MOE
+    d = wl.dims
+    w = synth.model_weights(wl)
+    x = synth.inputs(wl)
+    dc = model.DiffusionCache(d, model.weights_to_device(w, d, "cuda"), t_cfg=0.5, t_attn=0.6, interval=2)
+    dc.prepare_context(dev(np.stack([x["txt"], np.zeros_like(x["txt"])])), dev(x["clip"]))
+    y = dc.cfg.pair.build_cond_y(dev(x["img_lat"]))
+    xb = dev(np.stack([x["x0"], x["x0"]]))
+    dec = []
+    for t, dt, tau in O.schedule(wl.steps):
+        dec.append((dc.cfg.fresh(tau), dc.attn.fresh(tau)))
+        dc.cfg_euler_step(xb, y, tau, dt, wl.cfg_scale)
+    wd.wd_check()
+    want_x, want_dec = O.sample_diffusion_cache(x["x0"], x["img_lat"], w, x["txt"], x["clip"], d, wl.steps,
+                                                wl.cfg_scale, 0.5, 0.6, 2)
+    assert dec == want_dec == [(True, True), (True, True), (False, False), (False, True)]
+    assert rel(host(xb[0]), want_x) < TOL_F32

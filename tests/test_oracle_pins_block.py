@@ -379,3 +379,23 @@ def test_attention_cache_pin_catches_a_cache_that_is_never_read(monkeypatch):
     broken, _, _ = O.sample_attn_cache(x["x0"], x["img_lat"], w, x["txt"], x["clip"], d, wl.steps, wl.cfg_scale,
                                        t_attn=0.6, interval=2)
     np.testing.assert_array_equal(broken, plain)
+
+
+def test_diffusion_cache_reduces_to_each_cache_alone():
+    """Both caches at once: with the attention cache never taken it is the CFG
+    cache; with the CFG cache never taken it is the attention cache."""
+    wl = synth.TINY_MOE
+    d, w, x = wl.dims, synth.model_weights(wl), synth.inputs(wl)
+    args = (x["x0"], x["img_lat"], w, x["txt"], x["clip"], d, wl.steps, wl.cfg_scale)
+    cfg_only, _, fresh_cfg = O.sample_cfg_cache(*args, 0.5)
+    both, dec = O.sample_diffusion_cache(*args, 0.5, 0.6, 1)
+    assert [b for b, _ in dec] == fresh_cfg == [True, True, False, False]
+    np.testing.assert_array_equal(both, cfg_only)
+    attn_only, _, fresh_attn = O.sample_attn_cache(*args, 0.6, 2)
+    both, dec = O.sample_diffusion_cache(*args, -1.0, 0.6, 2)      # t_cfg < 0: both rows every step
+    assert [f for _, f in dec] == fresh_attn == [True, True, False, True]
+    np.testing.assert_array_equal(both, attn_only)
+    # together: the conditional-only steps reuse the conditional row's stored outputs
+    both, dec = O.sample_diffusion_cache(*args, 0.5, 0.6, 2)
+    assert dec == [(True, True), (True, True), (False, False), (False, True)]
+    assert np.abs(both - cfg_only).max() > 1e-6 and np.abs(both - attn_only).max() > 1e-6
