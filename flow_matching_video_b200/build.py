@@ -38,6 +38,8 @@ def build(verbose: bool = False, force: bool = False) -> str:
     tmp = f"{OUT}.{os.getpid()}.tmp"
     cmd = [NVCC, "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
            "-Xcompiler", "-fPIC", "-shared", "-o", tmp, os.path.join(SRC, "wd_lib.cu")]
+    # compile-time options of the kernels, e.g. WD_NVCC_DEFINES="WD_ATTN_SELF_BK=64"
+    cmd += ["-D" + d for d in os.environ.get("WD_NVCC_DEFINES", "").split()]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)

@@ -31,14 +31,19 @@
 namespace wd {
 namespace tca {
 
-constexpr int BQ = 128, BKV = 128, DH = 128;
-constexpr int TILE_BYTES = 128 * 128 * 2;   // one 128 x 128 tile of 2-byte elements (two 64-column halves)
+constexpr int BQ = 128, DH = 128;
+constexpr int TILE_BYTES = 128 * 128 * 2;   // one 128 x 128 Q tile of 2-byte elements (two 64-column halves)
 constexpr int HALF_BYTES = TILE_BYTES / 2;
-#ifndef WD_ATTN_RING
-#define WD_ATTN_RING 4   // K/V tiles in flight (32 KB each)
-#endif
-constexpr int RING = WD_ATTN_RING;
+constexpr int RING_BYTES = 4 * TILE_BYTES;  // K/V tiles in flight: 128 KB of shared memory
 constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
+
+#ifndef WD_ATTN_SELF_BK
+#define WD_ATTN_SELF_BK 128   // keys per block of the self-attention (128, or 64 with double-buffered S)
+#endif
+
+#ifndef WD_ATTN_ISSUERS
+#define WD_ATTN_ISSUERS 1   // MMA issuing threads of the self-attention (1, or 2: one per Q tile)
+#endif
 
 #ifndef WD_ATTN_SPLIT
 #define WD_ATTN_SPLIT 1   // softmax warps per TMEM lane quarter (1 or 2), each owning 128/SPLIT key columns
@@ -46,35 +51,53 @@ constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
 constexpr int SPLIT = WD_ATTN_SPLIT;
 static_assert(SPLIT == 1 || SPLIT == 2, "WD_ATTN_SPLIT must be 1 or 2");
 
-template <int NQ, int NSEG, typename TI>
+template <int NQ, int NSEG, typename TI, int BK = 128>
 struct Cfg {
+  static_assert(BK == 128 || BK == 64, "keys per block: 128 or 64");
+  static constexpr int BKV = BK;
+  // one K or V tile: BK keys x 128 dims, stored as two 64-dim halves of BK rows x 128 bytes
+  static constexpr int KV_BYTES = BK * DH * 2;
+  static constexpr int KV_HALF = KV_BYTES / 2;
+  static constexpr int RING = RING_BYTES / KV_BYTES;
   // 2 warps (loader, MMA) + per Q tile 4*SPLIT softmax warps: SPLIT per TMEM
-  // lane quarter (32 query rows), each owning 128/SPLIT of the key columns.
+  // lane quarter (32 query rows), each owning BK/SPLIT of the key columns.
   static constexpr int SM_WARPS = 4 * SPLIT;
   static constexpr int COLS = BKV / SPLIT;
-  static constexpr int THREADS = 64 + 32 * SM_WARPS * NQ;
+  static_assert(COLS % 64 == 0, "each softmax warp owns a multiple of 64 key columns");
+  // MMA issuing threads: one for all tiles, or (two tiles of one segment) one per tile,
+  // so that one issuer's waits overlap the other's MMAs
+  static constexpr int ISSUERS = (NSEG == 1 && NQ == 2) ? WD_ATTN_ISSUERS : 1;
+  static_assert(ISSUERS == 1 || ISSUERS == NQ, "one issuer, or one per Q tile");
+  static constexpr int THREADS = 32 * (1 + ISSUERS) + 32 * SM_WARPS * NQ;
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = NQ * TILE_BYTES;
-  static constexpr int XCH_OFF = RING_OFF + RING * TILE_BYTES;     // row-max / row-sum exchange
+  static constexpr int XCH_OFF = RING_OFF + RING_BYTES;     // row-max / row-sum exchange
   static constexpr int XCH_BYTES = NQ * (2 * 2 * 128 + 2 * 2 * 128) * 4;
   static constexpr int BAR_OFF = XCH_OFF + XCH_BYTES;
   static constexpr int SMEM = 1024 + BAR_OFF + 512;
-  static_assert(SMEM <= 232448, "shared memory budget of one CTA exceeded (reduce WD_ATTN_RING)");
+  static_assert(SMEM <= 232448, "shared memory budget of one CTA exceeded");
   static constexpr int TMEM_COLS = 512;
-  // TMEM columns.  One segment: S_t, O_t per tile (two tiles).  Two segments
-  // (one tile): O and O' in the middle and two S buffers, so that S of block
-  // n + 1 is computed while the softmax works on block n.
-  static constexpr bool DB = NSEG == 2;   // double-buffered S
-  static_assert(!DB || NQ == 1, "two key segments use one Q tile");
-  static constexpr int NBUF = DB ? 2 : NQ;   // S/P buffers (and their barriers)
-  __host__ __device__ static constexpr int buf(int t, int n) { return DB ? (n & 1) : t; }
+  // TMEM columns (512):
+  //  - one segment, 128-key blocks: S_t, O_t per tile (two tiles), one S buffer each;
+  //  - one segment, 64-key blocks: O_0, O_1 in columns 0-255, then two 64-column S
+  //    buffers per tile, so that S of block n + 1 is computed while the softmax
+  //    works on block n (double buffering);
+  //  - two segments (one tile): O and O' in the middle and two 128-column S buffers.
+  static constexpr bool DB = NSEG == 2 || BK == 64;   // double-buffered S
+  static_assert(NSEG == 1 || (NQ == 1 && BK == 128), "two key segments use one Q tile of 128-key blocks");
+  static constexpr int NBUF = DB ? 2 * NQ : NQ;   // S/P buffers (and their barriers)
+  __host__ __device__ static constexpr int buf(int t, int n) { return DB ? 2 * t + (n & 1) : t; }
   __host__ __device__ static constexpr uint32_t par(int n) { return DB ? ((n >> 1) & 1u) : (n & 1u); }
-  __host__ __device__ static constexpr int s_col(int t, int n) { return DB ? ((n & 1) ? 384 : 0) : t * 256; }
-  __host__ __device__ static constexpr int o_col(int t, int seg) { return DB ? 128 + 128 * seg : t * 256 + 128; }
+  __host__ __device__ static constexpr int s_col(int t, int n) {
+    return NSEG == 2 ? ((n & 1) ? 384 : 0) : (BK == 64 ? 256 + 128 * t + 64 * (n & 1) : t * 256);
+  }
+  __host__ __device__ static constexpr int o_col(int t, int seg) {
+    return NSEG == 2 ? 128 + 128 * seg : (BK == 64 ? 128 * t : t * 256 + 128);
+  }
   // Q K^T: both K-major; P V: P from TMEM, V MN-major (dh contiguous).  P is
   // held in the operands' type (A and B of one MMA share their type).
   static constexpr bool HALF = std::is_same<TI, f16>::value;
-  static constexpr uint32_t IDESC_S = HALF ? idesc_f16(128, 128, 0, 0) : idesc_bf16(128, 128, 0, 0);
+  static constexpr uint32_t IDESC_S = HALF ? idesc_f16(128, BK, 0, 0) : idesc_bf16(128, BK, 0, 0);
   static constexpr uint32_t IDESC_O = HALF ? idesc_f16(128, 128, 0, 1) : idesc_bf16(128, 128, 0, 1);
 };
 
@@ -123,16 +146,38 @@ __device__ __forceinline__ float exp2_fma(float x) {
   return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
 }
 
+// The same on two lanes at once with the packed fp32 instructions (f32x2): each
+// lane's operations and roundings are those of exp2_fma, in fewer instructions.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
+  const float2 magic = make_float2(12582912.f, 12582912.f);
+  const float2 t = fadd2(x, magic);
+  const float2 f = fsub2(x, fsub2(t, magic));
+  const float2 c3 = make_float2(0.0551716648f, 0.0551716648f), c2 = make_float2(0.2426111251f, 0.2426111251f);
+  const float2 c1 = make_float2(0.6932609677f, 0.6932609677f), c0 = make_float2(0.9999280572f, 0.9999280572f);
+  const float2 q = ffma2(ffma2(ffma2(c3, f, c2), f, c1), f, c0);
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
+#ifndef WD_EXP2_PACKED
+#define WD_EXP2_PACKED 0   // 1: the FMA-pipe exponentials of a pair of keys in one packed evaluation
+#endif
+
 #ifndef WD_EXP2_EMU_PER8
 #define WD_EXP2_EMU_PER8 1   // of every 8 exponentials, this many run on the FMA pipe
 #endif
+#ifndef WD_ATTN_ILP
+#define WD_ATTN_ILP 0   // 1: row max and row sum over four independent chains (shorter dependency chains)
+#endif
 
-template <int NQ, int NSEG, typename TI>
-__global__ void __launch_bounds__(Cfg<NQ, NSEG, TI>::THREADS, 1)
+template <int NQ, int NSEG, typename TI, int BK>
+__global__ void __launch_bounds__(Cfg<NQ, NSEG, TI, BK>::THREADS, 1)
 k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK0,
           const __grid_constant__ CUtensorMap tmV0, const __grid_constant__ CUtensorMap tmK1,
           const __grid_constant__ CUtensorMap tmV1, const Params p) {
-  using C = Cfg<NQ, NSEG, TI>;
+  using C = Cfg<NQ, NSEG, TI, BK>;
+  constexpr int RING = C::RING, BKV = C::BKV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
@@ -141,7 +186,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   uint64_t* kv_empty = kv_full + RING;     // RING
   uint64_t* s_full = kv_empty + RING;      // NBUF
   uint64_t* p_full = s_full + C::NBUF;     // NBUF: all of P written
-  uint64_t* p_half = p_full + C::NBUF;     // NBUF: keys 0-63 of P written
+  uint64_t* p_half = p_full + C::NBUF;     // NBUF: the first half of the block's keys of P written
   uint64_t* pv_done = p_half + C::NBUF;    // NBUF: P V of the block in that buffer completed (double buffering)
   uint64_t* o_done = pv_done + C::NBUF;    // NQ
   uint64_t* tdone = o_done + NQ;           // 1
@@ -162,7 +207,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < RING; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+    for (int s = 0; s < RING; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], C::ISSUERS); }
     for (int i = 0; i < C::NBUF; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], C::SM_WARPS);
@@ -170,7 +215,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       mbar_init(&pv_done[i], 1);
     }
     for (int t = 0; t < NQ; ++t) mbar_init(&o_done[t], 1);
-    mbar_init(tdone, 1);
+    mbar_init(tdone, C::ISSUERS);
     for (int i = 0; i < 4 * NQ; ++i) { mbar_init(&mx_bar[i], 2); mbar_init(&fin_bar[i], 2); }
     fence_mbar_init();
   }
@@ -200,10 +245,10 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           const int seq = 2 * n + kv, slot = seq % RING;
           const uint32_t ph = (seq / RING) & 1u;
           if (!mbar_wait(&kv_empty[slot], ph ^ 1u, SITE_KVE)) { ok = false; break; }
-          mbar_arrive_expect_tx(&kv_full[slot], TILE_BYTES);
+          mbar_arrive_expect_tx(&kv_full[slot], C::KV_BYTES);
           const int col = h * DH;
           for (int hf = 0; hf < 2; ++hf)
-            tma_load_3d(smem + C::RING_OFF + slot * TILE_BYTES + hf * HALF_BYTES, kv ? tv : tk, col + hf * 64, j0,
+            tma_load_3d(smem + C::RING_OFF + slot * C::KV_BYTES + hf * C::KV_HALF, kv ? tv : tk, col + hf * 64, j0,
                         bb, &kv_full[slot]);
           issued |= 1u << slot;
           last_par = (last_par & ~(1u << slot)) | (ph << slot);
@@ -214,13 +259,22 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         if (issued & (1u << s)) mbar_wait(&kv_full[s], (last_par >> s) & 1u, SITE_DRAIN);
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp <= C::ISSUERS) {
+    // ------------------------------------------------------------ MMA issuer(s)
+    // tiles [t_lo, t_hi) of this issuer: all of them, or its own one
+    const int t_lo = C::ISSUERS == 1 ? 0 : warp - 1, t_hi = C::ISSUERS == 1 ? NQ : warp;
     if (lane == 0) {
       bool ok = mbar_wait(q_full, 0, SITE_Q);
       tc_fence_after();
       const uint32_t q0 = smem_u32(smem + C::Q_OFF);
       const uint32_t r0 = smem_u32(smem + C::RING_OFF);
+      // Shared-memory descriptors as (low, high) halves: the high halves are
+      // fixed, the start address in the low half steps by 16-byte units.
+      const uint64_t dq0 = sdesc_sw128(q0, 16, 1024), dk0 = sdesc_sw128(r0, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(r0, C::KV_HALF, 1024);
+      const uint32_t q_lo = static_cast<uint32_t>(dq0), k_lo = static_cast<uint32_t>(dk0);
+      const uint32_t v_lo = static_cast<uint32_t>(dv0);
+      const uint32_t s_hi = static_cast<uint32_t>(dq0 >> 32), v_hi = static_cast<uint32_t>(dv0 >> 32);
       // P_t V_j for block n of tile t
       auto issue_pv = [&](int t, int n) -> bool {
         const int vseq = 2 * n + 1, vslot = vseq % RING;
@@ -228,41 +282,45 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         const int first = (n == 0) || (n == nb0);
         const int bi = C::buf(t, n);
         const uint32_t d = tmem + C::o_col(t, sg);
-        const uint32_t pa = tmem + C::s_col(t, n), vb = r0 + vslot * TILE_BYTES;
-        // With one softmax warp per lane quarter, P arrives in two halves (keys
-        // 0-63, then 64-127): the first four k-steps start as soon as the first
+        const uint32_t pa = tmem + C::s_col(t, n), vb_lo = v_lo + vslot * (C::KV_BYTES >> 4);
+        // With one softmax warp per lane quarter, P arrives in two halves of the
+        // block's keys: the first half of the k-steps starts as soon as the first
         // half is in TMEM.
+        constexpr int KK = BKV / 16;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           if (SPLIT == 1 || half == 0) {
             uint64_t* bar = (SPLIT == 1 && half == 0) ? &p_half[bi] : &p_full[bi];
             if (!MMA_WAIT(bar, C::par(n), SITE_P)) return false;
           }
-          if (half == 0 && !MMA_WAIT(&kv_full[vslot], (vseq / RING) & 1u, SITE_KVF)) return false;
+          // the V tile: waited for by this issuer's first tile (its other tiles read the same tile)
+          if (half == 0 && t == t_lo && !MMA_WAIT(&kv_full[vslot], (vseq / RING) & 1u, SITE_KVF)) return false;
           tc_fence_after();
 #pragma unroll
-          for (int kk = half * 4; kk < half * 4 + 4; ++kk) {
+          for (int kk = half * KK / 2; kk < (half + 1) * KK / 2; ++kk) {
             // A = P: 16 keys = 8 TMEM columns of packed bf16 pairs; each softmax
             // warp's keys sit over the first half of its own S columns:
             // key 16 kk lives at column (16kk / COLS) * COLS + (16kk % COLS) / 2
-            const uint64_t bd = sdesc_sw128(vb + kk * 2048, HALF_BYTES, 1024);
-            umma_ts(d, pa + (16 * kk / C::COLS) * C::COLS + (16 * kk % C::COLS) / 2, bd, C::IDESC_O,
-                    (!first || kk) ? 1u : 0u);
+            // B = V rows 16 kk .. 16 kk + 15: 2048 bytes on within each 64-dim half
+            umma_ts_lh(d, pa + (16 * kk / C::COLS) * C::COLS + (16 * kk % C::COLS) / 2, vb_lo + kk * (2048 >> 4), v_hi,
+                       C::IDESC_O, (!first || kk) ? 1u : 0u);
           }
         }
         if (C::DB) umma_commit(&pv_done[bi]);
-        if (t == NQ - 1) umma_commit(&kv_empty[vslot]);
+        if (t == t_hi - 1) umma_commit(&kv_empty[vslot]);
         return true;
       };
       // S_t = Q_t K_n^T into tile t's S buffer for block n (K tile already waited for)
       auto issue_s = [&](int t, int n) {
         const int kslot = (2 * n) % RING;
         const uint32_t d = tmem + C::s_col(t, n);
-        const uint32_t qa = q0 + t * TILE_BYTES, kb = r0 + kslot * TILE_BYTES;
+        const uint32_t qa = q_lo + t * (TILE_BYTES >> 4), kb = k_lo + kslot * (C::KV_BYTES >> 4);
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-          umma_ss(d, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), C::IDESC_S, kk ? 1u : 0u);
+          // 16 dims per step: 32 bytes into a 128-byte row of the step's 64-dim half
+          const uint32_t oq = ((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4;
+          const uint32_t ok_ = ((kk >> 2) * C::KV_HALF + (kk & 3) * 32) >> 4;
+          umma_ss_lh(d, qa + oq, s_hi, kb + ok_, s_hi, C::IDESC_S, kk ? 1u : 0u);
         }
         umma_commit(&s_full[C::buf(t, n)]);
       };
@@ -273,34 +331,37 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         return true;
       };
       if constexpr (C::DB) {
-        // One tile, two S buffers: S of blocks 0 and 1 first; then per block
-        // P V, and S of the block two ahead into the buffer that P V has read.
+        // Two S buffers per tile: S of blocks 0 and 1 first; then per block and
+        // tile P V, and S of the block two ahead into the buffer that P V has
+        // read (the MMAs of one thread run in issue order).
         for (int n = 0; n < 2 && n < NB && ok; ++n) {
           if (!wait_k(n)) { ok = false; break; }
-          issue_s(0, n);
+          for (int t = t_lo; t < t_hi; ++t) issue_s(t, n);
           umma_commit(&kv_empty[(2 * n) % RING]);
         }
         for (int n = 0; n < NB && ok; ++n) {
-          if (!issue_pv(0, n)) { ok = false; break; }
-          if (n + 2 < NB) {
-            if (!wait_k(n + 2)) { ok = false; break; }
-            issue_s(0, n + 2);
-            umma_commit(&kv_empty[(2 * (n + 2)) % RING]);
+          for (int t = t_lo; t < t_hi && ok; ++t) {
+            if (!issue_pv(t, n)) { ok = false; break; }
+            if (n + 2 < NB) {
+              if (t == t_lo && !wait_k(n + 2)) { ok = false; break; }
+              issue_s(t, n + 2);
+            }
           }
+          if (ok && n + 2 < NB) umma_commit(&kv_empty[(2 * (n + 2)) % RING]);
         }
-        if (ok) umma_commit(&o_done[0]);
+        for (int t = t_lo; t < t_hi && ok; ++t) umma_commit(&o_done[t]);
       } else {
         for (int n = 0; n < NB && ok; ++n) {
-          for (int t = 0; t < NQ && ok; ++t) {
+          for (int t = t_lo; t < t_hi && ok; ++t) {
             // P_t V of the previous block first: it needs only P_t and that V tile,
             // not the next K tile.
             if (n > 0 && !issue_pv(t, n - 1)) { ok = false; break; }
-            if (t == 0 && !wait_k(n)) { ok = false; break; }
+            if (t == t_lo && !wait_k(n)) { ok = false; break; }
             issue_s(t, n);
           }
           if (ok) umma_commit(&kv_empty[(2 * n) % RING]);
         }
-        for (int t = 0; t < NQ && ok; ++t) {
+        for (int t = t_lo; t < t_hi && ok; ++t) {
           if (!issue_pv(t, NB - 1)) { ok = false; break; }
           umma_commit(&o_done[t]);
         }
@@ -311,8 +372,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax warps
-    constexpr int COLS = C::COLS, CH = COLS / 32;
-    const int sw = warp - 2;
+    constexpr int COLS = C::COLS, CH = COLS / 32;      // this warp's key columns of a block
+    constexpr int OCOLS = DH / SPLIT, OCH = OCOLS / 32;   // ... and its output columns (of dh)
+    const int sw = warp - 1 - C::ISSUERS;
     const int t = sw / C::SM_WARPS;        // Q tile
     const int hc = SPLIT == 2 ? (sw >> 2) & 1 : 0;   // key part of this warp: columns [COLS hc, COLS hc + COLS)
     const int quarter = warp & 3;          // TMEM lanes this warp may access
@@ -345,12 +407,26 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             if (c * 32 + k >= valid) a[c][k] = __float_as_uint(-INFINITY);
       }
       float mx = -INFINITY;
+      if constexpr (WD_ATTN_ILP) {
+        // four chains, each over every fourth pair of columns, then combined
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < CH; c += 2)
+        for (int c = 0; c < CH; c += 2)
 #pragma unroll
-        for (int k = 0; k < 32; k += 2)
-          mx = fmax3(mx, fmax3(__uint_as_float(a[c][k]), __uint_as_float(a[c][k + 1]), __uint_as_float(a[c + 1][k])),
-                     __uint_as_float(a[c + 1][k + 1]));
+          for (int k = 0; k < 32; k += 2)
+            m4[(k >> 1) & 3] = fmax3(m4[(k >> 1) & 3],
+                                     fmax3(__uint_as_float(a[c][k]), __uint_as_float(a[c][k + 1]),
+                                           __uint_as_float(a[c + 1][k])),
+                                     __uint_as_float(a[c + 1][k + 1]));
+        mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < CH; c += 2)
+#pragma unroll
+          for (int k = 0; k < 32; k += 2)
+            mx = fmax3(mx, fmax3(__uint_as_float(a[c][k]), __uint_as_float(a[c][k + 1]), __uint_as_float(a[c + 1][k])),
+                       __uint_as_float(a[c + 1][k + 1]));
+      }
       if constexpr (SPLIT == 2) {   // the two warps of a lane quarter swap their row maxima
         float* slot = xmax + ((n & 1) * NQ + t) * 256;
         slot[hc * 128 + r] = mx;
@@ -374,9 +450,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       if (__any_sync(0xffffffffu, grow) && !first) {
         if (C::DB && !mbar_wait_warp(&pv_done[C::buf(t, n - 1)], C::par(n - 1), SITE_O)) { ok = false; break; }
         if (C::DB) tc_fence_after();
-        const uint32_t o_addr = tmem + lane_base + C::o_col(t, sg) + hc * COLS;
+        const uint32_t o_addr = tmem + lane_base + C::o_col(t, sg) + hc * OCOLS;
 #pragma unroll 1
-        for (int c = 0; c < CH; ++c) {
+        for (int c = 0; c < OCH; ++c) {
           uint32_t o[32];
           tmem_ld32(o_addr + c * 32, o);
           tmem_wait_ld();
@@ -390,6 +466,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       // own S columns: chunk c of 16 keys -> 8 columns at 8c (masked keys hold
       // -inf, so their exponential is 0)
       float2 rs2 = make_float2(0.f, 0.f);
+      [[maybe_unused]] float2 rs4[4] = {rs2, rs2, rs2, rs2};   // four partial sums (WD_ATTN_ILP)
       const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(neg_m, neg_m);
 #pragma unroll
       for (int c = 0; c < 2 * CH; ++c) {
@@ -399,13 +476,21 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           const int kk = (c & 1) * 16 + k;
           const float2 arg = ffma2(make_float2(__uint_as_float(a[c >> 1][kk]), __uint_as_float(a[c >> 1][kk + 1])),
                                    sc2, nm2);
-          const float e0 = ((k & 7) >= 8 - WD_EXP2_EMU_PER8) ? exp2_fma(arg.x) : ex2(arg.x);
-          const float e1 = (((k + 1) & 7) >= 8 - WD_EXP2_EMU_PER8) ? exp2_fma(arg.y) : ex2(arg.y);
-          rs2 = fadd2(rs2, make_float2(e0, e1));
+          float e0, e1;
+          if (WD_EXP2_PACKED && (k & 7) >= 8 - WD_EXP2_EMU_PER8 && ((k + 1) & 7) >= 8 - WD_EXP2_EMU_PER8) {
+            const float2 e = exp2_fma2(arg);
+            e0 = e.x;
+            e1 = e.y;
+          } else {
+            e0 = ((k & 7) >= 8 - WD_EXP2_EMU_PER8) ? exp2_fma(arg.x) : ex2(arg.x);
+            e1 = (((k + 1) & 7) >= 8 - WD_EXP2_EMU_PER8) ? exp2_fma(arg.y) : ex2(arg.y);
+          }
+          if constexpr (WD_ATTN_ILP) rs4[(k >> 1) & 3] = fadd2(rs4[(k >> 1) & 3], make_float2(e0, e1));
+          else rs2 = fadd2(rs2, make_float2(e0, e1));
           pk[k >> 1] = C::HALF ? pack_f16x2(e0, e1) : pack_bf16x2(e0, e1);
         }
         tmem_st8(s_addr + c * 8, pk);
-        if (SPLIT == 1 && c == CH - 1) {   // keys 0-63 of P are written: release the first half of P V
+        if (SPLIT == 1 && c == CH - 1) {   // the first half of the block's P is written: release its P V
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
@@ -413,6 +498,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         }
       }
       tmem_wait_st();
+      if constexpr (WD_ATTN_ILP) rs2 = fadd2(fadd2(rs4[0], rs4[1]), fadd2(rs4[2], rs4[3]));
       l = l * alpha + (rs2.x + rs2.y);     // this warp's share of the row sum
       tc_fence_before();
       __syncwarp();
@@ -437,18 +523,18 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       const int row = l0 + t * BQ + r;
       const float inv1 = 1.f / l;
       const float inv0 = NSEG == 2 ? 1.f / l_first : 0.f;
-      bf16* dst = p.o + (static_cast<int64_t>(b) * p.Lq + row) * p.o_rs + h * DH + hc * COLS;
+      bf16* dst = p.o + (static_cast<int64_t>(b) * p.Lq + row) * p.o_rs + h * DH + hc * OCOLS;
 #pragma unroll 1
-      for (int c = 0; c < CH; ++c) {
+      for (int c = 0; c < OCH; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_base + C::o_col(t, NSEG - 1) + hc * COLS + c * 32, o);
+        tmem_ld32(tmem + lane_base + C::o_col(t, NSEG - 1) + hc * OCOLS + c * 32, o);
         tmem_wait_ld();
         float v[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(o[k]) * inv1;
         if (NSEG == 2) {
           uint32_t o2[32];
-          tmem_ld32(tmem + lane_base + C::o_col(t, 0) + hc * COLS + c * 32, o2);
+          tmem_ld32(tmem + lane_base + C::o_col(t, 0) + hc * OCOLS + c * 32, o2);
           tmem_wait_ld();
 #pragma unroll
           for (int k = 0; k < 32; ++k) v[k] += __uint_as_float(o2[k]) * inv0;
@@ -474,9 +560,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 
 // ------------------------------------------------------------------ host side
 // 3D tensor map (bf16 or IEEE half elements) over [batches, rows, cols] (cols contiguous, row stride
-// `rs` elements, batch stride `bs` elements); box = 64 cols x 128 rows x 1.
+// `rs` elements, batch stride `bs` elements); box = 64 cols x box_rows rows x 1.
 static wd_status make_tmap_3d(CUtensorMap* m, CUtensorMapDataType type, const void* base, int64_t cols, int64_t rows,
-                              int64_t batches, int64_t rs, int64_t bs) {
+                              int64_t batches, int64_t rs, int64_t bs, int box_rows = 128) {
   auto fn = encode_fn();
   if (!fn) { set_error("cuTensorMapEncodeTiled unavailable"); return WD_ERR_CUDA; }
   if (batches > 1 && (bs * 2) % 16) { set_error("attention: batch stride not 16-byte aligned"); return WD_ERR_ALIGN; }
@@ -484,7 +570,7 @@ static wd_status make_tmap_3d(CUtensorMap* m, CUtensorMapDataType type, const vo
                         static_cast<cuuint64_t>(batches)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(rs) * 2,
                            static_cast<cuuint64_t>(batches > 1 ? bs : rs * rows) * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = fn(m, type, 3, const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -493,21 +579,21 @@ static wd_status make_tmap_3d(CUtensorMap* m, CUtensorMapDataType type, const vo
   return WD_OK;
 }
 
-template <int NQ, int NSEG, typename TI>
+template <int NQ, int NSEG, typename TI, int BK>
 static wd_status launch_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk0, const CUtensorMap& tv0,
                                 const CUtensorMap& tk1, const CUtensorMap& tv1, const tca::Params& p, int batch,
                                 int heads, bool cross, cudaStream_t st) {
-  using C = tca::Cfg<NQ, NSEG, TI>;
+  using C = tca::Cfg<NQ, NSEG, TI, BK>;
   static bool attr[16] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr[dev & 15]) {
-    cudaFuncSetAttribute(tca::k_attn_tc<NQ, NSEG, TI>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaFuncSetAttribute(tca::k_attn_tc<NQ, NSEG, TI, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     attr[dev & 15] = true;
   }
   dim3 grid((p.Lq + tca::BQ * NQ - 1) / (tca::BQ * NQ), heads, batch);
   Trace tr(cross ? KC_ATTN_CROSS : KC_ATTN_SELF, st);
-  tca::k_attn_tc<NQ, NSEG, TI><<<grid, C::THREADS, C::SMEM, st>>>(tq, tk0, tv0, tk1, tv1, p);
+  tca::k_attn_tc<NQ, NSEG, TI, BK><<<grid, C::THREADS, C::SMEM, st>>>(tq, tk0, tv0, tk1, tv1, p);
   return launch_status("attention_tc");
 }
 
@@ -531,8 +617,11 @@ static wd_status attention_tc_t(const AttnArgs<TI, bf16>& a, cudaStream_t st) {
   // Each map covers D columns from its own base pointer.
   WD_TRY(make_tmap_3d(&tq, ty, a.q, D, a.Lq, a.batch, a.q_rs, a.q_rs * a.Lq));
   const int64_t b1 = a.kv1_bs ? a.batch : 1;
-  WD_TRY(make_tmap_3d(&tk0, ty, a.k1, D, a.n1, b1, a.kv1_rs, a.kv1_bs));
-  WD_TRY(make_tmap_3d(&tv0, ty, a.v1, D, a.n1, b1, a.kv1_rs, a.kv1_bs));
+  // keys per block: the self-attention's (one segment) or 128 (two segments)
+  constexpr int BK1 = WD_ATTN_SELF_BK;
+  const int bk = a.k2 ? 128 : BK1;
+  WD_TRY(make_tmap_3d(&tk0, ty, a.k1, D, a.n1, b1, a.kv1_rs, a.kv1_bs, bk));
+  WD_TRY(make_tmap_3d(&tv0, ty, a.v1, D, a.n1, b1, a.kv1_rs, a.kv1_bs, bk));
   tca::Params p{};
   p.Lq = a.Lq;
   p.seg[0] = tca::Seg{a.n1, a.kv1_bs == 0};
@@ -544,9 +633,9 @@ static wd_status attention_tc_t(const AttnArgs<TI, bf16>& a, cudaStream_t st) {
     WD_TRY(make_tmap_3d(&tk1, ty, a.k2, D, a.n2, b2, a.kv2_rs, a.kv2_bs));
     WD_TRY(make_tmap_3d(&tv1, ty, a.v2, D, a.n2, b2, a.kv2_rs, a.kv2_bs));
     p.seg[1] = tca::Seg{a.n2, a.kv2_bs == 0};
-    return launch_attn_tc<1, 2, TI>(tq, tk0, tv0, tk1, tv1, p, a.batch, a.heads, a.cross, st);
+    return launch_attn_tc<1, 2, TI, 128>(tq, tk0, tv0, tk1, tv1, p, a.batch, a.heads, a.cross, st);
   }
-  return launch_attn_tc<2, 1, TI>(tq, tk0, tv0, tk0, tv0, p, a.batch, a.heads, a.cross, st);
+  return launch_attn_tc<2, 1, TI, BK1>(tq, tk0, tv0, tk0, tv0, p, a.batch, a.heads, a.cross, st);
 }
 
 wd_status attention_tc(const AttnArgs<bf16, bf16>& a, cudaStream_t st) { return attention_tc_t<bf16>(a, st); }

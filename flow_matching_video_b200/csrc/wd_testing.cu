@@ -10,12 +10,15 @@
 
 namespace wd {
 
-__global__ void k_test_exp2(const float* __restrict__ x, float* __restrict__ y_fma, float* __restrict__ y_mufu,
-                            float* __restrict__ y_lib, int64_t n) {
+__global__ void k_test_exp2(const float* __restrict__ x, float* __restrict__ y_fma, float* __restrict__ y_fma2,
+                            float* __restrict__ y_mufu, float* __restrict__ y_lib, int64_t n) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const float v = x[i];
     y_fma[i] = tca::exp2_fma(v);
+    // the packed form on the pair (x[i], x[i ^ 1]): lane 0 is x[i]
+    const int64_t j = ((i ^ 1) < n) ? (i ^ 1) : i;   // the partner index, inside [0, n)
+    y_fma2[i] = tca::exp2_fma2(make_float2(v, x[j])).x;
     y_mufu[i] = tca::ex2(v);
     y_lib[i] = exp2f(v);
   }
@@ -40,14 +43,15 @@ __global__ void k_test_wait_timeout(uint64_t limit_ns, unsigned site, int* out) 
 
 extern "C" {
 
-wd_status wd_test_exp2(const float* x, float* y_fma, float* y_mufu, float* y_lib, int64_t n, wd_stream stream) {
+wd_status wd_test_exp2(const float* x, float* y_fma, float* y_fma2, float* y_mufu, float* y_lib, int64_t n,
+                       wd_stream stream) {
   using namespace wd;
-  WD_NEED(x); WD_NEED(y_fma); WD_NEED(y_mufu); WD_NEED(y_lib);
+  WD_NEED(x); WD_NEED(y_fma); WD_NEED(y_fma2); WD_NEED(y_mufu); WD_NEED(y_lib);
   if (n <= 0) { set_error("wd_test_exp2: n = %lld", (long long)n); return WD_ERR_SHAPE; }
   const int64_t blocks = (n + 255) / 256;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Trace tr(KC_SMALL, st);
-  k_test_exp2<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0, st>>>(x, y_fma, y_mufu, y_lib, n);
+  k_test_exp2<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0, st>>>(x, y_fma, y_fma2, y_mufu, y_lib, n);
   return launch_status("test_exp2");
 }
 

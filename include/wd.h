@@ -333,14 +333,17 @@ wd_status wd_gemm_fp8(int M, int N, int K, const void* Aq, const float* sa, cons
  * Two entry points that exist only so that tests can reach pieces of the
  * kernels no output of the path exposes on its own.  Not part of the step. */
 
-/* Evaluates, for each of the n fp32 values x[i], the three 2^x of the
- * attention kernels' world: y_fma[i] = the FMA-pipe 2^x that the softmax of
- * the tensor-core attention uses for some of its exponentials (range
- * reduction to x = j + f, |f| <= 1/2, a degree-3 polynomial in f with a
- * stated relative error below 7.5e-5, inputs below -125 clamped to -125),
- * y_mufu[i] = the MUFU approximation ex2.approx.ftz.f32 used for the rest,
- * y_lib[i] = CUDA's exp2f.  All device arrays of n floats; n > 0. */
-wd_status wd_test_exp2(const float* x, float* y_fma, float* y_mufu, float* y_lib, int64_t n, wd_stream stream);
+/* Evaluates, for each of the n fp32 values x[i], the 2^x of the attention
+ * kernels' world: y_fma[i] = the FMA-pipe 2^x that the softmax of the
+ * tensor-core attention uses for some of its exponentials (range reduction
+ * to x = j + f, |f| <= 1/2, a degree-3 polynomial in f with a stated relative
+ * error below 7.5e-5, inputs below -125 clamped to -125); y_fma2[i] = the
+ * same function in its packed two-lane form (f32x2 instructions), evaluated
+ * on the pair (x[i], x[i^1]), which must equal y_fma[i]; y_mufu[i] = the MUFU
+ * approximation ex2.approx.ftz.f32 used for the rest; y_lib[i] = CUDA's
+ * exp2f.  All device arrays of n floats; n > 0. */
+wd_status wd_test_exp2(const float* x, float* y_fma, float* y_fma2, float* y_mufu, float* y_lib, int64_t n,
+                       wd_stream stream);
 
 /* Launches one warp that waits on an mbarrier phase nothing completes, with
  * the library's bounded wait given a limit of limit_ns (at most 100 ms, not

@@ -364,17 +364,20 @@ def test_exp2_fma_within_its_stated_bound(wd):
     [-130, 0] plus every half-integer (where the range reduction's rounding
     switches the integer part) and its float32 neighbours: relative error at
     most 7.5e-5 against float64 2^x, the bound its polynomial was fitted to;
-    inputs below -125 give 2^-125 within the same bound.  The MUFU ex2 and
-    CUDA's exp2f are checked beside it."""
+    inputs below -125 give 2^-125 within the same bound.  Its packed
+    two-lane form must give the same values; the MUFU ex2 and CUDA's exp2f
+    are checked beside it."""
     halves = np.arange(-130.0, 0.5, 0.5, dtype=np.float32)
     x = np.concatenate([np.linspace(-130.0, 0.0, 2_000_001, dtype=np.float32), halves,
                         np.nextafter(halves, np.float32(1)), np.nextafter(halves, np.float32(-200)),
                         np.float32([-1e-30, -1e-7, -0.0, -125.0, -125.5, -126.0, -1000.0])]).astype(np.float32)
     gx = dev(x)
-    outs = [torch.empty_like(gx) for _ in range(3)]
+    outs = [torch.empty_like(gx) for _ in range(4)]
     wd.wd_test_exp2(gx, *outs)
     wd.wd_check()
-    y_fma, y_mufu, y_lib = (o.cpu().numpy().astype(np.float64) for o in outs)
+    y_fma, y_fma2, y_mufu, y_lib = (o.cpu().numpy().astype(np.float64) for o in outs)
+    # the packed two-lane form computes the same function, lane by lane
+    np.testing.assert_array_equal(y_fma2, y_fma)
     x64 = x.astype(np.float64)
     ref = np.exp2(np.maximum(x64, -125.0))
     r_fma = np.abs(y_fma / ref - 1.0)
