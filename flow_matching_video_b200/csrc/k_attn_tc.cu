@@ -117,6 +117,8 @@ struct Params {
   bf16* o;
   int64_t o_rs;
   float scale_log2;
+  float* lse;   // one segment, optional: [batch, heads, Lq] row log-sum-exp (log2 units)
+  int heads;
 };
 
 // Bounded waits: the MMA thread alone, the softmax warps as whole warps.
@@ -161,14 +163,14 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 }
 
 #ifndef WD_EXP2_PACKED
-#define WD_EXP2_PACKED 0   // 1: the FMA-pipe exponentials of a pair of keys in one packed evaluation
+#define WD_EXP2_PACKED 1   // 1: the FMA-pipe exponentials of a pair of keys in one packed evaluation
 #endif
 
 #ifndef WD_EXP2_EMU_PER8
-#define WD_EXP2_EMU_PER8 1   // of every 8 exponentials, this many run on the FMA pipe
+#define WD_EXP2_EMU_PER8 2   // of every 8 exponentials, this many run on the FMA pipe
 #endif
 #ifndef WD_ATTN_ILP
-#define WD_ATTN_ILP 0   // 1: row max and row sum over four independent chains (shorter dependency chains)
+#define WD_ATTN_ILP 1   // 1: row max and row sum over four independent chains (shorter dependency chains)
 #endif
 
 template <int NQ, int NSEG, typename TI, int BK>
@@ -522,6 +524,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       tc_fence_after();
       const int row = l0 + t * BQ + r;
       const float inv1 = 1.f / l;
+      // the row's log-sum-exp in log2 units: the reference max plus log2 of the sum relative to it
+      if (NSEG == 1 && p.lse && hc == 0 && row < p.Lq)
+        p.lse[(static_cast<int64_t>(b) * p.heads + h) * p.Lq + row] = m + __log2f(l);
       const float inv0 = NSEG == 2 ? 1.f / l_first : 0.f;
       bf16* dst = p.o + (static_cast<int64_t>(b) * p.Lq + row) * p.o_rs + h * DH + hc * OCOLS;
 #pragma unroll 1
@@ -628,6 +633,8 @@ static wd_status attention_tc_t(const AttnArgs<TI, bf16>& a, cudaStream_t st) {
   p.o = a.o;
   p.o_rs = a.o_rs;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(a.dh));
+  p.lse = a.k2 ? nullptr : a.lse;
+  p.heads = a.heads;
   if (a.k2) {
     const int64_t b2 = a.kv2_bs ? a.batch : 1;
     WD_TRY(make_tmap_3d(&tk1, ty, a.k2, D, a.n2, b2, a.kv2_rs, a.kv2_bs));

@@ -169,6 +169,11 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
+      // Shared-memory descriptors as (low, high) halves: the high half is fixed and
+      // the start-address field in the low half steps by 16-byte units.
+      const uint64_t da0 = sdesc_sw128(smem_u32(sA), 16, 1024), db0 = sdesc_sw128(smem_u32(sB), 16, 1024);
+      const uint32_t a_lo0 = static_cast<uint32_t>(da0), b_lo0 = static_cast<uint32_t>(db0);
+      const uint32_t d_hi = static_cast<uint32_t>(da0 >> 32);
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, SITE_TEMPTY)) { ok = false; break; }
         tc_fence_after();
@@ -176,16 +181,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         for (int k = 0; k < k_iters; ++k) {
           if (!mbar_wait(&full[stage], phase, SITE_FULL)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
-          const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
+          const uint32_t a_lo = a_lo0 + stage * (C::A_BYTES >> 4), b_lo = b_lo0 + stage * (C::B_BYTES >> 4);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {   // 32 bytes of K per MMA: 16 bf16 or 32 e4m3 elements
             if constexpr (F8)
-              umma_ss_f8(d, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), C::IDESC_F8,
-                         (k | kk) != 0);
+              umma_ss_f8_lh(d, a_lo + kk * 2, d_hi, b_lo + kk * 2, d_hi, C::IDESC_F8, (k | kk) != 0);
             else
-              umma_ss(d, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), C::IDESC,
-                      (k | kk) != 0);
+              umma_ss_lh(d, a_lo + kk * 2, d_hi, b_lo + kk * 2, d_hi, C::IDESC, (k | kk) != 0);
           }
           umma_commit(&empty[stage]);   // frees the smem slot once these MMAs have read it
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }

@@ -186,6 +186,10 @@ __global__ void __launch_bounds__(256) k_attn_simt(AttnArgs<T, TO> a, float qsca
       const float inv = 1.f / lrow[i];
 #pragma unroll
       for (int c = 0; c < CW; ++c) out[i][c] += o[i][c] * inv;
+      // one segment: the row's log-sum-exp in log2 units (the scores carry log2(e) already)
+      const int l = q0 + ty * 4 + i;
+      if (a.lse && !a.k2 && tx == 0 && l < a.Lq)
+        a.lse[(static_cast<int64_t>(b) * a.heads + h) * a.Lq + l] = mrow[i] + log2f(lrow[i]);
     }
   }
 #pragma unroll

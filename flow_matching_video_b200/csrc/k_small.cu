@@ -331,6 +331,58 @@ __global__ void __launch_bounds__(256) k_patch_gather(const float* __restrict__ 
 }
 
 
+// ============================================================ merging attention over key parts
+// For a query row, the attention over the union of disjoint key sets is the
+// average of the attentions over each set weighted by each set's share of the
+// softmax denominator: with row log-sum-exps lse_r, lse_p (log2 units) and
+// M = max(lse_r, lse_p), o = (2^(lse_r - M) o_r + 2^(lse_p - M) o_p) / (2^(lse_r - M) + 2^(lse_p - M))
+// and lse = M + log2(2^(lse_r - M) + 2^(lse_p - M)).  One warp per (batch, head, row).
+template <typename TP>
+__global__ void __launch_bounds__(256) k_attn_merge(int batch, int Lq, int heads, int dh, float* __restrict__ o_run,
+                                                    float* __restrict__ lse_run, const TP* __restrict__ o_part,
+                                                    const float* __restrict__ lse_part, int first, TP* __restrict__ out) {
+  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;   // (b, h, l)
+  const int lane = threadIdx.x & 31;
+  if (w >= static_cast<int64_t>(batch) * heads * Lq) return;
+  const int l = static_cast<int>(w % Lq);
+  const int64_t bh = w / Lq;
+  const int h = static_cast<int>(bh % heads);
+  const int64_t b = bh / heads;
+  const int64_t base = (b * Lq + l) * static_cast<int64_t>(heads) * dh + static_cast<int64_t>(h) * dh;
+  const float lp = lse_part[w];
+  float wr = 0.f, wp = 1.f, lnew = lp;
+  if (!first) {
+    const float lr = lse_run[w];
+    const float M = fmaxf(lr, lp);
+    const float a = exp2f(lr - M), c = exp2f(lp - M), sum = a + c;
+    wr = a / sum;
+    wp = c / sum;
+    lnew = M + log2f(sum);
+  }
+  for (int d = lane; d < dh; d += 32) {
+    const float v = (first ? 0.f : wr * o_run[base + d]) + wp * to_f<TP>(o_part[base + d]);
+    o_run[base + d] = v;
+    if (out) out[base + d] = from_f<TP>(v);
+  }
+  __syncwarp();
+  if (lane == 0) lse_run[w] = lnew;
+}
+
+template <typename TP>
+wd_status attn_merge(int batch, int Lq, int heads, int dh, float* o_run, float* lse_run, const TP* o_part,
+                     const float* lse_part, int first, TP* out, cudaStream_t st) {
+  if (batch <= 0 || Lq <= 0 || heads <= 0 || dh <= 0) { set_error("attention merge: empty shape"); return WD_ERR_SHAPE; }
+  const int64_t threads = static_cast<int64_t>(batch) * heads * Lq * 32;
+  Trace tr(KC_SMALL, st);
+  k_attn_merge<TP><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(batch, Lq, heads, dh, o_run, lse_run,
+                                                                               o_part, lse_part, first, out);
+  return launch_status("attention_merge");
+}
+template wd_status attn_merge<bf16>(int, int, int, int, float*, float*, const bf16*, const float*, int, bf16*,
+                                    cudaStream_t);
+template wd_status attn_merge<float>(int, int, int, int, float*, float*, const float*, const float*, int, float*,
+                                     cudaStream_t);
+
 // ============================================================ e4m3 row quantisation
 // One warp per row: amax over the row, scale = amax / 448 (IEEE division), then
 // q = e4m3(x / scale) with round-to-nearest-even and saturation at +-448 (the

@@ -644,4 +644,46 @@ wd_status wd_attention(int dtype, int batch, int Lq, int heads, int dh, const vo
   return WD_ERR_DTYPE;
 }
 
+// One key segment with the rows' log-sum-exps, and the merge of two such results.
+wd_status wd_attention_lse(int dtype, int batch, int Lq, int heads, int dh, const void* q, const void* k, const void* v,
+                           int n, int kv_shared, void* o, float* lse, wd_stream stream) {
+  WD_NEED(q); WD_NEED(k); WD_NEED(v); WD_NEED(o); WD_NEED(lse);
+  if (batch <= 0 || Lq <= 0 || heads <= 0 || n <= 0) { set_error("attention sizes"); return WD_ERR_SHAPE; }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t D = static_cast<int64_t>(heads) * dh;
+  auto fill = [&](auto a) {
+    a.q_rs = D; a.kv1_rs = D; a.kv1_bs = kv_shared ? 0 : n * D; a.n1 = n;
+    a.o_rs = D; a.batch = batch; a.Lq = Lq; a.heads = heads; a.dh = dh; a.lse = lse;
+    return a;
+  };
+  if (dtype == WD_BF16) {
+    AttnArgs<bf16, bf16> a{};
+    a.q = static_cast<const bf16*>(q); a.k1 = static_cast<const bf16*>(k); a.v1 = static_cast<const bf16*>(v);
+    a.o = static_cast<bf16*>(o);
+    return attention(fill(a), st);
+  }
+  if (dtype == WD_F32) {
+    AttnArgs<float, float> a{};
+    a.q = static_cast<const float*>(q); a.k1 = static_cast<const float*>(k); a.v1 = static_cast<const float*>(v);
+    a.o = static_cast<float*>(o);
+    return attention(fill(a), st);
+  }
+  set_error("wd_attention_lse: dtype %d (WD_BF16 or WD_F32)", dtype);
+  return WD_ERR_DTYPE;
+}
+
+wd_status wd_attention_merge(int dtype, int batch, int Lq, int heads, int dh, float* o_run, float* lse_run,
+                             const void* o_part, const float* lse_part, int first, void* out, wd_stream stream) {
+  WD_NEED(o_run); WD_NEED(lse_run); WD_NEED(o_part); WD_NEED(lse_part); WD_OPT(out);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == WD_BF16)
+    return attn_merge<bf16>(batch, Lq, heads, dh, o_run, lse_run, static_cast<const bf16*>(o_part), lse_part, first,
+                            static_cast<bf16*>(out), st);
+  if (dtype == WD_F32)
+    return attn_merge<float>(batch, Lq, heads, dh, o_run, lse_run, static_cast<const float*>(o_part), lse_part, first,
+                             static_cast<float*>(out), st);
+  set_error("wd_attention_merge: dtype %d (WD_BF16 or WD_F32)", dtype);
+  return WD_ERR_DTYPE;
+}
+
 }  // extern "C"

@@ -131,7 +131,17 @@ struct AttnArgs {
   TO* o; int64_t o_rs;
   int batch, Lq, heads, dh;
   bool cross;                                  // counted as cross-attention in the launch trace
+  // one segment only, optional: lse[(b*heads + h)*Lq + l] = log2 sum_j 2^(q k_j^T log2(e) / sqrt(dh)),
+  // the row's log-sum-exp in log2 units (for merging attentions over parts of the keys)
+  float* lse;
 };
+// Merge of attentions over disjoint key sets (the ring level of sequence parallelism):
+// o_run, lse_run (fp32, [batch, Lq, heads*dh] and [batch, heads, Lq]) absorb the part
+// (o_part in TP, lse_part); first: the part is copied; out (TP, optional): the merged
+// output rounded to TP.
+template <typename TP>
+wd_status attn_merge(int batch, int Lq, int heads, int dh, float* o_run, float* lse_run, const TP* o_part,
+                     const float* lse_part, int first, TP* out, cudaStream_t st);
 template <typename TI, typename TO>
 wd_status attention_simt(const AttnArgs<TI, TO>& a, cudaStream_t st);
 // Tensor-core attention (dh = 128; other head sizes go to attention_simt).

@@ -200,3 +200,161 @@ class SeqParallelDiT:
         wd.wd_euler_cfg_step(xb[0], v[0], v[1], cfg_scale, dt)
         xb[1].copy_(xb[0])
         return xb
+
+
+# ------------------------------------------------------------------ 2D context parallelism: Ulysses x ring
+class CP2DBlock:
+    """One rank's part of a block under the two-level context parallelism of
+    "Wan（通义万相）..." 5.2: U ranks per Ulysses group (heads split inside the
+    group) times R groups on a ring (the sequence split across groups).
+
+    Rank r = g * U + u holds token slice r of L / (U R) tokens.  Group g's U
+    slices form chunk g (L / R tokens).  Per block:
+      1. q|k|v of the rank's slice (RoPE at the tokens' places in the grid);
+      2. all-to-all inside the group: head group u of chunk g -> [B, L/R, 3D/U];
+      3. the ring: the R ranks with the same u pass their chunks' keys and
+         values around; at step s a rank attends its queries (chunk g) to the
+         keys of chunk g - s and merges the result by log-sum-exp;
+      4. all-to-all back inside the group: the slice's output with every head;
+      5. the rest of the block on the slice.
+    With R = 1 it is the Ulysses block; with U = 1 a pure ring.
+
+    ops: qkv / post as for UlyssesBlock, plus
+      ops.attention_lse(q, k, v, heads) -> (o [B, m, heads*dh], lse [B, heads, m])
+      ops.merge(o_run, lse_run, o_part, lse_part, first, out)   (in place)
+      ops.merge_state(q, heads) -> (o_run fp32, lse_run fp32) buffers"""
+
+    def __init__(self, ops, rank: int, U: int, R: int, L: int, heads: int):
+        if heads % U:
+            raise ValueError(f"{heads} heads do not split evenly over {U} ranks")
+        self.ops, self.U, self.R = ops, U, R
+        self.g, self.u = divmod(rank, U)
+        self.tok0, self.n = token_slices(L, U * R)[rank]
+        self.heads_local = heads // U
+
+    # the Ulysses exchanges are those of UlyssesBlock, inside the group
+    def stage_qkv(self, blk: int, X_local: torch.Tensor) -> torch.Tensor:
+        return heads_send(self.ops.qkv(blk, self.tok0, self.n, X_local), self.U)
+
+    def ring_begin(self, recv_qkv: torch.Tensor):
+        """-> (q [B, m, Dg], kv [2, B, m, Dg]) of this group's chunk for this head group."""
+        qkv = heads_recv(recv_qkv)
+        Dg = qkv.shape[2] // 3
+        q = qkv[:, :, :Dg].contiguous()
+        kv = torch.stack([qkv[:, :, Dg:2 * Dg], qkv[:, :, 2 * Dg:]]).contiguous()
+        return q, kv
+
+    def ring_step(self, q: torch.Tensor, kv: torch.Tensor, state, step: int):
+        """Merge the attention of q to the keys/values kv into state (o_run,
+        lse_run, out); the last step also writes the merged output, in the
+        storage type, to out."""
+        o, lse = self.ops.attention_lse(q, kv[0], kv[1], self.heads_local)
+        if state is None:
+            state = self.ops.merge_state(q, self.heads_local) + (torch.empty_like(q),)
+        self.ops.merge(state[0], state[1], o, lse, step == 0, state[2] if step == self.R - 1 else None)
+        return state
+
+    def ring_end(self, state) -> torch.Tensor:
+        """The merged output -> the send buffer of the return all-to-all."""
+        return tokens_send(state[2], self.U)
+
+    def stage_post(self, blk: int, recv_o: torch.Tensor, X_local: torch.Tensor):
+        self.ops.post(blk, tokens_recv(recv_o), X_local)
+
+    def forward(self, blk: int, X_local: torch.Tensor, a2a, ring_pass) -> torch.Tensor:
+        """a2a(recv, send): all_to_all_single inside the Ulysses group;
+        ring_pass(kv) -> the kv of the previous rank on the ring (this rank's
+        kv goes to the next)."""
+        send = self.stage_qkv(blk, X_local)
+        recv = torch.empty_like(send)
+        a2a(recv, send)
+        q, kv = self.ring_begin(recv)
+        state = None
+        for s in range(self.R):
+            state = self.ring_step(q, kv, state, s)
+            if s + 1 < self.R:
+                kv = ring_pass(kv)
+        send = self.ring_end(state)
+        recv = torch.empty_like(send)
+        a2a(recv, send)
+        self.stage_post(blk, recv, X_local)
+        return X_local
+
+
+def cp2d_block_in_one_process(blocks, X_locals, blk: int):
+    """All U x R ranks of CP2DBlock in this process, one after the other: the
+    all-to-alls by copying inside each group, the ring by handing each group's
+    keys and values to the next group (for checking without several processes;
+    no rank waits for another)."""
+    U, R = blocks[0].U, blocks[0].R
+
+    def a2a_groups(sends):
+        out = [None] * (U * R)
+        for g in range(R):
+            grp = list(range(g * U, (g + 1) * U))
+            for j, r in enumerate(grp):
+                out[r] = torch.stack([sends[s][j] for s in grp])
+        return out
+    recv = a2a_groups([b.stage_qkv(blk, X) for b, X in zip(blocks, X_locals)])
+    qs, kvs = zip(*[b.ring_begin(rv) for b, rv in zip(blocks, recv)])
+    kvs = list(kvs)
+    states = [None] * (U * R)
+    for s in range(R):
+        states = [b.ring_step(q, kv, st, s) for b, q, kv, st in zip(blocks, qs, kvs, states)]
+        # rank g*U + u receives the kv of rank ((g - 1) mod R)*U + u
+        kvs = [kvs[((r // U - 1) % R) * U + r % U] for r in range(U * R)]
+    recv = a2a_groups([b.ring_end(st) for b, st in zip(blocks, states)])
+    for b, rv, X in zip(blocks, recv, X_locals):
+        b.stage_post(blk, rv, X)
+
+
+def cp2d_groups(U: int, R: int):
+    """The process groups of the two levels (every rank must call this, in the
+    same order): the Ulysses groups {g U .. g U + U - 1} and the ring groups
+    {u, U + u, ...}.  Returns (ulysses_groups, ring_groups)."""
+    import torch.distributed as dist
+    ul = [dist.new_group(list(range(g * U, (g + 1) * U))) for g in range(R)]
+    rg = [dist.new_group(list(range(u, U * R, U))) for u in range(U)]
+    return ul, rg
+
+
+def ring_pass_fn(rank: int, U: int, R: int):
+    """ring_pass(kv): send kv to the next rank on this rank's ring, receive the
+    previous rank's (point-to-point, both posted before either is waited on)."""
+    import torch.distributed as dist
+    g, u = divmod(rank, U)
+    nxt, prv = ((g + 1) % R) * U + u, ((g - 1) % R) * U + u
+
+    def ring_pass(kv):
+        recv = torch.empty_like(kv)
+        reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, kv, nxt), dist.P2POp(dist.irecv, recv, prv)])
+        for q in reqs:
+            q.wait()
+        return recv
+    return ring_pass
+
+
+class LibwdRingOps(LibwdOps):
+    """LibwdOps plus the ring's attention with log-sum-exp and its merge."""
+
+    def attention_lse(self, q, k, v, heads):
+        net, wd = self.net, self.wd
+        B, m, Dh = q.shape
+        o = torch.empty_like(q)
+        lse = torch.empty((B, heads, m), dtype=torch.float32, device=q.device)
+        dt = wd.WD_BF16 if q.dtype == torch.bfloat16 else wd.WD_F32
+        wd.wd_attention_lse(dt, B, m, heads, Dh // heads, q, k, v, k.shape[1], 0, o, lse)
+        return o, lse
+
+    def merge_state(self, q, heads):
+        B, m, Dh = q.shape
+        return (torch.empty((B, m, Dh), dtype=torch.float32, device=q.device),
+                torch.empty((B, heads, m), dtype=torch.float32, device=q.device))
+
+    def merge(self, o_run, lse_run, o_part, lse_part, first, out=None):
+        wd = self.wd
+        B, m, Dh = o_part.shape
+        heads = lse_part.shape[1]
+        dt = wd.WD_BF16 if o_part.dtype == torch.bfloat16 else wd.WD_F32
+        wd.wd_attention_merge(dt, B, m, heads, Dh // heads, o_run, lse_run, o_part, lse_part, first, out)
+

@@ -73,6 +73,8 @@ SIGNATURES = {
     "wd_euler_cfg_step": (_I, [_P, _P, _P, _F, _F, _S, _P]),
     "wd_gemm": (_I, [_I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P]),
     "wd_attention": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P, _I, _I, _P, _P]),
+    "wd_attention_lse": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P, _P]),
+    "wd_attention_merge": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P]),
     "wd_quant_rows_e4m3": (_I, [_I, _I, _I, _P, _P, _P, _P]),
     "wd_gemm_fp8": (_I, [_I, _I, _I, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P]),
     "wd_test_exp2": (_I, [_P, _P, _P, _P, _P, _L, _P]),
@@ -242,6 +244,16 @@ def wd_test_wait_timeout(limit_ns: int, site: int, out, stream=None):
 def wd_check_status(stream=None) -> int:
     """wd_check's status code without raising (tests of the error path)."""
     return int(_lib.wd_check(_stream(stream)))
+
+
+def wd_attention_lse(dtype, batch, Lq, heads, dh, q, k, v, n, kv_shared, o, lse, stream=None):
+    _ok(_lib.wd_attention_lse(dtype, batch, Lq, heads, dh, _p(q), _p(k), _p(v), n, int(kv_shared), _p(o), _p(lse),
+                              _stream(stream)), "wd_attention_lse")
+
+
+def wd_attention_merge(dtype, batch, Lq, heads, dh, o_run, lse_run, o_part, lse_part, first, out=None, stream=None):
+    _ok(_lib.wd_attention_merge(dtype, batch, Lq, heads, dh, _p(o_run), _p(lse_run), _p(o_part), _p(lse_part),
+                                int(first), _p(out), _stream(stream)), "wd_attention_merge")
 
 
 def wd_set_debug_flags(flags: int):

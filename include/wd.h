@@ -306,6 +306,26 @@ wd_status wd_attention(int dtype, int batch, int Lq, int heads, int dh, const vo
                        int n1, int kv1_shared, const void* k2, const void* v2, int n2, int kv2_shared, void* o,
                        wd_stream stream);
 
+/* The same attention for one key segment (k, v [batch or 1, n, heads*dh]),
+ * also writing each row's log-sum-exp lse [batch, heads, Lq] fp32,
+ * lse = log2 sum_j 2^(log2(e) q k_j^T / sqrt(dh)) (log2 units).  dtype WD_BF16
+ * or WD_F32.  With it, attentions over disjoint parts of the keys can be
+ * merged (wd_attention_merge): the ring level of the sequence parallelism of
+ * [WAN] 5.2, where each GPU holds a part of the keys and values. */
+wd_status wd_attention_lse(int dtype, int batch, int Lq, int heads, int dh, const void* q, const void* k, const void* v,
+                           int n, int kv_shared, void* o, float* lse, wd_stream stream);
+
+/* Merges one part's attention into a running result: o_run [batch, Lq,
+ * heads*dh] and lse_run [batch, heads, Lq] (fp32, updated in place) absorb
+ * o_part (dtype: WD_BF16 or WD_F32) and lse_part from wd_attention_lse over a
+ * disjoint set of keys: with M = max(lse_run, lse_part), a = 2^(lse_run - M),
+ * c = 2^(lse_part - M): o_run = (a o_run + c o_part) / (a + c), lse_run =
+ * M + log2(a + c).  first != 0: o_run and lse_run are set to the part (their
+ * old contents are not read).  out (optional, dtype, same layout as o_part)
+ * receives the merged output rounded to dtype. */
+wd_status wd_attention_merge(int dtype, int batch, int Lq, int heads, int dh, float* o_run, float* lse_run,
+                             const void* o_part, const float* lse_part, int first, void* out, wd_stream stream);
+
 /* FP8 building blocks ([WAN] 5.3: FP8 GEMM with per-token activation and
  * per-channel weight scales).  No counterpart is wired into wd_block_forward:
  * the block runs bf16; these are the next step's kernels, exposed to be

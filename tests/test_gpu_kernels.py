@@ -403,3 +403,53 @@ def test_bounded_wait_runs_out_reports_and_recovers(wd):
     assert wd.wd_check_status() == 0
     got, want, bound = _gemm_case(wd, wd.WD_BF16, 300, 192, 72, 3)
     assert_within(got, want, bound)
+
+
+# ------------------------------------------------------------------ attention over key parts: log-sum-exp and merge
+@pytest.mark.parametrize("dtype,dh,Lq,n", [("bf16", 128, 300, 1000), ("bf16", 128, 2048, 2048), ("f32", 32, 130, 200)])
+def test_attention_lse_and_merge_over_key_parts(wd, dtype, dh, Lq, n):
+    """wd_attention_lse returns each row's log-sum-exp (log2 units) of the
+    scaled scores; merging the attentions over three disjoint key parts by
+    log-sum-exp (wd_attention_merge) gives the attention over all keys.
+    Bounds: the log-sum-exp within 2e-4 (fp32 sums of 2^x, each within the
+    FMA-pipe 2^x's 7.5e-5); the merged output within the attention bound of
+    each part (its weights sum to 1) plus the rounding of the output."""
+    is_bf = dtype == "bf16"
+    dt = wd.WD_BF16 if is_bf else wd.WD_F32
+    tdt = torch.bfloat16 if is_bf else torch.float32
+    rng = np.random.default_rng(Lq + n + dh)
+    B, h = 2, 2
+    q, k, v = (rng.standard_normal((B, m, h * dh)).astype(np.float32) for m in (Lq, n, n))
+    if is_bf:
+        q, k, v = (bf(a).astype(np.float32) for a in (q, k, v))
+    qd, kd, vd = dev(q, tdt), dev(k, tdt), dev(v, tdt)
+    # exact attention and log-sum-exp per (batch, head, row)
+    qa, ka, va = (a.astype(np.float64).reshape(B, -1, h, dh) for a in (q, k, v))
+    s = np.einsum("bmhd,bnhd->bhmn", qa, ka) / np.sqrt(dh)
+    p = np.exp(s - s.max(-1, keepdims=True))
+    p /= p.sum(-1, keepdims=True)
+    want_o = np.einsum("bhmn,bnhd->bmhd", p, va).reshape(B, Lq, h * dh)
+    sm = s.max(-1, keepdims=True)
+    want_lse = (sm[..., 0] + np.log(np.exp(s - sm).sum(-1))) / np.log(2.0)
+    o = torch.empty((B, Lq, h * dh), device="cuda", dtype=tdt)
+    lse = torch.empty((B, h, Lq), device="cuda")
+    wd.wd_attention_lse(dt, B, Lq, h, dh, qd, kd, vd, n, 0, o, lse)
+    wd.wd_check()
+    assert np.abs(host(lse) - want_lse).max() <= 2e-4
+    # three parts of the keys, merged in turn
+    o_run = torch.empty((B, Lq, h * dh), device="cuda")
+    lse_run = torch.empty((B, h, Lq), device="cuda")
+    out = torch.empty((B, Lq, h * dh), device="cuda", dtype=tdt)
+    cuts = [0, n // 5, (3 * n) // 4, n]
+    for j in range(3):
+        a, b_ = cuts[j], cuts[j + 1]
+        op = torch.empty((B, Lq, h * dh), device="cuda", dtype=tdt)
+        lp = torch.empty((B, h, Lq), device="cuda")
+        wd.wd_attention_lse(dt, B, Lq, h, dh, qd, kd[:, a:b_].contiguous(), vd[:, a:b_].contiguous(), b_ - a, 0, op, lp)
+        wd.wd_attention_merge(dt, B, Lq, h, dh, o_run, lse_run, op, lp, j == 0, out if j == 2 else None)
+    wd.wd_check()
+    assert np.abs(host(lse_run) - want_lse).max() <= 3e-4
+    u_out = BF16_HALF_ULP if is_bf else 2 * U32
+    vbar = np.einsum("bhmn,bnhd->bmhd", p, np.abs(va)).reshape(B, Lq, h * dh)
+    bound = 2 * u_out * np.abs(want_o) + (4 * BF16_HALF_ULP if is_bf else 1e-5) * vbar + 1e-6
+    assert_within(host(out), want_o, bound)

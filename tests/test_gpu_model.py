@@ -470,3 +470,38 @@ def test_tiny_fp32_diffusion_cache_sampler(mods):
                                                 wl.cfg_scale, 0.5, 0.6, 2)
     assert dec == want_dec == [(True, True), (True, True), (False, False), (False, True)]
     assert rel(host(xb[0]), want_x) < TOL_F32
+
+
+@pytest.mark.parametrize("U,R", [(2, 1), (1, 2), (2, 2), (1, 4)])
+def test_cp2d_ranks_emulated_on_one_gpu(mods, U, R):
+    """The two-level context parallelism of "Wan（通义万相）..." 5.2 (Ulysses
+    inside groups of U ranks x a ring over R groups), U x R ranks run one
+    after the other on this GPU through seq_parallel's orchestration and
+    libwd's split, log-sum-exp and merge entry points (480p/81, batch 2).
+    R = 1 is the Ulysses block: bit for bit the fused block.  With a ring the
+    attention is merged from R partial outputs, each rounded to bf16 before the
+    fp32 merge: the block's contribution stays within the bf16 bar of the
+    fused block's (measured and printed)."""
+    model, wd = mods
+    from flow_matching_video_b200 import seq_parallel as SP
+    wl = synth.STACK_480P81
+    net, w, x, txt, y, d = setup(mods, wl, blocks=[0])
+    B = wl.batch
+    rng = np.random.default_rng(5)
+    X0 = dev(rng.standard_normal((B, d.L, d.D)) * 0.5)
+    net.e0.copy_(dev(O.time_mod(w, 400.0, d.D)[1]))
+    net.X.copy_(X0)
+    wd.wd_block_forward(net.cd, net.block_w[0], net.e0, net.kv[0], B, net.X, net.ws)
+    want = net.X.clone()
+    ops = SP.LibwdRingOps(net)
+    blocks = [SP.CP2DBlock(ops, r, U, R, d.L, d.heads) for r in range(U * R)]
+    X_locals = [X0[:, b.tok0:b.tok0 + b.n].contiguous() for b in blocks]
+    SP.cp2d_block_in_one_process(blocks, X_locals, 0)
+    wd.wd_check()
+    got = torch.cat(X_locals, dim=1)
+    if R == 1:
+        assert torch.equal(got, want)
+    else:
+        e = rel(host(got - X0), host(want - X0))
+        print(f"\n[cp2d U={U} R={R}] contribution vs the fused block: {e:.3e}")
+        assert e < TOL_BF16

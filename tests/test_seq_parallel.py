@@ -140,3 +140,99 @@ def test_ulysses_gloo_ranks_equal_the_whole_block(world):
         assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
         got = np.concatenate([out[r] for r in range(world)], axis=1)
     np.testing.assert_allclose(got, want, atol=1e-10, rtol=0)
+
+
+# ------------------------------------------------------------------ 2D context parallelism (Ulysses x ring)
+class OracleRingOps(OracleOps):
+    """The oracle's pieces plus attention with the rows' log-sum-exp and the merge."""
+
+    def attention_lse(self, q, k, v, heads):
+        B, m, Dh = q.shape
+        dh = Dh // heads
+        n = k.shape[1]
+        qa = q.numpy().reshape(B, m, heads, dh)
+        ka, va = k.numpy().reshape(B, n, heads, dh), v.numpy().reshape(B, n, heads, dh)
+        o = np.stack([O.attention(qa[b], ka[b], va[b]).reshape(m, Dh) for b in range(B)])
+        s = np.einsum("bmhd,bnhd->bhmn", qa, ka) / np.sqrt(dh) / np.log(2.0)   # log2 units
+        mx = s.max(axis=-1, keepdims=True)
+        lse = (mx + np.log2(np.exp2(s - mx).sum(axis=-1, keepdims=True)))[..., 0]
+        return torch.from_numpy(o), torch.from_numpy(lse)
+
+    def merge_state(self, q, heads):
+        B, m, Dh = q.shape
+        return torch.zeros((B, m, Dh), dtype=torch.float64), torch.zeros((B, heads, m), dtype=torch.float64)
+
+    def merge(self, o_run, lse_run, o_part, lse_part, first, out=None):
+        B, m, Dh = o_part.shape
+        heads = lse_part.shape[1]
+        if first:
+            o_run.copy_(o_part)
+            lse_run.copy_(lse_part)
+        else:
+            M = torch.maximum(lse_run, lse_part)
+            a, c = torch.exp2(lse_run - M), torch.exp2(lse_part - M)
+            wa = (a / (a + c)).permute(0, 2, 1).repeat_interleave(Dh // heads, dim=2)
+            wc = (c / (a + c)).permute(0, 2, 1).repeat_interleave(Dh // heads, dim=2)
+            o_run.copy_(wa * o_run + wc * o_part)
+            lse_run.copy_(M + torch.log2(a + c))
+        if out is not None:
+            out.copy_(o_run)
+
+
+@pytest.mark.parametrize("U,R", [(1, 2), (2, 2), (1, 4), (4, 1), (2, 1)])
+def test_cp2d_in_one_process_equals_the_whole_block(U, R):
+    d, w, kv, X, e0 = tiny_case()
+    want = O.block_forward(X, e0, w, 0, kv, d)
+    ops = OracleRingOps(d, w, kv, e0)
+    blocks = [SP.CP2DBlock(ops, r, U, R, d.L, d.heads) for r in range(U * R)]
+    X_locals = [torch.from_numpy(X[:, b.tok0:b.tok0 + b.n].copy()) for b in blocks]
+    SP.cp2d_block_in_one_process(blocks, X_locals, 0)
+    np.testing.assert_allclose(torch.cat(X_locals, dim=1).numpy(), want, atol=1e-10, rtol=0)
+
+
+def test_ring_merge_by_log_sum_exp_is_the_attention_over_all_keys():
+    rng = np.random.default_rng(9)
+    q = torch.from_numpy(rng.standard_normal((2, 5, 8)))
+    k, v = torch.from_numpy(rng.standard_normal((2, 12, 8))), torch.from_numpy(rng.standard_normal((2, 12, 8)))
+    ops = OracleRingOps(None, None, None, None)
+    o_all, lse_all = ops.attention_lse(q, k, v, 2)
+    st = ops.merge_state(q, 2)
+    for j, sl in enumerate([slice(0, 3), slice(3, 10), slice(10, 12)]):
+        o, lse = ops.attention_lse(q, k[:, sl].contiguous(), v[:, sl].contiguous(), 2)
+        ops.merge(st[0], st[1], o, lse, j == 0)
+    np.testing.assert_allclose(st[0].numpy(), o_all.numpy(), atol=1e-12)
+    np.testing.assert_allclose(st[1].numpy(), lse_all.numpy(), atol=1e-12)
+
+
+def _cp2d_rank(rank, U, R, port, out):
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=U * R, timeout=datetime.timedelta(seconds=60))
+    try:
+        d, w, kv, X, e0 = tiny_case()
+        ul, rg = SP.cp2d_groups(U, R)
+        blk = SP.CP2DBlock(OracleRingOps(d, w, kv, e0), rank, U, R, d.L, d.heads)
+        X_local = torch.from_numpy(X[:, blk.tok0:blk.tok0 + blk.n].copy())
+        blk.forward(0, X_local, SP.nccl_exchange(ul[blk.g]), SP.ring_pass_fn(rank, U, R))
+        out[rank] = X_local.numpy()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("U,R", [(1, 2), (2, 2)])
+def test_cp2d_gloo_ranks_equal_the_whole_block(U, R):
+    d, w, kv, X, e0 = tiny_case()
+    want = O.block_forward(X, e0, w, 0, kv, d)
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_cp2d_rank, args=(r, U, R, port, out)) for r in range(U * R)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(120)
+        assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+        got = np.concatenate([out[r] for r in range(U * R)], axis=1)
+    np.testing.assert_allclose(got, want, atol=1e-10, rtol=0)
