@@ -255,10 +255,14 @@ def run_ours(args, rank, world, local_rank):
         from flow_matching_video_b200.seq_parallel import SeqParallelDiT
         net = model.DiT(d, weights, B, dev)
         net.prepare_context(txt, clip)
-        runner = SeqParallelDiT(net, rank, world)
+        runner = SeqParallelDiT(net, rank, world, ring=args.ring)
         rows_local = B / world       # each rank carries 1/world of the tokens through the blocks
     else:
-        if args.cfg_cache is not None:   # the sampler with the CFG cache: late steps run the conditional row alone
+        if args.cfg_cache is not None and args.attn_cache is not None:   # both caches ("diffusion cache")
+            t_attn, interval = args.attn_cache
+            runner = model.DiffusionCache(d, weights, args.cfg_cache, t_attn, int(interval), dev)
+            net, attn_cache = runner.cfg.pair, runner.attn
+        elif args.cfg_cache is not None:   # the sampler with the CFG cache: late steps run the conditional row alone
             runner = model.CfgCache(d, weights, args.cfg_cache, dev)
             net = runner.pair
         elif args.attn_cache is not None:   # the sampler with the attention cache
@@ -361,18 +365,28 @@ def run_ours(args, rank, world, local_rank):
     # the whole job's algorithmic work per step: one CFG step (both rows) per video
     flops = step_flops(d, B) * (world if mode == "replicas" else 1)
     cache_note = None
-    if args.cfg_cache is not None:
-        # timed steps that ran only the conditional row do half the work of a CFG step
-        fresh = sum(1 for i in range(args.steps) if sched[(args.warmup + i) % n_sched][2] / 1000.0 > args.cfg_cache)
-        flops *= (fresh + 0.5 * (args.steps - fresh)) / args.steps
-        cache_note = {"t_cfg": args.cfg_cache, "steps_with_both_rows": fresh, "steps_conditional_only": args.steps - fresh}
-    if attn_cache is not None:
-        # a reusing step skips, per block and row, the q/k/v projection and the self-attention
-        reuse = sum(1 for f in timed_fresh if not f)
-        skipped = B * d.blocks * (2.0 * d.L * d.D * 3 * d.D + block_flops(d)["attn_self"])
-        flops -= skipped * reuse / args.steps
-        cache_note = {"t_attn": attn_cache.t_attn, "interval": attn_cache.interval,
-                      "steps_recomputing": len(timed_fresh) - reuse, "steps_reusing": reuse}
+    if args.cfg_cache is not None or attn_cache is not None:
+        # the work each timed step did: a step of the CFG cache that ran the conditional row alone
+        # does half of a CFG step; a step of the attention cache that reused the attention outputs
+        # skips, per block and row, the q/k/v projection and the self-attention
+        per_row = step_flops(d, B) / B
+        skipped_row = d.blocks * (2.0 * d.L * d.D * 3 * d.D + block_flops(d)["attn_self"])
+        work, n_both = 0.0, 0
+        for i in range(args.steps):
+            both = args.cfg_cache is None or sched[(args.warmup + i) % n_sched][2] / 1000.0 > args.cfg_cache
+            rows = B if both else 1
+            n_both += both
+            reuse = attn_cache is not None and not timed_fresh[i]
+            work += rows * (per_row - (skipped_row if reuse else 0.0))
+        flops = work / args.steps * (world if mode == "replicas" else 1)
+        cache_note = {}
+        if args.cfg_cache is not None:
+            cache_note.update(t_cfg=args.cfg_cache, steps_with_both_rows=n_both,
+                              steps_conditional_only=args.steps - n_both)
+        if attn_cache is not None:
+            reuse = sum(1 for f in timed_fresh if not f)
+            cache_note.update(t_attn=attn_cache.t_attn, interval=attn_cache.interval,
+                              steps_recomputing=len(timed_fresh) - reuse, steps_reusing=reuse)
     tflops = flops / (ms / 1e3) / 1e12
     # roofline of the dominant kernel (self-attention), timed live with events
     n_att, ms_att = tr["attn_self"]
@@ -399,7 +413,8 @@ def run_ours(args, rank, world, local_rank):
                    "tokens": d.L, "batch": B, "blocks": d.blocks, "D": d.D, "heads": d.heads, "ffn": d.ffn,
                    "parallelism": ("single GPU" if world == 1 and mode == "replicas" else
                                    {"replicas": f"replicas x{world}", "cfg-split": "CFG rows split over 2 GPUs",
-                                    "ulysses": f"Ulysses sequence parallel x{world}"}[mode]),
+                                    "ulysses": (f"Ulysses sequence parallel x{world}" if args.ring == 1 else
+                                                f"Ulysses x{world // args.ring} inside {args.ring} ring groups")}[mode]),
                    "l2": (f"no flush: per-step working set ({wbytes / 1e9:.1f} GB weights, "
                           f"{net.X.numel() * 4 / 1e9:.1f} GB residual stream) exceeds L2")},
         "tflops": tflops, "pct_bf16_peak": tflops / pk["bf16_tflops"],
@@ -415,7 +430,7 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": traffic_for("attn_self", os.path.join(ROOT, "flow_matching_video_b200", "csrc",
                                                                       "k_attn_tc.cu"))},
         "kernel_time_share": share,
-        **({("attn_cache" if attn_cache is not None else "cfg_cache"): cache_note} if cache_note else {}),
+        **({"cache": cache_note} if cache_note else {}),
         "clocks": clk,
     }
     if cpu is not None:
@@ -454,6 +469,8 @@ def main():
                     help="one video on two GPUs: rank 0 the text row, rank 1 the zeroed-text row (--gpus 2)")
     ap.add_argument("--seq-parallel", action="store_true",
                     help="one video on all GPUs: the blocks under head-sharded (Ulysses) sequence parallelism")
+    ap.add_argument("--ring", type=int, default=1, metavar="R",
+                    help="with --seq-parallel: R ring groups (Ulysses inside each group of N/R GPUs, a ring across them)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -160,20 +160,33 @@ class LibwdOps:
 
 
 class SeqParallelDiT:
-    """A whole DiT forward with the blocks under Ulysses sequence parallelism
-    on `world` GPUs (one process each).  Every rank holds the full model
-    (weights, context K/V) and the full-size buffers of `net`; the time MLP
-    and the patch embedding run on every rank (they are tiny), each rank keeps
-    its token slice of the residual stream through the blocks, and an
-    all-gather of the slices before the head gives every rank the velocity."""
+    """A whole DiT forward with the blocks under context parallelism on
+    `world` GPUs (one process each): Ulysses over all of them (ring = 1), or
+    the two-level scheme with `ring` groups of world / ring ranks.  Every rank
+    holds the full model (weights, context K/V) and the full-size buffers of
+    `net`; the time MLP and the patch embedding run on every rank (they are
+    tiny), each rank keeps its token slice of the residual stream through the
+    blocks, and an all-gather of the slices before the head gives every rank
+    the velocity.  Every rank must construct it (it creates the process groups
+    of the two levels in the same order on all ranks)."""
 
-    def __init__(self, net, rank: int, world: int, group=None, exchange=None):
+    def __init__(self, net, rank: int, world: int, group=None, exchange=None, ring: int = 1):
         import torch.distributed as dist
         self.net, self.rank, self.world, self.group = net, rank, world, group
         d = net.dims
-        self.block = UlyssesBlock(LibwdOps(net), rank, world, d.L, d.heads)
-        self.exchange = exchange or nccl_exchange(group)
         self._dist = dist
+        if world % ring:
+            raise ValueError(f"{world} ranks do not form {ring} ring groups")
+        self.ring = ring
+        if ring == 1:
+            self.block = UlyssesBlock(LibwdOps(net), rank, world, d.L, d.heads)
+            self.exchange = exchange or nccl_exchange(group)
+        else:
+            U = world // ring
+            ul, _ = cp2d_groups(U, ring)
+            self.block = CP2DBlock(LibwdRingOps(net), rank, U, ring, d.L, d.heads)
+            self.exchange = exchange or nccl_exchange(ul[self.block.g])
+            self.ring_pass = ring_pass_fn(rank, U, ring)
         B, n = net.batch, self.block.n
         self.X_local = torch.empty((B, n, d.D), dtype=torch.float32, device=net.X.device)
         self._gather = torch.empty((world, B, n, d.D), dtype=torch.float32, device=net.X.device)
@@ -185,7 +198,10 @@ class SeqParallelDiT:
         wd.wd_patch_embed(net.cd, x_t, y, net.w["pe.w"], net.w["pe.b"], net.batch, net.X, net.ws)
         self.X_local.copy_(net.X[:, blk.tok0:blk.tok0 + blk.n])
         for i in range(net.dims.blocks):
-            blk.forward(i, self.X_local, self.exchange)
+            if self.ring == 1:
+                blk.forward(i, self.X_local, self.exchange)
+            else:
+                blk.forward(i, self.X_local, self.exchange, self.ring_pass)
         self._dist.all_gather_into_tensor(self._gather, self.X_local.unsqueeze(0).contiguous(), group=self.group)
         net.X.copy_(self._gather.permute(1, 0, 2, 3).reshape(net.X.shape))
         wd.wd_unpatchify(net.cd, net.head_w, net.e, net.batch, net.X, net.v, net.ws)
