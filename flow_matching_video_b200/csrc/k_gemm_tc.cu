@@ -429,6 +429,7 @@ wd_status gemm_tc_fp8(int M, int N, int K, const uint8_t* A, int64_t lda, const 
     case EPI_GELU: return launch_tc<256, EPI_GELU, true>(ta, tb, ep, M, N, K, st);
     case EPI_F32: return launch_tc<256, EPI_F32, true>(ta, tb, ep, M, N, K, st);
     case EPI_RESID: return launch_tc<256, EPI_RESID, true>(ta, tb, ep, M, N, K, st);
+    case EPI_STORE_F16: return launch_tc<256, EPI_STORE_F16, true>(ta, tb, ep, M, N, K, st);
   }
   set_error("gemm_fp8: bad epilogue %d", mode);
   return WD_ERR_ARG;

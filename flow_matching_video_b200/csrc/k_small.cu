@@ -96,6 +96,9 @@ __global__ void __launch_bounds__(256) k_time_matvec(const float* __restrict__ W
 //   mul = gamma, add = beta                         (affine LayerNorm)
 // norm = LayerNorm (no affine) or RMSNorm.  One warp per row; each lane holds
 // NV float4 of the row in registers (D = 128 * NV), so x is read once.
+// OutT = uint8_t: the row is quantised to e4m3 as by k_quant_rows_e4m3 (scale =
+// amax / 448, codes e4m3(v / scale), IEEE division, saturating), from the fp32
+// values, and the scale written to scale[row] (the FP8 block's GEMM inputs).
 struct NormArgs {
   const float* x;
   int64_t rows;
@@ -105,6 +108,7 @@ struct NormArgs {
   int rms;
   float eps;
   void* out;
+  float* scale;                             // OutT = uint8_t: per-row e4m3 scales
 };
 
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
@@ -140,6 +144,7 @@ __global__ void __launch_bounds__(256) k_norm_mod(NormArgs a) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
   const float rstd = rsqrtf(q / a.D + a.eps);
+  float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int c = (i * 32 + lane) * 4;
@@ -157,12 +162,31 @@ __global__ void __launch_bounds__(256) k_norm_mod(NormArgs a) {
     const float o1 = (v[i].y - mean) * rstd * mul.y + add.y;
     const float o2 = (v[i].z - mean) * rstd * mul.z + add.z;
     const float o3 = (v[i].w - mean) * rstd * mul.w + add.w;
-    if constexpr (sizeof(OutT) == 2) {
+    if constexpr (std::is_same<OutT, uint8_t>::value) {   // kept for the quantisation below
+      v[i] = make_float4(o0, o1, o2, o3);
+      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(o0), fabsf(o1)), fmaxf(fabsf(o2), fabsf(o3))));
+    } else if constexpr (sizeof(OutT) == 2) {
       uint2 pk = make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
       *reinterpret_cast<uint2*>(static_cast<bf16*>(a.out) + row * a.D + c) = pk;
     } else {
       *reinterpret_cast<float4*>(static_cast<float*>(a.out) + row * a.D + c) = make_float4(o0, o1, o2, o3);
     }
+  }
+  if constexpr (std::is_same<OutT, uint8_t>::value) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float sc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = (i * 32 + lane) * 4;
+      const float e[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      uint32_t w = 0u;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        w |= static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(e[j], sc), __NV_SATFINITE, __NV_E4M3)) << (8 * j);
+      *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(a.out) + row * a.D + c) = w;
+    }
+    if (lane == 0) a.scale[row] = sc;
   }
 }
 

@@ -191,6 +191,35 @@ static wd_status self_attention_t(const wd_dims* d, int batch, int heads, const 
   return attention(a, st);
 }
 
+// The decoupled cross-attention ("图解 Wan2.1 I2V" 5.4) of n_tok queries per sample:
+// qc [batch, n_tok, D] in the cross operand type, kv the block's K/V cache, oc [batch, n_tok, D].
+template <typename T>
+static wd_status cross_attention_t(const wd_dims* d, const void* kv, int batch, int64_t n_tok, const void* qc, T* oc,
+                                   cudaStream_t st) {
+  const int D = d->D, dh = D / d->heads;
+  using CT = typename CrossT<T>::type;
+  const size_t es = sizeof(CT);
+  const char* kvp = static_cast<const char*>(kv);
+  const size_t n_img_b = up256(static_cast<size_t>(d->n_img) * D * es);
+  const size_t n_txt_b = up256(static_cast<size_t>(batch) * d->n_txt * D * es);
+  const CT* k_img = reinterpret_cast<const CT*>(kvp);
+  const CT* v_img = reinterpret_cast<const CT*>(kvp + n_img_b);
+  const CT* k_txt = reinterpret_cast<const CT*>(kvp + 2 * n_img_b);
+  const CT* v_txt = reinterpret_cast<const CT*>(kvp + 2 * n_img_b + n_txt_b);
+  AttnArgs<CT, T> a{};
+  a.q = static_cast<const CT*>(qc); a.q_rs = D;
+  a.cross = true;
+  if (d->n_img > 0) {
+    a.k1 = k_img; a.v1 = v_img; a.kv1_rs = D; a.kv1_bs = 0; a.n1 = d->n_img;
+    a.k2 = k_txt; a.v2 = v_txt; a.kv2_rs = D; a.kv2_bs = static_cast<int64_t>(d->n_txt) * D; a.n2 = d->n_txt;
+  } else {   // text-to-video: one stream, text keys only ("图解 Wan2.1 I2V" 9)
+    a.k1 = k_txt; a.v1 = v_txt; a.kv1_rs = D; a.kv1_bs = static_cast<int64_t>(d->n_txt) * D; a.n1 = d->n_txt;
+  }
+  a.o = oc; a.o_rs = D;
+  a.batch = batch; a.Lq = static_cast<int>(n_tok); a.heads = d->heads; a.dh = dh;
+  return attention(a, st);
+}
+
 template <typename T>
 static wd_status block_post_t(const wd_dims* d, const wd_block_weights* w, const float* e0, const void* kv, int batch,
                               int64_t n_tok, const T* o, float* X, const Ws& ws, cudaStream_t st) {
@@ -201,16 +230,6 @@ static wd_status block_post_t(const wd_dims* d, const wd_block_weights* w, const
   T* Bf = static_cast<T*>(ws.b);
   const int rms = d->norm == WD_NORM_RMS;
   const float* mod = w->mod;
-  // cross K/V cache parts
-  using CT = typename CrossT<T>::type;
-  const size_t es = sizeof(CT);
-  const char* kvp = static_cast<const char*>(kv);
-  const size_t n_img_b = up256(static_cast<size_t>(d->n_img) * D * es);
-  const size_t n_txt_b = up256(static_cast<size_t>(batch) * d->n_txt * D * es);
-  const CT* k_img = reinterpret_cast<const CT*>(kvp);
-  const CT* v_img = reinterpret_cast<const CT*>(kvp + n_img_b);
-  const CT* k_txt = reinterpret_cast<const CT*>(kvp + 2 * n_img_b);
-  const CT* v_txt = reinterpret_cast<const CT*>(kvp + 2 * n_img_b + n_txt_b);
 
   // 5. X += gate1 * (o Wo^T + b)
   WD_TRY(gemm<T>(M, D, D, o, D, w->o_w, D, EPI_RESID, epi(X, D, w->o_b, e0 + 2 * D, mod + 2 * D), st));
@@ -218,20 +237,7 @@ static wd_status block_post_t(const wd_dims* d, const wd_block_weights* w, const
   WD_TRY(norm_rows<T>(d, X, rows, nullptr, nullptr, nullptr, nullptr, w->cn_g, w->cn_b, 0, Bf, st));
   WD_TRY(gemm<T>(M, D, D, Bf, D, w->cq_w, D, CrossT<T>::store, epi(A, D, w->cq_b), st));
   // 8. oc = attn(qc, K_img, V_img) + attn(qc, K_txt, V_txt)
-  {
-    AttnArgs<CT, T> a{};
-    a.q = reinterpret_cast<const CT*>(A); a.q_rs = D;
-    a.cross = true;
-    if (d->n_img > 0) {
-      a.k1 = k_img; a.v1 = v_img; a.kv1_rs = D; a.kv1_bs = 0; a.n1 = d->n_img;
-      a.k2 = k_txt; a.v2 = v_txt; a.kv2_rs = D; a.kv2_bs = static_cast<int64_t>(d->n_txt) * D; a.n2 = d->n_txt;
-    } else {   // text-to-video: one stream, text keys only ("图解 Wan2.1 I2V" 9)
-      a.k1 = k_txt; a.v1 = v_txt; a.kv1_rs = D; a.kv1_bs = static_cast<int64_t>(d->n_txt) * D; a.n1 = d->n_txt;
-    }
-    a.o = Bf; a.o_rs = D;
-    a.batch = batch; a.Lq = static_cast<int>(n_tok); a.heads = d->heads; a.dh = dh;
-    WD_TRY(attention(a, st));
-  }
+  WD_TRY(cross_attention_t<T>(d, kv, batch, n_tok, A, Bf, st));
   // 9. X += oc Wco^T + b
   WD_TRY(gemm<T>(M, D, D, Bf, D, w->co_w, D, EPI_RESID, epi(X, D, w->co_b), st));
   // 10. h2 = norm(X)(1 + scale2) + shift2;  11. u = GELU(h2 W1^T + b1);  12. X += gate2 * (u W2^T + b2)
@@ -239,6 +245,90 @@ static wd_status block_post_t(const wd_dims* d, const wd_block_weights* w, const
   WD_TRY(gemm<T>(M, F, D, Bf, D, w->f1_w, D, EPI_GELU, epi(A, F, w->f1_b), st));
   WD_TRY(gemm<T>(M, D, F, A, F, w->f2_w, F, EPI_RESID, epi(X, D, w->f2_b, e0 + 5 * D, mod + 5 * D), st));
   return WD_OK;
+}
+
+// ------------------------------------------------------------------ FP8 block
+// The block of block_forward_t with its six linear layers on e4m3 operands
+// ("Wan（通义万相）..." 5.3: FP8 GEMM, per-token activation scales; here per-output-
+// channel weight scales): each GEMM input is quantised per row -- the three norms
+// quantise their fp32 output in the same kernel, the attention outputs and the FFN
+// hidden (bf16) go through the row quantiser -- and the GEMMs scale their fp32
+// accumulators by both scales before the usual epilogues.  The attentions, the
+// QK-norm + RoPE and the residual stream are those of the bf16 block.
+// Workspace: the bf16 block's, then the e4m3 activations [rows, max(D, ffn)] and
+// their row scales [rows].
+struct Ws8 {
+  Ws base;
+  uint8_t* q;
+  float* s;
+  size_t bytes;
+};
+static Ws8 ws_layout_fp8(const wd_dims* d, int batch, void* base) {
+  Ws8 w;
+  w.base = ws_layout(d, batch, base);
+  const size_t rows = static_cast<size_t>(batch) * tokens(d);
+  const size_t nq = up256(rows * static_cast<size_t>(d->ffn > d->D ? d->ffn : d->D));
+  const size_t ns = up256(rows * sizeof(float));
+  char* p = base ? static_cast<char*>(base) + w.base.bytes : nullptr;
+  w.q = reinterpret_cast<uint8_t*>(p);
+  w.s = p ? reinterpret_cast<float*>(p + nq) : nullptr;
+  w.bytes = w.base.bytes + nq + ns;
+  return w;
+}
+
+static wd_status block_forward_fp8_t(const wd_dims* d, const wd_block_weights* w, const wd_block_weights_fp8* w8,
+                                     const float* e0, const void* kv, int batch, float* X, const Ws8& ws,
+                                     cudaStream_t st) {
+  const int D = d->D, F = d->ffn, dh = D / d->heads;
+  const int64_t L = tokens(d), rows = batch * L;
+  const int M = static_cast<int>(rows);
+  bf16* A = static_cast<bf16*>(ws.base.a);
+  bf16* Bf = static_cast<bf16*>(ws.base.b);
+  uint8_t* Q = ws.q;
+  float* S = ws.s;
+  const int rms = d->norm == WD_NORM_RMS;
+  const float* mod = w->mod;
+  // e4m3 GEMM on the quantised activations Q (row scales S) and a quantised weight
+  auto g8 = [&](int N, int K, const void* wq, const float* wsc, const float* bias, int mode, void* out, int64_t ldo,
+                const float* ga, const float* gb) -> wd_status {
+    Epi ep = epi(out, ldo, bias, ga, gb);
+    ep.sa = S;
+    ep.sb = wsc;
+    return gemm_tc_fp8(M, N, K, Q, K, static_cast<const uint8_t*>(wq), K, mode, ep, st);
+  };
+  // norm (+ modulate or affine) with its output quantised into Q, S
+  auto nq = [&](const float* sh_a, const float* sh_b, const float* sc_a, const float* sc_b, const float* g,
+                const float* be, int rms_) -> wd_status {
+    NormArgs a{};
+    a.x = X; a.rows = rows; a.D = D;
+    a.sh_a = sh_a; a.sh_b = sh_b; a.sc_a = sc_a; a.sc_b = sc_b; a.gamma = g; a.beta = be;
+    a.rms = rms_; a.eps = d->eps; a.out = Q; a.scale = S;
+    return norm_mod<uint8_t>(a, st);
+  };
+  // 1. h = norm(X)(1 + scale1) + shift1, quantised;  2. q|k|v = h Wqkv^T + b
+  WD_TRY(nq(e0, mod, e0 + D, mod + D, nullptr, nullptr, rms));
+  WD_TRY(g8(3 * D, D, w8->qkv_q, w8->qkv_s, w->qkv_b, EPI_STORE, A, 3 * D, nullptr, nullptr));
+  // 3. QK-RMSNorm + 3D RoPE;  4. self-attention -> o (bf16)
+  { Trace tr(KC_SMALL, st); k_rope_table<<<64, 256, 0, st>>>(ws.base.rope, d->T, d->H / 2, d->W / 2, dh); }
+  WD_TRY(launch_status("rope_table"));
+  WD_TRY(qknorm_rope<bf16>(A, rows, *d, w->g_q, w->g_k, ws.base.rope, L, 0, st));
+  WD_TRY(self_attention_t<bf16>(d, batch, d->heads, A, Bf, st));
+  // 5. X += gate1 * (o Wo^T + b), o quantised
+  WD_TRY(quant_rows_e4m3<bf16>(M, D, Bf, Q, S, st));
+  WD_TRY(g8(D, D, w8->o_q, w8->o_s, w->o_b, EPI_RESID, X, D, e0 + 2 * D, mod + 2 * D));
+  // 6. hc = LN_affine(X), quantised;  7. qc = hc Wcq^T + b (IEEE half)
+  WD_TRY(nq(nullptr, nullptr, nullptr, nullptr, w->cn_g, w->cn_b, 0));
+  WD_TRY(g8(D, D, w8->cq_q, w8->cq_s, w->cq_b, EPI_STORE_F16, A, D, nullptr, nullptr));
+  // 8. decoupled cross-attention -> oc (bf16);  9. X += oc Wco^T + b, oc quantised
+  WD_TRY(cross_attention_t<bf16>(d, kv, batch, L, A, Bf, st));
+  WD_TRY(quant_rows_e4m3<bf16>(M, D, Bf, Q, S, st));
+  WD_TRY(g8(D, D, w8->co_q, w8->co_s, w->co_b, EPI_RESID, X, D, nullptr, nullptr));
+  // 10. h2 = norm(X)(1 + scale2) + shift2, quantised;  11. u = GELU(h2 W1^T + b1) (bf16)
+  WD_TRY(nq(e0 + 3 * D, mod + 3 * D, e0 + 4 * D, mod + 4 * D, nullptr, nullptr, rms));
+  WD_TRY(g8(F, D, w8->f1_q, w8->f1_s, w->f1_b, EPI_GELU, A, F, nullptr, nullptr));
+  // 12. X += gate2 * (u W2^T + b2), u quantised
+  WD_TRY(quant_rows_e4m3<bf16>(M, F, A, Q, S, st));
+  return g8(D, F, w8->f2_q, w8->f2_s, w->f2_b, EPI_RESID, X, D, e0 + 5 * D, mod + 5 * D);
 }
 
 template <typename T>
@@ -539,6 +629,33 @@ wd_status wd_block_post(const wd_dims* d, const wd_block_weights* w, const float
   return block_post_t<float>(d, w, e0, kv, batch, n_tok, static_cast<const float*>(o), X, L, st);
 }
 
+size_t wd_workspace_bytes_fp8(const wd_dims* d, int batch) {
+  if (check_dims(d) != WD_OK || check_batch(batch) != WD_OK) return 0;
+  return ws_layout_fp8(d, batch, nullptr).bytes;
+}
+
+wd_status wd_block_forward_fp8(const wd_dims* d, const wd_block_weights* w, const wd_block_weights_fp8* w8,
+                               const float* e0, const void* kv, int batch, float* X, void* ws, size_t ws_bytes,
+                               wd_stream stream) {
+  WD_TRY(check_dims(d));
+  WD_TRY(check_batch(batch));
+  if (d->dtype != WD_BF16) { set_error("wd_block_forward_fp8: the FP8 block is the bf16 model's"); return WD_ERR_UNSUPPORTED; }
+  if (d->D % 256 || d->ffn % 256) {
+    set_error("wd_block_forward_fp8: D=%d and ffn=%d must be multiples of 256", d->D, d->ffn);
+    return WD_ERR_SHAPE;
+  }
+  if (!w || !w8) { set_error("block weights NULL"); return WD_ERR_ARG; }
+  WD_NEED(w->qkv_b); WD_NEED(w->g_q); WD_NEED(w->g_k); WD_NEED(w->o_b); WD_NEED(w->cn_g); WD_NEED(w->cn_b);
+  WD_NEED(w->cq_b); WD_NEED(w->co_b); WD_NEED(w->f1_b); WD_NEED(w->f2_b); WD_NEED(w->mod);
+  WD_NEED(w8->qkv_q); WD_NEED(w8->o_q); WD_NEED(w8->cq_q); WD_NEED(w8->co_q); WD_NEED(w8->f1_q); WD_NEED(w8->f2_q);
+  WD_NEED(w8->qkv_s); WD_NEED(w8->o_s); WD_NEED(w8->cq_s); WD_NEED(w8->co_s); WD_NEED(w8->f1_s); WD_NEED(w8->f2_s);
+  WD_NEED(e0); WD_NEED(kv); WD_NEED(X); WD_NEED(ws);
+  const Ws8 L = ws_layout_fp8(d, batch, ws);
+  if (ws_bytes < L.bytes) { set_error("workspace %zu < %zu bytes", ws_bytes, L.bytes); return WD_ERR_WORKSPACE; }
+  if (static_cast<int64_t>(batch) * tokens(d) > 0x7fffffff) { set_error("too many rows"); return WD_ERR_SHAPE; }
+  return block_forward_fp8_t(d, w, w8, e0, kv, batch, X, L, static_cast<cudaStream_t>(stream));
+}
+
 wd_status wd_unpatchify(const wd_dims* d, const wd_head_weights* w, const float* e, int batch, const float* X, float* v,
                         void* ws, size_t ws_bytes, wd_stream stream) {
   WD_TRY(check_dims(d));
@@ -596,7 +713,10 @@ wd_status wd_gemm_fp8(int M, int N, int K, const void* Aq, const float* sa, cons
                       const float* bias, int epilogue, void* out, const float* gate_a, const float* gate_b,
                       wd_stream stream) {
   WD_NEED(Aq); WD_NEED(sa); WD_NEED(Bq); WD_NEED(sb); WD_NEED(out); WD_OPT(bias); WD_OPT(gate_a); WD_OPT(gate_b);
-  if (epilogue < 0 || epilogue > EPI_RESID) { set_error("gemm_fp8: epilogue %d (0-3)", epilogue); return WD_ERR_ARG; }
+  if (epilogue < 0 || (epilogue > EPI_RESID && epilogue != EPI_STORE_F16)) {
+    set_error("gemm_fp8: epilogue %d (0-3, 5)", epilogue);
+    return WD_ERR_ARG;
+  }
   Epi ep = epi(out, N, bias, gate_a, gate_b);
   ep.sa = sa;
   ep.sb = sb;

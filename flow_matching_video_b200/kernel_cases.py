@@ -4,8 +4,9 @@
 
 CASE is one of attn_self, attn_cross, gemm_qkv, gemm_o, gemm_ffn1, gemm_ffn2,
 euler, euler_hbm, gemm_fp8_qkv, gemm_fp8_o, gemm_fp8_ffn1, gemm_fp8_ffn2,
-quant_ffn_hidden, block_480p17 (one block, 17 frames, L = 7800, batch 1) and
-block_480p81 (one block, L = 32760, batch 2).
+quant_ffn_hidden, block_480p17 (one block, 17 frames, L = 7800, batch 1),
+block_480p81 (one block, L = 32760, batch 2) and block_480p81_fp8 (the same block
+with its six linear layers on e4m3 operands).
 Shapes are those of one block of the 30-block 480p/81-frame model (L = 32760
 tokens per sample, D = 1536, 12 heads x 128, FFN 8960, 257 image + 512 text
 keys); euler_hbm streams 2^26 elements so that every launch reads HBM.
@@ -74,12 +75,14 @@ def make_case(name: str, B: int):
         return (lambda: wd.wd_quant_rows_e4m3(wd.WD_BF16, rows, F, x, q, sc)), 3.0 * rows * F + 4.0 * rows, "B", B
     d = synth.Dims(D=D, heads=H, ffn=F, blocks=1, T=21, H=60, W=104, n_txt=NT, c_txt=4096, n_img=NI,
                    c_img=1280, dtype="bf16")
-    blocks = {"block_480p17": synth.BLOCK_480P17, "block_480p81": synth.STACK_480P81}
+    blocks = {"block_480p17": synth.BLOCK_480P17, "block_480p81": synth.STACK_480P81,
+              "block_480p81_fp8": synth.STACK_480P81}
     if name in blocks:   # one DiT block (wd_block_forward) at the workload's batch; FLOPs as in the bench
         wl = blocks[name]
+        fp8 = name.endswith("_fp8")   # the block with its linear layers on e4m3 operands
         dd = synth.Dims(**{**wl.dims.__dict__, "blocks": 1})
         net = model.DiT(dd, model.random_weights_on_device(synth.Workload(wl.name, dd, wl.batch, wl.seed), "cuda"),
-                        wl.batch)
+                        wl.batch, fp8=fp8)
         x = synth.inputs(wl)
         txt = torch.from_numpy(np.stack([x["txt"], 0 * x["txt"]][:wl.batch])).to("cuda", torch.bfloat16)
         net.prepare_context(txt, torch.from_numpy(x["clip"]).to("cuda", torch.bfloat16))
@@ -87,6 +90,9 @@ def make_case(name: str, B: int):
         net.e0.normal_(std=0.1)
         Lb, Db, Fb = dd.L, dd.D, dd.ffn
         flops = wl.batch * (2.0 * Lb * Db * (6 * Db + 2 * Fb) + 4.0 * Lb * Lb * Db + 4.0 * Lb * (dd.n_img + dd.n_txt) * Db)
+        if fp8:
+            return (lambda: wd.wd_block_forward_fp8(net.cd, net.block_w[0], net.block_w8[0], net.e0, net.kv[0],
+                                                    wl.batch, net.X, net.ws)), flops, "FLOP", wl.batch
         return (lambda: wd.wd_block_forward(net.cd, net.block_w[0], net.e0, net.kv[0], wl.batch, net.X, net.ws)), \
             flops, "FLOP", wl.batch
     if name in ("euler", "euler_hbm"):

@@ -69,10 +69,14 @@ def random_weights_on_device(wl: synth.Workload, device) -> dict:
 class DiT:
     """The DiT of one workload on one device, with its buffers for `batch` rows."""
 
-    def __init__(self, dims: synth.Dims, weights: dict, batch: int, device="cuda", buffers_from: "DiT" = None):
+    def __init__(self, dims: synth.Dims, weights: dict, batch: int, device="cuda", buffers_from: "DiT" = None,
+                 fp8: bool = False):
         """buffers_from: another DiT of the same dims and batch whose workspace,
         residual stream and output buffers this one shares (the experts of a
-        timestep MoE run one at a time); the context and K/V cache stay per model."""
+        timestep MoE run one at a time); the context and K/V cache stay per model.
+        fp8: the blocks run wd_block_forward_fp8 ("Wan（通义万相）..." 5.3), with the six
+        matrices of every block quantised once here by the library's row
+        quantiser (per output channel)."""
         self.dims = dims
         self.cd = wd.make_dims(dims)
         self.batch = batch
@@ -91,6 +95,19 @@ class DiT:
         self.block_w = [wd.wd_block_weights(*(p(f"blk{i}." + names[f]) for f in wd.BLOCK_FIELDS))
                         for i in range(dims.blocks)]
         self.head_w = wd.wd_head_weights(p("head.mod"), p("head.w"), p("head.b"))
+        self.fp8 = fp8
+        self.q8, self.block_w8 = {}, []
+        if fp8:
+            for i in range(dims.blocks):
+                ptrs = {}
+                for nm in ("qkv", "o", "cq", "co", "f1", "f2"):
+                    wt = self.w[f"blk{i}.{nm}.w"]
+                    q = torch.empty(wt.shape, dtype=torch.uint8, device=wt.device)
+                    sc = torch.empty(wt.shape[0], dtype=torch.float32, device=wt.device)
+                    wd.wd_quant_rows_e4m3(wd.WD_BF16, wt.shape[0], wt.shape[1], wt, q, sc)
+                    self.q8[(i, nm)] = (q, sc)
+                    ptrs[nm + "_q"], ptrs[nm + "_s"] = q.data_ptr(), sc.data_ptr()
+                self.block_w8.append(wd.wd_block_weights_fp8(*(ptrs[f] for f in wd.FP8_FIELDS)))
         L, D = dims.L, dims.D
         dev = self.device
         self.ctx = torch.empty(wd.wd_ctx_bytes(self.cd, batch), dtype=torch.uint8, device=dev)
@@ -101,7 +118,8 @@ class DiT:
             src = buffers_from
             self.ws, self.X, self.e, self.e0, self.v = src.ws, src.X, src.e, src.e0, src.v
             return
-        self.ws = torch.empty(wd.wd_workspace_bytes(self.cd, batch), dtype=torch.uint8, device=dev)
+        ws_bytes = wd.wd_workspace_bytes_fp8(self.cd, batch) if fp8 else wd.wd_workspace_bytes(self.cd, batch)
+        self.ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
         self.X = torch.empty((batch, L, D), dtype=torch.float32, device=dev)
         self.e = torch.empty(D, dtype=torch.float32, device=dev)
         self.e0 = torch.empty((6, D), dtype=torch.float32, device=dev)
@@ -127,7 +145,11 @@ class DiT:
         wd.wd_time_mod(self.cd, self.time_w, tau, self.e, self.e0, stream)
         wd.wd_patch_embed(self.cd, x_t, y, self.w["pe.w"], self.w["pe.b"], self.batch, self.X, self.ws, stream)
         for i in range(self.dims.blocks):
-            wd.wd_block_forward(self.cd, self.block_w[i], self.e0, self.kv[i], self.batch, self.X, self.ws, stream)
+            if self.fp8:
+                wd.wd_block_forward_fp8(self.cd, self.block_w[i], self.block_w8[i], self.e0, self.kv[i], self.batch,
+                                        self.X, self.ws, stream)
+            else:
+                wd.wd_block_forward(self.cd, self.block_w[i], self.e0, self.kv[i], self.batch, self.X, self.ws, stream)
         wd.wd_unpatchify(self.cd, self.head_w, self.e, self.batch, self.X, self.v, self.ws, stream)
         return self.v
 

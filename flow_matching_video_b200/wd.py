@@ -47,6 +47,8 @@ BLOCK_FIELDS = ["qkv_w", "qkv_b", "g_q", "g_k", "o_w", "o_b", "cn_g", "cn_b", "c
                 "f2_w", "f2_b", "mod"]
 wd_block_weights = _ptr_struct("wd_block_weights", BLOCK_FIELDS)
 wd_head_weights = _ptr_struct("wd_head_weights", ["mod", "w", "b"])
+FP8_FIELDS = ["qkv_q", "o_q", "cq_q", "co_q", "f1_q", "f2_q", "qkv_s", "o_s", "cq_s", "co_s", "f1_s", "f2_s"]
+wd_block_weights_fp8 = _ptr_struct("wd_block_weights_fp8", FP8_FIELDS)
 
 # exported symbol -> (restype, argtypes)
 _P, _I, _F, _S, _L = C.c_void_p, C.c_int, C.c_float, C.c_size_t, C.c_int64
@@ -69,6 +71,9 @@ SIGNATURES = {
     "wd_block_qkv": (_I, [_PD, C.POINTER(wd_block_weights), _P, _I, _L, _L, _P, _P, _P, _S, _P]),
     "wd_block_self_attention": (_I, [_PD, _I, _I, _P, _P, _P]),
     "wd_block_post": (_I, [_PD, C.POINTER(wd_block_weights), _P, _P, _I, _L, _P, _P, _P, _S, _P]),
+    "wd_workspace_bytes_fp8": (_S, [_PD, _I]),
+    "wd_block_forward_fp8": (_I, [_PD, C.POINTER(wd_block_weights), C.POINTER(wd_block_weights_fp8), _P, _P, _I, _P,
+                                  _P, _S, _P]),
     "wd_unpatchify": (_I, [_PD, C.POINTER(wd_head_weights), _P, _I, _P, _P, _P, _S, _P]),
     "wd_euler_cfg_step": (_I, [_P, _P, _P, _F, _F, _S, _P]),
     "wd_gemm": (_I, [_I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P]),
@@ -199,6 +204,15 @@ def wd_block_self_attention(dims, batch, heads, qkv, o, stream=None):
 def wd_block_post(dims, w: wd_block_weights, e0, kv, batch, n_tok, o, X, ws, stream=None):
     _ok(_lib.wd_block_post(C.byref(dims), C.byref(w), _p(e0), _p(kv), batch, n_tok, _p(o), _p(X), _p(ws),
                            ws.numel() * ws.element_size(), _stream(stream)), "wd_block_post")
+
+
+def wd_workspace_bytes_fp8(dims: wd_dims, batch: int) -> int:
+    return _lib.wd_workspace_bytes_fp8(C.byref(dims), batch)
+
+
+def wd_block_forward_fp8(dims, w: wd_block_weights, w8: wd_block_weights_fp8, e0, kv, batch, X, ws, stream=None):
+    _ok(_lib.wd_block_forward_fp8(C.byref(dims), C.byref(w), C.byref(w8), _p(e0), _p(kv), batch, _p(X), _p(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream)), "wd_block_forward_fp8")
 
 
 def wd_unpatchify(dims, w: wd_head_weights, e, batch, X, v, ws, stream=None):

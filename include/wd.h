@@ -113,6 +113,16 @@ typedef struct {
   const float *mod;
 } wd_block_weights;
 
+/* The six linear layers of one block quantised for the FP8 block
+ * (wd_block_forward_fp8): e4m3 matrices [out, in] (one byte per element) and
+ * their per-output-channel scales [out] fp32 from wd_quant_rows_e4m3, so that
+ * W ~ scale[row] * q.  The biases, gains and modulation stay in
+ * wd_block_weights. */
+typedef struct {
+  const void *qkv_q, *o_q, *cq_q, *co_q, *f1_q, *f2_q;
+  const float *qkv_s, *o_s, *cq_s, *co_s, *f1_s, *f2_s;
+} wd_block_weights_fp8;
+
 /* Head ([I2V] 5.5): mod [2,D] (shift, scale biases added to e), w [64,D]
  * in dtype, b [64] fp32.  Output feature c*4 + kh*2 + kw. */
 typedef struct {
@@ -232,6 +242,21 @@ wd_status wd_block_self_attention(const wd_dims* d, int batch, int heads, const 
 wd_status wd_block_post(const wd_dims* d, const wd_block_weights* w, const float* e0, const void* kv, int batch,
                         int64_t n_tok, const void* o, float* X, void* ws, size_t ws_bytes, wd_stream stream);
 
+/* The block of wd_block_forward with its six linear layers on e4m3
+ * operands ([WAN] 5.3: FP8 GEMM with per-token activation scales; here with
+ * per-output-channel weight scales, w8).  Each GEMM input is quantised per
+ * token row (scale = row amax / 448, codes rounded to nearest-even with
+ * saturation, as wd_quant_rows_e4m3): the outputs of the three norms are
+ * quantised from fp32 in the norm kernel, the attention outputs and the FFN
+ * hidden (bf16) by the row quantiser.  The self- and cross-attention, QK-norm
+ * + RoPE and the fp32 residual stream are those of the bf16 block.  WD_BF16
+ * models with D and ffn multiples of 256 only (else WD_ERR_UNSUPPORTED /
+ * WD_ERR_SHAPE).  ws: wd_workspace_bytes_fp8(d, batch) bytes. */
+size_t wd_workspace_bytes_fp8(const wd_dims* d, int batch);
+wd_status wd_block_forward_fp8(const wd_dims* d, const wd_block_weights* w, const wd_block_weights_fp8* w8,
+                               const float* e0, const void* kv, int batch, float* X, void* ws, size_t ws_bytes,
+                               wd_stream stream);
+
 /* Head and unpatchify ([I2V] 5.5): z = LN(X)(1 + e + mod[1]) + e + mod[0],
  * p = z w^T + b, v[b,c,f,2y+kh,2x+kw] = p[b, l, c*4+kh*2+kw].
  * X [batch,L,D] fp32, e [D] fp32 -> v [batch,16,T,H,W] fp32. */
@@ -344,7 +369,7 @@ wd_status wd_quant_rows_e4m3(int dtype, int rows, int K, const void* x, void* q,
  * the epilogues of wd_gemm: 0 out bf16 = v, 1 out bf16 = GELU(v), 2 out fp32
  * = v, 3 out fp32 += (gate_a + gate_b) * v.  Aq [M,K] and Bq [N,K] e4m3 from
  * wd_quant_rows_e4m3, sa [M], sb [N] their scales; N a multiple of 256, K a
- * multiple of 16; out [M,N]. */
+ * multiple of 16; out [M,N].  Epilogue 5 (out IEEE half = v) as for wd_gemm. */
 wd_status wd_gemm_fp8(int M, int N, int K, const void* Aq, const float* sa, const void* Bq, const float* sb,
                       const float* bias, int epilogue, void* out, const float* gate_a, const float* gate_b,
                       wd_stream stream);

@@ -318,7 +318,22 @@ def _mod(e0, w: dict, blk: int):
     return np.asarray(e0, F64) + np.asarray(w[f"blk{blk}.mod"], F64)
 
 
-def block_qkv(x, e0, w: dict, blk: int, dims, tok, rnd: bool = False, want=("q", "k", "v")):
+def linear_fp8(x, w, b=None):
+    """A Linear layer as the FP8 GEMM of [WAN] 5.3: x quantised per row (token),
+    W [out, in] per output channel (quant_rows_e4m3), the product of the codes
+    exact, both scales applied, then the bias."""
+    qx, sx = quant_rows_e4m3(x)
+    qw, sw = quant_rows_e4m3(w)
+    return gemm_fp8(qx, sx, qw, sw, b)
+
+
+def _lin(x, w, b, rnd: bool, fp8: bool):
+    """The block's Linear layers: on e4m3 operands (fp8), else on operands stored
+    as the GPU stores them (rnd) or exact."""
+    return linear_fp8(x, w, b) if fp8 else linear(_st(x, rnd), w, b)
+
+
+def block_qkv(x, e0, w: dict, blk: int, dims, tok, rnd: bool = False, want=("q", "k", "v"), fp8: bool = False):
     """The projections of the self-attention for some tokens of one sample
     ([I2V] 5.2, 5.3 (1) and (2)): x [n, D] are the residual-stream rows of the
     tokens whose sequence indices are `tok` [n];
@@ -328,20 +343,21 @@ def block_qkv(x, e0, w: dict, blk: int, dims, tok, rnd: bool = False, want=("q",
     token's (frame, row, column) in the grid; v split into heads.
     Returns {name: [n, heads, dh]} for the names in `want`.
     Reading: QK-RMSNorm over D before the head split (the page's
-    RMSNorm(Linear_q(x)))."""
+    RMSNorm(Linear_q(x))).  fp8: the projection as an FP8 GEMM whose input h is
+    quantised from its fp32 value (not from a bf16 copy)."""
     p = f"blk{blk}."
     D, nh, dh, eps = dims.D, dims.heads, dims.dh, dims.eps
     shift1, scale1 = _mod(e0, w, blk)[:2]
     tok = np.asarray(tok)
     n = len(tok)
     pf, py, px = (a[tok] for a in grid_positions(dims.T, dims.Hp, dims.Wp))
-    h = _st(adaln_modulate(x, shift1, scale1, eps, dims.norm), rnd)
+    h = adaln_modulate(x, shift1, scale1, eps, dims.norm)
     wqkv, bqkv = w[p + "qkv.w"], w[p + "qkv.b"]
     out = {}
     for j, name in enumerate(("q", "k", "v")):
         if name not in want:
             continue
-        a = _st(linear(h, wqkv[j * D:(j + 1) * D], bqkv[j * D:(j + 1) * D]), rnd)
+        a = _st(_lin(h, wqkv[j * D:(j + 1) * D], bqkv[j * D:(j + 1) * D], rnd, fp8), rnd)
         if name == "v":
             out[name] = a.reshape(n, nh, dh)
         else:
@@ -350,7 +366,7 @@ def block_qkv(x, e0, w: dict, blk: int, dims, tok, rnd: bool = False, want=("q",
     return out
 
 
-def block_self_attention(X, e0, w: dict, blk: int, dims, rnd: bool = False, rows=None):
+def block_self_attention(X, e0, w: dict, blk: int, dims, rnd: bool = False, rows=None, fp8: bool = False):
     """The attention output o of a block's self-attention for the token rows
     `rows` of every sample (default all): o = softmax(q k^T / sqrt(dh)) v per
     head over all L keys, heads concatenated -> [B, len(rows), D], the input of
@@ -361,13 +377,13 @@ def block_self_attention(X, e0, w: dict, blk: int, dims, rnd: bool = False, rows
     rows = np.arange(L) if rows is None else np.asarray(rows)
     o = np.empty((B, len(rows), D))
     for b in range(B):
-        kv = block_qkv(X[b], e0, w, blk, dims, np.arange(L), rnd, want=("k", "v"))
-        q = block_qkv(X[b][rows], e0, w, blk, dims, rows, rnd, want=("q",))["q"]
+        kv = block_qkv(X[b], e0, w, blk, dims, np.arange(L), rnd, want=("k", "v"), fp8=fp8)
+        q = block_qkv(X[b][rows], e0, w, blk, dims, rows, rnd, want=("q",), fp8=fp8)["q"]
         o[b] = _st(attention(q, kv["k"], kv["v"]).reshape(len(rows), D), rnd)
     return o
 
 
-def block_after_attention(Xr, o, e0, w: dict, blk: int, kv: dict, dims, rnd: bool = False):
+def block_after_attention(Xr, o, e0, w: dict, blk: int, kv: dict, dims, rnd: bool = False, fp8: bool = False):
     """The rest of the block for some token rows, given their self-attention
     output o [B, n, D] and their residual-stream rows Xr [B, n, D]
     ([I2V] 5.2-5.5):
@@ -375,7 +391,9 @@ def block_after_attention(Xr, o, e0, w: dict, blk: int, kv: dict, dims, rnd: boo
     X  += Linear_co(attn(qc, K_img, V_img) + attn(qc, K_txt, V_txt)),
           qc = Linear_cq(LN_affine(X))                (no adaLN, no gate)
     X  += gate2 * Linear_2(GELU(Linear_1(norm(X)(1+scale2)+shift2)))
-    Reading: the cross-attention input gets a LayerNorm with affine gains."""
+    Reading: the cross-attention input gets a LayerNorm with affine gains.
+    fp8: the four Linear layers as FP8 GEMMs; the norms' outputs are quantised
+    from their fp32 values, o, oc and the FFN hidden after their bf16 store."""
     p = f"blk{blk}."
     D, nh, dh, eps = dims.D, dims.heads, dims.dh, dims.eps
     Xr = np.asarray(Xr, F64)
@@ -383,10 +401,10 @@ def block_after_attention(Xr, o, e0, w: dict, blk: int, kv: dict, dims, rnd: boo
     shift1, scale1, gate1, shift2, scale2, gate2 = _mod(e0, w, blk)
     out = np.empty((B, n, D))
     for b in range(B):
-        xr = Xr[b] + gate1 * linear(o[b], w[p + "o.w"], w[p + "o.b"])
+        xr = Xr[b] + gate1 * _lin(o[b], w[p + "o.w"], w[p + "o.b"], rnd, fp8)
         # ---- decoupled cross-attention (not modulated, not gated)
-        hc = _st(layer_norm(xr, eps, w[p + "cn.g"], w[p + "cn.b"]), rnd)
-        qc = _st16(linear(hc, w[p + "cq.w"], w[p + "cq.b"]), rnd).reshape(n, nh, dh)
+        hc = layer_norm(xr, eps, w[p + "cn.g"], w[p + "cn.b"])
+        qc = _st16(_lin(hc, w[p + "cq.w"], w[p + "cq.b"], rnd, fp8), rnd).reshape(n, nh, dh)
         kt, vt = kv["k_txt"][b], kv["v_txt"][b]
         o_txt = attention(qc, kt.reshape(-1, nh, dh), vt.reshape(-1, nh, dh))
         if "k_img" in kv:
@@ -395,15 +413,15 @@ def block_after_attention(Xr, o, e0, w: dict, blk: int, kv: dict, dims, rnd: boo
             oc = _st((o_img + o_txt).reshape(n, D), rnd)
         else:   # text-to-video: single-stream cross-attention ([I2V] 9)
             oc = _st(o_txt.reshape(n, D), rnd)
-        xr = xr + linear(oc, w[p + "co.w"], w[p + "co.b"])
+        xr = xr + _lin(oc, w[p + "co.w"], w[p + "co.b"], rnd, fp8)
         # ---- gated FFN
-        h2 = _st(adaln_modulate(xr, shift2, scale2, eps, dims.norm), rnd)
-        u = _st(gelu(linear(h2, w[p + "f1.w"], w[p + "f1.b"])), rnd)
-        out[b] = xr + gate2 * linear(u, w[p + "f2.w"], w[p + "f2.b"])
+        h2 = adaln_modulate(xr, shift2, scale2, eps, dims.norm)
+        u = _st(gelu(_lin(h2, w[p + "f1.w"], w[p + "f1.b"], rnd, fp8)), rnd)
+        out[b] = xr + gate2 * _lin(u, w[p + "f2.w"], w[p + "f2.b"], rnd, fp8)
     return out
 
 
-def block_forward(X, e0, w: dict, blk: int, kv: dict, dims, rnd: bool = False, rows=None):
+def block_forward(X, e0, w: dict, blk: int, kv: dict, dims, rnd: bool = False, rows=None, fp8: bool = False):
     """One DiT block ([I2V] 5.2-5.5), order self-attention -> cross -> FFN:
     block_self_attention, then block_after_attention.
 
@@ -411,11 +429,12 @@ def block_forward(X, e0, w: dict, blk: int, kv: dict, dims, rnd: bool = False, r
     [B, n_txt, D], k_img/v_img [n_img, D]).  ``rows`` (optional index array)
     computes the output only for those token rows of every sample; keys and
     values still cover all L tokens, so the result is exact for those rows.
+    fp8: the six Linear layers as FP8 GEMMs ([WAN] 5.3), as the GPU's FP8 block.
     """
     X = np.asarray(X, F64)
     rows = np.arange(X.shape[1]) if rows is None else np.asarray(rows)
-    o = block_self_attention(X, e0, w, blk, dims, rnd, rows)
-    return block_after_attention(X[:, rows], o, e0, w, blk, kv, dims, rnd)
+    o = block_self_attention(X, e0, w, blk, dims, rnd, rows, fp8)
+    return block_after_attention(X[:, rows], o, e0, w, blk, kv, dims, rnd, fp8)
 
 
 # ---------------------------------------------------------------- head
@@ -431,7 +450,7 @@ def head_unpatchify(X, e, w: dict, dims, rnd: bool = False):
 
 
 # ---------------------------------------------------------------- whole DiT
-def dit_forward(x_t, y, tau: float, w: dict, kvs: list, dims, rnd: bool = False, attn=None):
+def dit_forward(x_t, y, tau: float, w: dict, kvs: list, dims, rnd: bool = False, attn=None, fp8: bool = False):
     """v = DiT(concat(x_t, y), tau, context) for a batch ([I2V] 5, 7).
     attn (optional, the attention cache of [WAN] 5.3): a dict with "o", a
     list holding per block the self-attention output o [B, L, D] last
@@ -442,7 +461,7 @@ def dit_forward(x_t, y, tau: float, w: dict, kvs: list, dims, rnd: bool = False,
     X = patch_embed(x_t, y, w["pe.w"], w["pe.b"], rnd)
     for i in range(dims.blocks):
         if attn is None:
-            X = block_forward(X, e0, w, i, kvs[i], dims, rnd)
+            X = block_forward(X, e0, w, i, kvs[i], dims, rnd, fp8=fp8)
             continue
         if not attn["reuse"]:
             attn["o"][i] = block_self_attention(X, e0, w, i, dims, rnd)

@@ -399,3 +399,39 @@ def test_diffusion_cache_reduces_to_each_cache_alone():
     both, dec = O.sample_diffusion_cache(*args, 0.5, 0.6, 2)
     assert dec == [(True, True), (True, True), (False, False), (False, True)]
     assert np.abs(both - cfg_only).max() > 1e-6 and np.abs(both - attn_only).max() > 1e-6
+
+
+# ------------------------------------------------------------------ the FP8 block ("Wan（通义万相）..." 5.3)
+def _e4m3_grid_rows(rows, cols, rng):
+    """Rows whose values are e4m3 values times a power of two, each row holding
+    +-448 x its scale, so that per-row quantisation is lossless."""
+    grid = np.unique(np.abs(O.e4m3(rng.standard_normal(4000) * 50)))
+    v = rng.choice(grid, size=(rows, cols)) * rng.choice([-1.0, 1.0], size=(rows, cols))
+    v[:, 0] = 448.0
+    return v * np.exp2(rng.integers(-12, -2, size=(rows, 1)).astype(np.float64))
+
+
+def test_linear_fp8_is_exact_on_representable_operands():
+    rng = np.random.default_rng(21)
+    x, w, b = _e4m3_grid_rows(9, 48, rng), _e4m3_grid_rows(16, 48, rng), rng.standard_normal(16)
+    np.testing.assert_array_equal(O.linear_fp8(x, w, b), O.linear(x, w, b))
+    # a planted mistake that drops the weight scales is caught
+    qx, sx = O.quant_rows_e4m3(x)
+    qw, sw = O.quant_rows_e4m3(w)
+    assert np.abs(O.gemm_fp8(qx, sx, qw, np.ones_like(sw), b) - O.linear(x, w, b)).max() > 1.0
+
+
+def test_fp8_block_is_the_block_within_e4m3_precision():
+    """The FP8 block differs from the exact block by the e4m3 rounding of its
+    GEMM inputs (half a step: 2^-4 relative per element), far less than the
+    block's own contribution, and by more than float64 noise (the quantisation
+    is really applied)."""
+    d, w, txt, clip, X = _tiny(D=48, ffn=40)
+    e0 = RNG.standard_normal((6, d.D)) * 0.3
+    ctx_t, ctx_i = O.context_embed(w, txt, clip)
+    kv = O.cross_kv(w, 0, ctx_t, ctx_i)
+    exact = O.block_forward(X, e0, w, 0, kv, d)
+    f8 = O.block_forward(X, e0, w, 0, kv, d, fp8=True)
+    contrib = np.sqrt(((exact - X) ** 2).mean())
+    err = np.abs(f8 - exact).max()
+    assert 1e-6 * contrib < err < 0.25 * contrib
