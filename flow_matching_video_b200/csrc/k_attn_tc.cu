@@ -41,6 +41,10 @@ constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
 #define WD_ATTN_SELF_BK 128   // keys per block of the self-attention (128, or 64 with double-buffered S)
 #endif
 
+#ifndef WD_ATTN_P_PARTS
+#define WD_ATTN_P_PARTS 2   // releases of a block's P to its P V (one softmax warp per lane quarter): 1, 2 or 4
+#endif
+
 #ifndef WD_ATTN_ISSUERS
 #define WD_ATTN_ISSUERS 1   // MMA issuing threads of the self-attention (1, or 2: one per Q tile)
 #endif
@@ -64,6 +68,10 @@ struct Cfg {
   static constexpr int SM_WARPS = 4 * SPLIT;
   static constexpr int COLS = BKV / SPLIT;
   static_assert(COLS % 64 == 0, "each softmax warp owns a multiple of 64 key columns");
+  // P of a block is handed to its P V in PP parts (each part's k-steps start once it is in TMEM)
+  static constexpr int PP = SPLIT == 1 ? WD_ATTN_P_PARTS : 1;
+  static_assert(PP == 1 || PP == 2 || PP == 4, "P released in 1, 2 or 4 parts");
+  static constexpr int PPB = PP > 1 ? PP - 1 : 1;   // barriers for the parts before the last
   // MMA issuing threads: one for all tiles, or (two tiles of one segment) one per tile,
   // so that one issuer's waits overlap the other's MMAs
   static constexpr int ISSUERS = (NSEG == 1 && NQ == 2) ? WD_ATTN_ISSUERS : 1;
@@ -188,8 +196,8 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   uint64_t* kv_empty = kv_full + RING;     // RING
   uint64_t* s_full = kv_empty + RING;      // NBUF
   uint64_t* p_full = s_full + C::NBUF;     // NBUF: all of P written
-  uint64_t* p_half = p_full + C::NBUF;     // NBUF: the first half of the block's keys of P written
-  uint64_t* pv_done = p_half + C::NBUF;    // NBUF: P V of the block in that buffer completed (double buffering)
+  uint64_t* p_part = p_full + C::NBUF;     // NBUF x PPB: the first parts of the block's P written
+  uint64_t* pv_done = p_part + C::NBUF * C::PPB;   // NBUF: P V of the block in that buffer completed (double buffering)
   uint64_t* o_done = pv_done + C::NBUF;    // NQ
   uint64_t* tdone = o_done + NQ;           // 1
   uint64_t* mx_bar = tdone + 1;            // NQ x 4: the two warps of a lane quarter swap row maxima
@@ -213,7 +221,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     for (int i = 0; i < C::NBUF; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], C::SM_WARPS);
-      mbar_init(&p_half[i], C::SM_WARPS);
+      for (int j = 0; j < C::PPB; ++j) mbar_init(&p_part[i * C::PPB + j], C::SM_WARPS);
       mbar_init(&pv_done[i], 1);
     }
     for (int t = 0; t < NQ; ++t) mbar_init(&o_done[t], 1);
@@ -285,21 +293,18 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         const int bi = C::buf(t, n);
         const uint32_t d = tmem + C::o_col(t, sg);
         const uint32_t pa = tmem + C::s_col(t, n), vb_lo = v_lo + vslot * (C::KV_BYTES >> 4);
-        // With one softmax warp per lane quarter, P arrives in two halves of the
-        // block's keys: the first half of the k-steps starts as soon as the first
-        // half is in TMEM.
+        // P arrives in PP parts of the block's keys: the k-steps of a part start as
+        // soon as that part is in TMEM.
         constexpr int KK = BKV / 16;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          if (SPLIT == 1 || half == 0) {
-            uint64_t* bar = (SPLIT == 1 && half == 0) ? &p_half[bi] : &p_full[bi];
-            if (!MMA_WAIT(bar, C::par(n), SITE_P)) return false;
-          }
+        for (int part = 0; part < C::PP; ++part) {
+          uint64_t* bar = part < C::PP - 1 ? &p_part[bi * C::PPB + part] : &p_full[bi];
+          if (!MMA_WAIT(bar, C::par(n), SITE_P)) return false;
           // the V tile: waited for by this issuer's first tile (its other tiles read the same tile)
-          if (half == 0 && t == t_lo && !MMA_WAIT(&kv_full[vslot], (vseq / RING) & 1u, SITE_KVF)) return false;
+          if (part == 0 && t == t_lo && !MMA_WAIT(&kv_full[vslot], (vseq / RING) & 1u, SITE_KVF)) return false;
           tc_fence_after();
 #pragma unroll
-          for (int kk = half * KK / 2; kk < (half + 1) * KK / 2; ++kk) {
+          for (int kk = part * KK / C::PP; kk < (part + 1) * KK / C::PP; ++kk) {
             // A = P: 16 keys = 8 TMEM columns of packed bf16 pairs; each softmax
             // warp's keys sit over the first half of its own S columns:
             // key 16 kk lives at column (16kk / COLS) * COLS + (16kk % COLS) / 2
@@ -492,11 +497,14 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           pk[k >> 1] = C::HALF ? pack_f16x2(e0, e1) : pack_bf16x2(e0, e1);
         }
         tmem_st8(s_addr + c * 8, pk);
-        if (SPLIT == 1 && c == CH - 1) {   // the first half of the block's P is written: release its P V
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&p_half[bi]);
+        if constexpr (C::PP > 1) {   // a part of the block's P is written: release its P V
+          constexpr int per = 2 * CH / C::PP;   // 16-key chunks per part
+          if ((c + 1) % per == 0 && c + 1 < 2 * CH) {
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_part[bi * C::PPB + (c + 1) / per - 1]);
+          }
         }
       }
       tmem_wait_st();
