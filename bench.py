@@ -270,7 +270,7 @@ def run_ours(args, rank, world, local_rank):
             runner = attn_cache = model.AttnCache(d, weights, t_attn, int(interval), B, dev)
             net = runner.net
         else:
-            runner = net = model.DiT(d, weights, B, dev, fp8=args.fp8)
+            runner = net = model.DiT(d, weights, B, dev, fp8=args.fp8 is not None, fp8_ffn2=args.fp8 != "no-ffn2")
         runner.prepare_context(txt, clip)
         rows_local = B
     y = None if d.t2v else net.build_cond_y(torch.from_numpy(x["img_lat"]).to(dev))
@@ -407,7 +407,8 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak" if mode == "replicas" else "strong",
-        "vs_baseline": None, "dtype": "bf16 (e4m3 GEMMs)" if args.fp8 else "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": ({"all": "bf16 (e4m3 GEMMs)", "no-ffn2": "bf16 (e4m3 GEMMs but FFN2)"}[args.fp8]
+                                        if args.fp8 else "bf16"), "data": "synthetic",
         "config": {"workload": wl.name, "video": f"{4 * (d.T - 1) + 1} frames {8 * d.H}x{8 * d.W}",
                    "latent": [16, d.T, d.H, d.W],
                    "tokens": d.L, "batch": B, "blocks": d.blocks, "D": d.D, "heads": d.heads, "ffn": d.ffn,
@@ -469,8 +470,9 @@ def main():
                     help="one video on two GPUs: rank 0 the text row, rank 1 the zeroed-text row (--gpus 2)")
     ap.add_argument("--seq-parallel", action="store_true",
                     help="one video on all GPUs: the blocks under head-sharded (Ulysses) sequence parallelism")
-    ap.add_argument("--fp8", action="store_true",
-                    help="the blocks' six linear layers as e4m3 GEMMs (per-token / per-channel scales); attention bf16")
+    ap.add_argument("--fp8", nargs="?", const="all", default=None, choices=("all", "no-ffn2"),
+                    help="the blocks' linear layers as e4m3 GEMMs (per-token / per-channel scales; attention bf16): "
+                         "all six, or all but the FFN's second layer (no-ffn2: the FFN hidden stays bf16)")
     ap.add_argument("--ring", type=int, default=1, metavar="R",
                     help="with --seq-parallel: R ring groups (Ulysses inside each group of N/R GPUs, a ring across them)")
     args = ap.parse_args()

@@ -326,7 +326,9 @@ static wd_status block_forward_fp8_t(const wd_dims* d, const wd_block_weights* w
   // 10. h2 = norm(X)(1 + scale2) + shift2, quantised;  11. u = GELU(h2 W1^T + b1) (bf16)
   WD_TRY(nq(e0 + 3 * D, mod + 3 * D, e0 + 4 * D, mod + 4 * D, nullptr, nullptr, rms));
   WD_TRY(g8(F, D, w8->f1_q, w8->f1_s, w->f1_b, EPI_GELU, A, F, nullptr, nullptr));
-  // 12. X += gate2 * (u W2^T + b2), u quantised
+  // 12. X += gate2 * (u W2^T + b2): u quantised, or (no e4m3 FFN2 weight) the bf16 GEMM on u
+  if (!w8->f2_q)
+    return gemm<bf16>(M, D, F, A, F, w->f2_w, F, EPI_RESID, epi(X, D, w->f2_b, e0 + 5 * D, mod + 5 * D), st);
   WD_TRY(quant_rows_e4m3<bf16>(M, F, A, Q, S, st));
   return g8(D, F, w8->f2_q, w8->f2_s, w->f2_b, EPI_RESID, X, D, e0 + 5 * D, mod + 5 * D);
 }
@@ -647,8 +649,9 @@ wd_status wd_block_forward_fp8(const wd_dims* d, const wd_block_weights* w, cons
   if (!w || !w8) { set_error("block weights NULL"); return WD_ERR_ARG; }
   WD_NEED(w->qkv_b); WD_NEED(w->g_q); WD_NEED(w->g_k); WD_NEED(w->o_b); WD_NEED(w->cn_g); WD_NEED(w->cn_b);
   WD_NEED(w->cq_b); WD_NEED(w->co_b); WD_NEED(w->f1_b); WD_NEED(w->f2_b); WD_NEED(w->mod);
-  WD_NEED(w8->qkv_q); WD_NEED(w8->o_q); WD_NEED(w8->cq_q); WD_NEED(w8->co_q); WD_NEED(w8->f1_q); WD_NEED(w8->f2_q);
-  WD_NEED(w8->qkv_s); WD_NEED(w8->o_s); WD_NEED(w8->cq_s); WD_NEED(w8->co_s); WD_NEED(w8->f1_s); WD_NEED(w8->f2_s);
+  WD_NEED(w8->qkv_q); WD_NEED(w8->o_q); WD_NEED(w8->cq_q); WD_NEED(w8->co_q); WD_NEED(w8->f1_q);
+  WD_NEED(w8->qkv_s); WD_NEED(w8->o_s); WD_NEED(w8->cq_s); WD_NEED(w8->co_s); WD_NEED(w8->f1_s);
+  if (w8->f2_q) { WD_NEED(w8->f2_s); } else { WD_NEED(w->f2_w); }   // no e4m3 FFN2: the bf16 weight
   WD_NEED(e0); WD_NEED(kv); WD_NEED(X); WD_NEED(ws);
   const Ws8 L = ws_layout_fp8(d, batch, ws);
   if (ws_bytes < L.bytes) { set_error("workspace %zu < %zu bytes", ws_bytes, L.bytes); return WD_ERR_WORKSPACE; }

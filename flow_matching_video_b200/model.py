@@ -70,13 +70,14 @@ class DiT:
     """The DiT of one workload on one device, with its buffers for `batch` rows."""
 
     def __init__(self, dims: synth.Dims, weights: dict, batch: int, device="cuda", buffers_from: "DiT" = None,
-                 fp8: bool = False):
+                 fp8: bool = False, fp8_ffn2: bool = True):
         """buffers_from: another DiT of the same dims and batch whose workspace,
         residual stream and output buffers this one shares (the experts of a
         timestep MoE run one at a time); the context and K/V cache stay per model.
         fp8: the blocks run wd_block_forward_fp8 ("Wan（通义万相）..." 5.3), with the six
         matrices of every block quantised once here by the library's row
-        quantiser (per output channel)."""
+        quantiser (per output channel); fp8_ffn2=False keeps the FFN's second
+        layer in bf16 (its input, the FFN hidden, is then not quantised)."""
         self.dims = dims
         self.cd = wd.make_dims(dims)
         self.batch = batch
@@ -101,6 +102,9 @@ class DiT:
             for i in range(dims.blocks):
                 ptrs = {}
                 for nm in ("qkv", "o", "cq", "co", "f1", "f2"):
+                    if nm == "f2" and not fp8_ffn2:
+                        ptrs["f2_q"] = ptrs["f2_s"] = None
+                        continue
                     wt = self.w[f"blk{i}.{nm}.w"]
                     q = torch.empty(wt.shape, dtype=torch.uint8, device=wt.device)
                     sc = torch.empty(wt.shape[0], dtype=torch.float32, device=wt.device)

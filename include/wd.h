@@ -251,7 +251,10 @@ wd_status wd_block_post(const wd_dims* d, const wd_block_weights* w, const float
  * hidden (bf16) by the row quantiser.  The self- and cross-attention, QK-norm
  * + RoPE and the fp32 residual stream are those of the bf16 block.  WD_BF16
  * models with D and ffn multiples of 256 only (else WD_ERR_UNSUPPORTED /
- * WD_ERR_SHAPE).  ws: wd_workspace_bytes_fp8(d, batch) bytes. */
+ * WD_ERR_SHAPE).  ws: wd_workspace_bytes_fp8(d, batch) bytes.  With
+ * w8->f2_q NULL the FFN's second layer stays bf16 (w->f2_w): the FFN hidden
+ * is then not quantised, which saves its extra pass over the largest
+ * activation of the block. */
 size_t wd_workspace_bytes_fp8(const wd_dims* d, int batch);
 wd_status wd_block_forward_fp8(const wd_dims* d, const wd_block_weights* w, const wd_block_weights_fp8* w8,
                                const float* e0, const void* kv, int batch, float* X, void* ws, size_t ws_bytes,

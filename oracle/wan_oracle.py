@@ -393,7 +393,8 @@ def block_after_attention(Xr, o, e0, w: dict, blk: int, kv: dict, dims, rnd: boo
     X  += gate2 * Linear_2(GELU(Linear_1(norm(X)(1+scale2)+shift2)))
     Reading: the cross-attention input gets a LayerNorm with affine gains.
     fp8: the four Linear layers as FP8 GEMMs; the norms' outputs are quantised
-    from their fp32 values, o, oc and the FFN hidden after their bf16 store."""
+    from their fp32 values, o, oc and the FFN hidden after their bf16 store.
+    fp8 = "no-ffn2": the FFN's second layer stays bf16."""
     p = f"blk{blk}."
     D, nh, dh, eps = dims.D, dims.heads, dims.dh, dims.eps
     Xr = np.asarray(Xr, F64)
@@ -417,7 +418,7 @@ def block_after_attention(Xr, o, e0, w: dict, blk: int, kv: dict, dims, rnd: boo
         # ---- gated FFN
         h2 = adaln_modulate(xr, shift2, scale2, eps, dims.norm)
         u = _st(gelu(_lin(h2, w[p + "f1.w"], w[p + "f1.b"], rnd, fp8)), rnd)
-        out[b] = xr + gate2 * _lin(u, w[p + "f2.w"], w[p + "f2.b"], rnd, fp8)
+        out[b] = xr + gate2 * _lin(u, w[p + "f2.w"], w[p + "f2.b"], rnd, fp8 and fp8 != "no-ffn2")
     return out
 
 

@@ -49,7 +49,7 @@ def host(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def setup(mods, wl, blocks=None, fp8=False):
+def setup(mods, wl, blocks=None, fp8=False, fp8_ffn2=True):
     model, wd = mods
     d = wl.dims
     w = synth.model_weights(wl, blocks=blocks)
@@ -61,7 +61,7 @@ def setup(mods, wl, blocks=None, fp8=False):
         ren = {f"blk{b}.": f"blk{j}." for j, b in enumerate(blocks)}
         wdev = {next((ren[p] + k[len(p):] for p in ren if k.startswith(p)), k): v for k, v in w.items()}
     dw = model.weights_to_device(wdev, d, "cuda")
-    net = model.DiT(d, dw, wl.batch, fp8=fp8)
+    net = model.DiT(d, dw, wl.batch, fp8=fp8, fp8_ffn2=fp8_ffn2)
     tdt = net.tdtype
     txt = np.stack([x["txt"], np.zeros_like(x["txt"])]) if wl.batch == 2 else x["txt"][None]
     if d.t2v:   # text-to-video: no CLIP context, no y
@@ -540,11 +540,14 @@ def _oracle_moved(monkeypatch, fn, seed=17, size=1e-3):
         return fn()
 
 
+@pytest.mark.parametrize("mode", ["all", "no-ffn2"])
 @pytest.mark.parametrize("wl,n_rows,tau", [(synth.STACK_480P81, 192, 700.0), (synth.BLOCK_480P17, 256, 300.0)],
                          ids=lambda v: getattr(v, "name", str(v)))
-def test_block_fp8(mods, monkeypatch, wl, n_rows, tau):
+def test_block_fp8(mods, monkeypatch, wl, n_rows, tau, mode):
+    """The FP8 block (all six linear layers on e4m3 operands, or all but the
+    FFN's second layer) against the oracle's FP8 block in the same mode."""
     model, wd = mods
-    net, w, x, txt, y, d = setup(mods, wl, blocks=[0], fp8=True)
+    net, w, x, txt, y, d = setup(mods, wl, blocks=[0], fp8=True, fp8_ffn2=mode == "all")
     B, L, D = wl.batch, d.L, d.D
     x_t = np.stack([x["x0"]] * B)
     X_in = O.patch_embed(x_t, O.build_cond_y(x["img_lat"]), w["pe.w"], w["pe.b"], rnd=True)
@@ -558,7 +561,7 @@ def test_block_fp8(mods, monkeypatch, wl, n_rows, tau):
     rows = np.unique(np.concatenate([rng.choice(L, n_rows, replace=False), np.arange(L - 70, L), [0]]))
     got = host(net.X)[:, rows]
     kvs = oracle_context(w, txt, x["clip"], d, True)
-    f8 = lambda: O.block_forward(X_in, e0, w, 0, kvs[0], d, rnd=True, rows=rows, fp8=True)
+    f8 = lambda: O.block_forward(X_in, e0, w, 0, kvs[0], d, rnd=True, rows=rows, fp8=True if mode == "all" else mode)
     want8, moved = f8(), _oracle_moved(monkeypatch, f8)
     want16 = O.block_forward(X_in, e0, w, 0, kvs[0], d, rnd=True, rows=rows)
     c = lambda a: a - X_in[:, rows]
@@ -566,7 +569,7 @@ def test_block_fp8(mods, monkeypatch, wl, n_rows, tau):
            "x": max(TOL_BF16, 2 * rel(moved, want8))}
     err = {"max": rel(c(got), c(want8)), "rms": _rms_rel(c(got), c(want8)), "x": rel(got, want8)}
     e16 = rel(c(got), c(want16))
-    print(f"\n[{wl.name} FP8 block] vs the FP8 oracle: contribution max {err['max']:.3e} (bar {bar['max']:.3e}), "
+    print(f"\n[{wl.name} FP8 block, {mode}] vs the FP8 oracle: contribution max {err['max']:.3e} (bar {bar['max']:.3e}), "
           f"rms {err['rms']:.3e} (bar {bar['rms']:.3e}), X_out {err['x']:.3e} (bar {bar['x']:.3e}); "
           f"contribution vs the bf16 oracle {e16:.3e}")
     for k in err:

@@ -20,6 +20,8 @@ rows and columns swapped, RMSNorm per head instead of over D, a RoPE turning
 the wrong way or reading the wrong coordinate, the text and image key weights
 swapped, the unconditional row keeping its text.  The pin must fail on each.
 """
+import unittest.mock as um
+
 import numpy as np
 import pytest
 import torch
@@ -435,3 +437,21 @@ def test_fp8_block_is_the_block_within_e4m3_precision():
     contrib = np.sqrt(((exact - X) ** 2).mean())
     err = np.abs(f8 - exact).max()
     assert 1e-6 * contrib < err < 0.25 * contrib
+
+
+def test_fp8_block_without_fp8_ffn2_is_the_fp8_block_with_an_exact_last_layer():
+    """fp8="no-ffn2" keeps only the FFN's second layer exact: planting the
+    exact Linear into that one call of the full FP8 block gives it bit for
+    bit, and it differs from both."""
+    d, w, txt, clip, X = _tiny(D=48, ffn=40)
+    e0 = RNG.standard_normal((6, d.D)) * 0.3
+    ctx_t, ctx_i = O.context_embed(w, txt, clip)
+    kv = O.cross_kv(w, 0, ctx_t, ctx_i)
+    exact = O.block_forward(X, e0, w, 0, kv, d)
+    f8 = O.block_forward(X, e0, w, 0, kv, d, fp8=True)
+    part = O.block_forward(X, e0, w, 0, kv, d, fp8="no-ffn2")
+    assert np.abs(part - f8).max() > 0 and np.abs(part - exact).max() > 0
+    lin8 = O.linear_fp8
+    with um.patch.object(O, "linear_fp8", lambda x, wt, b=None: O.linear(x, wt, b) if wt is w["blk0.f2.w"] else lin8(x, wt, b)):
+        planted = O.block_forward(X, e0, w, 0, kv, d, fp8=True)
+    np.testing.assert_array_equal(planted, part)
