@@ -366,12 +366,13 @@ def block_qkv(x, e0, w: dict, blk: int, dims, tok, rnd: bool = False, want=("q",
     return out
 
 
-def block_self_attention(X, e0, w: dict, blk: int, dims, rnd: bool = False, rows=None, fp8: bool = False):
+def block_self_attention(X, e0, w: dict, blk: int, dims, rnd: bool = False, rows=None, fp8: bool = False,
+                         attn8: bool = False):
     """The attention output o of a block's self-attention for the token rows
     `rows` of every sample (default all): o = softmax(q k^T / sqrt(dh)) v per
     head over all L keys, heads concatenated -> [B, len(rows), D], the input of
     Linear_o ([I2V] 5.3).  Keys and values cover every token, so the rows are
-    exact."""
+    exact.  attn8: the FP8 attention (attention_fp8) on the stored q, k, v."""
     X = np.asarray(X, F64)
     B, L, D = X.shape
     rows = np.arange(L) if rows is None else np.asarray(rows)
@@ -379,7 +380,8 @@ def block_self_attention(X, e0, w: dict, blk: int, dims, rnd: bool = False, rows
     for b in range(B):
         kv = block_qkv(X[b], e0, w, blk, dims, np.arange(L), rnd, want=("k", "v"), fp8=fp8)
         q = block_qkv(X[b][rows], e0, w, blk, dims, rows, rnd, want=("q",), fp8=fp8)["q"]
-        o[b] = _st(attention(q, kv["k"], kv["v"]).reshape(len(rows), D), rnd)
+        att = attention_fp8 if attn8 else attention
+        o[b] = _st(att(q, kv["k"], kv["v"]).reshape(len(rows), D), rnd)
     return o
 
 
@@ -422,7 +424,8 @@ def block_after_attention(Xr, o, e0, w: dict, blk: int, kv: dict, dims, rnd: boo
     return out
 
 
-def block_forward(X, e0, w: dict, blk: int, kv: dict, dims, rnd: bool = False, rows=None, fp8: bool = False):
+def block_forward(X, e0, w: dict, blk: int, kv: dict, dims, rnd: bool = False, rows=None, fp8: bool = False,
+                  attn8: bool = False):
     """One DiT block ([I2V] 5.2-5.5), order self-attention -> cross -> FFN:
     block_self_attention, then block_after_attention.
 
@@ -431,10 +434,11 @@ def block_forward(X, e0, w: dict, blk: int, kv: dict, dims, rnd: bool = False, r
     computes the output only for those token rows of every sample; keys and
     values still cover all L tokens, so the result is exact for those rows.
     fp8: the six Linear layers as FP8 GEMMs ([WAN] 5.3), as the GPU's FP8 block.
+    attn8: the self-attention as the FP8 attention of [WAN] 5.3.
     """
     X = np.asarray(X, F64)
     rows = np.arange(X.shape[1]) if rows is None else np.asarray(rows)
-    o = block_self_attention(X, e0, w, blk, dims, rnd, rows, fp8)
+    o = block_self_attention(X, e0, w, blk, dims, rnd, rows, fp8, attn8)
     return block_after_attention(X[:, rows], o, e0, w, blk, kv, dims, rnd, fp8)
 
 
@@ -451,7 +455,8 @@ def head_unpatchify(X, e, w: dict, dims, rnd: bool = False):
 
 
 # ---------------------------------------------------------------- whole DiT
-def dit_forward(x_t, y, tau: float, w: dict, kvs: list, dims, rnd: bool = False, attn=None, fp8: bool = False):
+def dit_forward(x_t, y, tau: float, w: dict, kvs: list, dims, rnd: bool = False, attn=None, fp8: bool = False,
+                attn8: bool = False):
     """v = DiT(concat(x_t, y), tau, context) for a batch ([I2V] 5, 7).
     attn (optional, the attention cache of [WAN] 5.3): a dict with "o", a
     list holding per block the self-attention output o [B, L, D] last
@@ -462,7 +467,7 @@ def dit_forward(x_t, y, tau: float, w: dict, kvs: list, dims, rnd: bool = False,
     X = patch_embed(x_t, y, w["pe.w"], w["pe.b"], rnd)
     for i in range(dims.blocks):
         if attn is None:
-            X = block_forward(X, e0, w, i, kvs[i], dims, rnd, fp8=fp8)
+            X = block_forward(X, e0, w, i, kvs[i], dims, rnd, fp8=fp8, attn8=attn8)
             continue
         if not attn["reuse"]:
             attn["o"][i] = block_self_attention(X, e0, w, i, dims, rnd)
@@ -707,3 +712,92 @@ def gemm_fp8(qa, sa, qb, sb, bias=None):
     acc = np.asarray(qa, F64) @ np.asarray(qb, F64).T
     out = acc * np.asarray(sa, F64)[:, None] * np.asarray(sb, F64)[None, :]
     return out + np.asarray(bias, F64) if bias is not None else out
+
+
+# ---------------------------------------------------------------- FP8 attention ([WAN] 5.3)
+I8_MAX = 127.0
+
+
+def quant_rows_int8(x):
+    """Per-row symmetric INT8 quantisation for the attention's Q K^T product
+    ([WAN] 5.3 "FlashAttention3 FP8": the Q/K inner product in INT8).
+    Reading: scale_r = amax_r / 127 and q = round-half-even(x / scale_r), both
+    computed in fp32 (IEEE division), as for the e4m3 quantiser; an all-zero row
+    gets scale 1.  Returns (codes [rows, K] float64 holding integers in
+    [-127, 127], scale [rows] float32)."""
+    x = np.asarray(x, dtype=np.float32)
+    amax = np.abs(x).max(axis=1)
+    scale = np.where(amax > 0, amax / np.float32(I8_MAX), np.float32(1.0)).astype(np.float32)
+    y = (x / scale[:, None]).astype(np.float32)
+    return np.clip(np.rint(y.astype(F64)), -I8_MAX, I8_MAX), scale
+
+
+def quant_blocks_int8(x, bk: int = 128):
+    """INT8 quantisation with one scale per block of bk consecutive rows (the
+    keys of one attention block): each block is quantised as one row by
+    quant_rows_int8.  Returns (codes [rows, K], scale [ceil(rows / bk)] float32)."""
+    x = np.asarray(x, dtype=np.float32)
+    rows, K = x.shape
+    nb = -(-rows // bk)
+    codes, scale = np.empty((rows, K)), np.empty(nb, np.float32)
+    for n in range(nb):
+        blk = x[n * bk:(n + 1) * bk]
+        c, s = quant_rows_int8(blk.reshape(1, -1))
+        codes[n * bk:(n + 1) * bk], scale[n] = c.reshape(blk.shape), s[0]
+    return codes, scale
+
+
+def quant_cols_e4m3(x):
+    """Per-column (per channel over all rows) e4m3 quantisation of the
+    attention's values: quant_rows_e4m3 of the transpose.  Returns (codes
+    [rows, K], scale [K] float32)."""
+    codes, scale = quant_rows_e4m3(np.asarray(x, dtype=np.float32).T)
+    return codes.T, scale
+
+
+def attention_fp8_head(q, k, v, bk: int = 128, theta: float = 8.0, quant_p: bool = True):
+    """One head of the FP8 attention of [WAN] 5.3 ("FlashAttention3 FP8": the
+    Q/K inner product in INT8, O = P V in FP8, accumulation across key blocks
+    in FP32), q [Nq, dh], k/v [Nk, dh] -> [Nq, dh].
+
+    Reading (the page names the precisions only):
+    * Q in INT8 per row (token) and K in INT8 per block of bk keys, so that
+      S = (q8 k8^T) sq_r sk_n exactly (integer products); V in e4m3 per channel.
+    * The softmax runs blockwise over the keys in order, as the accumulation
+      across blocks implies: per block n, logits t = S log2(e) / sqrt(dh)
+      (log2 units), the block's row maximum mx; the reference m moves to mx only
+      when mx exceeds it by more than theta (log2 units), and then the running
+      O and l are scaled by 2^(m_old - m).  p = 2^(t - m) <= 2^theta, its e4m3
+      rounding P8 (quant_p) enters O += P8 v8, and the unrounded p enters l.
+    * out = O * sv / l.
+    With quant_p=False and any theta this is softmax(q k^T / sqrt(dh)) v of the
+    dequantised operands exactly; with quant_p the result depends on the
+    reference, hence on theta and bk, within e4m3 precision of P."""
+    q8, sq = quant_rows_int8(q)
+    k8, sk = quant_blocks_int8(k, bk)
+    v8, sv = quant_cols_e4m3(v)
+    Nq, dh = q8.shape
+    c = math.log2(math.e) / math.sqrt(dh)
+    m = np.full(Nq, -np.inf)
+    l = np.zeros(Nq)
+    O = np.zeros((Nq, v8.shape[1]))
+    for n in range(len(sk)):
+        js = slice(n * bk, min(k8.shape[0], (n + 1) * bk))
+        t = (q8 @ k8[js].T) * (np.asarray(sq, F64)[:, None] * F64(sk[n]) * c)
+        mx = t.max(axis=1)
+        m_new = np.where(mx > m + theta, mx, m)
+        alpha = np.exp2(m - m_new)
+        p = np.exp2(t - m_new[:, None])
+        O = O * alpha[:, None] + (e4m3(p) if quant_p else p) @ v8[js]
+        l = l * alpha + p.sum(axis=1)
+        m = m_new
+    return O * np.asarray(sv, F64)[None, :] / l[:, None]
+
+
+def attention_fp8(q, k, v, bk: int = 128, theta: float = 8.0, quant_p: bool = True):
+    """attention_fp8_head per head: q [Nq, h, dh], k/v [Nk, h, dh] -> [Nq, h, dh].
+    The quantisation scales of K and V cover every key of the head, so q may
+    hold any subset of the query rows."""
+    q, k, v = (np.asarray(a, F64) for a in (q, k, v))
+    return np.stack([attention_fp8_head(q[:, hh], k[:, hh], v[:, hh], bk, theta, quant_p)
+                     for hh in range(q.shape[1])], axis=1)
