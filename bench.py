@@ -270,7 +270,9 @@ def run_ours(args, rank, world, local_rank):
             runner = attn_cache = model.AttnCache(d, weights, t_attn, int(interval), B, dev)
             net = runner.net
         else:
-            runner = net = model.DiT(d, weights, B, dev, fp8=args.fp8 is not None, fp8_ffn2=args.fp8 != "no-ffn2")
+            runner = net = model.DiT(d, weights, B, dev, fp8=args.fp8 is not None,
+                                     fp8_ffn2=not (args.fp8 or "").startswith("no-ffn2"),
+                                     fp8_attention=(args.fp8 or "").endswith("+attn"))
         runner.prepare_context(txt, clip)
         rows_local = B
     y = None if d.t2v else net.build_cond_y(torch.from_numpy(x["img_lat"]).to(dev))
@@ -394,6 +396,9 @@ def run_ours(args, rank, world, local_rank):
     att_flops = (1 if mode == "cfg-split" else B) * block_flops(d)["attn_self"] / (world if mode == "ulysses" else 1)
     achieved = att_flops / (avg_att / 1e3) / 1e12
     peak_s = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    # the FP8 attention's products run at twice the bf16 rate (the nominal int8 / e4m3 : bf16 ratio)
+    attn8 = (args.fp8 or "").endswith("+attn")
+    peak_att = 2 * peak_s if attn8 else peak_s
     share = {k: round(v[1] / max(sum(u[1] for u in tr.values()), 1e-9), 4) for k, v in tr.items()}
     launches = sum(v[0] for v in tr.values())
     cpu = None
@@ -407,8 +412,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak" if mode == "replicas" else "strong",
-        "vs_baseline": None, "dtype": ({"all": "bf16 (e4m3 GEMMs)", "no-ffn2": "bf16 (e4m3 GEMMs but FFN2)"}[args.fp8]
-                                        if args.fp8 else "bf16"), "data": "synthetic",
+        "vs_baseline": None, "dtype": fp8_label(args.fp8), "data": "synthetic",
         "config": {"workload": wl.name, "video": f"{4 * (d.T - 1) + 1} frames {8 * d.H}x{8 * d.W}",
                    "latent": [16, d.T, d.H, d.W],
                    "tokens": d.L, "batch": B, "blocks": d.blocks, "D": d.D, "heads": d.heads, "ffn": d.ffn,
@@ -424,12 +428,17 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": value_e2e, "unit": "tokens/s",
                 "h2d_bytes_per_step": x_host.numel() * 4, "d2h_bytes_per_step": out_host.numel() * 4},
         "gpu_launches": launches,
-        "roofline": {"bound": "tensor", "kernel": "attention_tc self (k_attn_tc<2,1,bf16>)",
-                     "achieved": achieved, "peak": peak_s, "unit": "TFLOP/s", "frac": achieved / peak_s,
-                     "peak_source": f"{pk['_source']} bf16 sustained",
+        "roofline": {"bound": "tensor",
+                     "kernel": ("attention_fp8 self (k_attn_f8: INT8 Q K^T, e4m3 P V)" if attn8 else
+                                "attention_tc self (k_attn_tc<2,1,bf16>)"),
+                     "achieved": achieved, "peak": peak_att, "unit": "TFLOP/s", "frac": achieved / peak_att,
+                     "peak_source": (f"{pk['_source']} bf16 sustained x 2 (nominal int8/e4m3 : bf16 ratio)" if attn8
+                                     else f"{pk['_source']} bf16 sustained"),
                      "flops_per_launch": att_flops, "avg_launch_ms": avg_att, "launches": n_att,
-                     "traffic": traffic_for("attn_self", os.path.join(ROOT, "flow_matching_video_b200", "csrc",
-                                                                      "k_attn_tc.cu"))},
+                     "traffic": (traffic_for("attn_self_f8", os.path.join(ROOT, "flow_matching_video_b200", "csrc",
+                                                                          "k_attn_f8.cu")) if attn8 else
+                                 traffic_for("attn_self", os.path.join(ROOT, "flow_matching_video_b200", "csrc",
+                                                                       "k_attn_tc.cu")))},
         "kernel_time_share": share,
         **({"cache": cache_note} if cache_note else {}),
         "clocks": clk,
@@ -453,6 +462,14 @@ def launch_ranks(n: int) -> int:
     return subprocess.call(cmd)
 
 
+def fp8_label(mode):
+    """The dtype key of the JSON line for a --fp8 mode."""
+    if not mode:
+        return "bf16"
+    gemms = "e4m3 GEMMs but FFN2" if mode.startswith("no-ffn2") else "e4m3 GEMMs"
+    return f"bf16 ({gemms}, INT8/e4m3 attention)" if mode.endswith("+attn") else f"bf16 ({gemms})"
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -470,9 +487,11 @@ def main():
                     help="one video on two GPUs: rank 0 the text row, rank 1 the zeroed-text row (--gpus 2)")
     ap.add_argument("--seq-parallel", action="store_true",
                     help="one video on all GPUs: the blocks under head-sharded (Ulysses) sequence parallelism")
-    ap.add_argument("--fp8", nargs="?", const="all", default=None, choices=("all", "no-ffn2"),
-                    help="the blocks' linear layers as e4m3 GEMMs (per-token / per-channel scales; attention bf16): "
-                         "all six, or all but the FFN's second layer (no-ffn2: the FFN hidden stays bf16)")
+    ap.add_argument("--fp8", nargs="?", const="all", default=None,
+                    choices=("all", "no-ffn2", "all+attn", "no-ffn2+attn"),
+                    help="the blocks' linear layers as e4m3 GEMMs (per-token / per-channel scales): all six, or all "
+                         "but the FFN's second layer (no-ffn2: the FFN hidden stays bf16); +attn: the self-attention "
+                         "as the FP8 attention (INT8 Q K^T, e4m3 P V), else bf16")
     ap.add_argument("--ring", type=int, default=1, metavar="R",
                     help="with --seq-parallel: R ring groups (Ulysses inside each group of N/R GPUs, a ring across them)")
     args = ap.parse_args()

@@ -261,6 +261,8 @@ struct Ws8 {
   Ws base;
   uint8_t* q;
   float* s;
+  void* attn8;                 // the FP8 attention's operands (layout a8)
+  wd_attn_fp8_layout a8;
   size_t bytes;
 };
 static Ws8 ws_layout_fp8(const wd_dims* d, int batch, void* base) {
@@ -269,10 +271,14 @@ static Ws8 ws_layout_fp8(const wd_dims* d, int batch, void* base) {
   const size_t rows = static_cast<size_t>(batch) * tokens(d);
   const size_t nq = up256(rows * static_cast<size_t>(d->ffn > d->D ? d->ffn : d->D));
   const size_t ns = up256(rows * sizeof(float));
+  w.a8 = wd_attn_fp8_layout{};
+  const int dh = d->D / d->heads;
+  if (dh != 128 || attn_fp8_layout(batch, tokens(d), tokens(d), d->heads, dh, &w.a8) != WD_OK) w.a8.bytes = 0;
   char* p = base ? static_cast<char*>(base) + w.base.bytes : nullptr;
   w.q = reinterpret_cast<uint8_t*>(p);
   w.s = p ? reinterpret_cast<float*>(p + nq) : nullptr;
-  w.bytes = w.base.bytes + nq + ns;
+  w.attn8 = p ? p + nq + ns : nullptr;
+  w.bytes = w.base.bytes + nq + ns + w.a8.bytes;
   return w;
 }
 
@@ -312,7 +318,13 @@ static wd_status block_forward_fp8_t(const wd_dims* d, const wd_block_weights* w
   { Trace tr(KC_SMALL, st); k_rope_table<<<64, 256, 0, st>>>(ws.base.rope, d->T, d->H / 2, d->W / 2, dh); }
   WD_TRY(launch_status("rope_table"));
   WD_TRY(qknorm_rope<bf16>(A, rows, *d, w->g_q, w->g_k, ws.base.rope, L, 0, st));
-  WD_TRY(self_attention_t<bf16>(d, batch, d->heads, A, Bf, st));
+  if (w8->attention_fp8) {   // INT8 Q K^T, FP8 P V
+    WD_TRY(attn_fp8_quantize(batch, static_cast<int>(L), static_cast<int>(L), d->heads, A, 3 * D, A + D, A + 2 * D,
+                             3 * D, ws.attn8, ws.a8, st));
+    WD_TRY(attn_fp8(batch, static_cast<int>(L), static_cast<int>(L), d->heads, ws.attn8, ws.a8, Bf, D, st));
+  } else {
+    WD_TRY(self_attention_t<bf16>(d, batch, d->heads, A, Bf, st));
+  }
   // 5. X += gate1 * (o Wo^T + b), o quantised
   WD_TRY(quant_rows_e4m3<bf16>(M, D, Bf, Q, S, st));
   WD_TRY(g8(D, D, w8->o_q, w8->o_s, w->o_b, EPI_RESID, X, D, e0 + 2 * D, mod + 2 * D));
@@ -652,6 +664,10 @@ wd_status wd_block_forward_fp8(const wd_dims* d, const wd_block_weights* w, cons
   WD_NEED(w8->qkv_q); WD_NEED(w8->o_q); WD_NEED(w8->cq_q); WD_NEED(w8->co_q); WD_NEED(w8->f1_q);
   WD_NEED(w8->qkv_s); WD_NEED(w8->o_s); WD_NEED(w8->cq_s); WD_NEED(w8->co_s); WD_NEED(w8->f1_s);
   if (w8->f2_q) { WD_NEED(w8->f2_s); } else { WD_NEED(w->f2_w); }   // no e4m3 FFN2: the bf16 weight
+  if (w8->attention_fp8 && d->D / d->heads != 128) {
+    set_error("wd_block_forward_fp8: the FP8 attention needs 128-wide heads");
+    return WD_ERR_UNSUPPORTED;
+  }
   WD_NEED(e0); WD_NEED(kv); WD_NEED(X); WD_NEED(ws);
   const Ws8 L = ws_layout_fp8(d, batch, ws);
   if (ws_bytes < L.bytes) { set_error("workspace %zu < %zu bytes", ws_bytes, L.bytes); return WD_ERR_WORKSPACE; }
@@ -793,6 +809,34 @@ wd_status wd_attention_lse(int dtype, int batch, int Lq, int heads, int dh, cons
   }
   set_error("wd_attention_lse: dtype %d (WD_BF16 or WD_F32)", dtype);
   return WD_ERR_DTYPE;
+}
+
+wd_status wd_attention_fp8_layout(int batch, int64_t Lq, int64_t Lk, int heads, int dh, wd_attn_fp8_layout* out) {
+  WD_NEED(out);
+  return attn_fp8_layout(batch, Lq, Lk, heads, dh, out);
+}
+
+wd_status wd_attention_fp8_quantize(int batch, int64_t Lq, int64_t Lk, int heads, int dh, const void* q, int64_t q_rs,
+                                    const void* k, const void* v, int64_t kv_rs, void* buf, size_t buf_bytes,
+                                    wd_stream stream) {
+  WD_NEED(q); WD_NEED(k); WD_NEED(v); WD_NEED(buf);
+  wd_attn_fp8_layout L;
+  WD_TRY(attn_fp8_layout(batch, Lq, Lk, heads, dh, &L));
+  if (buf_bytes < L.bytes) { set_error("FP8 attention buffer %zu < %zu bytes", buf_bytes, L.bytes); return WD_ERR_WORKSPACE; }
+  if (reinterpret_cast<uintptr_t>(buf) & 255u) { set_error("FP8 attention buffer not 256-byte aligned"); return WD_ERR_ALIGN; }
+  return attn_fp8_quantize(batch, static_cast<int>(Lq), static_cast<int>(Lk), heads, static_cast<const bf16*>(q), q_rs,
+                           static_cast<const bf16*>(k), static_cast<const bf16*>(v), kv_rs, buf, L,
+                           static_cast<cudaStream_t>(stream));
+}
+
+wd_status wd_attention_fp8(int batch, int64_t Lq, int64_t Lk, int heads, int dh, const void* buf, size_t buf_bytes,
+                           void* o, int64_t o_rs, wd_stream stream) {
+  WD_NEED(buf); WD_NEED(o);
+  wd_attn_fp8_layout L;
+  WD_TRY(attn_fp8_layout(batch, Lq, Lk, heads, dh, &L));
+  if (buf_bytes < L.bytes) { set_error("FP8 attention buffer %zu < %zu bytes", buf_bytes, L.bytes); return WD_ERR_WORKSPACE; }
+  return attn_fp8(batch, static_cast<int>(Lq), static_cast<int>(Lk), heads, buf, L, static_cast<bf16*>(o), o_rs,
+                  static_cast<cudaStream_t>(stream));
 }
 
 wd_status wd_attention_merge(int dtype, int batch, int Lq, int heads, int dh, float* o_run, float* lse_run,

@@ -147,5 +147,12 @@ wd_status attention_simt(const AttnArgs<TI, TO>& a, cudaStream_t st);
 // Tensor-core attention (dh = 128; other head sizes go to attention_simt).
 wd_status attention_tc(const AttnArgs<bf16, bf16>& a, cudaStream_t st);
 wd_status attention_tc(const AttnArgs<f16, bf16>& a, cudaStream_t st);
+// FP8 attention (k_attn_f8.cu): the operand buffer's layout, the quantisation
+// of bf16 q, k, v into it and the attention on it (bf16 output).
+wd_status attn_fp8_layout(int batch, int64_t Lq, int64_t Lk, int heads, int dh, wd_attn_fp8_layout* L);
+wd_status attn_fp8_quantize(int batch, int Lq, int Lk, int heads, const bf16* q, int64_t q_rs, const bf16* k,
+                            const bf16* v, int64_t kv_rs, void* buf, const wd_attn_fp8_layout& L, cudaStream_t st);
+wd_status attn_fp8(int batch, int Lq, int Lk, int heads, const void* buf, const wd_attn_fp8_layout& L, bf16* o,
+                   int64_t o_rs, cudaStream_t st);
 
 }  // namespace wd

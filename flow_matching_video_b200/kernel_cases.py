@@ -2,11 +2,13 @@
 
     python -m flow_matching_video_b200.kernel_cases CASE [--batch B] [--iters N] [--warmup W]
 
-CASE is one of attn_self, attn_cross, gemm_qkv, gemm_o, gemm_ffn1, gemm_ffn2,
-euler, euler_hbm, gemm_fp8_qkv, gemm_fp8_o, gemm_fp8_ffn1, gemm_fp8_ffn2,
-quant_ffn_hidden, block_480p17 (one block, 17 frames, L = 7800, batch 1),
-block_480p81 (one block, L = 32760, batch 2) and block_480p81_fp8 (the same block
-with its six linear layers on e4m3 operands).
+CASE is one of attn_self, attn_cross, attn_fp8 (the FP8 self-attention on
+quantised operands), attn_fp8_quantize (the quantisation of q, k, v for it),
+gemm_qkv, gemm_o, gemm_ffn1, gemm_ffn2, euler, euler_hbm, gemm_fp8_qkv,
+gemm_fp8_o, gemm_fp8_ffn1, gemm_fp8_ffn2, quant_ffn_hidden, block_480p17 (one
+block, 17 frames, L = 7800, batch 1), block_480p81 (one block, L = 32760, batch
+2), block_480p81_fp8 (the same block with its six linear layers on e4m3
+operands) and block_480p81_fp8attn (and with the FP8 self-attention).
 Shapes are those of one block of the 30-block 480p/81-frame model (L = 32760
 tokens per sample, D = 1536, 12 heads x 128, FFN 8960, 257 image + 512 text
 keys); euler_hbm streams 2^26 elements so that every launch reads HBM.
@@ -42,6 +44,16 @@ def make_case(name: str, B: int):
     if name == "attn_self":
         q, k, v, o = bf(B, L, D), bf(B, L, D), bf(B, L, D), torch.empty(B, L, D, device="cuda", dtype=torch.bfloat16)
         return (lambda: wd.wd_attention(wd.WD_BF16, B, L, H, 128, q, k, v, L, 0, o)), 4.0 * B * L * L * D, "FLOP", B
+    if name in ("attn_fp8", "attn_fp8_quantize"):   # q|k|v fused as in the block
+        qkv, o = bf(B, L, 3 * D), torch.empty(B, L, D, device="cuda", dtype=torch.bfloat16)
+        lay = wd.wd_attention_fp8_layout(B, L, L, H, 128)
+        buf = torch.empty(lay.bytes, dtype=torch.uint8, device="cuda")
+        quant = lambda: wd.wd_attention_fp8_quantize(B, L, L, H, 128, qkv, 3 * D, qkv[..., D:], qkv[..., 2 * D:],
+                                                     3 * D, buf)
+        quant()
+        if name == "attn_fp8_quantize":   # bytes: q, k, v read (bf16), q8, k8, v8t written, v read twice
+            return quant, B * L * D * (2.0 * 4 + 3.0), "B", B
+        return (lambda: wd.wd_attention_fp8(B, L, L, H, 128, buf, o, D)), 4.0 * B * L * L * D, "FLOP", B
     if name == "attn_cross":   # IEEE half operands, bf16 output, as in the block
         q, o = hf(B, L, D), torch.empty(B, L, D, device="cuda", dtype=torch.bfloat16)
         ki, vi, kt, vt = hf(NI, D), hf(NI, D), hf(B, NT, D), hf(B, NT, D)
@@ -76,13 +88,13 @@ def make_case(name: str, B: int):
     d = synth.Dims(D=D, heads=H, ffn=F, blocks=1, T=21, H=60, W=104, n_txt=NT, c_txt=4096, n_img=NI,
                    c_img=1280, dtype="bf16")
     blocks = {"block_480p17": synth.BLOCK_480P17, "block_480p81": synth.STACK_480P81,
-              "block_480p81_fp8": synth.STACK_480P81}
+              "block_480p81_fp8": synth.STACK_480P81, "block_480p81_fp8attn": synth.STACK_480P81}
     if name in blocks:   # one DiT block (wd_block_forward) at the workload's batch; FLOPs as in the bench
         wl = blocks[name]
-        fp8 = name.endswith("_fp8")   # the block with its linear layers on e4m3 operands
+        fp8 = "_fp8" in name   # the block with its linear layers on e4m3 operands
         dd = synth.Dims(**{**wl.dims.__dict__, "blocks": 1})
         net = model.DiT(dd, model.random_weights_on_device(synth.Workload(wl.name, dd, wl.batch, wl.seed), "cuda"),
-                        wl.batch, fp8=fp8)
+                        wl.batch, fp8=fp8, fp8_attention=name.endswith("attn"))
         x = synth.inputs(wl)
         txt = torch.from_numpy(np.stack([x["txt"], 0 * x["txt"]][:wl.batch])).to("cuda", torch.bfloat16)
         net.prepare_context(txt, torch.from_numpy(x["clip"]).to("cuda", torch.bfloat16))

@@ -70,14 +70,16 @@ class DiT:
     """The DiT of one workload on one device, with its buffers for `batch` rows."""
 
     def __init__(self, dims: synth.Dims, weights: dict, batch: int, device="cuda", buffers_from: "DiT" = None,
-                 fp8: bool = False, fp8_ffn2: bool = True):
+                 fp8: bool = False, fp8_ffn2: bool = True, fp8_attention: bool = False):
         """buffers_from: another DiT of the same dims and batch whose workspace,
         residual stream and output buffers this one shares (the experts of a
         timestep MoE run one at a time); the context and K/V cache stay per model.
         fp8: the blocks run wd_block_forward_fp8 ("Wan（通义万相）..." 5.3), with the six
         matrices of every block quantised once here by the library's row
         quantiser (per output channel); fp8_ffn2=False keeps the FFN's second
-        layer in bf16 (its input, the FFN hidden, is then not quantised)."""
+        layer in bf16 (its input, the FFN hidden, is then not quantised);
+        fp8_attention: the self-attention as the page's FP8 attention (INT8
+        Q K^T, FP8 P V)."""
         self.dims = dims
         self.cd = wd.make_dims(dims)
         self.batch = batch
@@ -111,7 +113,8 @@ class DiT:
                     wd.wd_quant_rows_e4m3(wd.WD_BF16, wt.shape[0], wt.shape[1], wt, q, sc)
                     self.q8[(i, nm)] = (q, sc)
                     ptrs[nm + "_q"], ptrs[nm + "_s"] = q.data_ptr(), sc.data_ptr()
-                self.block_w8.append(wd.wd_block_weights_fp8(*(ptrs[f] for f in wd.FP8_FIELDS)))
+                self.block_w8.append(wd.wd_block_weights_fp8(*(ptrs[f] for f in wd.FP8_FIELDS),
+                                                             int(bool(fp8_attention))))
         L, D = dims.L, dims.D
         dev = self.device
         self.ctx = torch.empty(wd.wd_ctx_bytes(self.cd, batch), dtype=torch.uint8, device=dev)

@@ -48,7 +48,13 @@ BLOCK_FIELDS = ["qkv_w", "qkv_b", "g_q", "g_k", "o_w", "o_b", "cn_g", "cn_b", "c
 wd_block_weights = _ptr_struct("wd_block_weights", BLOCK_FIELDS)
 wd_head_weights = _ptr_struct("wd_head_weights", ["mod", "w", "b"])
 FP8_FIELDS = ["qkv_q", "o_q", "cq_q", "co_q", "f1_q", "f2_q", "qkv_s", "o_s", "cq_s", "co_s", "f1_s", "f2_s"]
-wd_block_weights_fp8 = _ptr_struct("wd_block_weights_fp8", FP8_FIELDS)
+wd_block_weights_fp8 = type("wd_block_weights_fp8", (C.Structure,),
+                            {"_fields_": [(f, C.c_void_p) for f in FP8_FIELDS] + [("attention_fp8", C.c_int)]})
+
+
+class wd_attn_fp8_layout(C.Structure):
+    _fields_ = [(f, C.c_size_t) for f in ("q8", "sq", "k8", "sk", "v8t", "sv", "v_amax", "bytes")] + \
+               [("lkp", C.c_int64)]
 
 # exported symbol -> (restype, argtypes)
 _P, _I, _F, _S, _L = C.c_void_p, C.c_int, C.c_float, C.c_size_t, C.c_int64
@@ -80,6 +86,9 @@ SIGNATURES = {
     "wd_attention": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P, _I, _I, _P, _P]),
     "wd_attention_lse": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P, _P]),
     "wd_attention_merge": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P]),
+    "wd_attention_fp8_layout": (_I, [_I, _L, _L, _I, _I, C.POINTER(wd_attn_fp8_layout)]),
+    "wd_attention_fp8_quantize": (_I, [_I, _L, _L, _I, _I, _P, _L, _P, _P, _L, _P, _S, _P]),
+    "wd_attention_fp8": (_I, [_I, _L, _L, _I, _I, _P, _S, _P, _L, _P]),
     "wd_quant_rows_e4m3": (_I, [_I, _I, _I, _P, _P, _P, _P]),
     "wd_gemm_fp8": (_I, [_I, _I, _I, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P]),
     "wd_test_exp2": (_I, [_P, _P, _P, _P, _P, _L, _P]),
@@ -268,6 +277,22 @@ def wd_attention_lse(dtype, batch, Lq, heads, dh, q, k, v, n, kv_shared, o, lse,
 def wd_attention_merge(dtype, batch, Lq, heads, dh, o_run, lse_run, o_part, lse_part, first, out=None, stream=None):
     _ok(_lib.wd_attention_merge(dtype, batch, Lq, heads, dh, _p(o_run), _p(lse_run), _p(o_part), _p(lse_part),
                                 int(first), _p(out), _stream(stream)), "wd_attention_merge")
+
+
+def wd_attention_fp8_layout(batch, Lq, Lk, heads, dh) -> wd_attn_fp8_layout:
+    out = wd_attn_fp8_layout()
+    _ok(_lib.wd_attention_fp8_layout(batch, Lq, Lk, heads, dh, C.byref(out)), "wd_attention_fp8_layout")
+    return out
+
+
+def wd_attention_fp8_quantize(batch, Lq, Lk, heads, dh, q, q_rs, k, v, kv_rs, buf, stream=None):
+    _ok(_lib.wd_attention_fp8_quantize(batch, Lq, Lk, heads, dh, _p(q), q_rs, _p(k), _p(v), kv_rs, _p(buf),
+                                       buf.numel() * buf.element_size(), _stream(stream)), "wd_attention_fp8_quantize")
+
+
+def wd_attention_fp8(batch, Lq, Lk, heads, dh, buf, o, o_rs, stream=None):
+    _ok(_lib.wd_attention_fp8(batch, Lq, Lk, heads, dh, _p(buf), buf.numel() * buf.element_size(), _p(o), o_rs,
+                              _stream(stream)), "wd_attention_fp8")
 
 
 def wd_set_debug_flags(flags: int):

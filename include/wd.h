@@ -121,6 +121,7 @@ typedef struct {
 typedef struct {
   const void *qkv_q, *o_q, *cq_q, *co_q, *f1_q, *f2_q;
   const float *qkv_s, *o_s, *cq_s, *co_s, *f1_s, *f2_s;
+  int attention_fp8;   /* 0: the block's self-attention in bf16; 1: the FP8 attention (wd_attention_fp8) */
 } wd_block_weights_fp8;
 
 /* Head ([I2V] 5.5): mod [2,D] (shift, scale biases added to e), w [64,D]
@@ -254,7 +255,9 @@ wd_status wd_block_post(const wd_dims* d, const wd_block_weights* w, const float
  * WD_ERR_SHAPE).  ws: wd_workspace_bytes_fp8(d, batch) bytes.  With
  * w8->f2_q NULL the FFN's second layer stays bf16 (w->f2_w): the FFN hidden
  * is then not quantised, which saves its extra pass over the largest
- * activation of the block. */
+ * activation of the block.  With w8->attention_fp8 the self-attention is the
+ * FP8 attention of [WAN] 5.3 (wd_attention_fp8_quantize + wd_attention_fp8 on
+ * the block's q, k, v). */
 size_t wd_workspace_bytes_fp8(const wd_dims* d, int batch);
 wd_status wd_block_forward_fp8(const wd_dims* d, const wd_block_weights* w, const wd_block_weights_fp8* w8,
                                const float* e0, const void* kv, int batch, float* X, void* ws, size_t ws_bytes,
@@ -354,9 +357,54 @@ wd_status wd_attention_lse(int dtype, int batch, int Lq, int heads, int dh, cons
 wd_status wd_attention_merge(int dtype, int batch, int Lq, int heads, int dh, float* o_run, float* lse_run,
                              const void* o_part, const float* lse_part, int first, void* out, wd_stream stream);
 
-/* FP8 building blocks ([WAN] 5.3: FP8 GEMM with per-token activation and
- * per-channel weight scales).  No counterpart is wired into wd_block_forward:
- * the block runs bf16; these are the next step's kernels, exposed to be
+/* FP8 attention ([WAN] 5.3, "FlashAttention3 FP8": the Q/K inner product in
+ * INT8, O = P V in FP8, accumulation across key blocks in FP32), non-causal,
+ * one key segment, head dim 128, bf16 q, k, v and output.
+ *
+ * Operands, in one device buffer laid out by wd_attention_fp8_layout (byte
+ * offsets, each 256-byte aligned; the buffer itself 256-byte aligned):
+ *   q8  int8 [batch, Lq, heads*128], one scale per (row, head): sq [batch, heads, Lq]
+ *   k8  int8 [batch, Lk, heads*128], one scale per (128-key block, head): sk [batch, heads, ceil(Lk/128)]
+ *   v8t e4m3 [batch, heads, 128, lkp] (V transposed: keys contiguous; lkp = Lk rounded up to 16,
+ *       keys Lk..lkp zero), one scale per (channel, head, batch): sv [batch, heads*128]
+ *   v_amax scratch [batch, heads*128]
+ * Scales: int8 amax/127, e4m3 amax/448 (fp32, IEEE division; 1 for an all-zero
+ * row, block or channel); codes: round to nearest even (int8 clamped to
+ * +-127; e4m3 saturating at +-448).
+ * Attention: per 128-key block, S = q8 k8^T exactly (int32), logits
+ * t = S sq sk log2(e)/sqrt(128) (log2 units), the online softmax with a lazy
+ * reference max m (moved to the block's row max only when that exceeds m by
+ * more than 8; the running O and l are then scaled by 2^(m_old - m)),
+ * p = 2^(t - m) rounded to e4m3 for O += P8 v8 (fp32 accumulation) while l
+ * sums the unrounded p; out = O sv / l rounded to bf16.  The result depends on
+ * that reference within e4m3 precision of P (the oracle follows the same
+ * blocks and rule).
+ * Errors: dh != 128 -> WD_ERR_UNSUPPORTED; empty shapes, Lq or Lk above 2^30 ->
+ * WD_ERR_SHAPE; a buffer smaller than layout.bytes -> WD_ERR_WORKSPACE;
+ * misaligned pointers or strides -> WD_ERR_ALIGN. */
+typedef struct {
+  size_t q8, sq, k8, sk, v8t, sv, v_amax;   /* byte offsets in the buffer */
+  size_t bytes;                             /* the buffer's size */
+  int64_t lkp;                              /* keys per V^T row */
+} wd_attn_fp8_layout;
+wd_status wd_attention_fp8_layout(int batch, int64_t Lq, int64_t Lk, int heads, int dh, wd_attn_fp8_layout* out);
+
+/* Quantises q [batch, Lq, heads*dh] (row stride q_rs elements; 8-byte aligned)
+ * and k, v [batch, Lk, heads*dh] (row stride kv_rs; k 8-byte, v 16-byte
+ * aligned; strides multiples of 8) into buf (two kernels and a memset, on
+ * stream).  q, k, v may be the column blocks of one fused q|k|v buffer. */
+wd_status wd_attention_fp8_quantize(int batch, int64_t Lq, int64_t Lk, int heads, int dh, const void* q, int64_t q_rs,
+                                    const void* k, const void* v, int64_t kv_rs, void* buf, size_t buf_bytes,
+                                    wd_stream stream);
+
+/* The attention on the quantised operands in buf (from
+ * wd_attention_fp8_quantize with the same shape): o [batch, Lq, heads*dh]
+ * bf16, row stride o_rs elements (16-byte aligned, a multiple of 8). */
+wd_status wd_attention_fp8(int batch, int64_t Lq, int64_t Lk, int heads, int dh, const void* buf, size_t buf_bytes,
+                           void* o, int64_t o_rs, wd_stream stream);
+
+/* FP8 GEMM building blocks ([WAN] 5.3: FP8 GEMM with per-token activation and
+ * per-channel weight scales), used by wd_block_forward_fp8 and exposed to be
  * checked and measured on their own. */
 
 /* Per-row e4m3 quantisation: for each row r of x [rows, K] (dtype WD_BF16 or

@@ -453,3 +453,99 @@ def test_attention_lse_and_merge_over_key_parts(wd, dtype, dh, Lq, n):
     vbar = np.einsum("bhmn,bnhd->bmhd", p, np.abs(va)).reshape(B, Lq, h * dh)
     bound = 2 * u_out * np.abs(want_o) + (4 * BF16_HALF_ULP if is_bf else 1e-5) * vbar + 1e-6
     assert_within(host(out), want_o, bound)
+
+
+# ------------------------------------------------------------------ FP8 attention ("Wan（通义万相）..." 5.3)
+# (batch, L, heads): ragged small cases, and the 480x832x81 block's self-attention (L = 32760, 12 heads, batch 2)
+ATTN8_CASES = [(2, 300, 2), (1, 129, 1), (2, 32760, 12)]
+
+
+def _qkv8(batch, L, heads, seed):
+    """A fused bf16 q|k|v buffer [batch, L, 3D] (host float32 copy, device bf16)
+    with per-channel spreads, so that the rows, key blocks and value channels
+    all get different scales."""
+    rng = np.random.default_rng(seed)
+    D = heads * 128
+    x = rng.standard_normal((batch, L, 3 * D), dtype=np.float32)
+    x[..., :2 * D] *= rng.uniform(0.5, 2.0, 2 * D).astype(np.float32)
+    x[..., 2 * D:] *= rng.uniform(0.2, 3.0, D).astype(np.float32)
+    x[:, : min(L, 40), :D] *= 3.0                                 # a few large rows of q
+    t = torch.from_numpy(x).to(torch.bfloat16)                      # round to nearest even, as O.bf16
+    return t.float().numpy(), t.to("cuda")
+
+
+def _attn8_run(wd, batch, L, heads, seed):
+    qh, qd = _qkv8(batch, L, heads, seed)
+    D = heads * 128
+    lay = wd.wd_attention_fp8_layout(batch, L, L, heads, 128)
+    buf = torch.empty(lay.bytes, dtype=torch.uint8, device="cuda")
+    wd.wd_attention_fp8_quantize(batch, L, L, heads, 128, qd, 3 * D, qd[..., D:], qd[..., 2 * D:], 3 * D, buf)
+    o = torch.empty((batch, L, D), dtype=torch.bfloat16, device="cuda")
+    wd.wd_attention_fp8(batch, L, L, heads, 128, buf, o, D)
+    wd.wd_check()
+    return qh, lay, buf, o
+
+
+@pytest.mark.parametrize("batch,L,heads", ATTN8_CASES)
+def test_attention_fp8_operands_bit_exact(wd, batch, L, heads):
+    """The quantised operands byte for byte against the oracle's quantisers:
+    q8 and sq per (row, head), k8 and sk per (128-key block, head), v8t (V
+    transposed, e4m3) and sv per (channel, head, batch), the padding keys of
+    v8t zero."""
+    qh, lay, buf, _ = _attn8_run(wd, batch, L, heads, seed=L + heads)
+    D, nb, lkp = heads * 128, (L + 127) // 128, lay.lkp
+    cut = lambda off, n, dt: buf[off:off + n * torch.tensor([], dtype=dt).element_size()].view(dt)
+    q8 = cut(lay.q8, batch * L * D, torch.int8).reshape(batch, L, D).cpu().numpy()
+    k8 = cut(lay.k8, batch * L * D, torch.int8).reshape(batch, L, D).cpu().numpy()
+    sq = cut(lay.sq, batch * heads * L, torch.float32).reshape(batch, heads, L).cpu().numpy()
+    sk = cut(lay.sk, batch * heads * nb, torch.float32).reshape(batch, heads, nb).cpu().numpy()
+    sv = cut(lay.sv, batch * D, torch.float32).reshape(batch, D).cpu().numpy()
+    v8 = cut(lay.v8t, batch * D * lkp, torch.float8_e4m3fn).reshape(batch, heads, 128, lkp).double().cpu().numpy()
+    for b in range(batch):
+        for h in range(heads):
+            cs = slice(h * 128, (h + 1) * 128)
+            cq, s_q = O.quant_rows_int8(qh[b, :, cs])
+            np.testing.assert_array_equal(q8[b, :, cs], cq)
+            np.testing.assert_array_equal(sq[b, h], s_q)
+            ck, s_k = O.quant_blocks_int8(qh[b, :, D:][:, cs], 128)
+            np.testing.assert_array_equal(k8[b, :, cs], ck)
+            np.testing.assert_array_equal(sk[b, h], s_k)
+            cv, s_v = O.quant_cols_e4m3(qh[b, :, 2 * D:][:, cs])
+            np.testing.assert_array_equal(v8[b, h, :, :L], cv.T)
+            np.testing.assert_array_equal(sv[b, cs], s_v)
+            assert not v8[b, h, :, L:].any()
+
+
+@pytest.mark.parametrize("batch,L,heads,n_rows", [(2, 300, 2, None), (1, 129, 1, None), (2, 32760, 12, 64)])
+def test_attention_fp8(wd, monkeypatch, batch, L, heads, n_rows):
+    """The FP8 attention against the oracle's (the same quantisers, key blocks
+    and reference rule) on every row of the small cases and on sampled rows
+    plus the ragged tail of the 480p one.  The two differ where the rounding of
+    p to e4m3 decides differently: the GPU's 2^x errs by up to 7.5e-5 (FMA
+    pipe) and its fp32 logits by a few ulp.  The bar is derived from the oracle
+    itself: twice its movement when every p is moved by 1e-4 (seeded), plus
+    the rounding of the output to bf16.  Against the exact attention of the
+    unquantised inputs the FP8 error is printed and bounded by 0.5 of the
+    output's RMS (max error / RMS)."""
+    qh, lay, buf, o = _attn8_run(wd, batch, L, heads, seed=7 * L + heads)
+    D = heads * 128
+    rows = np.arange(L)
+    if n_rows is not None:
+        rng = np.random.default_rng(L)
+        rows = np.unique(np.concatenate([rng.choice(L, n_rows, replace=False), np.arange(L - 40, L), [0, 5]]))
+    got = o.float().cpu().numpy()[:, rows].astype(np.float64).reshape(batch, len(rows), heads, 128)
+    split = lambda b: (qh[b, rows, :D].reshape(len(rows), heads, 128), qh[b, :, D:2 * D].reshape(L, heads, 128),
+                       qh[b, :, 2 * D:].reshape(L, heads, 128))
+    want = np.stack([O.attention_fp8(*split(b)) for b in range(batch)])
+    prng = np.random.default_rng(99)
+    with monkeypatch.context() as m:
+        m.setattr(O.np, "exp2", lambda a, _e=np.exp2: _e(a) * (1 + 1e-4 * prng.standard_normal(np.shape(a)))
+                  if np.ndim(a) == 2 else _e(a))
+        moved = np.stack([O.attention_fp8(*split(b)) for b in range(batch)])
+    exact = np.stack([O.attention(*split(b)) for b in range(batch)])
+    err, bar = rel(got, want), 2 * rel(moved, want) + rel(bf(want), want)
+    e_exact = rel(got, exact)
+    print(f"\n[FP8 attention b={batch} L={L} h={heads}] vs the oracle's FP8 attention {err:.3e} (bar {bar:.3e}); "
+          f"vs the exact attention {e_exact:.3e}")
+    assert err <= bar
+    assert e_exact < 0.5

@@ -49,7 +49,7 @@ def host(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def setup(mods, wl, blocks=None, fp8=False, fp8_ffn2=True):
+def setup(mods, wl, blocks=None, fp8=False, fp8_ffn2=True, fp8_attention=False):
     model, wd = mods
     d = wl.dims
     w = synth.model_weights(wl, blocks=blocks)
@@ -61,7 +61,7 @@ def setup(mods, wl, blocks=None, fp8=False, fp8_ffn2=True):
         ren = {f"blk{b}.": f"blk{j}." for j, b in enumerate(blocks)}
         wdev = {next((ren[p] + k[len(p):] for p in ren if k.startswith(p)), k): v for k, v in w.items()}
     dw = model.weights_to_device(wdev, d, "cuda")
-    net = model.DiT(d, dw, wl.batch, fp8=fp8, fp8_ffn2=fp8_ffn2)
+    net = model.DiT(d, dw, wl.batch, fp8=fp8, fp8_ffn2=fp8_ffn2, fp8_attention=fp8_attention)
     tdt = net.tdtype
     txt = np.stack([x["txt"], np.zeros_like(x["txt"])]) if wl.batch == 2 else x["txt"][None]
     if d.t2v:   # text-to-video: no CLIP context, no y
@@ -529,25 +529,33 @@ def _rms_rel(a, b):
     return float(np.sqrt(((a - b) ** 2).mean() / (b * b).mean()))
 
 
-def _oracle_moved(monkeypatch, fn, seed=17, size=1e-3):
+def _oracle_moved(monkeypatch, fn, seed=17, size=1e-3, p_size=1e-4):
     """fn() with the oracle's attention and GELU outputs multiplied by
-    (1 + size * N(0, 1)), seeded; the oracle itself is restored after."""
+    (1 + size * N(0, 1)), seeded, and the FP8 attention's probabilities p (its
+    only two-dimensional exp2) by (1 + p_size * N(0, 1)), the size of the
+    GPU's 2^x error; the oracle itself is restored after."""
     rng = np.random.default_rng(seed)
-    att, gel = O.attention, O.gelu
+    att, att8, gel = O.attention, O.attention_fp8, O.gelu
+    mv = lambda o: o * (1 + size * rng.standard_normal(np.shape(o)))
     with monkeypatch.context() as m:
-        m.setattr(O, "attention", lambda q, k, v: (lambda o: o * (1 + size * rng.standard_normal(o.shape)))(att(q, k, v)))
-        m.setattr(O, "gelu", lambda z: (lambda g: g * (1 + size * rng.standard_normal(np.shape(g))))(gel(z)))
+        m.setattr(O, "attention", lambda q, k, v: mv(att(q, k, v)))
+        m.setattr(O, "attention_fp8", lambda q, k, v: mv(att8(q, k, v)))
+        m.setattr(O, "gelu", lambda z: mv(gel(z)))
+        m.setattr(O.np, "exp2", lambda a, _e=np.exp2: _e(a) * (1 + p_size * rng.standard_normal(np.shape(a)))
+                  if np.ndim(a) == 2 else _e(a))
         return fn()
 
 
-@pytest.mark.parametrize("mode", ["all", "no-ffn2"])
+@pytest.mark.parametrize("mode", ["all", "no-ffn2", "all+attn"])
 @pytest.mark.parametrize("wl,n_rows,tau", [(synth.STACK_480P81, 192, 700.0), (synth.BLOCK_480P17, 256, 300.0)],
                          ids=lambda v: getattr(v, "name", str(v)))
 def test_block_fp8(mods, monkeypatch, wl, n_rows, tau, mode):
     """The FP8 block (all six linear layers on e4m3 operands, or all but the
-    FFN's second layer) against the oracle's FP8 block in the same mode."""
+    FFN's second layer; +attn: with the FP8 attention) against the oracle's FP8
+    block in the same mode."""
     model, wd = mods
-    net, w, x, txt, y, d = setup(mods, wl, blocks=[0], fp8=True, fp8_ffn2=mode == "all")
+    net, w, x, txt, y, d = setup(mods, wl, blocks=[0], fp8=True, fp8_ffn2=not mode.startswith("no-ffn2"),
+                                 fp8_attention=mode.endswith("+attn"))
     B, L, D = wl.batch, d.L, d.D
     x_t = np.stack([x["x0"]] * B)
     X_in = O.patch_embed(x_t, O.build_cond_y(x["img_lat"]), w["pe.w"], w["pe.b"], rnd=True)
@@ -561,7 +569,8 @@ def test_block_fp8(mods, monkeypatch, wl, n_rows, tau, mode):
     rows = np.unique(np.concatenate([rng.choice(L, n_rows, replace=False), np.arange(L - 70, L), [0]]))
     got = host(net.X)[:, rows]
     kvs = oracle_context(w, txt, x["clip"], d, True)
-    f8 = lambda: O.block_forward(X_in, e0, w, 0, kvs[0], d, rnd=True, rows=rows, fp8=True if mode == "all" else mode)
+    f8 = lambda: O.block_forward(X_in, e0, w, 0, kvs[0], d, rnd=True, rows=rows,
+                                 fp8="no-ffn2" if mode.startswith("no-ffn2") else True, attn8=mode.endswith("+attn"))
     want8, moved = f8(), _oracle_moved(monkeypatch, f8)
     want16 = O.block_forward(X_in, e0, w, 0, kvs[0], d, rnd=True, rows=rows)
     c = lambda a: a - X_in[:, rows]
