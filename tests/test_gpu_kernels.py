@@ -525,8 +525,9 @@ def test_attention_fp8(wd, monkeypatch, batch, L, heads, n_rows):
     pipe) and its fp32 logits by a few ulp.  The bar is derived from the oracle
     itself: twice its movement when every p is moved by 1e-4 (seeded), plus
     the rounding of the output to bf16.  Against the exact attention of the
-    unquantised inputs the FP8 error is printed and bounded by 0.5 of the
-    output's RMS (max error / RMS)."""
+    unquantised inputs the GPU may be no farther than the oracle's FP8
+    attention is, plus that bar (the INT8 logits of sharp rows already move the
+    oracle by 0.7-0.9 of the output's RMS on these inputs); both are printed."""
     qh, lay, buf, o = _attn8_run(wd, batch, L, heads, seed=7 * L + heads)
     D = heads * 128
     rows = np.arange(L)
@@ -544,8 +545,8 @@ def test_attention_fp8(wd, monkeypatch, batch, L, heads, n_rows):
         moved = np.stack([O.attention_fp8(*split(b)) for b in range(batch)])
     exact = np.stack([O.attention(*split(b)) for b in range(batch)])
     err, bar = rel(got, want), 2 * rel(moved, want) + rel(bf(want), want)
-    e_exact = rel(got, exact)
+    e_exact, o_exact = rel(got, exact), rel(want, exact)
     print(f"\n[FP8 attention b={batch} L={L} h={heads}] vs the oracle's FP8 attention {err:.3e} (bar {bar:.3e}); "
-          f"vs the exact attention {e_exact:.3e}")
+          f"vs the exact attention {e_exact:.3e} (the oracle's FP8 attention: {o_exact:.3e})")
     assert err <= bar
-    assert e_exact < 0.5
+    assert e_exact <= o_exact + bar
