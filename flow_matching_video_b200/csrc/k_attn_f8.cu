@@ -107,9 +107,21 @@ __device__ __forceinline__ float2 exp2_fma2_f8(float2 x) {
                      __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
+// Of every 8 exponentials, this many on the FMA pipe (even values: keys go in
+// pairs).  0: all on MUFU.  The softmax here is issue-bound (int32 -> float
+// conversion and e4m3 packing come on top of the bf16 kernel's work), so the
+// polynomial's extra instructions cost more than the MUFU time they free
+// (B200, 480p block, batch 2: 10.06 ms with 0, 11.38 ms with 2, 12.11 with 4).
 #ifndef WD_F8_EXP2_EMU_PER8
-#define WD_F8_EXP2_EMU_PER8 2   // of every 8 exponentials, this many on the FMA pipe
+#define WD_F8_EXP2_EMU_PER8 0
 #endif
+// int32 S -> float (exact either way): 1 uses the conversion instruction; 0 adds
+// the bits of 1.5 * 2^23 and subtracts 1.5 * 2^23 as a float.  The conversion
+// was faster (B200, 480p block, batch 2: 10.37 against 10.96 ms).
+#ifndef WD_F8_CVT
+#define WD_F8_CVT 1
+#endif
+constexpr float S_OFF = WD_F8_CVT ? 0.f : MAGIC_F;   // the offset the float values of S carry
 
 // e4m3 codes of two floats, x in the low byte (round to nearest even, saturating)
 __device__ __forceinline__ uint32_t e4m3x2(float x, float y) {
@@ -258,11 +270,12 @@ k_attn_f8(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, a[c]);
       tmem_wait_ld();
-      // int32 -> 1.5 * 2^23 + s as float bits (exact); masked keys -> -inf
+      // int32 -> float: 1.5 * 2^23 + s as float bits, or s itself (exact either way); masked keys -> -inf
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int k = 0; k < 32; ++k) a[c][k] += MAGIC;
+        for (int k = 0; k < 32; ++k)
+          a[c][k] = WD_F8_CVT ? __float_as_uint(__int2float_rn(static_cast<int>(a[c][k]))) : a[c][k] + MAGIC;
       if (valid < BK) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -279,7 +292,7 @@ k_attn_f8(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                                    fmax3(__uint_as_float(a[c][k]), __uint_as_float(a[c][k + 1]),
                                          __uint_as_float(a[c + 1][k])),
                                    __uint_as_float(a[c + 1][k + 1]));
-      const float mx = (fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) - MAGIC_F) * cl;
+      const float mx = (fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) - S_OFF) * cl;
       const bool grow = mx > m + RESCALE_THRESHOLD;
       const float m_new = grow ? mx : m;
       const float alpha = grow ? ex2f(m - m_new) : 1.f;
@@ -311,7 +324,8 @@ k_attn_f8(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           float e[4];
 #pragma unroll
           for (int j = 0; j < 4; j += 2) {
-            const float2 x = fsub2(make_float2(__uint_as_float(a[c][k + j]), __uint_as_float(a[c][k + j + 1])), mg2);
+            float2 x = make_float2(__uint_as_float(a[c][k + j]), __uint_as_float(a[c][k + j + 1]));
+            if (!WD_F8_CVT) x = fsub2(x, mg2);
             const float2 arg = ffma2(x, cl2, nm2);
             if (((k + j) & 7) >= 8 - WD_F8_EXP2_EMU_PER8) {
               const float2 y = exp2_fma2_f8(arg);
@@ -323,7 +337,7 @@ k_attn_f8(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             }
             rs4[((k + j) >> 1) & 3] = fadd2(rs4[((k + j) >> 1) & 3], make_float2(e[j], e[j + 1]));
           }
-          pk[k >> 2] = e4m3x2(e[0], e[1]) | (e4m3x2(e[2], e[3]) << 16);
+          pk[k >> 2] = e4m3x2(e[0], e[1]) | (e4m3x2(e[2], e[3]) << 16);   // keys k..k+3, low byte first
         }
         tmem_st8(s_addr + c * 8, pk);
         if (c == 1) {   // keys 0..63 written: release the first half of P V
@@ -392,11 +406,6 @@ struct PrepArgs {
   unsigned* v_amax;                       // [batch, heads*128], zeroed before the launch
 };
 
-__device__ __forceinline__ void load4(const bf16* src, float (&x)[4]) {
-  const uint2 u = *reinterpret_cast<const uint2*>(src);
-  const float2 a = unpack_bf16x2(u.x), c = unpack_bf16x2(u.y);
-  x[0] = a.x; x[1] = a.y; x[2] = c.x; x[3] = c.y;
-}
 __device__ __forceinline__ uint32_t i8x4(const float (&x)[4], float s) {
   uint32_t w = 0;
 #pragma unroll
@@ -409,46 +418,58 @@ __device__ __forceinline__ uint32_t i8x4(const float (&x)[4], float s) {
 
 __global__ void __launch_bounds__(256) k_attn8_prep(PrepArgs a) {
   __shared__ float red[8][128];
-  __shared__ float kmax_s;
+  __shared__ float kred[8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int D = a.heads * 128, col = h * 128 + lane * 4;
   const int64_t bh = static_cast<int64_t>(b) * a.heads + h;
-  // ---- Q: per row
+  const int r0 = tile * 128 + warp * 16;   // this warp's first row
+  // every load of the warp's 16 rows issued before any arithmetic (rows past the end read as 0)
+  uint2 uq[16], uk[16], uv[16];
+#pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const int l = tile * 128 + warp * 16 + i;
-    if (l >= a.Lq) break;
+    const int l = r0 + i;
+    uq[i] = l < a.Lq ? *reinterpret_cast<const uint2*>(a.q + (static_cast<int64_t>(b) * a.Lq + l) * a.q_rs + col)
+                     : make_uint2(0u, 0u);
+    const int64_t off = (static_cast<int64_t>(b) * a.Lk + l) * a.kv_rs + col;
+    uk[i] = l < a.Lk ? *reinterpret_cast<const uint2*>(a.k + off) : make_uint2(0u, 0u);
+    uv[i] = l < a.Lk ? *reinterpret_cast<const uint2*>(a.v + off) : make_uint2(0u, 0u);
+  }
+  auto unpack = [](uint2 u, float (&x)[4]) {
+    const float2 p0 = unpack_bf16x2(u.x), p1 = unpack_bf16x2(u.y);
+    x[0] = p0.x; x[1] = p0.y; x[2] = p1.x; x[3] = p1.y;
+  };
+  // ---- Q: one scale per row
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int l = r0 + i;
     float x[4];
-    load4(a.q + (static_cast<int64_t>(b) * a.Lq + l) * a.q_rs + col, x);
+    unpack(uq[i], x);
     float am = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
     const float s = am > 0.f ? __fdiv_rn(am, 127.f) : 1.f;
-    *reinterpret_cast<uint32_t*>(a.q8 + (static_cast<int64_t>(b) * a.Lq + l) * D + col) = i8x4(x, s);
-    if (lane == 0) a.sq[bh * a.Lq + l] = s;
+    if (l < a.Lq) {
+      *reinterpret_cast<uint32_t*>(a.q8 + (static_cast<int64_t>(b) * a.Lq + l) * D + col) = i8x4(x, s);
+      if (lane == 0) a.sq[bh * a.Lq + l] = s;
+    }
   }
-  // ---- K (one scale for the tile) and V (per-channel maxima)
-  if (tile * 128 >= a.Lk) return;                        // CTA-uniform
-  float kx[16][4], vm[4] = {0.f, 0.f, 0.f, 0.f}, km = 0.f;
+  if (tile * 128 >= a.Lk) return;                        // CTA-uniform: no keys in this tile
+  // ---- K (one scale for the tile's 128 keys) and V (per-channel maxima over the tile)
+  float km = 0.f, vm[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const int l = tile * 128 + warp * 16 + i;
-    if (l < a.Lk) {
-      const int64_t off = (static_cast<int64_t>(b) * a.Lk + l) * a.kv_rs + col;
-      load4(a.k + off, kx[i]);
-      float vx[4];
-      load4(a.v + off, vx);
+    float x[4], y[4];
+    unpack(uk[i], x);
+    unpack(uv[i], y);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) { km = fmaxf(km, fabsf(kx[i][j])); vm[j] = fmaxf(vm[j], fabsf(vx[j])); }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) kx[i][j] = 0.f;
-    }
+    for (int j = 0; j < 4; ++j) { km = fmaxf(km, fabsf(x[j])); vm[j] = fmaxf(vm[j], fabsf(y[j])); }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) km = fmaxf(km, __shfl_xor_sync(0xffffffffu, km, o));
 #pragma unroll
   for (int j = 0; j < 4; ++j) red[warp][lane * 4 + j] = vm[j];
+  if (lane == 0) kred[warp] = km;
   __syncthreads();
   if (threadIdx.x < 128) {
     float m = 0.f;
@@ -456,22 +477,17 @@ __global__ void __launch_bounds__(256) k_attn8_prep(PrepArgs a) {
     for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w][threadIdx.x]);
     atomicMax(&a.v_amax[static_cast<int64_t>(b) * D + h * 128 + threadIdx.x], __float_as_uint(m));
   }
-  __syncthreads();
-  if (lane == 0) red[0][warp] = km;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float m = 0.f;
-    for (int w = 0; w < 8; ++w) m = fmaxf(m, red[0][w]);
-    kmax_s = m;
-  }
-  __syncthreads();
-  const float km_all = kmax_s;
+  float km_all = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) km_all = fmaxf(km_all, kred[w]);
   const float s = km_all > 0.f ? __fdiv_rn(km_all, 127.f) : 1.f;
   if (threadIdx.x == 0) a.sk[bh * a.nb + tile] = s;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const int l = tile * 128 + warp * 16 + i;
-    if (l < a.Lk) *reinterpret_cast<uint32_t*>(a.k8 + (static_cast<int64_t>(b) * a.Lk + l) * D + col) = i8x4(kx[i], s);
+    const int l = r0 + i;
+    float x[4];
+    unpack(uk[i], x);
+    if (l < a.Lk) *reinterpret_cast<uint32_t*>(a.k8 + (static_cast<int64_t>(b) * a.Lk + l) * D + col) = i8x4(x, s);
   }
 }
 
@@ -499,28 +515,27 @@ __global__ void __launch_bounds__(256) k_attn8_vt(VtArgs a) {
     if (tile == 0) a.sv[static_cast<int64_t>(b) * D + h * 128 + threadIdx.x] = s;
   }
   __syncthreads();
-  // thread -> key r = tid & 127, channels 64 g .. 64 g + 63
+  // thread -> key r = tid & 127, channels 64 g .. 64 g + 63: all eight 16-byte loads first
   const int r = threadIdx.x & 127, g = threadIdx.x >> 7;
   const int l = tile * 128 + r;
-  for (int c = 0; c < 64; c += 8) {
-    const int d = g * 64 + c;
-    uint8_t codes[8];
-    if (l < a.Lk) {
-      const uint4 u = *reinterpret_cast<const uint4*>(a.v + (static_cast<int64_t>(b) * a.Lk + l) * a.kv_rs + h * 128 + d);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  uint4 u[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = unpack_bf16x2(w[j]);
-        codes[2 * j] = static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(f.x, sc[d + 2 * j]), __NV_SATFINITE, __NV_E4M3));
-        codes[2 * j + 1] =
-            static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(f.y, sc[d + 2 * j + 1]), __NV_SATFINITE, __NV_E4M3));
-      }
-    } else {
+  for (int c = 0; c < 8; ++c)
+    u[c] = l < a.Lk ? *reinterpret_cast<const uint4*>(a.v + (static_cast<int64_t>(b) * a.Lk + l) * a.kv_rs + h * 128 +
+                                                      g * 64 + c * 8)
+                    : make_uint4(0u, 0u, 0u, 0u);   // keys past the end: code 0
 #pragma unroll
-      for (int j = 0; j < 8; ++j) codes[j] = 0;
+  for (int c = 0; c < 8; ++c) {
+    const int d = g * 64 + c * 8;
+    const uint32_t w[4] = {u[c].x, u[c].y, u[c].z, u[c].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = unpack_bf16x2(w[j]);
+      tile_t[d + 2 * j][r] =
+          static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(f.x, sc[d + 2 * j]), __NV_SATFINITE, __NV_E4M3));
+      tile_t[d + 2 * j + 1][r] =
+          static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(f.y, sc[d + 2 * j + 1]), __NV_SATFINITE, __NV_E4M3));
     }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) tile_t[d + j][r] = codes[j];
   }
   __syncthreads();
   // rows of 128 keys (the last tile: up to lkp, a multiple of 16), 16 bytes per store

@@ -28,6 +28,16 @@ constexpr int BM = 128, BK = 64;
 // the MMAs of a tile), one otherwise.
 template <int MODE> __host__ __device__ constexpr int epi_wg() { return MODE == EPI_GELU ? 2 : 1; }
 template <int MODE> __host__ __device__ constexpr int threads() { return 64 + 128 * epi_wg<MODE>(); }
+// Epilogues with a 2-byte output go out through TMA stores: each epilogue warp
+// packs 32 rows x 64 columns (one 128-byte row per output row) into a
+// 128-byte-swizzled staging tile and one lane stores the box, so global memory
+// sees whole 128-byte rows instead of 16-byte pieces of 32 rows.  Staging
+// buffers per warp: two with one epilogue warpgroup, one with two.
+template <int MODE> __host__ __device__ constexpr bool staged2() {
+  return MODE == EPI_STORE || MODE == EPI_GELU || MODE == EPI_STORE_F16;
+}
+template <int MODE> __host__ __device__ constexpr int stg_bufs() { return epi_wg<MODE>() == 1 ? 2 : 1; }
+constexpr int STG2_TILE = 32 * 128;   // bytes of one staging tile: 32 rows x 64 two-byte columns
 
 template <int BN>
 struct Cfg {
@@ -40,8 +50,14 @@ struct Cfg {
   // gated residual: per epilogue warp two 32 x 32 fp32 staging tiles for the TMA reduce-add
   static constexpr int RESID_STAGE_BYTES = 32 * 32 * 4;
   static constexpr int STG_BYTES = 4 * 2 * RESID_STAGE_BYTES;
-  static constexpr int smem(int mode) { return 1024 + STAGES * STAGE_BYTES + (mode == EPI_RESID ? STG_BYTES : 0) + BAR_BYTES; }
+  // staging bytes in front of the barriers: the residual tiles, or the 2-byte store tiles (32 KB either way)
+  __host__ __device__ static constexpr int stg(int mode) {
+    return mode == EPI_RESID ? STG_BYTES
+                             : ((mode == EPI_STORE || mode == EPI_GELU || mode == EPI_STORE_F16) ? 8 * STG2_TILE : 0);
+  }
+  static constexpr int smem(int mode) { return 1024 + STAGES * STAGE_BYTES + stg(mode) + BAR_BYTES; }
   static_assert(1024 + STAGES * STAGE_BYTES + STG_BYTES + BAR_BYTES <= 232448, "shared memory budget of one CTA exceeded");
+  static_assert(8 * STG2_TILE <= STG_BYTES, "2-byte staging within the residual staging budget");
   static constexpr uint32_t IDESC = idesc_bf16(BM, BN, 0, 0);
   static constexpr uint32_t IDESC_F8 = idesc_e4m3(BM, BN, 0, 0);
 };
@@ -51,13 +67,13 @@ enum : unsigned { SITE_EMPTY = 0x101, SITE_FULL = 0x102, SITE_TFULL = 0x103, SIT
 
 // ------------------------------------------------------------------ epilogue on 32 columns
 // One thread = one output row m; columns n .. n+31 come from the accumulator.
+// The values before the store: FP8 scales (row scale sm = sa[m], passed in so
+// that rows past M need not read it), bias, GELU.
 template <int MODE>
-__device__ __forceinline__ void epilogue32(const Epi& ep, int64_t m, int n, const uint32_t (&r)[32]) {
-  float v[32];
+__device__ __forceinline__ void epi_values32(const Epi& ep, float sm, int n, const uint32_t (&r)[32], float (&v)[32]) {
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
   if (ep.sa) {   // FP8 operands: acc * (sa[m] * sb[n])
-    const float sm = ep.sa[m];
 #pragma unroll
     for (int j = 0; j < 32; j += 4) {
       const float4 b = __ldg(reinterpret_cast<const float4*>(ep.sb + n + j));
@@ -71,11 +87,25 @@ __device__ __forceinline__ void epilogue32(const Epi& ep, int64_t m, int n, cons
       v[j] += b.x; v[j + 1] += b.y; v[j + 2] += b.z; v[j + 3] += b.w;
     }
   }
-  if constexpr (MODE == EPI_STORE || MODE == EPI_GELU) {
-    if constexpr (MODE == EPI_GELU) {
+  if constexpr (MODE == EPI_GELU) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
-    }
+    for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+  }
+}
+// 8 values packed as 2-byte elements of the epilogue's output type
+template <int MODE>
+__device__ __forceinline__ uint4 pack8(const float* v) {
+  if constexpr (MODE == EPI_STORE_F16)
+    return make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]), pack_f16x2(v[6], v[7]));
+  else
+    return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+
+template <int MODE>
+__device__ __forceinline__ void epilogue32(const Epi& ep, int64_t m, int n, const uint32_t (&r)[32]) {
+  float v[32];
+  epi_values32<MODE>(ep, ep.sa ? ep.sa[m] : 0.f, n, r, v);
+  if constexpr (MODE == EPI_STORE || MODE == EPI_GELU) {
     uint4* dst = reinterpret_cast<uint4*>(static_cast<bf16*>(ep.out) + m * ep.ldo + n);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -111,7 +141,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::STAGES * C::A_BYTES;
   float* stg = reinterpret_cast<float*>(sB + C::STAGES * C::B_BYTES);   // 1024-byte aligned
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES + (MODE == EPI_RESID ? C::STG_BYTES : 0));
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES + C::stg(MODE));
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;   // [2]
   uint64_t* tempty = tfull + 2;          // [2]
@@ -257,6 +287,37 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           }
           ++chunk;
         }
+      } else if constexpr (staged2<MODE>() && COLS % 64 == 0) {
+        // 64 columns at a time: values packed into this warp's staging tile
+        // (row `lane`, 16-byte chunk j at chunk j ^ (lane & 7)), then one lane
+        // stores the 32 x 64 box; rows past M inside the box are clipped by the TMA.
+        constexpr int NB = stg_bufs<MODE>();
+        const float sm = (ep.sa && m < M) ? ep.sa[m] : 0.f;
+#pragma unroll 1
+        for (int c = c_begin; c < c_begin + COLS; c += 64) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tbase + c, r0);
+          tmem_ld32(tbase + c + 32, r1);
+          uint8_t* tile = reinterpret_cast<uint8_t*>(stg) + ((warp - 2) * NB + (chunk % NB)) * STG2_TILE;
+          if (lane == 0) bulk_wait_group_read<NB - 1>();   // the store that last read this tile is done with it
+          __syncwarp();
+          tmem_wait_ld();
+          uint4* row = reinterpret_cast<uint4*>(tile + lane * 128);
+          float v[32];
+          epi_values32<MODE>(ep, sm, n0 + c, r0, v);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) row[j ^ (lane & 7)] = pack8<MODE>(v + 8 * j);
+          epi_values32<MODE>(ep, sm, n0 + c + 32, r1, v);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) row[(4 + j) ^ (lane & 7)] = pack8<MODE>(v + 8 * j);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && m0 + q * 32 < M) {
+            tma_store_2d(tile, &tmX, n0 + c, m0 + q * 32);
+            bulk_commit_group();
+          }
+          ++chunk;
+        }
       } else {
 #pragma unroll 1
         for (int c = c_begin; c < c_begin + COLS; c += 32) {
@@ -271,7 +332,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       if (lane == 0) mbar_arrive(&tempty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
-    if (MODE == EPI_RESID && lane == 0) bulk_wait_group<0>();   // reductions performed before exit
+    if ((MODE == EPI_RESID || (staged2<MODE>() && COLS % 64 == 0)) && lane == 0)
+      bulk_wait_group<0>();   // reductions and stores performed before exit
   }
 
   tc_fence_before();
@@ -339,6 +401,22 @@ static wd_status make_tmap_f32(CUtensorMap* m, const void* base, int64_t rows, i
   return WD_OK;
 }
 
+// 2D tensor map over a 2-byte output [rows, cols] (bf16, or IEEE half), row
+// stride ld elements; box 64 x 32 (one 128-byte row per box row), 128-byte swizzle.
+static wd_status make_tmap_2b(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld, bool half) {
+  auto fn = encode_fn();
+  if (!fn) { set_error("cuTensorMapEncodeTiled unavailable"); return WD_ERR_CUDA; }
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, half ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) { set_error("cuTensorMapEncodeTiled (2-byte out) failed (%d)", static_cast<int>(r)); return WD_ERR_CUDA; }
+  return WD_OK;
+}
+
 template <int BN, int MODE, bool F8 = false>
 static wd_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const Epi& ep, int M, int N, int K,
                            cudaStream_t st) {
@@ -352,8 +430,10 @@ static wd_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const E
   }
   const int tiles = ((M + tcg::BM - 1) / tcg::BM) * (N / BN);
   const int grid = tiles < sm_count() ? tiles : sm_count();
-  CUtensorMap tx = ta;   // unused unless the epilogue adds into the fp32 residual
+  CUtensorMap tx = ta;   // the residual (fp32) or 2-byte output map of the TMA epilogues, else unused
   if (MODE == EPI_RESID) WD_TRY(make_tmap_f32(&tx, ep.out, M, N, ep.ldo, 32, 32));
+  if (tcg::staged2<MODE>() && (BN / tcg::epi_wg<MODE>()) % 64 == 0)
+    WD_TRY(make_tmap_2b(&tx, ep.out, M, N, ep.ldo, MODE == EPI_STORE_F16));
   Trace tr(KC_GEMM, st);
   tcg::k_gemm_tc<BN, MODE, F8><<<grid, tcg::threads<MODE>(), C::smem(MODE), st>>>(ta, tb, tx, ep, M, N, K);
   return launch_status("gemm_tc");

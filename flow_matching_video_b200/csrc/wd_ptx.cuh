@@ -153,6 +153,14 @@ __device__ __forceinline__ void tma_reduce_add_2d(const void* src, const CUtenso
                "r"(smem_u32(src)), "r"(c0), "r"(c1)
                : "memory");
 }
+// Tiled TMA store of a shared-memory box into global memory (bulk group; the
+// coordinates must not be negative, the innermost one 16-byte aligned).
+__device__ __forceinline__ void tma_store_2d(const void* src, const CUtensorMap* tm, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tm)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until at most N of this thread's bulk groups still read their shared-memory source.
 template <int N>
