@@ -406,17 +406,21 @@ struct PrepArgs {
   unsigned* v_amax;                       // [batch, heads*128], zeroed before the launch
 };
 
+// Four int8 codes round-half-even(x / s), x[0] in the low byte.  The rounding to
+// an integer adds 1.5 * 2^23 (exact round-to-nearest-even for |y| < 2^22; here
+// |x / s| <= 127), which keeps it off the conversion unit.
 __device__ __forceinline__ uint32_t i8x4(const float (&x)[4], float s) {
   uint32_t w = 0;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const int c = max(-127, min(127, __float2int_rn(__fdiv_rn(x[j], s))));
+    const float y = __fdiv_rn(x[j], s);
+    const int c = max(-127, min(127, __float_as_int(__fadd_rn(y, MAGIC_F)) - static_cast<int>(MAGIC)));
     w |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * j);
   }
   return w;
 }
 
-__global__ void __launch_bounds__(256) k_attn8_prep(PrepArgs a) {
+__global__ void __launch_bounds__(256, 2) k_attn8_prep(PrepArgs a) {
   __shared__ float red[8][128];
   __shared__ float kred[8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -424,16 +428,13 @@ __global__ void __launch_bounds__(256) k_attn8_prep(PrepArgs a) {
   const int D = a.heads * 128, col = h * 128 + lane * 4;
   const int64_t bh = static_cast<int64_t>(b) * a.heads + h;
   const int r0 = tile * 128 + warp * 16;   // this warp's first row
-  // every load of the warp's 16 rows issued before any arithmetic (rows past the end read as 0)
-  uint2 uq[16], uk[16], uv[16];
+  // each phase issues all its loads of the warp's 16 rows before any arithmetic (rows past the end read as 0)
+  uint2 uq[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int l = r0 + i;
     uq[i] = l < a.Lq ? *reinterpret_cast<const uint2*>(a.q + (static_cast<int64_t>(b) * a.Lq + l) * a.q_rs + col)
                      : make_uint2(0u, 0u);
-    const int64_t off = (static_cast<int64_t>(b) * a.Lk + l) * a.kv_rs + col;
-    uk[i] = l < a.Lk ? *reinterpret_cast<const uint2*>(a.k + off) : make_uint2(0u, 0u);
-    uv[i] = l < a.Lk ? *reinterpret_cast<const uint2*>(a.v + off) : make_uint2(0u, 0u);
   }
   auto unpack = [](uint2 u, float (&x)[4]) {
     const float2 p0 = unpack_bf16x2(u.x), p1 = unpack_bf16x2(u.y);
@@ -456,6 +457,14 @@ __global__ void __launch_bounds__(256) k_attn8_prep(PrepArgs a) {
   }
   if (tile * 128 >= a.Lk) return;                        // CTA-uniform: no keys in this tile
   // ---- K (one scale for the tile's 128 keys) and V (per-channel maxima over the tile)
+  uint2 uk[16], uv[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int l = r0 + i;
+    const int64_t off = (static_cast<int64_t>(b) * a.Lk + l) * a.kv_rs + col;
+    uk[i] = l < a.Lk ? *reinterpret_cast<const uint2*>(a.k + off) : make_uint2(0u, 0u);
+    uv[i] = l < a.Lk ? *reinterpret_cast<const uint2*>(a.v + off) : make_uint2(0u, 0u);
+  }
   float km = 0.f, vm[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
@@ -515,27 +524,29 @@ __global__ void __launch_bounds__(256) k_attn8_vt(VtArgs a) {
     if (tile == 0) a.sv[static_cast<int64_t>(b) * D + h * 128 + threadIdx.x] = s;
   }
   __syncthreads();
-  // thread -> key r = tid & 127, channels 64 g .. 64 g + 63: all eight 16-byte loads first
-  const int r = threadIdx.x & 127, g = threadIdx.x >> 7;
-  const int l = tile * 128 + r;
-  uint4 u[8];
+  // thread -> keys 4 kq .. 4 kq + 3, channels 16 cg .. 16 cg + 15 (one 32-byte sector of each row):
+  // all loads first, then one 32-bit word of four keys' codes per channel into the transposed tile
+  const int kq = threadIdx.x & 31, cg = threadIdx.x >> 5;
+  uint4 u[4][2];
 #pragma unroll
-  for (int c = 0; c < 8; ++c)
-    u[c] = l < a.Lk ? *reinterpret_cast<const uint4*>(a.v + (static_cast<int64_t>(b) * a.Lk + l) * a.kv_rs + h * 128 +
-                                                      g * 64 + c * 8)
-                    : make_uint4(0u, 0u, 0u, 0u);   // keys past the end: code 0
+  for (int i = 0; i < 4; ++i) {
+    const int l = tile * 128 + 4 * kq + i;
+    const bf16* src = a.v + (static_cast<int64_t>(b) * a.Lk + l) * a.kv_rs + h * 128 + 16 * cg;
+    u[i][0] = l < a.Lk ? *reinterpret_cast<const uint4*>(src) : make_uint4(0u, 0u, 0u, 0u);   // keys past the end: 0
+    u[i][1] = l < a.Lk ? *reinterpret_cast<const uint4*>(src + 8) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  auto val = [&](int i, int c) {   // key 4 kq + i, channel 16 cg + c
+    const uint4 q = u[i][c >> 3];
+    const uint32_t w = ((c & 7) >> 1) == 0 ? q.x : ((c & 7) >> 1) == 1 ? q.y : ((c & 7) >> 1) == 2 ? q.z : q.w;
+    const float2 f = unpack_bf16x2(w);
+    return (c & 1) ? f.y : f.x;
+  };
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const int d = g * 64 + c * 8;
-    const uint32_t w[4] = {u[c].x, u[c].y, u[c].z, u[c].w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = unpack_bf16x2(w[j]);
-      tile_t[d + 2 * j][r] =
-          static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(f.x, sc[d + 2 * j]), __NV_SATFINITE, __NV_E4M3));
-      tile_t[d + 2 * j + 1][r] =
-          static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(f.y, sc[d + 2 * j + 1]), __NV_SATFINITE, __NV_E4M3));
-    }
+  for (int c = 0; c < 16; ++c) {
+    const float s = sc[16 * cg + c];
+    const uint32_t lo = e4m3x2(__fdiv_rn(val(0, c), s), __fdiv_rn(val(1, c), s));
+    const uint32_t hi = e4m3x2(__fdiv_rn(val(2, c), s), __fdiv_rn(val(3, c), s));
+    *reinterpret_cast<uint32_t*>(&tile_t[16 * cg + c][4 * kq]) = lo | (hi << 16);
   }
   __syncthreads();
   // rows of 128 keys (the last tile: up to lkp, a multiple of 16), 16 bytes per store
