@@ -45,6 +45,14 @@ constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
 #define WD_ATTN_P_PARTS 2   // releases of a block's P to its P V (one softmax warp per lane quarter): 1, 2 or 4
 #endif
 
+#ifndef WD_ATTN_ILP
+#define WD_ATTN_ILP 1   // 1: row max and row sum over four independent chains (shorter dependency chains)
+#endif
+
+#ifndef WD_ATTN_SPEC
+#define WD_ATTN_SPEC 0   // 1: no separate row-max pass before the exponentials (speculative reference)
+#endif
+
 #ifndef WD_ATTN_ISSUERS
 #define WD_ATTN_ISSUERS 1   // MMA issuing threads of the self-attention (1, or 2: one per Q tile)
 #endif
@@ -72,6 +80,8 @@ struct Cfg {
   static constexpr int PP = SPLIT == 1 ? WD_ATTN_P_PARTS : 1;
   static_assert(PP == 1 || PP == 2 || PP == 4, "P released in 1, 2 or 4 parts");
   static constexpr int PPB = PP > 1 ? PP - 1 : 1;   // barriers for the parts before the last
+  // speculative softmax (see the softmax warps): one thread per row, P released in at most two parts
+  static constexpr bool SPEC = WD_ATTN_SPEC && SPLIT == 1 && PP <= 2 && WD_ATTN_ILP;
   // MMA issuing threads: one for all tiles, or (two tiles of one segment) one per tile,
   // so that one issuer's waits overlap the other's MMAs
   static constexpr int ISSUERS = (NSEG == 1 && NQ == 2) ? WD_ATTN_ISSUERS : 1;
@@ -176,9 +186,6 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 
 #ifndef WD_EXP2_EMU_PER8
 #define WD_EXP2_EMU_PER8 2   // of every 8 exponentials, this many run on the FMA pipe
-#endif
-#ifndef WD_ATTN_ILP
-#define WD_ATTN_ILP 1   // 1: row max and row sum over four independent chains (shorter dependency chains)
 #endif
 
 template <int NQ, int NSEG, typename TI, int BK>
@@ -413,6 +420,104 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           for (int k = 0; k < 32; ++k)
             if (c * 32 + k >= valid) a[c][k] = __float_as_uint(-INFINITY);
       }
+      // exponentials of 16-key chunk c against the reference -nm2, packed into TMEM over this
+      // warp's own S columns (chunk c -> 8 columns at 8c), summed into rs4 / rs2
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+      auto emit = [&](int c, float2 nm2, float2 (&rs4)[4], float2& rs2) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int k = 0; k < 16; k += 2) {
+          const int kk = (c & 1) * 16 + k;
+          const float2 arg = ffma2(make_float2(__uint_as_float(a[c >> 1][kk]), __uint_as_float(a[c >> 1][kk + 1])),
+                                   sc2, nm2);
+          float e0, e1;
+          if (WD_EXP2_PACKED && (k & 7) >= 8 - WD_EXP2_EMU_PER8 && ((k + 1) & 7) >= 8 - WD_EXP2_EMU_PER8) {
+            const float2 e = exp2_fma2(arg);
+            e0 = e.x;
+            e1 = e.y;
+          } else {
+            e0 = ((k & 7) >= 8 - WD_EXP2_EMU_PER8) ? exp2_fma(arg.x) : ex2(arg.x);
+            e1 = (((k + 1) & 7) >= 8 - WD_EXP2_EMU_PER8) ? exp2_fma(arg.y) : ex2(arg.y);
+          }
+          if constexpr (WD_ATTN_ILP) rs4[(k >> 1) & 3] = fadd2(rs4[(k >> 1) & 3], make_float2(e0, e1));
+          else rs2 = fadd2(rs2, make_float2(e0, e1));
+          pk[k >> 1] = C::HALF ? pack_f16x2(e0, e1) : pack_bf16x2(e0, e1);
+        }
+        tmem_st8(s_addr + c * 8, pk);
+      };
+      // O_t *= alpha on this warp's output columns for rows whose reference max moved,
+      // before any of this block's P V can start.  With one S buffer per tile, P V of
+      // the previous block has completed (its commit precedes the S commit waited on);
+      // with two, S of this block was issued before that P V, so wait for it.
+      auto rescale_o = [&](float alpha) -> bool {
+        if (C::DB && !mbar_wait_warp(&pv_done[C::buf(t, n - 1)], C::par(n - 1), SITE_O)) return false;
+        if (C::DB) tc_fence_after();
+        const uint32_t o_addr = tmem + lane_base + C::o_col(t, sg) + hc * OCOLS;
+#pragma unroll 1
+        for (int c = 0; c < OCH; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_addr + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_st32(o_addr + c * 32, o);
+        }
+        tmem_wait_st();
+        return true;
+      };
+      if constexpr (C::SPEC) {
+        if (!first) {
+          // Speculative pass: the first half's exponentials run against the current
+          // reference m while the row maximum is taken beside them (no pass before).
+          // The maximum is checked before that half's P is released; if a row's grew
+          // past the threshold, the warp moves those rows' reference, rescales O and
+          // redoes the half, so P, l and O end as with the maximum taken first.
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int c = 0; c < CH; c += 2)
+#pragma unroll
+            for (int k = 0; k < 32; k += 2)
+              m4[(k >> 1) & 3] = fmax3(m4[(k >> 1) & 3],
+                                       fmax3(__uint_as_float(a[c][k]), __uint_as_float(a[c][k + 1]),
+                                             __uint_as_float(a[c + 1][k])),
+                                       __uint_as_float(a[c + 1][k + 1]));
+          float2 rs2s = make_float2(0.f, 0.f);
+          float2 rs4s[4] = {rs2s, rs2s, rs2s, rs2s};
+          float2 nm2 = make_float2(-m, -m);
+#pragma unroll
+          for (int c = 0; c < CH; ++c) emit(c, nm2, rs4s, rs2s);
+          const float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * p.scale_log2;
+          const bool grow = mx > m + RESCALE_THRESHOLD;
+          float alpha = 1.f;
+          if (__any_sync(0xffffffffu, grow)) {
+            const float m_new = grow ? mx : m;
+            alpha = grow ? ex2(m - m_new) : 1.f;
+            m = m_new;
+            tmem_wait_st();   // the first half's stores land before they are rewritten
+            if (!rescale_o(alpha)) { ok = false; break; }
+            nm2 = make_float2(-m, -m);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) rs4s[j] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < CH; ++c) emit(c, nm2, rs4s, rs2s);
+          }
+          if constexpr (C::PP == 2) {   // the first half of P is written: release its P V
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_part[bi * C::PPB]);
+          }
+#pragma unroll
+          for (int c = CH; c < 2 * CH; ++c) emit(c, nm2, rs4s, rs2s);
+          tmem_wait_st();
+          const float2 rsum = fadd2(fadd2(rs4s[0], rs4s[1]), fadd2(rs4s[2], rs4s[3]));
+          l = l * alpha + (rsum.x + rsum.y);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[bi]);
+          continue;
+        }
+      }
       float mx = -INFINITY;
       if constexpr (WD_ATTN_ILP) {
         // four chains, each over every fourth pair of columns, then combined
@@ -449,54 +554,16 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       const float alpha = grow ? ex2(m - m_new) : 1.f;
       m = m_new;
       const float neg_m = -m;
-      // O_t *= alpha on this warp's output columns for rows whose reference
-      // max moved, before any of this block's P V can start.  With one S
-      // buffer per tile, P V of the previous block has completed (its commit
-      // precedes the S commit waited on above); with two, S of this block was
-      // issued before that P V, so wait for it.
-      if (__any_sync(0xffffffffu, grow) && !first) {
-        if (C::DB && !mbar_wait_warp(&pv_done[C::buf(t, n - 1)], C::par(n - 1), SITE_O)) { ok = false; break; }
-        if (C::DB) tc_fence_after();
-        const uint32_t o_addr = tmem + lane_base + C::o_col(t, sg) + hc * OCOLS;
-#pragma unroll 1
-        for (int c = 0; c < OCH; ++c) {
-          uint32_t o[32];
-          tmem_ld32(o_addr + c * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st32(o_addr + c * 32, o);
-        }
-        tmem_wait_st();
-      }
+      if (__any_sync(0xffffffffu, grow) && !first && !rescale_o(alpha)) { ok = false; break; }
       // P = exp2(s * scale - m) as packed pairs (operand type) into TMEM over this warp's
       // own S columns: chunk c of 16 keys -> 8 columns at 8c (masked keys hold
       // -inf, so their exponential is 0)
       float2 rs2 = make_float2(0.f, 0.f);
       [[maybe_unused]] float2 rs4[4] = {rs2, rs2, rs2, rs2};   // four partial sums (WD_ATTN_ILP)
-      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(neg_m, neg_m);
+      const float2 nm2 = make_float2(neg_m, neg_m);
 #pragma unroll
       for (int c = 0; c < 2 * CH; ++c) {
-        uint32_t pk[8];
-#pragma unroll
-        for (int k = 0; k < 16; k += 2) {
-          const int kk = (c & 1) * 16 + k;
-          const float2 arg = ffma2(make_float2(__uint_as_float(a[c >> 1][kk]), __uint_as_float(a[c >> 1][kk + 1])),
-                                   sc2, nm2);
-          float e0, e1;
-          if (WD_EXP2_PACKED && (k & 7) >= 8 - WD_EXP2_EMU_PER8 && ((k + 1) & 7) >= 8 - WD_EXP2_EMU_PER8) {
-            const float2 e = exp2_fma2(arg);
-            e0 = e.x;
-            e1 = e.y;
-          } else {
-            e0 = ((k & 7) >= 8 - WD_EXP2_EMU_PER8) ? exp2_fma(arg.x) : ex2(arg.x);
-            e1 = (((k + 1) & 7) >= 8 - WD_EXP2_EMU_PER8) ? exp2_fma(arg.y) : ex2(arg.y);
-          }
-          if constexpr (WD_ATTN_ILP) rs4[(k >> 1) & 3] = fadd2(rs4[(k >> 1) & 3], make_float2(e0, e1));
-          else rs2 = fadd2(rs2, make_float2(e0, e1));
-          pk[k >> 1] = C::HALF ? pack_f16x2(e0, e1) : pack_bf16x2(e0, e1);
-        }
-        tmem_st8(s_addr + c * 8, pk);
+        emit(c, nm2, rs4, rs2);
         if constexpr (C::PP > 1) {   // a part of the block's P is written: release its P V
           constexpr int per = 2 * CH / C::PP;   // 16-key chunks per part
           if ((c + 1) % per == 0 && c + 1 < 2 * CH) {
