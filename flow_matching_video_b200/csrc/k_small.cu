@@ -457,11 +457,76 @@ __global__ void __launch_bounds__(256) k_quant_rows_e4m3(const T* __restrict__ x
   if (lane == 0) scale[row] = s;
 }
 
+// The same quantisation for bf16 rows read once: the row stays in registers
+// between its maximum and its codes.  WPR warps per row (1 for K <= 2048, 8 for
+// K <= 16384; their maxima meet in shared memory), 256 threads per block, each
+// thread holding up to 8 chunks of 8 consecutive elements.
+template <int WPR>
+__global__ void __launch_bounds__(256) k_quant_rows_e4m3_reg(const bf16* __restrict__ x, int rows, int K,
+                                                              uint8_t* __restrict__ q, float* __restrict__ scale) {
+  constexpr int NV = 8, TPR = 32 * WPR, RPB = 8 / WPR;
+  __shared__ float red[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rib = warp / WPR, tir = (warp % WPR) * 32 + lane;   // row in block, thread in row
+  const int row = blockIdx.x * RPB + rib;
+  const bool live = row < rows;
+  const bf16* xr = x + static_cast<int64_t>(live ? row : 0) * K;
+  uint4 u[NV];
+  float amax = 0.f;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int k = (j * TPR + tir) * 8;
+    u[j] = (live && k < K) ? *reinterpret_cast<const uint4*>(xr + k) : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t w[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = unpack_bf16x2(w[i]);
+      amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  if constexpr (WPR > 1) {
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < WPR; ++w) amax = fmaxf(amax, red[rib * WPR + w]);
+  }
+  const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+  uint8_t* qr = q + static_cast<int64_t>(live ? row : 0) * K;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int k = (j * TPR + tir) * 8;
+    if (!live || k >= K) continue;
+    const uint32_t w[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+    uint32_t c[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = unpack_bf16x2(w[i]);
+      const uint32_t pair = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(
+          make_float2(__fdiv_rn(f.x, s), __fdiv_rn(f.y, s)), __NV_SATFINITE, __NV_E4M3));   // f.x in the low byte
+      c[i >> 1] |= pair << (16 * (i & 1));
+    }
+    *reinterpret_cast<uint2*>(qr + k) = make_uint2(c[0], c[1]);
+  }
+  if (live && tir == 0) scale[row] = s;
+}
+
 template <typename T>
 wd_status quant_rows_e4m3(int rows, int K, const T* x, uint8_t* q, float* scale, cudaStream_t st) {
   if (rows <= 0 || K <= 0 || K % 8) { set_error("quant_rows: rows=%d, K=%d (K a multiple of 8)", rows, K); return WD_ERR_SHAPE; }
-  const int64_t threads = static_cast<int64_t>(rows) * 32;
   Trace tr(KC_SMALL, st);
+  if constexpr (std::is_same<T, bf16>::value) {
+    if (K <= 2048) {          // one warp per row, 8 rows per block
+      k_quant_rows_e4m3_reg<1><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(x, rows, K, q, scale);
+      return launch_status("quant_rows_e4m3");
+    }
+    if (K <= 16384) {         // one block of 8 warps per row
+      k_quant_rows_e4m3_reg<8><<<static_cast<unsigned>(rows), 256, 0, st>>>(x, rows, K, q, scale);
+      return launch_status("quant_rows_e4m3");
+    }
+  }
+  const int64_t threads = static_cast<int64_t>(rows) * 32;
   k_quant_rows_e4m3<T><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(x, rows, K, q, scale);
   return launch_status("quant_rows_e4m3");
 }

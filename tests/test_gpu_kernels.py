@@ -297,7 +297,10 @@ def _e4m3_bytes(vals):
     return torch.from_numpy(np.ascontiguousarray(vals)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
 
 
-@pytest.mark.parametrize("rows,K,dtype", [(257, 1536, "bf16"), (3, 8, "bf16"), (130, 8960, "bf16"), (64, 136, "f32")])
+# one warp per row (K <= 2048), eight warps per row (K <= 16384) and the two-pass kernel (longer rows, fp32),
+# each at its boundaries and with row counts that leave a block part-filled
+@pytest.mark.parametrize("rows,K,dtype", [(257, 1536, "bf16"), (3, 8, "bf16"), (5, 2048, "bf16"), (130, 8960, "bf16"),
+                                          (7, 2056, "bf16"), (9, 16384, "bf16"), (2, 16392, "bf16"), (64, 136, "f32")])
 def test_quant_rows_e4m3_bit_exact(wd, rows, K, dtype):
     rng = np.random.default_rng(rows + K)
     x = (rng.standard_normal((rows, K)) * np.exp(rng.uniform(-4, 4, (rows, 1)))).astype(np.float32)
