@@ -15,6 +15,9 @@
 //              quarter of the accumulator for its warpgroup's share of the
 //              columns (tcgen05.ld), applies the epilogue and stores; they
 //              release the TMEM buffer so the next tile's MMAs overlap it.
+//              The 2-byte outputs and the residual go out through shared-memory
+//              staging tiles and TMA stores / reduce-adds (whole 128-byte rows);
+//              fp32 stores and the unpatchify scatter store from registers.
 #include "wd_internal.cuh"
 
 #include <cudaTypedefs.h>
