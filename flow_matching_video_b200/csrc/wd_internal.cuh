@@ -147,7 +147,7 @@ wd_status attention_simt(const AttnArgs<TI, TO>& a, cudaStream_t st);
 // Tensor-core attention (dh = 128; other head sizes go to attention_simt).
 wd_status attention_tc(const AttnArgs<bf16, bf16>& a, cudaStream_t st);
 wd_status attention_tc(const AttnArgs<f16, bf16>& a, cudaStream_t st);
-// Two key segments on the tensor cores (k_attn_cross.cu: persistent over Q tiles).
+// Two key segments on the tensor cores, computed side by side (k_attn_cross.cu).
 template <typename TI>
 wd_status attention_cross_tc(const AttnArgs<TI, bf16>& a, cudaStream_t st);
 // FP8 attention (k_attn_f8.cu): the operand buffer's layout, the quantisation
