@@ -49,10 +49,6 @@ constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
 #define WD_ATTN_ILP 1   // 1: row max and row sum over four independent chains (shorter dependency chains)
 #endif
 
-#ifndef WD_ATTN_CROSS_CHAINS
-#define WD_ATTN_CROSS_CHAINS 1   // two key segments: k_attn_cross.cu, the segments side by side (0: one after the other)
-#endif
-
 #ifndef WD_ATTN_SPEC
 #define WD_ATTN_SPEC 0   // 1: no separate row-max pass before the exponentials (speculative reference)
 #endif
@@ -695,7 +691,6 @@ static wd_status attention_tc_t(const AttnArgs<TI, bf16>& a, cudaStream_t st) {
     set_error("attention_tc: operands must be 16-byte aligned with row strides multiple of 8");
     return WD_ERR_ALIGN;
   }
-  if (WD_ATTN_CROSS_CHAINS && a.k2) return attention_cross_tc<TI>(a, st);   // two key segments side by side
   const CUtensorMapDataType ty =
       std::is_same<TI, f16>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap tq, tk0, tv0, tk1, tv1;
@@ -715,7 +710,7 @@ static wd_status attention_tc_t(const AttnArgs<TI, bf16>& a, cudaStream_t st) {
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(a.dh));
   p.lse = a.k2 ? nullptr : a.lse;
   p.heads = a.heads;
-  if (a.k2) {   // the two segments one after the other (WD_ATTN_CROSS_CHAINS=0)
+  if (a.k2) {
     const int64_t b2 = a.kv2_bs ? a.batch : 1;
     WD_TRY(make_tmap_3d(&tk1, ty, a.k2, D, a.n2, b2, a.kv2_rs, a.kv2_bs));
     WD_TRY(make_tmap_3d(&tv1, ty, a.v2, D, a.n2, b2, a.kv2_rs, a.kv2_bs));

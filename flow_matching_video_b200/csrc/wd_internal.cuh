@@ -147,9 +147,6 @@ wd_status attention_simt(const AttnArgs<TI, TO>& a, cudaStream_t st);
 // Tensor-core attention (dh = 128; other head sizes go to attention_simt).
 wd_status attention_tc(const AttnArgs<bf16, bf16>& a, cudaStream_t st);
 wd_status attention_tc(const AttnArgs<f16, bf16>& a, cudaStream_t st);
-// Two key segments on the tensor cores, computed side by side (k_attn_cross.cu).
-template <typename TI>
-wd_status attention_cross_tc(const AttnArgs<TI, bf16>& a, cudaStream_t st);
 // FP8 attention (k_attn_f8.cu): the operand buffer's layout, the quantisation
 // of bf16 q, k, v into it and the attention on it (bf16 output).
 wd_status attn_fp8_layout(int batch, int64_t Lq, int64_t Lk, int heads, int dh, wd_attn_fp8_layout* L);

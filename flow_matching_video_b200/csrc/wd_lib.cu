@@ -6,7 +6,6 @@
 #include "k_gemm_tc.cu"
 #include "k_attn_tc.cu"
 #include "k_attn_f8.cu"
-#include "k_attn_cross.cu"
 #include "wd_api.cu"
 #include "wd_noalloc.cu"
 #include "wd_testing.cu"
