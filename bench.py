@@ -406,6 +406,8 @@ def run_ours(args, rank, world, local_rank):
     attn8 = (args.fp8 or "").endswith("+attn")
     peak_att = 2 * peak_s if attn8 else peak_s
     share = {k: round(v[1] / max(sum(u[1] for u in tr.values()), 1e-9), 4) for k, v in tr.items()}
+    # the event-timed kernels of one step (traced re-run); ms_per_step minus this is time between kernels
+    kernel_ms = sum(v[1] for v in tr.values()) / args.steps
     launches = sum(v[0] for v in tr.values())
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -446,6 +448,7 @@ def run_ours(args, rank, world, local_rank):
                                  traffic_for("attn_self", os.path.join(ROOT, "flow_matching_video_b200", "csrc",
                                                                        "k_attn_tc.cu")))},
         "kernel_time_share": share,
+        "kernel_ms_per_step": kernel_ms,
         **({"cache": cache_note} if cache_note else {}),
         "clocks": clk,
     }
