@@ -159,3 +159,33 @@ def test_bf16_model_needs_128_wide_heads(wd):
     d = wd.make_dims(synth.TINY.dims)
     assert wd.wd_workspace_bytes(d, 2) > 0
     assert wd.wd_debug_flags() == 0
+
+
+def test_fp8_attention_layout_and_refusals(wd):
+    """The FP8 attention's operand layout (256-byte aligned regions in order,
+    each large enough, the V^T rows padded to 16 keys), and its refusals before
+    any CUDA call: head sizes other than 128, empty shapes, short or misaligned
+    buffers, misaligned operands."""
+    lib = wd.lib()
+    B, Lq, Lk, H = 2, 300, 301, 2
+    D, nb = H * 128, (Lk + 127) // 128
+    lay = wd.wd_attention_fp8_layout(B, Lq, Lk, H, 128)
+    assert lay.lkp == 304
+    regions = [("q8", B * Lq * D), ("sq", 4 * B * H * Lq), ("k8", B * Lk * D), ("sk", 4 * B * H * nb),
+               ("v8t", B * D * lay.lkp), ("sv", 4 * B * D), ("v_amax", 4 * B * D)]
+    ends = [getattr(lay, n) for n, _ in regions[1:]] + [lay.bytes]
+    for (name, size), end in zip(regions, ends):
+        off = getattr(lay, name)
+        assert off % 256 == 0 and end - off >= size, name
+    out = wd.wd_attn_fp8_layout()
+    assert lib.wd_attention_fp8_layout(B, Lq, Lk, H, 64, C.byref(out)) == 8          # dh 64: unsupported
+    assert lib.wd_attention_fp8_layout(B, 0, Lk, H, 128, C.byref(out)) == 2          # no queries
+    assert lib.wd_attention_fp8_layout(B, Lq, 0, H, 128, C.byref(out)) == 2          # no keys
+    q, k, v, buf = 0x10000, 0x20000, 0x30000, 0x100000
+    # quantise: buffer too small, then a buffer off its 256-byte alignment, then a misaligned v
+    assert lib.wd_attention_fp8_quantize(B, Lq, Lk, H, 128, q, 3 * D, k, v, 3 * D, buf, lay.bytes - 1, None) == 5
+    assert lib.wd_attention_fp8_quantize(B, Lq, Lk, H, 128, q, 3 * D, k, v, 3 * D, buf + 16, lay.bytes, None) == 4
+    assert lib.wd_attention_fp8_quantize(B, Lq, Lk, H, 128, q, 3 * D, k, v + 8, 3 * D, buf, lay.bytes, None) == 4
+    # attention: buffer too small, head size 64
+    assert lib.wd_attention_fp8(B, Lq, Lk, H, 128, buf, lay.bytes - 1, 0x200000, D, None) == 5
+    assert lib.wd_attention_fp8(B, Lq, Lk, H, 64, buf, lay.bytes, 0x200000, D, None) == 8
