@@ -4,7 +4,8 @@
 
 CASE is one of attn_self, attn_cross, attn_fp8 (the FP8 self-attention on
 quantised operands), attn_fp8_quantize (the quantisation of q, k, v for it),
-gemm_qkv, gemm_o, gemm_ffn1, gemm_ffn2, euler, euler_hbm, gemm_fp8_qkv,
+gemm_qkv, gemm_o, gemm_ffn1, gemm_ffn2, gemm_ffn1_store (FFN1's shape without the
+GELU), euler, euler_hbm, gemm_fp8_qkv,
 gemm_fp8_o, gemm_fp8_ffn1, gemm_fp8_ffn2, quant_ffn_hidden, block_480p17 (one
 block, 17 frames, L = 7800, batch 1), block_480p81 (one block, L = 32760, batch
 2), block_480p81_fp8 (the same block with its six linear layers on e4m3
@@ -60,7 +61,8 @@ def make_case(name: str, B: int):
         return (lambda: wd.wd_attention(wd.WD_F16, B, L, H, 128, q, ki, vi, NI, 1, o, kt, vt, NT, 0),
                 4.0 * B * L * (NI + NT) * D, "FLOP", B)
     gemms = {"gemm_qkv": (3 * D, D, wd.EPI_STORE), "gemm_o": (D, D, wd.EPI_RESID),
-             "gemm_ffn1": (F, D, wd.EPI_GELU), "gemm_ffn2": (D, F, wd.EPI_RESID)}
+             "gemm_ffn1": (F, D, wd.EPI_GELU), "gemm_ffn2": (D, F, wd.EPI_RESID),
+             "gemm_ffn1_store": (F, D, wd.EPI_STORE)}   # FFN1's shape with a plain bf16 store: the GELU's cost
     if name in gemms:
         N, K, epi = gemms[name]
         A, W, bias = bf(rows, K), bf(N, K) * 0.02, torch.zeros(N, device="cuda")
