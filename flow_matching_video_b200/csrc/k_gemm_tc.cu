@@ -27,8 +27,8 @@ namespace tcg {
 
 constexpr int BM = 128, BK = 64;
 // Epilogue warpgroups per mode, each taking an equal share of a tile's columns:
-// two for the GELU epilogue (erf per element; with e4m3 operands it outlasts
-// the MMAs of a tile), one otherwise.
+// two for the GELU epilogue (a reciprocal and an exponential per element; with
+// e4m3 operands it would outlast the MMAs of a tile on one), one otherwise.
 template <int MODE> __host__ __device__ constexpr int epi_wg() { return MODE == EPI_GELU ? 2 : 1; }
 template <int MODE> __host__ __device__ constexpr int threads() { return 64 + 128 * epi_wg<MODE>(); }
 // Epilogues with a 2-byte output go out through TMA stores: each epilogue warp
@@ -92,7 +92,7 @@ __device__ __forceinline__ void epi_values32(const Epi& ep, float sm, int n, con
   }
   if constexpr (MODE == EPI_GELU) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+    for (int j = 0; j < 32; ++j) v[j] = gelu_as(v[j]);
   }
 }
 // 8 values packed as 2-byte elements of the epilogue's output type

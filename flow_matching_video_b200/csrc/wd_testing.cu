@@ -1,7 +1,9 @@
-// wd_testing.cu — two entry points that exist only to test pieces of the
+// wd_testing.cu — entry points that exist only to test pieces of the
 // kernels that no output of the path exposes on its own:
 //   wd_test_exp2          the FMA-pipe 2^x of the attention softmax (and the
 //                         MUFU ex2 beside it) evaluated on caller data;
+//   wd_test_gelu          the GEMM epilogue's GELU (and the erff form of the
+//                         CUDA-core path) evaluated on caller data;
 //   wd_test_wait_timeout  one bounded mbarrier wait that nothing completes,
 //                         with a short limit, so the timeout path (error
 //                         word, drain, return, wd_check) can be exercised
@@ -21,6 +23,15 @@ __global__ void k_test_exp2(const float* __restrict__ x, float* __restrict__ y_f
     y_fma2[i] = tca::exp2_fma2(make_float2(v, x[j])).x;
     y_mufu[i] = tca::ex2(v);
     y_lib[i] = exp2f(v);
+  }
+}
+
+__global__ void k_test_gelu(const float* __restrict__ x, float* __restrict__ y_as, float* __restrict__ y_erf,
+                            int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    y_as[i] = gelu_as(x[i]);
+    y_erf[i] = gelu_erf(x[i]);
   }
 }
 
@@ -53,6 +64,17 @@ wd_status wd_test_exp2(const float* x, float* y_fma, float* y_fma2, float* y_muf
   Trace tr(KC_SMALL, st);
   k_test_exp2<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0, st>>>(x, y_fma, y_fma2, y_mufu, y_lib, n);
   return launch_status("test_exp2");
+}
+
+wd_status wd_test_gelu(const float* x, float* y_as, float* y_erf, int64_t n, wd_stream stream) {
+  using namespace wd;
+  WD_NEED(x); WD_NEED(y_as); WD_NEED(y_erf);
+  if (n <= 0) { set_error("wd_test_gelu: n = %lld", (long long)n); return WD_ERR_SHAPE; }
+  const int64_t blocks = (n + 255) / 256;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Trace tr(KC_SMALL, st);
+  k_test_gelu<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0, st>>>(x, y_as, y_erf, n);
+  return launch_status("test_gelu");
 }
 
 wd_status wd_test_wait_timeout(uint64_t limit_ns, unsigned site, int* out, wd_stream stream) {

@@ -392,6 +392,31 @@ def test_exp2_fma_within_its_stated_bound(wd):
     assert np.abs(y_fma[in_range] / y_lib[in_range] - 1.0).max() <= 7.5e-5 + 2.0 ** -22
 
 
+def test_gelu_epilogue_within_its_bound(wd):
+    """The tensor-core GEMM epilogue's GELU (Abramowitz and Stegun 7.1.26 for
+    the normal tail probability) on a dense grid over [-30, 30] plus the sign
+    change and far arguments: within 1e-6 (|GELU(x)| + 1) of the float64
+    GELU, the function-error allowance of the GEMM tests, and within 1e-6 of
+    the erff form that the CUDA-core path uses; exact 0 at 0, x itself far
+    right, 0 far left."""
+    from scipy.special import erfc
+    x = np.concatenate([np.linspace(-30.0, 30.0, 4_000_001, dtype=np.float32),
+                        np.float32([0.0, -0.0, 1e-30, -1e-30, 1e-7, -1e-7, 50.0, -50.0, 1e4, -1e4])])
+    gx = dev(x)
+    y_as, y_erf = torch.empty_like(gx), torch.empty_like(gx)
+    wd.wd_test_gelu(gx, y_as, y_erf)
+    wd.wd_check()
+    ya, ye = (t.cpu().numpy().astype(np.float64) for t in (y_as, y_erf))
+    x64 = x.astype(np.float64)
+    exact = 0.5 * x64 * erfc(-x64 / np.sqrt(2.0))
+    err = np.abs(ya - exact)
+    assert np.all(err <= 1e-6 * (np.abs(exact) + 1.0)), (err.max(), x[err.argmax()])
+    assert np.abs(ya - ye).max() <= 1e-6
+    assert ya[x == 0.0].max() == 0.0 and ya[x == 0.0].min() == 0.0
+    far = np.abs(x64) >= 50.0
+    np.testing.assert_array_equal(ya[far], np.where(x64[far] > 0, x64[far], 0.0))
+
+
 def test_bounded_wait_runs_out_reports_and_recovers(wd):
     """A wait that nothing completes, with a 1 ms limit: the kernel returns,
     wd_check reports WD_ERR_TIMEOUT with the site and clears the error word,
@@ -456,6 +481,47 @@ def test_attention_lse_and_merge_over_key_parts(wd, dtype, dh, Lq, n):
     vbar = np.einsum("bhmn,bnhd->bmhd", p, np.abs(va)).reshape(B, Lq, h * dh)
     bound = 2 * u_out * np.abs(want_o) + (4 * BF16_HALF_ULP if is_bf else 1e-5) * vbar + 1e-6
     assert_within(host(out), want_o, bound)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_attention_bf16_reference_moves(wd, seed):
+    """Key groups whose scores rise far above every earlier key block's (by
+    more than 58 in log2 units for most rows), so the online softmax must move
+    its reference and rescale O and the row sum deep into the row: head 0,
+    keys 300-309 scaled by 40 (in key block 2); head 1, keys 300-309 scaled
+    by 4 (a rise within the lazy threshold for some rows) and keys 600-609 by
+    40 (the second half of block 4).  Output and log-sum-exp against the
+    exact attention, with the bounds of the other attention tests; the
+    log-sum-exp bound adds the fp32 accumulation bound of the scores
+    (dh * 2^-24 * sum |q_i k_i|)."""
+    B, Lq, h, dh, n = 1, 300, 2, 128, 640
+    rng = np.random.default_rng(500 + seed)
+    q, k, v = (rng.standard_normal((B, m, h * dh)) for m in (Lq, n, n))
+    k[:, 300:310, :dh] *= 40.0
+    k[:, 300:310, dh:] *= 4.0
+    k[:, 600:610, dh:] *= 40.0
+    q, k, v = (bf(a.astype(np.float32)).astype(np.float32) for a in (q, k, v))
+    qa, ka, va = (a.astype(np.float64).reshape(B, -1, h, dh) for a in (q, k, v))
+    s = np.einsum("bmhd,bnhd->bhmn", qa, ka) / np.sqrt(dh)
+    sm = s.max(-1, keepdims=True)
+    p = np.exp(s - sm)
+    want_lse = (sm[..., 0] + np.log(p.sum(-1))) / np.log(2.0)
+    p /= p.sum(-1, keepdims=True)
+    want = np.einsum("bhmn,bnhd->bmhd", p, va).reshape(B, Lq, h * dh)
+    pv_abs = np.einsum("bhmn,bnhd->bmhd", p, np.abs(va)).reshape(B, Lq, h * dh)
+    # the rows really jump: by more than 58 (log2 units) above all earlier keys, in both heads
+    s2 = s / np.log(2.0)
+    assert (s2[0, 0, :, 300:310].max(-1) - s2[0, 0, :, :256].max(-1) > 58).mean() > 0.5
+    assert (s2[0, 1, :, 600:610].max(-1) - s2[0, 1, :, :512].max(-1) > 58).mean() > 0.5
+    o = torch.empty((B, Lq, h * dh), device="cuda", dtype=torch.bfloat16)
+    lse = torch.empty((B, h, Lq), device="cuda")
+    wd.wd_attention_lse(wd.WD_BF16, B, Lq, h, dh, dev(q, torch.bfloat16), dev(k, torch.bfloat16),
+                        dev(v, torch.bfloat16), n, 0, o, lse)
+    wd.wd_check()
+    bound = BF16_HALF_ULP * np.abs(want) + 2 * BF16_HALF_ULP * pv_abs + 1e-6
+    assert_within(host(o), want, bound)
+    acc = dh * 2.0 ** -24 * np.einsum("bmhd,bnhd->bhmn", np.abs(qa), np.abs(ka)).max(-1) / np.sqrt(dh) / np.log(2.0)
+    assert np.all(np.abs(host(lse) - want_lse) <= 2e-4 + acc)
 
 
 # ------------------------------------------------------------------ FP8 attention ("Wan（通义万相）..." 5.3)
