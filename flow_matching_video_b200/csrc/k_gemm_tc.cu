@@ -72,28 +72,36 @@ enum : unsigned { SITE_EMPTY = 0x101, SITE_FULL = 0x102, SITE_TFULL = 0x103, SIT
 // One thread = one output row m; columns n .. n+31 come from the accumulator.
 // The values before the store: FP8 scales (row scale sm = sa[m], passed in so
 // that rows past M need not read it), bias, GELU.
+// Pairs of columns go through the packed fp32 instructions (f32x2), which
+// round each lane as the scalar ones would.
 template <int MODE>
 __device__ __forceinline__ void epi_values32(const Epi& ep, float sm, int n, const uint32_t (&r)[32], float (&v)[32]) {
+  float2 w[16];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+  for (int j = 0; j < 16; ++j) w[j] = make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
   if (ep.sa) {   // FP8 operands: acc * (sa[m] * sb[n])
+    const float2 sm2 = make_float2(sm, sm);
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
-      const float4 b = __ldg(reinterpret_cast<const float4*>(ep.sb + n + j));
-      v[j] *= sm * b.x; v[j + 1] *= sm * b.y; v[j + 2] *= sm * b.z; v[j + 3] *= sm * b.w;
+    for (int j = 0; j < 16; j += 2) {
+      const float4 b = __ldg(reinterpret_cast<const float4*>(ep.sb + n + 2 * j));
+      w[j] = fmul2(w[j], fmul2(sm2, make_float2(b.x, b.y)));
+      w[j + 1] = fmul2(w[j + 1], fmul2(sm2, make_float2(b.z, b.w)));
     }
   }
   if (ep.bias) {
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
-      const float4 b = __ldg(reinterpret_cast<const float4*>(ep.bias + n + j));
-      v[j] += b.x; v[j + 1] += b.y; v[j + 2] += b.z; v[j + 3] += b.w;
+    for (int j = 0; j < 16; j += 2) {
+      const float4 b = __ldg(reinterpret_cast<const float4*>(ep.bias + n + 2 * j));
+      w[j] = fadd2(w[j], make_float2(b.x, b.y));
+      w[j + 1] = fadd2(w[j + 1], make_float2(b.z, b.w));
     }
   }
   if constexpr (MODE == EPI_GELU) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = gelu_as(v[j]);
+    for (int j = 0; j < 16; ++j) w[j] = gelu_as2(w[j]);
   }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) { v[2 * j] = w[j].x; v[2 * j + 1] = w[j].y; }
 }
 // 8 values packed as 2-byte elements of the epilogue's output type
 template <int MODE>

@@ -112,6 +112,15 @@ __device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return o;
 }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 o;
+  asm("{\n\t.reg .b64 x, y, r;\n\t"
+      "mov.b64 x, {%2, %3};\n\tmov.b64 y, {%4, %5};\n\t"
+      "mul.f32x2 r, x, y;\n\tmov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(o.x), "=f"(o.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return o;
+}
 // max of three (one instruction on sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float o;

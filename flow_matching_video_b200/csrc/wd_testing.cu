@@ -26,11 +26,14 @@ __global__ void k_test_exp2(const float* __restrict__ x, float* __restrict__ y_f
   }
 }
 
-__global__ void k_test_gelu(const float* __restrict__ x, float* __restrict__ y_as, float* __restrict__ y_erf,
-                            int64_t n) {
+__global__ void k_test_gelu(const float* __restrict__ x, float* __restrict__ y_as, float* __restrict__ y_as2,
+                            float* __restrict__ y_erf, int64_t n) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     y_as[i] = gelu_as(x[i]);
+    // the packed form on the pair (x[i], x[i ^ 1]): lane 0 is x[i]
+    const int64_t j = ((i ^ 1) < n) ? (i ^ 1) : i;
+    y_as2[i] = gelu_as2(make_float2(x[i], x[j])).x;
     y_erf[i] = gelu_erf(x[i]);
   }
 }
@@ -66,14 +69,14 @@ wd_status wd_test_exp2(const float* x, float* y_fma, float* y_fma2, float* y_muf
   return launch_status("test_exp2");
 }
 
-wd_status wd_test_gelu(const float* x, float* y_as, float* y_erf, int64_t n, wd_stream stream) {
+wd_status wd_test_gelu(const float* x, float* y_as, float* y_as2, float* y_erf, int64_t n, wd_stream stream) {
   using namespace wd;
-  WD_NEED(x); WD_NEED(y_as); WD_NEED(y_erf);
+  WD_NEED(x); WD_NEED(y_as); WD_NEED(y_as2); WD_NEED(y_erf);
   if (n <= 0) { set_error("wd_test_gelu: n = %lld", (long long)n); return WD_ERR_SHAPE; }
   const int64_t blocks = (n + 255) / 256;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Trace tr(KC_SMALL, st);
-  k_test_gelu<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0, st>>>(x, y_as, y_erf, n);
+  k_test_gelu<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0, st>>>(x, y_as, y_as2, y_erf, n);
   return launch_status("test_gelu");
 }
 

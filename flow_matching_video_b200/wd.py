@@ -92,7 +92,7 @@ SIGNATURES = {
     "wd_quant_rows_e4m3": (_I, [_I, _I, _I, _P, _P, _P, _P]),
     "wd_gemm_fp8": (_I, [_I, _I, _I, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P]),
     "wd_test_exp2": (_I, [_P, _P, _P, _P, _P, _L, _P]),
-    "wd_test_gelu": (_I, [_P, _P, _P, _L, _P]),
+    "wd_test_gelu": (_I, [_P, _P, _P, _P, _L, _P]),
     "wd_test_wait_timeout": (_I, [C.c_uint64, C.c_uint, _P, _P]),
     "wd_set_debug_flags": (None, [C.c_uint]),
     "wd_debug_flags": (C.c_uint, []),
@@ -261,8 +261,8 @@ def wd_test_exp2(x, y_fma, y_fma2, y_mufu, y_lib, stream=None):
         "wd_test_exp2")
 
 
-def wd_test_gelu(x, y_as, y_erf, stream=None):
-    _ok(_lib.wd_test_gelu(_p(x), _p(y_as), _p(y_erf), x.numel(), _stream(stream)), "wd_test_gelu")
+def wd_test_gelu(x, y_as, y_as2, y_erf, stream=None):
+    _ok(_lib.wd_test_gelu(_p(x), _p(y_as), _p(y_as2), _p(y_erf), x.numel(), _stream(stream)), "wd_test_gelu")
 
 
 def wd_test_wait_timeout(limit_ns: int, site: int, out, stream=None):

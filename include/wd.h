@@ -444,10 +444,12 @@ wd_status wd_test_exp2(const float* x, float* y_fma, float* y_fma2, float* y_muf
 /* Evaluates, for each of the n fp32 values x[i], the two GELUs of the library:
  * y_as[i] = the tensor-core GEMM epilogue's x * Phi(x), with the normal tail
  * probability from the rational approximation 7.1.26 of Abramowitz and Stegun
- * (erf within 1.5e-7), a MUFU reciprocal and a MUFU 2^x; y_erf[i] = the
- * CUDA-core path's 0.5 x (1 + erff(x / sqrt 2)).  All device arrays of n
- * floats; n > 0. */
-wd_status wd_test_gelu(const float* x, float* y_as, float* y_erf, int64_t n, wd_stream stream);
+ * (erf within 1.5e-7), a MUFU reciprocal and a MUFU 2^x; y_as2[i] = the same
+ * function in its packed two-lane form (f32x2 instructions, the one the
+ * epilogue runs), evaluated on the pair (x[i], x[i^1]), which must equal
+ * y_as[i]; y_erf[i] = the CUDA-core path's 0.5 x (1 + erff(x / sqrt 2)).
+ * All device arrays of n floats; n > 0. */
+wd_status wd_test_gelu(const float* x, float* y_as, float* y_as2, float* y_erf, int64_t n, wd_stream stream);
 
 /* Launches one warp that waits on an mbarrier phase nothing completes, with
  * the library's bounded wait given a limit of limit_ns (at most 100 ms, not

@@ -394,8 +394,8 @@ def test_exp2_fma_within_its_stated_bound(wd):
 
 def test_gelu_epilogue_within_its_bound(wd):
     """The tensor-core GEMM epilogue's GELU (Abramowitz and Stegun 7.1.26 for
-    the normal tail probability) on a dense grid over [-30, 30] plus the sign
-    change and far arguments: within 1e-6 (|GELU(x)| + 1) of the float64
+    the normal tail probability), scalar and packed two-lane forms, on a dense
+    grid over [-30, 30] plus the sign change and far arguments: within 1e-6 (|GELU(x)| + 1) of the float64
     GELU, the function-error allowance of the GEMM tests, and within 1e-6 of
     the erff form that the CUDA-core path uses; exact 0 at 0, x itself far
     right, 0 far left."""
@@ -403,10 +403,12 @@ def test_gelu_epilogue_within_its_bound(wd):
     x = np.concatenate([np.linspace(-30.0, 30.0, 4_000_001, dtype=np.float32),
                         np.float32([0.0, -0.0, 1e-30, -1e-30, 1e-7, -1e-7, 50.0, -50.0, 1e4, -1e4])])
     gx = dev(x)
-    y_as, y_erf = torch.empty_like(gx), torch.empty_like(gx)
-    wd.wd_test_gelu(gx, y_as, y_erf)
+    y_as, y_as2, y_erf = torch.empty_like(gx), torch.empty_like(gx), torch.empty_like(gx)
+    wd.wd_test_gelu(gx, y_as, y_as2, y_erf)
     wd.wd_check()
-    ya, ye = (t.cpu().numpy().astype(np.float64) for t in (y_as, y_erf))
+    ya, ya2, ye = (t.cpu().numpy().astype(np.float64) for t in (y_as, y_as2, y_erf))
+    # the packed two-lane form (the one the epilogue runs) computes the same function, lane by lane
+    np.testing.assert_array_equal(ya2, ya)
     x64 = x.astype(np.float64)
     exact = 0.5 * x64 * erfc(-x64 / np.sqrt(2.0))
     err = np.abs(ya - exact)
