@@ -262,6 +262,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         // at chunk j ^ (lane & 7)), then one lane reduces the tile into X in
         // L2, so no residual load waits in the SM.
         const bool gated = ep.gate_a || ep.gate_b;
+        // FP8 row scale of this thread's row, read once per tile (inside the column loop the
+        // compiler cannot keep it across the staging-tile stores)
+        const float rs = (ep.sa && m < M) ? ep.sa[m] : 0.f;
 #pragma unroll 1
         for (int c = c_begin; c < c_begin + COLS; c += 32) {
           uint32_t r[32];
@@ -284,9 +287,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             float4 a = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
                                    __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
             if (ep.sa) {   // FP8 operands: acc * (sa[m] * sb[n])
-              const float sm = m < M ? ep.sa[m] : 0.f;
               const float4 sb = __ldg(reinterpret_cast<const float4*>(ep.sb + n));
-              a.x *= sm * sb.x; a.y *= sm * sb.y; a.z *= sm * sb.z; a.w *= sm * sb.w;
+              a.x *= rs * sb.x; a.y *= rs * sb.y; a.z *= rs * sb.z; a.w *= rs * sb.w;
             }
             row[j ^ (lane & 7)] = make_float4(g.x * (a.x + bb.x), g.y * (a.y + bb.y), g.z * (a.z + bb.z), g.w * (a.w + bb.w));
           }
