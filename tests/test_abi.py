@@ -140,6 +140,10 @@ def test_empty_sizes_are_a_no_op_or_rejected_before_launch(wd):
     assert lib.wd_gemm_fp8(0, 256, 64, 0x1000, 0x2000, 0x3000, 0x4000, None, 0, 0x5000, None, None, None) == 2
     assert lib.wd_quant_rows_e4m3(1, 0, 64, 0x1000, 0x2000, 0x3000, None) == 2
     assert lib.wd_quant_rows_e4m3(1, 4, 12, 0x1000, 0x2000, 0x3000, None) == 2    # K not a multiple of 8
+    # the test-only entries: no values, or a missing output, are refused before any launch
+    assert lib.wd_test_gelu(0x1000, 0x2000, 0x3000, 0x4000, 0, None) == 2
+    assert lib.wd_test_gelu(0x1000, 0x2000, None, 0x4000, 16, None) == 1
+    assert lib.wd_test_exp2(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0, None) == 2
     # the FP8 GEMM's shape rules: N a multiple of 256, scales required
     assert lib.wd_gemm_fp8(8, 128, 64, 0x1000, 0x2000, 0x3000, 0x4000, None, 0, 0x5000, None, None, None) == 2
     assert lib.wd_gemm_fp8(8, 256, 64, 0x1000, None, 0x3000, 0x4000, None, 0, 0x5000, None, None, None) == 1
