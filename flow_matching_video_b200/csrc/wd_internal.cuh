@@ -76,7 +76,8 @@ __device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + e
 // |error| <= 1.5e-7 for y >= 0; the a_i below are the published ones halved.
 // Phi(x) = 1 - E for x >= 0 and E for x < 0, so the negative tail is never a
 // difference of nearly equal numbers.  Two MUFU operations (reciprocal, 2^x)
-// and seven FMA-pipe ones per value, against about thirty for the erff form.
+// and twelve FMA-pipe ones per value (about seven in the packed form below),
+// against about thirty issue slots for the erff form.
 __device__ __forceinline__ float gelu_as(float x) {
   float t, e;
   const float y = fabsf(x) * 0.70710678118654752f;
