@@ -178,7 +178,7 @@ def _block_parity(mods, wl, n_rows, tau, block=0, deep=None):
           f"contribution {errs[True][1]:.3e}; against the unrounded oracle: X_out {errs[False][0]:.3e}, "
           f"contribution {errs[False][1]:.3e}; rms(X_in) {np.sqrt((X_in ** 2).mean()):.3f}")
     assert errs[True][0] < TOL_BF16
-    # the block's own contribution, judged on its own scale
+    # the block's own contribution, measured against its own scale
     assert errs[True][1] < TOL_BF16
     assert errs[False][0] < TOL_BF16_UNROUNDED
     assert errs[False][1] < TOL_BF16_UNROUNDED
