@@ -12,13 +12,17 @@ the other pin file checks only with a branch switched off.
   "图解 Wan2.1 I2V" 5.4;
 * the text MLP and the CLIP MLPProj against torch ("图解 Wan2.1 I2V" 7);
 * the sampler's unconditional row: zeroed text, CLIP and y unchanged
-  ("图解 Wan2.1 I2V" Q5).
+  ("图解 Wan2.1 I2V" Q5);
+* the whole block with every branch on, against a torch restatement that runs
+  self-attention, cross-attention and feed-forward one after the other
+  ("图解 Wan2.1 I2V" 5.2-5.5).
 
 Each pin is also run against oracles with a plausible mistake planted
 (monkeypatched on the CPU, for the length of one test): the token grid with
 rows and columns swapped, RMSNorm per head instead of over D, a RoPE turning
 the wrong way or reading the wrong coordinate, the text and image key weights
-swapped, the unconditional row keeping its text.  The pin must fail on each.
+swapped, the unconditional row keeping its text, the block's branches all
+reading its input.  The pin must fail on each.
 """
 import unittest.mock as um
 
@@ -203,6 +207,71 @@ def test_self_attention_pin_catches_rope_on_values(monkeypatch):
         return orig_att(q, k, v)
     monkeypatch.setattr(O, "attention", att)
     assert _self_branch_error() > 1e-3
+
+
+# ------------------------------------------------------------------ the whole block, every branch on
+def block_torch(X, e0, w, d, kv):
+    """One block with all three branches on, restated with torch (float64):
+    the self-attention branch (self_branch_torch); then, on the stream it
+    leaves, the decoupled cross-attention (affine LayerNorm, query Linear, the
+    image and the text attention summed, output Linear; no adaLN, no gate);
+    then, on the stream after that, the gated GELU feed-forward with adaLN
+    ("图解 Wan2.1 I2V" 5.2-5.5)."""
+    B, D, h, dh = X.shape[0], d.D, d.heads, d.dh
+    mod = e0 + w["blk0.mod"]
+    x1 = T64(self_branch_torch(X, e0, w, d))
+    hc = TF.layer_norm(x1, (D,), T64(w["blk0.cn.g"]), T64(w["blk0.cn.b"]), eps=d.eps)
+    qc = TF.linear(hc, T64(w["blk0.cq.w"]), T64(w["blk0.cq.b"]))
+    sp = lambda t: t.reshape(t.shape[0], t.shape[1], h, dh).transpose(1, 2)
+
+    def sdpa(q, k, v):
+        return TF.scaled_dot_product_attention(sp(q), sp(k), sp(v)).transpose(1, 2).reshape(q.shape)
+    ki, vi = T64(kv["k_img"]).expand(B, -1, -1), T64(kv["v_img"]).expand(B, -1, -1)
+    oc = sdpa(qc, ki, vi) + sdpa(qc, T64(kv["k_txt"]), T64(kv["v_txt"]))
+    x2 = x1 + TF.linear(oc, T64(w["blk0.co.w"]), T64(w["blk0.co.b"]))
+    h2 = TF.layer_norm(x2, (D,), eps=d.eps) * (1 + T64(mod[4])) + T64(mod[3])
+    u = TF.gelu(TF.linear(h2, T64(w["blk0.f1.w"]), T64(w["blk0.f1.b"])))
+    return (x2 + T64(mod[5]) * TF.linear(u, T64(w["blk0.f2.w"]), T64(w["blk0.f2.b"]))).numpy()
+
+
+def _whole_block_error():
+    d, w, txt, clip, X = _tiny()
+    e0, w = _gated(w, d.D, 0.8, 1.3)
+    ctx_t, ctx_i = O.context_embed(w, txt, clip)
+    kv = O.cross_kv(w, 0, ctx_t, ctx_i)
+    got = O.block_forward(X, e0, w, 0, kv, d)
+    want = block_torch(X, e0, w, d, kv)
+    assert np.abs(want - X).max() > 1.0
+    return float(np.abs(got - want).max())
+
+
+def test_whole_block_against_torch_restatement():
+    assert _whole_block_error() < 1e-9
+
+
+def test_whole_block_pin_catches_branches_reading_the_block_input(monkeypatch):
+    """A plausible misreading of the order: the cross-attention and the
+    feed-forward both read the block's input instead of the stream the branch
+    before them left."""
+    def parallel(Xr, o, e0, w, blk, kv, dims, rnd=False, fp8=False):
+        p = f"blk{blk}."
+        D, nh, dh, eps = dims.D, dims.heads, dims.dh, dims.eps
+        _, _, gate1, shift2, scale2, gate2 = O._mod(e0, w, blk)
+        sp = lambda a: np.asarray(a).reshape(-1, nh, dh)
+        out = np.empty_like(np.asarray(Xr, np.float64))
+        for b in range(Xr.shape[0]):
+            x0 = Xr[b]
+            sa = gate1 * O.linear(o[b], w[p + "o.w"], w[p + "o.b"])
+            qc = sp(O.linear(O.layer_norm(x0, eps, w[p + "cn.g"], w[p + "cn.b"]), w[p + "cq.w"], w[p + "cq.b"]))
+            oc = (O.attention(qc, sp(kv["k_img"]), sp(kv["v_img"]))
+                  + O.attention(qc, sp(kv["k_txt"][b]), sp(kv["v_txt"][b]))).reshape(-1, D)
+            ca = O.linear(oc, w[p + "co.w"], w[p + "co.b"])
+            h2 = O.adaln_modulate(x0, shift2, scale2, eps, dims.norm)
+            ff = gate2 * O.linear(O.gelu(O.linear(h2, w[p + "f1.w"], w[p + "f1.b"])), w[p + "f2.w"], w[p + "f2.b"])
+            out[b] = x0 + sa + ca + ff
+        return out
+    monkeypatch.setattr(O, "block_after_attention", parallel)
+    assert _whole_block_error() > 1e-3
 
 
 # ------------------------------------------------------------------ cross-attention keys and values
