@@ -20,9 +20,10 @@ stores a bf16 tensor (GEMM operands, q/k/v, attention outputs, FFN hidden),
 and to IEEE half where it stores a half tensor (the cross-attention queries
 and K/V cache), so a bf16 run is compared with the same function.
 Parity pins: see tests/test_oracle_*.py.  Functions whose full output no page
-pins ("parity unpinned"): dit_forward / block_forward values beyond the
-invariants (AdaLN-Zero identity, attention and RoPE special cases) checked in
-the tests; the pages print no tensor values.
+pins ("parity unpinned" against the pages, which print no tensor values):
+dit_forward and block_forward.  The tests pin them by invariants (AdaLN-Zero
+identity, attention and RoPE special cases), branch by branch, and whole
+against a second implementation of the same readings in torch.
 """
 from __future__ import annotations
 

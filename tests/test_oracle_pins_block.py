@@ -15,14 +15,15 @@ the other pin file checks only with a branch switched off.
   ("图解 Wan2.1 I2V" Q5);
 * the whole block with every branch on, against a torch restatement that runs
   self-attention, cross-attention and feed-forward one after the other
-  ("图解 Wan2.1 I2V" 5.2-5.5).
+  ("图解 Wan2.1 I2V" 5.2-5.5), and the whole two-block model against a torch
+  restatement of time MLP, patch embedding, context, blocks and head.
 
 Each pin is also run against oracles with a plausible mistake planted
 (monkeypatched on the CPU, for the length of one test): the token grid with
 rows and columns swapped, RMSNorm per head instead of over D, a RoPE turning
 the wrong way or reading the wrong coordinate, the text and image key weights
 swapped, the unconditional row keeping its text, the block's branches all
-reading its input.  The pin must fail on each.
+reading its input, every block running with block 0's weights.  The pin must fail on each.
 """
 import unittest.mock as um
 
@@ -126,23 +127,24 @@ def rope_complex(x, pos, dh):
     return torch.cat(out, dim=-1)
 
 
-def self_branch_torch(X, e0, w, d):
+def self_branch_torch(X, e0, w, d, blk=0):
     """X + gate1 * Linear_o(attention) of one block, restated with torch:
     h = LayerNorm(X)(1 + scale1) + shift1; [q k v] = Linear_qkv(h);
     q, k = RMSNorm over D with gains; heads split; RoPE; SDPA; Linear_o."""
     B, L, D, h, dh = X.shape[0], d.L, d.D, d.heads, d.dh
-    mod = e0 + w["blk0.mod"]
+    p = f"blk{blk}."
+    mod = e0 + w[p + "mod"]
     Xt = T64(X)
     hh = TF.layer_norm(Xt, (D,), eps=d.eps) * (1 + T64(mod[1])) + T64(mod[0])
-    q, k, v = TF.linear(hh, T64(w["blk0.qkv.w"]), T64(w["blk0.qkv.b"])).split(D, dim=-1)
-    q = TF.rms_norm(q, (D,), weight=T64(w["blk0.gq"]), eps=d.eps)
-    k = TF.rms_norm(k, (D,), weight=T64(w["blk0.gk"]), eps=d.eps)
+    q, k, v = TF.linear(hh, T64(w[p + "qkv.w"]), T64(w[p + "qkv.b"])).split(D, dim=-1)
+    q = TF.rms_norm(q, (D,), weight=T64(w[p + "gq"]), eps=d.eps)
+    k = TF.rms_norm(k, (D,), weight=T64(w[p + "gk"]), eps=d.eps)
     pos = conv3d_token_grid(d.T, d.H, d.W)
     heads = lambda t: t.reshape(B, L, h, dh)
     q, k, v = rope_complex(heads(q), pos, dh), rope_complex(heads(k), pos, dh), heads(v)
     o = TF.scaled_dot_product_attention(q.transpose(1, 2), k.transpose(1, 2), v.transpose(1, 2))
     o = o.transpose(1, 2).reshape(B, L, D)
-    return (Xt + T64(mod[2]) * TF.linear(o, T64(w["blk0.o.w"]), T64(w["blk0.o.b"]))).numpy()
+    return (Xt + T64(mod[2]) * TF.linear(o, T64(w[p + "o.w"]), T64(w[p + "o.b"]))).numpy()
 
 
 def _self_branch_error():
@@ -210,7 +212,7 @@ def test_self_attention_pin_catches_rope_on_values(monkeypatch):
 
 
 # ------------------------------------------------------------------ the whole block, every branch on
-def block_torch(X, e0, w, d, kv):
+def block_torch(X, e0, w, d, kv, blk=0):
     """One block with all three branches on, restated with torch (float64):
     the self-attention branch (self_branch_torch); then, on the stream it
     leaves, the decoupled cross-attention (affine LayerNorm, query Linear, the
@@ -218,20 +220,21 @@ def block_torch(X, e0, w, d, kv):
     then, on the stream after that, the gated GELU feed-forward with adaLN
     ("图解 Wan2.1 I2V" 5.2-5.5)."""
     B, D, h, dh = X.shape[0], d.D, d.heads, d.dh
-    mod = e0 + w["blk0.mod"]
-    x1 = T64(self_branch_torch(X, e0, w, d))
-    hc = TF.layer_norm(x1, (D,), T64(w["blk0.cn.g"]), T64(w["blk0.cn.b"]), eps=d.eps)
-    qc = TF.linear(hc, T64(w["blk0.cq.w"]), T64(w["blk0.cq.b"]))
+    p = f"blk{blk}."
+    mod = e0 + w[p + "mod"]
+    x1 = T64(self_branch_torch(X, e0, w, d, blk))
+    hc = TF.layer_norm(x1, (D,), T64(w[p + "cn.g"]), T64(w[p + "cn.b"]), eps=d.eps)
+    qc = TF.linear(hc, T64(w[p + "cq.w"]), T64(w[p + "cq.b"]))
     sp = lambda t: t.reshape(t.shape[0], t.shape[1], h, dh).transpose(1, 2)
 
     def sdpa(q, k, v):
         return TF.scaled_dot_product_attention(sp(q), sp(k), sp(v)).transpose(1, 2).reshape(q.shape)
     ki, vi = T64(kv["k_img"]).expand(B, -1, -1), T64(kv["v_img"]).expand(B, -1, -1)
     oc = sdpa(qc, ki, vi) + sdpa(qc, T64(kv["k_txt"]), T64(kv["v_txt"]))
-    x2 = x1 + TF.linear(oc, T64(w["blk0.co.w"]), T64(w["blk0.co.b"]))
+    x2 = x1 + TF.linear(oc, T64(w[p + "co.w"]), T64(w[p + "co.b"]))
     h2 = TF.layer_norm(x2, (D,), eps=d.eps) * (1 + T64(mod[4])) + T64(mod[3])
-    u = TF.gelu(TF.linear(h2, T64(w["blk0.f1.w"]), T64(w["blk0.f1.b"])))
-    return (x2 + T64(mod[5]) * TF.linear(u, T64(w["blk0.f2.w"]), T64(w["blk0.f2.b"]))).numpy()
+    u = TF.gelu(TF.linear(h2, T64(w[p + "f1.w"]), T64(w[p + "f1.b"])))
+    return (x2 + T64(mod[5]) * TF.linear(u, T64(w[p + "f2.w"]), T64(w[p + "f2.b"]))).numpy()
 
 
 def _whole_block_error():
@@ -272,6 +275,69 @@ def test_whole_block_pin_catches_branches_reading_the_block_input(monkeypatch):
         return out
     monkeypatch.setattr(O, "block_after_attention", parallel)
     assert _whole_block_error() > 1e-3
+
+
+# ------------------------------------------------------------------ the whole model
+def dit_torch(x_t, y, tau, w, txt, clip, d):
+    """The DiT's velocity restated with torch (float64): the time MLP on the
+    sinusoid of tau ([cos, sin] at 10000^(-i/128)) giving e and the six
+    modulation rows e0; the patch embedding as a Conv3d of concat(x_t, y); the
+    text MLP and CLIP MLPProj; per block its cross keys and values and
+    block_torch; the head (LayerNorm modulated by e + its own two rows, a
+    Linear) and the inverse of the (1, 2, 2) patchify
+    ("图解 Wan2.1 I2V" 4.2, 5.1-5.5, 7)."""
+    W = lambda k: T64(w[k])
+    B, D, T, Hp, Wp = x_t.shape[0], d.D, d.T, d.Hp, d.Wp
+    fr = torch.pow(torch.tensor(10000.0, dtype=torch.float64), -torch.arange(128, dtype=torch.float64) / 128)
+    es = torch.cat([torch.cos(tau * fr), torch.sin(tau * fr)])
+    e = TF.linear(TF.silu(TF.linear(es, W("t1.w"), W("t1.b"))), W("t2.w"), W("t2.b"))
+    e0 = TF.linear(TF.silu(e), W("tp.w"), W("tp.b")).reshape(6, D)
+    x_in = torch.cat([T64(x_t), T64(y)[None].expand(B, -1, -1, -1, -1)], dim=1)
+    X = TF.conv3d(x_in, W("pe.w").reshape(D, 36, 1, 2, 2), W("pe.b"), stride=(1, 2, 2)).flatten(2).transpose(1, 2)
+    mlp = lambda x, a, b: TF.linear(TF.gelu(TF.linear(x, W(a + ".w"), W(a + ".b"))), W(b + ".w"), W(b + ".b"))
+    ctx_t, ctx_i = mlp(T64(txt), "txt1", "txt2"), mlp(T64(clip), "img1", "img2")
+    for i in range(d.blocks):
+        p = f"blk{i}."
+        kv = {n: TF.linear(c, W(p + k + ".w"), W(p + k + ".b")).numpy()
+              for n, c, k in (("k_txt", ctx_t, "ck"), ("v_txt", ctx_t, "cv"), ("k_img", ctx_i, "cki"),
+                              ("v_img", ctx_i, "cvi"))}
+        X = T64(block_torch(X.numpy(), e0.numpy(), w, d, kv, i))
+    z = TF.layer_norm(X, (D,), eps=d.eps) * (1 + e + W("head.mod")[1]) + e + W("head.mod")[0]
+    pt = TF.linear(z, W("head.w"), W("head.b"))                                   # [B, L, 16 * 1 * 2 * 2]
+    return pt.reshape(B, T, Hp, Wp, 16, 2, 2).permute(0, 4, 1, 2, 5, 3, 6).reshape(B, 16, T, 2 * Hp, 2 * Wp).numpy()
+
+
+def _whole_model_error():
+    d = synth.Dims(D=48, heads=2, ffn=40, blocks=2, T=2, H=4, W=6, n_txt=5, c_txt=12, n_img=4, c_img=10,
+                   dtype="f32")
+    wl = synth.Workload("pin2", d, batch=2, seed=98)
+    w = {k: v.astype(np.float64) for k, v in synth.model_weights(wl).items()}
+    for k in list(w):                      # larger weights so that every term matters
+        if k.endswith(".w"):
+            w[k] = w[k] * 6
+    x_t = RNG.standard_normal((2, 16, d.T, d.H, d.W))
+    y = RNG.standard_normal((20, d.T, d.H, d.W))
+    txt = RNG.standard_normal((2, d.n_txt, d.c_txt))
+    clip = RNG.standard_normal((d.n_img, d.c_img))
+    tau = 731.0
+    ctx_t, ctx_i = O.context_embed(w, txt, clip)
+    kvs = [O.cross_kv(w, i, ctx_t, ctx_i) for i in range(d.blocks)]
+    got = O.dit_forward(x_t, y, tau, w, kvs, d)
+    want = dit_torch(x_t, y, tau, w, txt, clip, d)
+    assert np.abs(want).max() > 1.0
+    return float(np.abs(got - want).max() / np.abs(want).max())
+
+
+def test_whole_model_against_torch_restatement():
+    assert _whole_model_error() < 1e-12
+
+
+def test_whole_model_pin_catches_every_block_reading_block_0(monkeypatch):
+    """A dropped index: every block runs with block 0's weights (and its own
+    cross keys and values)."""
+    orig = O.block_forward
+    monkeypatch.setattr(O, "block_forward", lambda X, e0, w, blk, kv, dims, *a, **k: orig(X, e0, w, 0, kv, dims, *a, **k))
+    assert _whole_model_error() > 1e-3
 
 
 # ------------------------------------------------------------------ cross-attention keys and values
