@@ -16,14 +16,16 @@ the other pin file checks only with a branch switched off.
 * the whole block with every branch on, against a torch restatement that runs
   self-attention, cross-attention and feed-forward one after the other
   ("图解 Wan2.1 I2V" 5.2-5.5), and the whole two-block model against a torch
-  restatement of time MLP, patch embedding, context, blocks and head.
+  restatement of time MLP, patch embedding, context, blocks and head, and the
+  three-step CFG Euler sampler around it.
 
 Each pin is also run against oracles with a plausible mistake planted
 (monkeypatched on the CPU, for the length of one test): the token grid with
 rows and columns swapped, RMSNorm per head instead of over D, a RoPE turning
 the wrong way or reading the wrong coordinate, the text and image key weights
 swapped, the unconditional row keeping its text, the block's branches all
-reading its input, every block running with block 0's weights.  The pin must fail on each.
+reading its input, every block running with block 0's weights, the guidance
+combination with its rows exchanged.  The pin must fail on each.
 """
 import unittest.mock as um
 
@@ -338,6 +340,52 @@ def test_whole_model_pin_catches_every_block_reading_block_0(monkeypatch):
     orig = O.block_forward
     monkeypatch.setattr(O, "block_forward", lambda X, e0, w, blk, kv, dims, *a, **k: orig(X, e0, w, 0, kv, dims, *a, **k))
     assert _whole_model_error() > 1e-3
+
+
+def sample_torch(x0, img_lat, w, txt, clip, d, steps, s):
+    """The CFG Euler sampler restated around dit_torch: y = the 4-channel mask
+    (all ones on latent frame 0, the default known first frame) stacked on the
+    image latent; the conditional row with the text, the unconditional row with
+    zeroed text (CLIP and y kept); at step k of N, tau = 1000 (1 - k/N) and
+    x += (1/N) (v_u + s (v_c - v_u)) ("图解 Wan2.1 I2V" 4.1, 7, Q5;
+    "Wan（通义万相）..." 2.7)."""
+    mask = np.zeros((4,) + img_lat.shape[1:])
+    mask[:, 0] = 1.0
+    y = np.concatenate([mask, img_lat])
+    txt2 = np.stack([txt, np.zeros_like(txt)])
+    x = np.asarray(x0, np.float64)
+    for k in range(steps):
+        v = dit_torch(np.stack([x, x]), y, 1000.0 * (1.0 - k / steps), w, txt2, clip, d)
+        x = x + (1.0 / steps) * (v[1] + s * (v[0] - v[1]))
+    return x
+
+
+def _sampler_error():
+    d = synth.Dims(D=48, heads=2, ffn=40, blocks=2, T=2, H=4, W=6, n_txt=5, c_txt=12, n_img=4, c_img=10,
+                   dtype="f32")
+    wl = synth.Workload("pin3", d, batch=2, seed=97)
+    w = {k: v.astype(np.float64) for k, v in synth.model_weights(wl).items()}
+    for k in list(w):
+        if k.endswith(".w"):
+            w[k] = w[k] * 6
+    x0 = RNG.standard_normal((16, d.T, d.H, d.W))
+    img_lat = RNG.standard_normal((16, d.T, d.H, d.W))
+    txt = RNG.standard_normal((d.n_txt, d.c_txt))
+    clip = RNG.standard_normal((d.n_img, d.c_img))
+    got, _ = O.sample(x0, img_lat, w, txt, clip, d, steps=3, cfg_scale=5.0)
+    want = sample_torch(x0, img_lat, w, txt, clip, d, 3, 5.0)
+    assert np.abs(want - x0).max() > 1.0
+    return float(np.abs(got - want).max() / np.abs(want).max())
+
+
+def test_sampler_against_torch_restatement():
+    assert _sampler_error() < 1e-12
+
+
+def test_sampler_pin_catches_swapped_guidance_rows(monkeypatch):
+    """The guidance combination with its rows exchanged (v_c + s (v_u - v_c))."""
+    monkeypatch.setattr(O, "cfg_combine", lambda v_c, v_u, s: np.asarray(v_c) + s * (np.asarray(v_u) - np.asarray(v_c)))
+    assert _sampler_error() > 1e-3
 
 
 # ------------------------------------------------------------------ cross-attention keys and values
