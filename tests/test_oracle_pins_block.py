@@ -231,8 +231,10 @@ def block_torch(X, e0, w, d, kv, blk=0):
 
     def sdpa(q, k, v):
         return TF.scaled_dot_product_attention(sp(q), sp(k), sp(v)).transpose(1, 2).reshape(q.shape)
-    ki, vi = T64(kv["k_img"]).expand(B, -1, -1), T64(kv["v_img"]).expand(B, -1, -1)
-    oc = sdpa(qc, ki, vi) + sdpa(qc, T64(kv["k_txt"]), T64(kv["v_txt"]))
+    oc = sdpa(qc, T64(kv["k_txt"]), T64(kv["v_txt"]))
+    if "k_img" in kv:   # the image-to-video model's second stream
+        ki, vi = T64(kv["k_img"]).expand(B, -1, -1), T64(kv["v_img"]).expand(B, -1, -1)
+        oc = sdpa(qc, ki, vi) + oc
     x2 = x1 + TF.linear(oc, T64(w[p + "co.w"]), T64(w[p + "co.b"]))
     h2 = TF.layer_norm(x2, (D,), eps=d.eps) * (1 + T64(mod[4])) + T64(mod[3])
     u = TF.gelu(TF.linear(h2, T64(w[p + "f1.w"]), T64(w[p + "f1.b"])))
@@ -294,23 +296,27 @@ def dit_torch(x_t, y, tau, w, txt, clip, d):
     es = torch.cat([torch.cos(tau * fr), torch.sin(tau * fr)])
     e = TF.linear(TF.silu(TF.linear(es, W("t1.w"), W("t1.b"))), W("t2.w"), W("t2.b"))
     e0 = TF.linear(TF.silu(e), W("tp.w"), W("tp.b")).reshape(6, D)
-    x_in = torch.cat([T64(x_t), T64(y)[None].expand(B, -1, -1, -1, -1)], dim=1)
-    X = TF.conv3d(x_in, W("pe.w").reshape(D, 36, 1, 2, 2), W("pe.b"), stride=(1, 2, 2)).flatten(2).transpose(1, 2)
+    x_in = T64(x_t) if y is None else torch.cat([T64(x_t), T64(y)[None].expand(B, -1, -1, -1, -1)], dim=1)
+    X = TF.conv3d(x_in, W("pe.w").reshape(D, x_in.shape[1], 1, 2, 2), W("pe.b"), stride=(1, 2, 2))
+    X = X.flatten(2).transpose(1, 2)
     mlp = lambda x, a, b: TF.linear(TF.gelu(TF.linear(x, W(a + ".w"), W(a + ".b"))), W(b + ".w"), W(b + ".b"))
-    ctx_t, ctx_i = mlp(T64(txt), "txt1", "txt2"), mlp(T64(clip), "img1", "img2")
+    ctx_t = mlp(T64(txt), "txt1", "txt2")
+    streams = [("k_txt", ctx_t, "ck"), ("v_txt", ctx_t, "cv")]
+    if clip is not None:   # image-to-video: the CLIP context and its own keys and values
+        ctx_i = mlp(T64(clip), "img1", "img2")
+        streams += [("k_img", ctx_i, "cki"), ("v_img", ctx_i, "cvi")]
     for i in range(d.blocks):
         p = f"blk{i}."
-        kv = {n: TF.linear(c, W(p + k + ".w"), W(p + k + ".b")).numpy()
-              for n, c, k in (("k_txt", ctx_t, "ck"), ("v_txt", ctx_t, "cv"), ("k_img", ctx_i, "cki"),
-                              ("v_img", ctx_i, "cvi"))}
+        kv = {n: TF.linear(c, W(p + k + ".w"), W(p + k + ".b")).numpy() for n, c, k in streams}
         X = T64(block_torch(X.numpy(), e0.numpy(), w, d, kv, i))
     z = TF.layer_norm(X, (D,), eps=d.eps) * (1 + e + W("head.mod")[1]) + e + W("head.mod")[0]
     pt = TF.linear(z, W("head.w"), W("head.b"))                                   # [B, L, 16 * 1 * 2 * 2]
     return pt.reshape(B, T, Hp, Wp, 16, 2, 2).permute(0, 4, 1, 2, 5, 3, 6).reshape(B, 16, T, 2 * Hp, 2 * Wp).numpy()
 
 
-def _whole_model_error():
-    d = synth.Dims(D=48, heads=2, ffn=40, blocks=2, T=2, H=4, W=6, n_txt=5, c_txt=12, n_img=4, c_img=10,
+def _whole_model_error(t2v=False):
+    n_img, c_img = (0, 0) if t2v else (4, 10)
+    d = synth.Dims(D=48, heads=2, ffn=40, blocks=2, T=2, H=4, W=6, n_txt=5, c_txt=12, n_img=n_img, c_img=c_img,
                    dtype="f32")
     wl = synth.Workload("pin2", d, batch=2, seed=98)
     w = {k: v.astype(np.float64) for k, v in synth.model_weights(wl).items()}
@@ -318,9 +324,9 @@ def _whole_model_error():
         if k.endswith(".w"):
             w[k] = w[k] * 6
     x_t = RNG.standard_normal((2, 16, d.T, d.H, d.W))
-    y = RNG.standard_normal((20, d.T, d.H, d.W))
+    y = None if t2v else RNG.standard_normal((20, d.T, d.H, d.W))
     txt = RNG.standard_normal((2, d.n_txt, d.c_txt))
-    clip = RNG.standard_normal((d.n_img, d.c_img))
+    clip = None if t2v else RNG.standard_normal((d.n_img, d.c_img))
     tau = 731.0
     ctx_t, ctx_i = O.context_embed(w, txt, clip)
     kvs = [O.cross_kv(w, i, ctx_t, ctx_i) for i in range(d.blocks)]
@@ -330,8 +336,11 @@ def _whole_model_error():
     return float(np.abs(got - want).max() / np.abs(want).max())
 
 
-def test_whole_model_against_torch_restatement():
-    assert _whole_model_error() < 1e-12
+@pytest.mark.parametrize("t2v", [False, True])
+def test_whole_model_against_torch_restatement(t2v):
+    """Image-to-video, and text-to-video (x_t alone through a 16-channel patch
+    embedding, text-only cross-attention; "图解 Wan2.1 I2V" 9)."""
+    assert _whole_model_error(t2v) < 1e-12
 
 
 def test_whole_model_pin_catches_every_block_reading_block_0(monkeypatch):
