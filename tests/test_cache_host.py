@@ -1,5 +1,6 @@
 """The samplers' caches in model.py (host code) against the oracle's rules, on
-the CPU ("Wan（通义万相）..." 5.3: CFG cache, attention cache, both at once).
+the CPU ("Wan（通义万相）..." 5.3: CFG cache, attention cache, both at once;
+7.2: the timestep MoE's choice of expert).
 The library calls are replaced by recorders, so only the decision and
 bookkeeping code of model.CfgCache, model.AttnCache and model.DiffusionCache
 runs; the oracle's samplers run with a stand-in DiT (zeros) so that their own
@@ -110,3 +111,29 @@ def test_diffusion_cache_takes_the_oracle_decisions(monkeypatch, no_library, ste
         dc.cfg_euler_step(xb, None, tau, dt, 5.0)
     got = [(batch == 2, fresh) for batch, fresh in no_library]
     assert got == _oracle_decisions(monkeypatch, "diffusion", steps, t_cfg=t_cfg, t_attn=t_attn, interval=interval)
+
+
+class _Expert:
+    def __init__(self):
+        self.steps = 0
+
+    def cfg_euler_step(self, xb, y, tau, dt, cfg_scale, stream=None):
+        self.steps += 1
+        return xb
+
+
+@pytest.mark.parametrize("steps,t_moe", [(4, 0.6), (12, 0.5), (12, 0.875), (12, 1.0), (12, -1.0), (7, 0.4)])
+def test_moe_runs_the_expert_the_oracle_picks(monkeypatch, steps, t_moe):
+    moe = model.MoE.__new__(model.MoE)
+    moe.high, moe.low, moe.t_moe = _Expert(), _Expert(), t_moe
+    xb = torch.zeros((2,) + SHAPE)
+    got = []
+    for _, dt, tau in O.schedule(steps):
+        before = moe.high.steps
+        moe.cfg_euler_step(xb, None, tau, dt, 5.0)
+        got.append("high" if moe.high.steps > before else "low")
+    monkeypatch.setattr(O, "dit_forward", lambda xb, *a, **k: np.zeros((xb.shape[0],) + SHAPE))
+    w = synth.model_weights(WL)
+    x = synth.inputs(WL)
+    used = O.sample_moe(x["x0"], x["img_lat"], w, w, x["txt"], x["clip"], WL.dims, steps, 5.0, t_moe)[2]
+    assert got == used
