@@ -312,7 +312,9 @@ wd_status wd_patch_embed_noalloc(const wd_dims* d, const float* x_t, const float
 /* C = epilogue(A B^T + bias) for A [M,K] and B [N,K] (a Linear weight), both
  * in `dtype` (wd_dtype), row-major with leading dimension K; bias [N] fp32 or
  * NULL.  epilogue 0: out [M,N] = v in dtype; 1: out = GELU(v) (erf form,
- * [I2V] 5.5) in dtype; 2: out = v in fp32; 3: out [M,N] fp32 += g*v with
+ * [I2V] 5.5; on the tensor cores the normal tail probability comes from
+ * Abramowitz-Stegun 7.1.26, within 3.3e-7 of the exact GELU, on the CUDA
+ * cores from erff) in dtype; 2: out = v in fp32; 3: out [M,N] fp32 += g*v with
  * g = gate_a + gate_b (either may be NULL; both NULL means 1) — the gated
  * residual of [I2V] 5.2; 5 (WD_BF16 only): out = v in IEEE half (the
  * cross-attention operands).  bf16 runs on the tcgen05 tensor cores (N a
