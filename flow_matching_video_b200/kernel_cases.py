@@ -30,6 +30,10 @@ from . import model, synth, wd  # noqa: E402
 
 L, D, H, F, NI, NT = 32760, 1536, 12, 8960, 257, 512
 
+CASES = ("attn_self", "attn_cross", "attn_fp8", "attn_fp8_quantize", "gemm_qkv", "gemm_o", "gemm_ffn1", "gemm_ffn2",
+         "gemm_ffn1_store", "euler", "euler_hbm", "gemm_fp8_qkv", "gemm_fp8_o", "gemm_fp8_ffn1", "gemm_fp8_ffn2",
+         "quant_ffn_hidden", "block_480p17", "block_480p81", "block_480p81_fp8", "block_480p81_fp8attn")
+
 
 def bf(*shape):
     return torch.randn(*shape, device="cuda").to(torch.bfloat16)
@@ -120,7 +124,7 @@ def make_case(name: str, B: int):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case")
+    ap.add_argument("case", choices=CASES)
     ap.add_argument("--batch", type=int, default=2)
     ap.add_argument("--iters", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=2)
